@@ -1,0 +1,420 @@
+"""Benchmark: W4A16 decode-sweep GEMV on B200 (plus the other hot-path rows as extras).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl ours|reference]
+
+Headline workload: the decode sweep of a synthetic Llama-style 1B stack (hidden 2048,
+intermediate 5632, 24 layers x 7 projections = 168 dyadic g64 matrices, 1,056,964,608
+weights), batch B bf16 N(0,1) activations. One step = one W4A16 GEMV over all 168 packed
+matrices (one grouped launch), inputs resident in HBM. The packed weights (535 MB) are
+larger than L2 (126 MB), so every step streams them from HBM; no flush is needed.
+
+value = effective weight bytes (packed nibbles + bf16 scales) streamed per second, GB/s.
+Multi-GPU: replicas only (the sweep has no exchange step); every rank runs the same
+sweep on its own GPU, time = max over ranks, value = all ranks' bytes / that time.
+--impl reference times the fp64 CPU oracle on host cores on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "W4A16 GEMV effective weight GB/s (% HBM peak); GEMM TFLOP/s; quantize Gweights/s"
+UNIT = "GB/s"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# inputs
+# ---------------------------------------------------------------------------------------
+
+def sweep_host_weights(threads: int = 8):
+    mats = workloads.sweep_matrices()
+    with ThreadPoolExecutor(threads) as ex:
+        ws = list(ex.map(lambda m: workloads.gaussian_outlier_weight(m[2], m[3], workloads.DECODE_SWEEP, m[4]), mats))
+    return mats, ws
+
+
+def build_sweep(wq, torch, dev, batch):
+    mats, host_w = sweep_host_weights()
+    packed = []
+    for (layer, name, n, k, idx), wb in zip(mats, host_w):
+        w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
+        pw, _ = wq.quantize_dyadic(w, 64)
+        packed.append(pw)
+        del w
+    xs_host = [workloads.activations(batch, k, workloads.DECODE_SWEEP, idx) for _, _, _, k, idx in mats]
+    xs = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in xs_host]
+    ys = [torch.empty((batch, n), dtype=torch.bfloat16, device=dev) for _, _, n, _, _ in mats]
+    torch.cuda.synchronize(dev)
+    return mats, packed, xs_host, xs, ys
+
+
+def sweep_bytes(mats, batch):
+    packed = sum(n * k // 2 for _, _, n, k, _ in mats)
+    scale = sum(n * (k // 64) * 2 for _, _, n, k, _ in mats)
+    xb = sum(batch * k * 2 for _, _, _, k, _ in mats)
+    yb = sum(batch * n * 2 for _, _, n, _, _ in mats)
+    return packed, scale, xb, yb
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+
+def time_region(torch, stream, fn, steps, warmup, barrier):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        fn()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return t0.elapsed_time(t1) / steps
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from w4a16_matmul_b200 import build as _build
+    _build.build()
+    import w4a16_matmul_b200 as wq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    B = args.batch
+    mats, packed, xs_host, xs, ys = build_sweep(wq, torch, dev, B)
+    stream = torch.cuda.current_stream(dev)
+    run = wq.GroupedGemv(packed, xs, ys)
+    pk_b, sc_b, x_b, y_b = sweep_bytes(mats, B)
+    weight_bytes = pk_b + sc_b
+    algo_bytes = pk_b + sc_b + x_b + y_b
+
+    clocks = ClockSampler(local)
+    # ---- headline: device-resident, one grouped launch per step ------------------------
+    clocks.start()
+    ms = time_region(torch, stream, run, args.steps, args.warmup, barrier)
+    clk = clocks.stop()
+    ms = max_over_ranks(ms)
+    value = world * weight_bytes / (ms * 1e-3) / 1e9
+    achieved = algo_bytes / (ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers ---------------------------
+    xs_pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in xs_host]
+    ys_pin = [torch.empty(y.shape, dtype=torch.bfloat16).pin_memory() for y in ys]
+
+    def e2e_step():
+        for xp, xd in zip(xs_pin, xs):
+            xd.copy_(xp, non_blocking=True)
+        run()
+        for yp, yd in zip(ys_pin, ys):
+            yp.copy_(yd, non_blocking=True)
+
+    ms_e2e = max_over_ranks(time_region(torch, stream, e2e_step, args.steps, args.warmup, barrier))
+    e2e = {"value": round(world * weight_bytes / (ms_e2e * 1e-3) / 1e9, 2), "unit": UNIT,
+           "h2d_bytes_per_step": x_b, "d2h_bytes_per_step": y_b, "ms_per_step": round(ms_e2e, 4)}
+
+    extras = {}
+    if not args.no_extras:
+        extras = run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrier,
+                            max_over_ranks)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u4+bf16->f32",
+        "data": "synthetic (seeded numpy PCG64, pages' value distributions)",
+        "config": {"workload": "decode sweep: 24 layers x {q,k,v,o,gate,up,down} dyadic g64, "
+                               "hidden 2048, intermediate 5632, 1,056,964,608 weights",
+                   "batch": B, "matrices": len(mats), "launch": "one grouped GEMV launch per step",
+                   "weight_bytes_per_step": weight_bytes, "l2": "inputs larger than L2 (535 MB/step)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": peaks["source"],
+                     "algorithmic_bytes_per_launch": algo_bytes, "kernel": "gemv_kernel (grouped)"},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "extras": extras,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args, mats, seconds=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrier, max_over_ranks):
+    """Secondary rows of the hot path, each on its own workload, timed the same way."""
+    out = {}
+    steps, warm = max(args.steps, 5), max(args.warmup, 3)
+    # decode sweep as 168 dependent-order launches captured in one CUDA graph
+    try:
+        g = torch.cuda.CUDAGraph()
+        s2 = torch.cuda.Stream(dev)
+        s2.wait_stream(stream)
+        with torch.cuda.stream(s2):
+            for pw, x, y in zip(packed, xs, ys):      # warm the path before capture
+                wq.gemv(pw, x, out=y)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s2):
+            for pw, x, y in zip(packed, xs, ys):
+                wq.gemv(pw, x, out=y)
+        ms = max_over_ranks(time_region(torch, stream, g.replay, steps, warm, barrier))
+        pk, sc, _, _ = sweep_bytes(mats, args.batch)
+        out["sweep_chain_graph"] = {"ms_per_step": round(ms, 4), "GB/s": round((pk + sc) / ms / 1e6, 1),
+                                    "launches_per_step": len(mats)}
+        del g
+    except Exception as e:  # report, never hide
+        out["sweep_chain_graph"] = {"error": repr(e)[:200]}
+    # other batch sizes of the grouped sweep
+    for b in (4, 16):
+        if b == args.batch:
+            continue
+        xs_b = [torch.randn((b, x.shape[1]), device=dev).to(torch.bfloat16) for x in xs]
+        ys_b = [torch.empty((b, y.shape[1]), dtype=torch.bfloat16, device=dev) for y in ys]
+        run_b = wq.GroupedGemv(packed, xs_b, ys_b)
+        ms = max_over_ranks(time_region(torch, stream, run_b, steps, warm, barrier))
+        pk, sc, xb, yb = sweep_bytes(mats, b)
+        out[f"sweep_batch{b}"] = {"ms_per_step": round(ms, 4), "GB/s": round((pk + sc) / ms / 1e6, 1),
+                                  "frac_hbm": round((pk + sc + xb + yb) / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    # dyadic quantisation of the whole stack (bf16 -> scale + packed), HBM-bound
+    try:
+        n_w = sum(n * k for _, _, n, k, _ in mats[:7])
+        wts = [torch.randn((n, k), device=dev).mul_(0.02).to(torch.bfloat16) for _, _, n, k, _ in mats[:7]]
+        outs = [(torch.empty((n, k // 64), dtype=torch.bfloat16, device=dev),
+                 torch.empty((n, k // 2), dtype=torch.uint8, device=dev)) for _, _, n, k, _ in mats[:7]]
+        import ctypes
+
+        def q():
+            for w, (s, p) in zip(wts, outs):
+                st = wq._lib.wq_quantize_dyadic(ctypes.c_void_p(w.data_ptr()), w.shape[0], w.shape[1], 64,
+                                                ctypes.c_void_p(s.data_ptr()), None,
+                                                ctypes.c_void_p(p.data_ptr()),
+                                                ctypes.c_void_p(stream.cuda_stream))
+                assert st == 0, wq.last_error()
+        ms = max_over_ranks(time_region(torch, stream, q, steps, warm, barrier))
+        byts = n_w * (2 + 0.5 + 2 / 64)
+        out["quantize_dyadic_layer"] = {"Gweights/s": round(n_w / ms / 1e6, 2),
+                                        "GB/s": round(byts / ms / 1e6, 1),
+                                        "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
+        # dense reconstruction of the same layer
+        def dq():
+            for pw in packed[:7]:
+                wq.dequant(pw)
+        ms = max_over_ranks(time_region(torch, stream, dq, steps, warm, barrier))
+        byts = n_w * (0.5 + 2 / 64 + 2)
+        out["dequant_layer"] = {"GB/s": round(byts / ms / 1e6, 1),
+                                "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
+        del wts, outs
+    except Exception as e:
+        out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle baseline / reference arm
+# ---------------------------------------------------------------------------------------
+
+def _oracle_sample_rows(mats, rows_per_matrix: int, seed: int = 0):
+    """A bounded sample of the sweep: `rows_per_matrix` rows of each of the 7 distinct
+    projection shapes of layer 0 (weights drawn and quantised by the oracle)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    sample = []
+    for layer, name, n, k, idx in mats[:7]:
+        rows = np.sort(rng.choice(n, min(rows_per_matrix, n), replace=False))
+        w = workloads.gaussian_outlier_weight(n, k, workloads.DECODE_SWEEP, idx)[rows]
+        s, c = oracle.dyadic_quantize(w, 64)
+        sample.append((oracle.pack(c), s, workloads.activations(1, k, workloads.DECODE_SWEEP, idx)))
+    return sample
+
+
+def cpu_baseline(args, mats, seconds: float = 15.0, batch: int | None = None):
+    import oracle
+    batch = batch or args.batch
+    threads = oracle.default_threads()
+    # calibrate on a small sample, then size the timed sample to ~`seconds`
+    small = _oracle_sample_rows(mats, 8)
+    t0 = time.perf_counter()
+    for packed, s, x in small:
+        oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, np.repeat(x, batch, 0), threads=threads)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    rows = int(max(8, min(4096, 8 * seconds / dt)))
+    sample = _oracle_sample_rows(mats, rows)
+    nbytes = sum(p.size + s.size * 2 for p, s, _ in sample)
+    t0 = time.perf_counter()
+    for packed, s, x in sample:
+        oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, np.repeat(x, batch, 0), threads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} rows of each of the 7 projection shapes of one sweep layer "
+                      f"(batch {batch}, fp64 dequant + dot), {dt:.1f} s"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    mats = workloads.sweep_matrices()
+    import oracle
+    threads = oracle.default_threads()
+    sample = _oracle_sample_rows(mats, args.ref_rows)
+    nbytes = sum(p.size + s.size * 2 for p, s, _ in sample)
+
+    def step():
+        for packed, s, x in sample:
+            oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, np.repeat(x, args.batch, 0), threads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = round(nbytes / dt / 1e9, 6)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded numpy PCG64, pages' value distributions)",
+            "config": {"workload": "decode sweep: 24 layers x {q,k,v,o,gate,up,down} dyadic g64, "
+                                   "hidden 2048, intermediate 5632, 1,056,964,608 weights",
+                       "batch": args.batch, "sample_rows_per_shape": args.ref_rows},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"{args.ref_rows} rows of each of the 7 projection shapes per step"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,215 @@
+/*
+ * wq.h -- C ABI of libwq: group-wise 4-bit weight coding and W4A16 matmul on B200
+ * (sm_100a).
+ *
+ * Sources cited below:
+ *   [DG]  "MiniCPM5-1B 验证: 6× 压缩, ppl 反超 fp, 1.2GB 显存, 50ms Triton 推理"
+ *         (DyadicGumbel 4-bit): §2.1 dyadic codebook, §2.2 block layout and
+ *         reconstruction, §2.3 hard argmin, §2.5 nibble pack and unpack-to-bf16.
+ *   [KM]  "K-Means量化技术：突破LLM低比特部署瓶颈": §1.2 per-block-64 k-means with
+ *         16 centroids, §2.2 LUT decoding, §4.1 kernel choice by batch size.
+ *   [G32] "int4-g32+warm 裸量化：原理与实验报告": §1.2 112-candidate shape grid,
+ *         §1.3 quantisation flow (candidate argmin, 25 Lloyd rounds, sign bit),
+ *         §2 storage format, §5.1-5.2 offline quantisation and inference.
+ *
+ * Conventions shared by every entry point
+ *   - Matrices are row-major. A weight W is [n, k] = (out, in); groups are runs of
+ *     `group` consecutive columns of one row. Activations x are [m, k], outputs y [m, n].
+ *   - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
+ *   - Every pointer is a DEVICE pointer (cudaMalloc / torch CUDA memory) of the current
+ *     device, 16-byte aligned, unless a parameter says it may be NULL. Host pointers are
+ *     rejected with WQ_EINVAL. The caller allocates and owns every buffer; the library
+ *     allocates nothing, frees nothing and keeps no pointer after a call returns.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream)
+ *     and runs asynchronously: buffers must stay alive until the stream is synchronised.
+ *   - Arguments are checked on the host before anything is launched; on any failure
+ *     nothing is launched and the status says why (details in wq_last_error()). A launch
+ *     failure reported by the CUDA runtime returns WQ_ECUDA.
+ *   - Inputs must be finite. NaN or Inf weights or activations give unspecified codes
+ *     and outputs (never a fault).
+ *   - Entry points are reentrant; concurrent calls on different streams are safe.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* wq_stream;
+
+typedef enum wq_status {
+    WQ_OK = 0,
+    WQ_EINVAL = 1,        /* bad size, NULL or non-device pointer, bad format field */
+    WQ_EALIGN = 2,        /* pointer not 16-byte aligned */
+    WQ_EUNSUPPORTED = 3,  /* valid request this build does not implement (e.g. group) */
+    WQ_ECUDA = 4,         /* the CUDA runtime reported an error (launch or attribute query) */
+    WQ_ETIMEOUT = 5       /* a bounded device-side wait gave up (reserved) */
+} wq_status;
+
+/* Static description of a status code. Never NULL. */
+const char* wq_status_string(int32_t status);
+
+/* Detail of the last failure on the calling host thread ("" if none). Thread-local;
+ * valid until the next failing call on that thread. */
+const char* wq_last_error(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int32_t wq_version(void);
+
+/* ------------------------------------------------------------------------------------ */
+/* Packed weight descriptor                                                              */
+/* ------------------------------------------------------------------------------------ */
+
+typedef enum wq_format {
+    /* [DG] §2.1-2.2: code idx in 0..15, w = step * (idx - 8), step = scale / 8, one bf16
+     * scale (the group's absmax) per group of 64 or 32. aux = bf16 [n, k/group]. */
+    WQ_FMT_DYADIC4 = 0,
+    /* [G32] §1.3-2: code = q | sign << 3 (q in 0..7 a magnitude level, sign 1 = negative),
+     * w = sign ? -level[q] : level[q]; 8 fp32 magnitude levels per group of 32.
+     * aux = fp32 [n, k/32, 8]. */
+    WQ_FMT_LLOYD8S = 1,
+    /* [KM] §1.2, §2.2: code = centroid index 0..15, w = centroid; 16 fp16 centroids per
+     * block of 64. aux = fp16 [n, k/64, 16]. */
+    WQ_FMT_LUT16 = 2
+} wq_format;
+
+typedef struct wq_weight {
+    int32_t fmt;            /* wq_format */
+    int32_t group;          /* DYADIC4: 64 or 32; LLOYD8S: 32; LUT16: 64 */
+    int64_t n;              /* rows (outputs), >= 1 */
+    int64_t k;              /* columns (inputs), >= 1, multiple of group */
+    const uint8_t* packed;  /* [n, k/2]: byte j of a row = code[2j] | code[2j+1] << 4
+                               ([DG] §2.5 "lo | hi << 4": even column in the low nibble) */
+    const void* aux;        /* per-group scale / levels / centroids, see wq_format */
+} wq_weight;
+
+/* ------------------------------------------------------------------------------------ */
+/* Producers                                                                             */
+/* ------------------------------------------------------------------------------------ */
+
+/* Dyadic 4-bit quantisation, [DG] §2.1-2.3 and §2.5. For every group of `group`
+ * consecutive weights of a row: scale = max |w| (stored as bf16, exact), and for every
+ * weight idx = argmin_j |w - (j - 8) * scale / 8| over j = 0..15, the lowest j on a tie.
+ *   w       bf16 [n, k], finite.
+ *   group   64 or 32; k % group == 0.
+ *   scale   out bf16 [n, k/group].
+ *   codes   out uint8 [n, k] (one code per byte), may be NULL.
+ *   packed  out uint8 [n, k/2] (two codes per byte, see wq_weight), may be NULL.
+ * At least one of codes / packed must be non-NULL. An all-zero group gets scale 0 and
+ * codes 0 (every code ties). Output is bit-exact (no floating-point freedom). */
+wq_status wq_quantize_dyadic(const uint16_t* w, int64_t n, int64_t k, int32_t group,
+                             uint16_t* scale, uint8_t* codes, uint8_t* packed,
+                             wq_stream stream);
+
+typedef enum wq_lloyd_mode {
+    /* [G32] §1.3: per group of 32 magnitudes, the lowest-MSE of the 112 candidate shapes
+     * of §1.2 gives 8 initial levels; `rounds` Lloyd rounds (nearest level, lowest index
+     * on a tie; level = mean of its members, an empty level keeps its value) and a
+     * final nearest assignment; sign kept as bit 3 of the code. codebook = fp32
+     * [n, k/32, 8] levels, params = the per-group byte family << 7 | b_rel index << 3 |
+     * beta index of [G32] §2, mse_trace = [n, k/32, rounds + 2] (candidate MSE, then the
+     * MSE after each assignment). */
+    WQ_LLOYD_G32_WARM = 0,
+    /* [KM] §1.2: per block of 64 signed weights, 16 centroids initialised at the
+     * (4i+2)-th smallest value, `rounds` Lloyd rounds as above, centroids rounded to
+     * fp16 and a final nearest assignment against the fp16 centroids. codebook = fp16
+     * [n, k/64, 16] (the LUT16 aux), params unused, mse_trace = [n, k/64, rounds + 1]. */
+    WQ_LLOYD_KMEANS16 = 1
+} wq_lloyd_mode;
+
+typedef struct wq_lloyd_params {
+    int32_t mode;    /* wq_lloyd_mode */
+    int32_t rounds;  /* Lloyd rounds, 0..64; the pages use 25 */
+} wq_lloyd_params;
+
+/* Codebook quantisation (Lloyd / k-means), [G32] §1.3 and §5.1, [KM] §1.2.
+ *   w         bf16 [n, k], finite; k % 32 == 0 (G32_WARM) or k % 64 == 0 (KMEANS16).
+ *   codes     out uint8 [n, k], may be NULL.
+ *   packed    out uint8 [n, k/2], may be NULL (at least one of codes / packed).
+ *   codebook  out, see wq_lloyd_mode.
+ *   params    out uint8 [n, k/32] (G32_WARM only), may be NULL.
+ *   mse_trace out fp32, see wq_lloyd_mode, may be NULL.
+ * Both modes take their decisions in double precision (G32_WARM screens the 112
+ * candidates in fp32 first and re-ranks the near-best ones in double). */
+wq_status wq_quantize_lloyd(const uint16_t* w, int64_t n, int64_t k, const wq_lloyd_params* p,
+                            uint8_t* codes, uint8_t* packed, void* codebook, uint8_t* params,
+                            float* mse_trace, wq_stream stream);
+
+/* ------------------------------------------------------------------------------------ */
+/* Packing and reconstruction                                                            */
+/* ------------------------------------------------------------------------------------ */
+
+/* [DG] §2.5 pack: packed[r, j] = codes[r, 2j] | codes[r, 2j+1] << 4. codes must be in
+ * 0..15 (higher bits are dropped). k even, k % 32 == 0. */
+wq_status wq_pack(const uint8_t* codes, int64_t n, int64_t k, uint8_t* packed, wq_stream stream);
+
+/* Inverse of wq_pack: codes[r, 2j] = packed & 15, codes[r, 2j+1] = packed >> 4. */
+wq_status wq_unpack(const uint8_t* packed, int64_t n, int64_t k, uint8_t* codes, wq_stream stream);
+
+/* Dense reconstruction of a packed weight ([DG] §2.5 unpack; [G32] §5.2; [KM] §2.2):
+ *   DYADIC4 -> bf16(step * (idx - 8)), one rounding to nearest even;
+ *   LLOYD8S -> bf16(+/- level[q]);
+ *   LUT16   -> the fp16 centroid itself (out holds fp16 patterns).
+ *   out  [n, k] 16-bit patterns. Bit-exact. */
+wq_status wq_dequant(const wq_weight* w, uint16_t* out, wq_stream stream);
+
+/* ------------------------------------------------------------------------------------ */
+/* W4A16 consumers                                                                       */
+/* ------------------------------------------------------------------------------------ */
+
+/* Decode-side W4A16 GEMV ([DG] §2.5/§3.2 fused unpack; [KM] §2.2, §4.1 small batch):
+ * y[b, r] = sum_c Wdeq[r, c] * x[b, c], fp32 accumulation, bf16 output (rounded to
+ * nearest even), for b < batch. Wdeq is the reconstruction wq_dequant gives (bf16 for
+ * DYADIC4 / LLOYD8S; for LUT16 the fp16 centroid, with x converted to fp16, exact for
+ * |x| in [2^-14, 65504]; |x| > 65504 is outside the contract).
+ *   w      packed weight (any format).
+ *   x      bf16 [batch, k].
+ *   batch  1..16.
+ *   y      out bf16 [batch, n].
+ * Within |y - y_ref| <= 2e-3 * sum_c |Wdeq[r, c]| * |x[b, c]| of the exact product y_ref.
+ * Needs no workspace; one kernel launch. */
+wq_status wq_gemv_w4a16(const wq_weight* w, const uint16_t* x, int32_t batch, uint16_t* y,
+                        wq_stream stream);
+
+/* Several independent GEMVs in ONE launch (e.g. the q/k/v projections of a decoder layer,
+ * which share an input, or a whole stack of layers with independent inputs). Problem i
+ * computes ys[i] = Wdeq(ws[i]) xs[i] as wq_gemv_w4a16 does. ws, xs, ys are HOST arrays
+ * of `count` entries (the pointers they hold are device pointers); all weights must have
+ * the same format and group. count in 1..WQ_GEMV_MAX_GROUPED. */
+#define WQ_GEMV_MAX_GROUPED 192
+wq_status wq_gemv_w4a16_grouped(const wq_weight* ws, const uint16_t* const* xs,
+                                uint16_t* const* ys, int32_t count, int32_t batch,
+                                wq_stream stream);
+
+/* Bytes of device workspace wq_gemm_w4a16 needs for this weight and m (0 if none). */
+size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
+
+/* Prefill-side W4A16 GEMM on the tcgen05 tensor cores ([KM] §4.1 large batch; [DG] §3.2
+ * "materialized" bf16 path fused): y[i, r] = sum_c Wdeq[r, c] * x[i, c] for i < m, fp32
+ * accumulation in tensor memory, bf16 output. Formats DYADIC4 (group 64 or 32).
+ *   x      bf16 [m, k]; m >= 1; k % 64 == 0.
+ *   y      out bf16 [m, n].
+ *   ws     device workspace of at least wq_gemm_workspace_bytes(w, m) bytes (NULL if 0).
+ * Same tolerance as wq_gemv_w4a16. */
+wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y,
+                        void* ws, size_t ws_bytes, wq_stream stream);
+
+/* ------------------------------------------------------------------------------------ */
+/* Failure injection (host side only)                                                    */
+/* ------------------------------------------------------------------------------------ */
+
+/* Make the next `count` entry points that would launch work fail with WQ_ECUDA before
+ * launching anything (for testing callers' error paths without a GPU fault). 0 clears.
+ * Process-wide. */
+void wq_debug_fail_next_launches(int32_t count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

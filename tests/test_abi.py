@@ -1,0 +1,71 @@
+"""CPU-side checks of the C ABI: the library loads, exports every function include/wq.h
+declares, and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+
+def test_library_exports_every_header_function(wq):
+    names = wq.header_functions()
+    expected = {"wq_status_string", "wq_last_error", "wq_version", "wq_quantize_dyadic",
+                "wq_quantize_lloyd", "wq_pack", "wq_unpack", "wq_dequant", "wq_gemv_w4a16",
+                "wq_gemv_w4a16_grouped", "wq_gemm_workspace_bytes", "wq_gemm_w4a16",
+                "wq_debug_fail_next_launches"}
+    assert expected <= set(names), set(names) ^ expected
+    for n in names:
+        assert hasattr(wq._lib, n), n
+
+
+def test_status_strings_and_version(wq):
+    for s in range(6):
+        assert wq._lib.wq_status_string(s).decode().startswith("WQ_")
+    assert wq._lib.wq_status_string(99).decode() == "unknown wq_status"
+    assert wq.version() >= 100
+
+
+def test_shape_and_group_checks_fail_before_any_cuda_call(wq):
+    lib = wq._lib
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    # unsupported group
+    assert lib.wq_quantize_dyadic(p, 4, 64, 16, p, p, p, None) == wq.WQ_EUNSUPPORTED
+    assert "group" in wq.last_error()
+    # k not a multiple of 32 / of the group, non-positive sizes
+    assert lib.wq_quantize_dyadic(p, 4, 48, 32, p, p, p, None) == wq.WQ_EINVAL
+    assert lib.wq_quantize_dyadic(p, 4, 96, 64, p, p, p, None) == wq.WQ_EINVAL
+    assert lib.wq_quantize_dyadic(p, 0, 64, 64, p, p, p, None) == wq.WQ_EINVAL
+    assert lib.wq_pack(p, 4, 30, p, None) == wq.WQ_EINVAL
+    # NULL weight descriptor, bad batch, bad lloyd params
+    assert lib.wq_gemv_w4a16(None, p, 1, p, None) == wq.WQ_EINVAL
+    d = wq.WqWeight(wq.FMT_DYADIC4, 64, 4, 64, p.value, p.value)
+    assert lib.wq_gemv_w4a16(ctypes.byref(d), p, 17, p, None) == wq.WQ_EINVAL
+    d.fmt = 7
+    assert lib.wq_dequant(ctypes.byref(d), p, None) == wq.WQ_EINVAL
+    prm = wq.WqLloydParams(5, 25)
+    assert lib.wq_quantize_lloyd(p, 4, 64, ctypes.byref(prm), p, p, p, None, None, None) == wq.WQ_EINVAL
+    prm = wq.WqLloydParams(0, 100)
+    assert lib.wq_quantize_lloyd(p, 4, 64, ctypes.byref(prm), p, p, p, None, None, None) == wq.WQ_EINVAL
+    assert lib.wq_gemv_w4a16_grouped(None, None, None, 1, 1, None) == wq.WQ_EINVAL
+
+
+def test_misaligned_and_host_pointers_are_rejected(wq):
+    lib = wq._lib
+    buf = (ctypes.c_uint8 * 256)()
+    base = ctypes.addressof(buf)
+    aligned = (base + 15) // 16 * 16
+    st = lib.wq_pack(ctypes.c_void_p(aligned + 1), 2, 64, ctypes.c_void_p(aligned), None)
+    assert st == wq.WQ_EALIGN
+    # a host pointer is never accepted (no GPU here: the attribute query fails; on a GPU
+    # box it reports unregistered host memory) -- either way WQ_EINVAL, nothing launched
+    st = lib.wq_pack(ctypes.c_void_p(aligned), 2, 64, ctypes.c_void_p(aligned + 128), None)
+    assert st == wq.WQ_EINVAL
+    assert "device memory" in wq.last_error() or "cudaPointerGetAttributes" in wq.last_error()
+
+
+def test_binding_refuses_cpu_tensors(wq):
+    with pytest.raises(ValueError):
+        wq.quantize_dyadic(torch.zeros(4, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        wq.pack(torch.zeros(4, 64, dtype=torch.uint8))

@@ -1,0 +1,151 @@
+"""GPU parity of the W4A16 GEMV against the oracle's fp64 product of its own
+reconstruction: |y - y_ref| <= 2e-3 * sum_c |Wdeq[r, c]| |x[b, c]| per output element
+(the stated tolerance), plus exact special cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from _util import bits, f32, to_dev, to_dev_bits
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+def _dyadic_weight(wq, n, k, group, seed):
+    w_bits = workloads.gaussian_outlier_weight(n, k, workloads.DYADIC_1, seed)
+    s, c = oracle.dyadic_quantize(w_bits, group)
+    packed = oracle.pack(c)
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, group, n, k, to_dev(packed), to_dev_bits(s))
+    return pw, packed, s
+
+
+def _check(y, y_ref, bound, rows=None):
+    y = f32(y)
+    if rows is not None:
+        y = y[:, rows]
+    err = np.abs(y - y_ref)
+    ok = err <= TOL * bound
+    assert ok.all(), f"max err/bound {np.max(err / np.maximum(bound, 1e-300)):.3g}"
+    return float(np.max(err / np.maximum(bound, 1e-300)))
+
+
+@pytest.mark.parametrize("batch", [1, 2, 4, 8, 9, 16])
+@pytest.mark.parametrize("n,k,group", [(8, 256, 64), (13, 320, 64), (37, 1088, 64),
+                                       (300, 2048, 64), (24, 2144, 32), (5, 32, 32)])
+def test_gemv_dyadic_matches_oracle(wq, n, k, group, batch):
+    pw, packed, s = _dyadic_weight(wq, n, k, group, n + k + group)
+    x_bits = workloads.activations(batch, k, workloads.DECODE_SWEEP, n)
+    y = wq.gemv(pw, to_dev_bits(x_bits))
+    y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, group, x_bits)
+    _check(y, y_ref, bound)
+
+
+@pytest.mark.parametrize("group", [64, 32])
+def test_gemv_one_hot_reproduces_dequantised_column_exactly(wq, group):
+    n, k = 40, 512
+    pw, packed, s = _dyadic_weight(wq, n, k, group, 5)
+    wd = oracle.dequant(oracle.DYADIC4, packed, s, group)
+    cols = [0, 1, 7, 31, 32, 63, 64, 255, 256, 511]
+    x = np.zeros((len(cols), k))
+    for i, c in enumerate(cols):
+        x[i, c] = 1.0
+    y = wq.gemv(pw, to_dev_bits(workloads.f64_to_bf16_bits(x)))
+    got = f32(y)
+    for i, c in enumerate(cols):
+        assert np.array_equal(got[i], oracle.bf16_to_f64(wd[:, c]))
+
+
+def test_gemv_all_codes_eight_is_exact_zero_and_unit_group_sums(wq):
+    n, k = 24, 384
+    packed = np.full((n, k // 2), 0x88, np.uint8)
+    s = workloads.f64_to_bf16_bits(np.random.default_rng(1).uniform(0.01, 3, (n, k // 64)))
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(packed), to_dev_bits(s))
+    x = workloads.activations(16, k, workloads.DECODE_SWEEP, 3)
+    assert np.all(f32(wq.gemv(pw, to_dev_bits(x))) == 0.0)
+    g = np.random.default_rng(2)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    scale = np.full((n, k // 64), 0x3E00, np.uint16)          # step 1/64: sums exact in bf16
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(oracle.pack(codes)), to_dev_bits(scale))
+    xs = np.zeros((6, k))
+    for grp in range(6):
+        xs[grp, grp * 64:(grp + 1) * 64] = 1.0
+    y = f32(wq.gemv(pw, to_dev_bits(workloads.f64_to_bf16_bits(xs))))
+    for grp in range(6):
+        expect = (codes[:, grp * 64:(grp + 1) * 64].astype(np.int64) - 8).sum(1) / 64.0
+        assert np.array_equal(y[grp], expect)
+
+
+@pytest.mark.parametrize("batch", [1, 4, 16])
+def test_grouped_gemv_equals_single_calls(wq, batch):
+    shapes = [(2048, 2048), (256, 2048), (300, 1088), (5632, 2048), (2048, 5632)]
+    ws, xs, xbits, packs = [], [], [], []
+    for i, (n, k) in enumerate(shapes):
+        pw, packed, s = _dyadic_weight(wq, n, k, 64, 100 + i)
+        ws.append(pw)
+        packs.append((packed, s))
+        xb = workloads.activations(batch, k, workloads.DECODE_SWEEP, 100 + i)
+        xbits.append(xb)
+        xs.append(to_dev_bits(xb))
+    ys = wq.gemv_grouped(ws, xs)
+    for w, x, y in zip(ws, xs, ys):
+        assert torch.equal(y, wq.gemv(w, x))
+    # and against the oracle on sampled rows
+    rng = np.random.default_rng(3)
+    for (packed, s), xb, y in zip(packs, xbits, ys):
+        rows = rng.choice(packed.shape[0], 64, replace=False)
+        y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, xb, rows=rows)
+        _check(y, y_ref, bound, rows)
+
+
+def test_decode_sweep_layer_full_size_sampled(wq):
+    """One layer of the decode-sweep stack at full size, quantised on the GPU, in the
+    grouped launch the benchmark times; sampled rows of every projection against the
+    oracle, at batch 1 and 16."""
+    mats = [m for m in workloads.sweep_matrices(1)]
+    ws, pk = [], []
+    for layer, name, n, k, idx in mats:
+        w_bits = workloads.gaussian_outlier_weight(n, k, workloads.DECODE_SWEEP, idx)
+        pw, _ = wq.quantize_dyadic(to_dev_bits(w_bits), 64)
+        ws.append(pw)
+        pk.append((pw.packed.cpu().numpy(), bits(pw.aux)))
+    rng = np.random.default_rng(4)
+    for batch in (1, 16):
+        xb = [workloads.activations(batch, k, workloads.DECODE_SWEEP, idx) for _, _, _, k, idx in mats]
+        ys = wq.gemv_grouped(ws, [to_dev_bits(x) for x in xb])
+        for (packed, s), x, y in zip(pk, xb, ys):
+            rows = rng.choice(packed.shape[0], 48, replace=False)
+            y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x, rows=rows)
+            _check(y, y_ref, bound, rows)
+
+
+def test_gemv_host_input_path(wq):
+    pw, packed, s = _dyadic_weight(wq, 64, 512, 64, 9)
+    x_bits = workloads.activations(2, 512, workloads.DECODE_SWEEP, 9)
+    xc = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16)
+    y = wq.gemv(pw, xc)
+    assert y.device.type == "cpu"
+    assert torch.equal(y, wq.gemv(pw, xc.cuda()).cpu())
+
+
+def test_gemv_lut16_matches_oracle(wq):
+    n, k = 96, 1024
+    g = np.random.default_rng(11)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    lut = oracle.f64_to_fp16(np.sort(g.standard_normal((n, k // 64, 16)), -1) * 0.01)
+    packed = oracle.pack(codes)
+    pw = wq.PackedWeight(wq.FMT_LUT16, 64, n, k, to_dev(packed), to_dev_bits(lut, torch.float16))
+    for batch in (1, 8, 16):
+        x_bits = workloads.activations(batch, k, workloads.LUT16, batch)
+        y = wq.gemv(pw, to_dev_bits(x_bits))
+        y_ref, bound = oracle.matmul_rows(oracle.LUT16, packed, lut, 64, x_bits)
+        _check(y, y_ref, bound)
+    # one-hot: the fp16 centroid rounded once to bf16
+    x = np.zeros((3, k))
+    x[0, 0] = x[1, 65] = x[2, 1023] = 1.0
+    y = f32(wq.gemv(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
+    wd = oracle.fp16_to_f64(oracle.dequant(oracle.LUT16, packed, lut, 64))
+    for i, c in enumerate([0, 65, 1023]):
+        assert np.array_equal(y[i], oracle.bf16_to_f64(oracle.f64_to_bf16(wd[:, c])))

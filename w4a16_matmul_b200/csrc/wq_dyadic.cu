@@ -1,0 +1,255 @@
+// wq_dyadic.cu -- dyadic 4-bit quantisation ("MiniCPM5-1B 验证: 6× 压缩…" §2.1-2.3),
+// nibble pack / unpack (§2.5) and dense reconstruction of all three packed formats.
+//
+// All four kernels are HBM-bound streams: one thread owns a 16-byte chunk of the widest
+// array it touches, loads are 128-bit and coalesced, grids are a multiple of the SM count
+// and loop grid-stride.
+#include "wq_internal.cuh"
+
+namespace wq {
+namespace {
+
+constexpr int kThreads = 256;
+
+int stream_grid(int64_t items, int per_sm_blocks = 8) {
+    int64_t blocks = (items + kThreads - 1) / kThreads;
+    int64_t cap = (int64_t)sm_count() * per_sm_blocks;
+    if (blocks > cap) blocks = cap;
+    return (int)(blocks < 1 ? 1 : blocks);
+}
+
+// ---------------------------------------------------------------------------------------
+// Quantisation: scale = max|w| per group; idx = #{j in 1..15 : w > (2j-17) * scale/16}.
+//
+// That count is the argmin over the 16 codes with the lowest index on a tie (the
+// midpoint between codes j-1 and j is (2j-17) * scale / 16, and a weight exactly on a
+// midpoint stays with the lower code). With t = 16 w / scale it equals
+// (ceil(t) + 16) >> 1 clamped to 0..15: the count only changes where t crosses an odd
+// integer. t is formed with one correctly rounded reciprocal per group and one multiply
+// (relative error <= 2^-23, |t| <= 16, so |error| < 2e-6). For bf16 w and scale with
+// 16 w / scale != u (u odd, |u| <= 15) the distance |16 w / scale - u| is at least
+// 2^-16, so t is on the right side of every odd integer except when w sits exactly on
+// a midpoint; that case can only overshoot by one, and is corrected by an exact
+// comparison against the midpoint below (a bf16 times an odd integer <= 17 over 16, exact
+// in fp32).
+// ---------------------------------------------------------------------------------------
+template <int G>
+__global__ void __launch_bounds__(kThreads)
+quantize_dyadic_kernel(const uint4* __restrict__ w, int64_t n_chunks, int64_t k,
+                       uint16_t* __restrict__ scale, uint2* __restrict__ codes,
+                       uint32_t* __restrict__ packed) {
+    constexpr int LANES = G / 8;                 // threads per group (8 or 4)
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t chunks_per_row = k / 8;
+    for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); c0 < n_chunks;
+         c0 += stride) {
+        const int64_t c = c0 + (threadIdx.x & 31);
+        const bool live = c < n_chunks;          // groups never straddle n_chunks
+        uint4 v = live ? ldg_nc_v4(w + c) : make_uint4(0, 0, 0, 0);
+        uint32_t h[8] = {v.x & 0xFFFF, v.x >> 16, v.y & 0xFFFF, v.y >> 16,
+                         v.z & 0xFFFF, v.z >> 16, v.w & 0xFFFF, v.w >> 16};
+        float f[8];
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            f[i] = bf16_bits_to_float(h[i]);
+            amax = fmaxf(amax, fabsf(f[i]));
+        }
+#pragma unroll
+        for (int off = 1; off < LANES; off <<= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+
+        uint32_t idx[8];
+        if (amax == 0.f) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) idx[i] = 0;            // every code ties
+        } else {
+            // keep 16/s and 17*s/16 finite for tiny and huge scales: rescale w and s by a
+            // power of two (exact; a weight that underflows is far below the smallest step)
+            const float ps = amax < 0x1p-96f ? 0x1p32f : (amax > 0x1p96f ? 0x1p-32f : 1.0f);
+            const float s = amax * ps;
+            const float c16 = 16.0f * __frcp_rn(s);
+            const float s16 = s * 0.0625f;
+            const float two_s16 = 2.0f * s16, m17 = -17.0f * s16;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float ws = f[i] * ps;
+                int cnt = (__float2int_ru(ws * c16) + 16) >> 1;
+                cnt = min(max(cnt, 0), 15);
+                // exact midpoint below code cnt: (2 cnt - 17) * s/16
+                const float mlo = fmaf((float)cnt, two_s16, m17);
+                if (cnt > 0 && !(ws > mlo)) cnt -= 1;
+                idx[i] = (uint32_t)cnt;
+            }
+        }
+        if (live) {
+            const uint32_t p = idx[0] | idx[1] << 4 | idx[2] << 8 | idx[3] << 12 |
+                               idx[4] << 16 | idx[5] << 20 | idx[6] << 24 | idx[7] << 28;
+            if (packed) packed[c] = p;
+            if (codes)
+                codes[c] = make_uint2(idx[0] | idx[1] << 8 | idx[2] << 16 | idx[3] << 24,
+                                      idx[4] | idx[5] << 8 | idx[6] << 16 | idx[7] << 24);
+            if ((threadIdx.x & (LANES - 1)) == 0) {
+                const int64_t row = c / chunks_per_row;
+                const int64_t col = (c - row * chunks_per_row) * 8;
+                scale[row * (k / G) + col / G] = (uint16_t)float_to_bf16_bits(amax);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+pack_kernel(const uint4* __restrict__ codes, int64_t n16, uint2* __restrict__ packed) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 c = ldg_nc_v4(codes + i);
+        const uint32_t in[4] = {c.x, c.y, c.z, c.w};
+        uint32_t out[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint32_t a = in[2 * j], b = in[2 * j + 1];
+            // bytes a = c0 c1 c2 c3 -> (c0 | c1 << 4) | (c2 | c3 << 4) << 8, then b above
+            const uint32_t lo = (a & 0x0F) | ((a >> 4) & 0xF0) | ((a >> 8) & 0x0F00) | ((a >> 12) & 0xF000);
+            const uint32_t hi = (b & 0x0F) | ((b >> 4) & 0xF0) | ((b >> 8) & 0x0F00) | ((b >> 12) & 0xF000);
+            out[j] = lo | hi << 16;
+        }
+        packed[i] = make_uint2(out[0], out[1]);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+unpack_kernel(const uint2* __restrict__ packed, int64_t n16, uint4* __restrict__ codes) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint2 p = packed[i];
+        const uint32_t in[2] = {p.x, p.y};
+        uint32_t out[4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint32_t v = in[j];
+            out[2 * j] = (v & 0x0F) | ((v & 0xF0) << 4) | ((v & 0x0F00) << 8) | ((v & 0xF000) << 12);
+            const uint32_t u = v >> 16;
+            out[2 * j + 1] = (u & 0x0F) | ((u & 0xF0) << 4) | ((u & 0x0F00) << 8) | ((u & 0xF000) << 12);
+        }
+        codes[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Dense reconstruction. One thread: 8 codes (one 32-bit packed word) -> 16 bytes.
+// ---------------------------------------------------------------------------------------
+
+// DYADIC4: bf16(step * (idx - 8)), step = scale / 8. The product is exact in fp32 (an
+// 8-bit significand times an integer of magnitude <= 8, scaled by 2^-3), so the bf16
+// conversion is the one and only rounding.
+__global__ void __launch_bounds__(kThreads)
+dequant_dyadic_kernel(const uint32_t* __restrict__ packed, const uint16_t* __restrict__ scale,
+                      int64_t n_words, int64_t k, int group, uint4* __restrict__ out) {
+    const int64_t words_per_row = k / 8;
+    const int64_t groups_per_row = k / group;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_words;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t p = packed[i];
+        const int64_t row = i / words_per_row;
+        const int64_t col = (i - row * words_per_row) * 8;
+        const float step = bf16_bits_to_float(ldg_u16(scale + row * groups_per_row + col / group)) * 0.125f;
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = step * (float)((int)((p >> (4 * j)) & 15) - 8);
+        out[i] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    }
+}
+
+// LLOYD8S: code = q | sign << 3; bf16(+/- level[q]) from the group's 8 fp32 levels.
+__global__ void __launch_bounds__(kThreads)
+dequant_lloyd_kernel(const uint32_t* __restrict__ packed, const float4* __restrict__ levels,
+                     int64_t n_words, uint4* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_words;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t p = packed[i];
+        const int64_t g = i / 4;                    // 32 codes per group = 4 words
+        const float4 l0 = levels[2 * g], l1 = levels[2 * g + 1];
+        const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t c = (p >> (4 * j)) & 15;
+            float a = lv[0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q) a = ((c & 7) == (uint32_t)q) ? lv[q] : a;
+            v[j] = (c & 8) ? -a : a;
+        }
+        out[i] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    }
+}
+
+// LUT16: the fp16 centroid itself.
+__global__ void __launch_bounds__(kThreads)
+dequant_lut16_kernel(const uint32_t* __restrict__ packed, const uint4* __restrict__ lut,
+                     int64_t n_words, uint4* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_words;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t p = packed[i];
+        const int64_t g = i / 8;                    // 64 codes per block = 8 words
+        const uint4 a = lut[2 * g], b = lut[2 * g + 1];
+        const uint32_t L[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t c = (p >> (4 * j)) & 15;
+            uint32_t r = L[0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q) r = ((c >> 1) == (uint32_t)q) ? L[q] : r;
+            h[j] = (c & 1) ? (r >> 16) : (r & 0xFFFF);
+        }
+        out[i] = make_uint4(h[0] | h[1] << 16, h[2] | h[3] << 16, h[4] | h[5] << 16, h[6] | h[7] << 16);
+    }
+}
+
+}  // namespace
+
+wq_status launch_quantize_dyadic(const uint16_t* w, int64_t n, int64_t k, int group,
+                                 uint16_t* scale, uint8_t* codes, uint8_t* packed,
+                                 cudaStream_t s) {
+    const int64_t chunks = n * k / 8;
+    const int grid = stream_grid(chunks);
+    if (group == 64)
+        quantize_dyadic_kernel<64><<<grid, kThreads, 0, s>>>((const uint4*)w, chunks, k, scale,
+                                                             (uint2*)codes, (uint32_t*)packed);
+    else
+        quantize_dyadic_kernel<32><<<grid, kThreads, 0, s>>>((const uint4*)w, chunks, k, scale,
+                                                             (uint2*)codes, (uint32_t*)packed);
+    return check_launch("quantize_dyadic");
+}
+
+wq_status launch_pack(const uint8_t* codes, int64_t n, int64_t k, uint8_t* packed, cudaStream_t s) {
+    const int64_t n16 = n * k / 16;
+    pack_kernel<<<stream_grid(n16), kThreads, 0, s>>>((const uint4*)codes, n16, (uint2*)packed);
+    return check_launch("pack");
+}
+
+wq_status launch_unpack(const uint8_t* packed, int64_t n, int64_t k, uint8_t* codes, cudaStream_t s) {
+    const int64_t n16 = n * k / 16;
+    unpack_kernel<<<stream_grid(n16), kThreads, 0, s>>>((const uint2*)packed, n16, (uint4*)codes);
+    return check_launch("unpack");
+}
+
+wq_status launch_dequant(const wq_weight& w, uint16_t* out, cudaStream_t s) {
+    const int64_t n_words = w.n * w.k / 8;
+    const int grid = stream_grid(n_words);
+    if (w.fmt == WQ_FMT_DYADIC4)
+        dequant_dyadic_kernel<<<grid, kThreads, 0, s>>>((const uint32_t*)w.packed,
+                                                        (const uint16_t*)w.aux, n_words, w.k,
+                                                        w.group, (uint4*)out);
+    else if (w.fmt == WQ_FMT_LLOYD8S)
+        dequant_lloyd_kernel<<<grid, kThreads, 0, s>>>((const uint32_t*)w.packed,
+                                                       (const float4*)w.aux, n_words, (uint4*)out);
+    else
+        dequant_lut16_kernel<<<grid, kThreads, 0, s>>>((const uint32_t*)w.packed,
+                                                       (const uint4*)w.aux, n_words, (uint4*)out);
+    return check_launch("dequant");
+}
+
+}  // namespace wq

@@ -1,0 +1,133 @@
+// wq_internal.cuh -- declarations shared by the translation units of libwq (sm_100a).
+// Nothing here is part of the public ABI (include/wq.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+#include <cstddef>
+
+#include "wq.h"
+
+namespace wq {
+
+// ---------------------------------------------------------------------------------------
+// Host-side status plumbing (wq_api.cu)
+// ---------------------------------------------------------------------------------------
+
+// Records a formatted failure message for wq_last_error() and returns `st`.
+wq_status fail(wq_status st, const char* fmt, ...);
+
+// Converts the CUDA runtime's last launch error into a status (clears it).
+wq_status check_launch(const char* what);
+
+// ---------------------------------------------------------------------------------------
+// Kernel launchers (each returns after enqueueing; arguments already validated)
+// ---------------------------------------------------------------------------------------
+
+wq_status launch_quantize_dyadic(const uint16_t* w, int64_t n, int64_t k, int group,
+                                 uint16_t* scale, uint8_t* codes, uint8_t* packed,
+                                 cudaStream_t s);
+wq_status launch_pack(const uint8_t* codes, int64_t n, int64_t k, uint8_t* packed, cudaStream_t s);
+wq_status launch_unpack(const uint8_t* packed, int64_t n, int64_t k, uint8_t* codes, cudaStream_t s);
+wq_status launch_dequant(const wq_weight& w, uint16_t* out, cudaStream_t s);
+
+struct GemvProblem {
+    const uint8_t* packed;
+    const void* aux;
+    const uint16_t* x;
+    uint16_t* y;
+    int32_t n, k;
+};
+wq_status launch_gemv(int fmt, int group, const GemvProblem* probs, int count, int batch,
+                      cudaStream_t s);
+
+wq_status launch_lloyd_g32(const uint16_t* w, int64_t n, int64_t k, int rounds, uint8_t* codes,
+                           uint8_t* packed, float* levels, uint8_t* params, float* trace,
+                           cudaStream_t s);
+wq_status launch_kmeans16(const uint16_t* w, int64_t n, int64_t k, int rounds, uint8_t* codes,
+                          uint8_t* packed, uint16_t* lut, float* trace, cudaStream_t s);
+
+size_t gemm_workspace_bytes(const wq_weight& w, int64_t m);
+wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
+                      size_t ws_bytes, cudaStream_t s);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// ---------------------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) {
+    return __uint_as_float(h << 16);
+}
+
+// fp32 -> bf16 bits, round to nearest even (finite inputs).
+__device__ __forceinline__ uint32_t float_to_bf16_bits(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// Two fp32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint4 ldg_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_u16(const void* p) {
+    unsigned short v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+// D += A * B on the legacy warp-level tensor-core path, m16n8k16, bf16 in, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Same with fp16 operands.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+}  // namespace wq
