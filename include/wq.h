@@ -199,6 +199,12 @@ size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
 wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y,
                         void* ws, size_t ws_bytes, wq_stream stream);
 
+/* Reads and clears the library's device-side error word. Kernels that wait on the GPU
+ * (the GEMM pipeline's mbarrier waits) give up after a bounded time instead of hanging and
+ * record a nonzero code there; *code receives it (0 = none). Synchronous (copies one int
+ * from the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_OK otherwise. */
+wq_status wq_device_error(int32_t* code);
+
 /* ------------------------------------------------------------------------------------ */
 /* Failure injection (host side only)                                                    */
 /* ------------------------------------------------------------------------------------ */

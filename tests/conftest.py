@@ -25,7 +25,7 @@ def pytest_collection_modifyitems(config, items):
 @pytest.fixture(scope="session")
 def wq():
     """The CUDA binding, built in-tree first if needed (nvcc cross-compiles on CPU)."""
-    from w4a16_matmul_b200 import build as _b
-    _b.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import w4a16_matmul_b200 as m
     return m

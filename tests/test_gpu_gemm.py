@@ -1,0 +1,86 @@
+"""GPU parity of the tcgen05 W4A16 GEMM against the oracle's fp64 product of its own
+reconstruction: |y - y_ref| <= 2e-3 * sum_k |Wdeq[n, k]| |x[m, k]| per element, plus exact
+special cases (one-hot activations reproduce a dequantised column; all-eight codes give
+zero) and the split-K workspace path used for small m."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from _util import f32, to_dev, to_dev_bits
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def _weight(wq, n, k, group, seed, workload=workloads.PREFILL):
+    w_bits = workloads.gaussian_outlier_weight(n, k, workload, seed)
+    s, c = oracle.dyadic_quantize(w_bits, group)
+    packed = oracle.pack(c)
+    return wq.PackedWeight(wq.FMT_DYADIC4, group, n, k, to_dev(packed), to_dev_bits(s)), packed, s
+
+
+def _check(y, y_ref, bound):
+    err = np.abs(f32(y) - y_ref)
+    ratio = err / np.maximum(bound, 1e-300)
+    assert np.all(err <= TOL * bound), f"max err/bound {ratio.max():.3g}"
+
+
+@pytest.mark.parametrize("m", [1, 16, 17, 100, 128, 129, 256, 300])
+@pytest.mark.parametrize("n,k,group", [(128, 256, 64), (200, 320, 64), (13, 64, 64), (256, 1024, 32)])
+def test_gemm_matches_oracle(wq, m, n, k, group):
+    pw, packed, s = _weight(wq, n, k, group, m * 7 + n + k)
+    x_bits = workloads.activations(m, k, workloads.PREFILL, n + m)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, group, x_bits)
+    _check(y, y_ref, bound)
+    assert wq.device_error() == 0
+
+
+def test_gemm_one_hot_and_zero_codes_exact(wq):
+    n, k = 256, 512
+    pw, packed, s = _weight(wq, n, k, 64, 3)
+    wd = oracle.bf16_to_f64(oracle.dequant(oracle.DYADIC4, packed, s, 64))
+    cols = np.arange(0, 512, 3)
+    x = np.zeros((len(cols), k))
+    x[np.arange(len(cols)), cols] = 1.0
+    y = f32(wq.gemm(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
+    assert np.array_equal(y, wd[:, cols].T)
+    zero = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(np.full((n, k // 2), 0x88, np.uint8)), pw.aux)
+    xr = to_dev_bits(workloads.activations(64, k, workloads.PREFILL, 9))
+    assert torch.count_nonzero(wq.gemm(zero, xr).float()).item() == 0
+
+
+def test_gemm_split_k_uses_workspace(wq):
+    pw, packed, s = _weight(wq, 1024, 8192, 64, 5)
+    assert wq.gemm_workspace_bytes(pw, 16) > 0            # small m splits K
+    x_bits = workloads.activations(16, 8192, workloads.PREFILL, 5)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    rows = np.arange(0, 1024, 7)
+    y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x_bits, rows=rows)
+    err = np.abs(f32(y)[:, rows] - y_ref)
+    assert np.all(err <= TOL * bound)
+
+
+@pytest.mark.parametrize("shape", workloads.PREFILL_SHAPES)
+@pytest.mark.parametrize("m", workloads.PREFILL_M)
+def test_gemm_full_size_sampled(wq, shape, m):
+    """The prefill workload at full size: (n, k) = (4096, 11008) / (11008, 4096), every m;
+    96 sampled weight rows x up to 128 sampled activation rows against the oracle."""
+    n, k = shape
+    w_bits = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 0 if n == 4096 else 1)
+    pw, _ = wq.quantize_dyadic(to_dev_bits(w_bits), 64)
+    x_bits = workloads.activations(m, k, workloads.PREFILL, m)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+    rng = np.random.default_rng(m + n)
+    rows = np.sort(rng.choice(n, 96, replace=False))
+    ms = np.sort(rng.choice(m, min(m, 128), replace=False))
+    packed = pw.packed.cpu().numpy()
+    s = pw.aux.view(torch.int16).cpu().numpy().view(np.uint16)
+    y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x_bits[ms], rows=rows)
+    got = f32(y)[np.ix_(ms, rows)]
+    assert np.all(np.abs(got - y_ref) <= TOL * bound)

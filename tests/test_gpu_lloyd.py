@@ -1,0 +1,157 @@
+"""GPU parity of the codebook producers against the oracle.
+
+Lloyd g32 ([G32] "int4-g32+warm 裸量化：原理与实验报告" §1.3): the GPU screens the 112
+candidates in fp32 and takes the Lloyd decisions in fp64. Where the oracle's best and the
+GPU's candidate differ, the two must be a near-tie (the GPU's choice is within 1e-4
+relative of the oracle's best MSE); those groups are re-run in the oracle from the GPU's
+candidate, and everything downstream is then compared: codes exactly wherever the
+nearest-level margin exceeds 1e-6 * gmax, levels within 1e-5 * gmax, the parameter byte
+exactly, the MSE trace within 1e-5 relative.
+
+k-means LUT16 ([KM] "K-Means量化技术：突破LLM低比特部署瓶颈" §1.2): both sides decide in
+fp64 with exact member sums, so codes and fp16 centroids must match bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from _util import bits, to_dev_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _cand_from_params(p):
+    p = p.astype(np.int64)
+    fam = p >> 7
+    return np.where(fam == 0, 7 * ((p >> 3) & 15) + (p & 7), 105 + ((p >> 3) & 15))
+
+
+def _check_lloyd(wq, w_bits, rounds=25, max_mismatch_frac=1e-3):
+    n, k = w_bits.shape
+    pw, ex = wq.quantize_lloyd(to_dev_bits(w_bits), wq.LLOYD_G32_WARM, rounds, codes=True, trace=True)
+    torch.cuda.synchronize()
+    g_codes = ex["codes"].cpu().numpy()
+    g_lv = pw.aux.cpu().numpy().astype(np.float64)
+    g_par = ex["params"].cpu().numpy()
+    g_tr = ex["trace"].cpu().numpy().astype(np.float64)
+    ref = oracle.lloyd(w_bits, 32, rounds)
+    gmax = np.abs(oracle.bf16_to_f64(w_bits)).reshape(n, k // 32, 32).max(-1)
+    g_cand = _cand_from_params(g_par)
+    mism = g_cand != ref["cand"]
+    frac = mism.mean()
+    assert frac <= max_mismatch_frac, f"{mism.sum()} candidate mismatches ({frac:.2%})"
+    if mism.any():
+        forced = oracle.lloyd(w_bits, 32, rounds, force_cand=np.where(mism, g_cand, -1).astype(np.int32))
+        # the GPU's candidate is a near-tie of the oracle's best
+        best = ref["trace"][..., 0]
+        gpu_c_mse = forced["trace"][..., 0]
+        assert np.all(gpu_c_mse[mism] <= best[mism] * (1 + 1e-4) + 1e-12 * gmax[mism] ** 2)
+        ref = forced
+    assert np.array_equal(g_par, ref["params"])
+    # packed bytes agree with the codes
+    assert np.array_equal(pw.packed.cpu().numpy(), oracle.pack(g_codes))
+    # codes exact where the nearest-level margin is not a near-tie
+    clear = ref["min_margin"] > 1e-6 * gmax
+    cmatch = (g_codes.reshape(n, k // 32, 32) == ref["codes"].reshape(n, k // 32, 32)).all(-1)
+    assert np.all(cmatch[clear]), f"{(~cmatch & clear).sum()} clear groups with different codes"
+    lv_err = np.abs(g_lv - ref["levels"])[clear]
+    assert np.all(lv_err <= 1e-5 * gmax[clear][:, None])
+    # the trace is stored as fp32: compare where the MSE is inside fp32's range, with an
+    # absolute floor of the smallest normal fp32
+    tr = ref["trace"]
+    inrange = (tr < 3.0e38)[clear]
+    diff = np.abs(g_tr - tr)[clear]
+    assert np.all((diff <= 1e-5 * tr[clear] + 2.0 ** -126)[inrange])
+    assert np.all(np.isinf(g_tr[clear][~inrange]))
+    # dequant of the GPU's own output is exactly the oracle's reconstruction of it
+    d = wq.dequant(pw)
+    assert np.array_equal(bits(d), oracle.dequant(oracle.LLOYD8S, pw.packed.cpu().numpy(),
+                                                  pw.aux.cpu().numpy(), 32))
+    return frac, (~clear).mean()
+
+
+def test_lloyd_g32_laplace_rowscaled(wq):
+    w = workloads.laplace_rowscaled_weight(96, 2048, index=0)
+    _check_lloyd(wq, w)
+
+
+def test_lloyd_g32_edge_groups(wq):
+    rng = np.random.default_rng(1)
+    w = workloads.laplace_rowscaled_weight(8, 512, index=1)
+    w[0, :32] = 0                                        # all zero (with a -0.0)
+    w[0, 5] = 0x8000
+    w[1, :32] = 0x3C80                                   # equal magnitudes, mixed signs
+    w[1, :32:3] |= 0x8000
+    w[2, :32] = 0
+    w[2, 7] = 0x3F80                                     # a single nonzero weight
+    w[3, :32] = workloads.f64_to_bf16_bits(rng.laplace(0, 1e-36, 32))   # tiny / subnormal
+    w[4, :32] = workloads.f64_to_bf16_bits(rng.laplace(0, 1e35, 32))    # huge
+    w[5, :32] = 0x3F80                                   # two magnitudes only
+    w[5, ::2] = 0x3E80
+    for rounds in (25, 0, 1):
+        _check_lloyd(wq, w, rounds)
+
+
+def test_lloyd_g32_full_size_matrix_sampled(wq):
+    """A full 2048x2048 matrix of the 224-matrix workload on the GPU; 64 sampled rows
+    (4096 groups) compared with the oracle."""
+    w = workloads.laplace_rowscaled_weight(2048, 2048, index=7)
+    pw, ex = wq.quantize_lloyd(to_dev_bits(w), wq.LLOYD_G32_WARM, 25, codes=True, trace=True)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(2).choice(2048, 64, replace=False))
+    sub = w[rows]
+    ref = oracle.lloyd(sub, 32, 25)
+    g_par = ex["params"].cpu().numpy()[rows]
+    g_cand = _cand_from_params(g_par)
+    assert (g_cand != ref["cand"]).mean() <= 1e-3
+    same = g_cand == ref["cand"]
+    gmax = np.abs(oracle.bf16_to_f64(sub)).reshape(64, 64, 32).max(-1)
+    clear = same & (ref["min_margin"] > 1e-6 * gmax)
+    g_codes = ex["codes"].cpu().numpy()[rows].reshape(64, 64, 32)
+    assert np.all((g_codes == ref["codes"].reshape(64, 64, 32)).all(-1)[clear])
+    g_lv = pw.aux.cpu().numpy()[rows].astype(np.float64)
+    assert np.all(np.abs(g_lv - ref["levels"])[clear] <= 1e-5 * gmax[clear][:, None])
+
+
+def _check_kmeans(wq, w_bits, rounds=25):
+    n, k = w_bits.shape
+    pw, ex = wq.quantize_lloyd(to_dev_bits(w_bits), wq.LLOYD_KMEANS16, rounds, codes=True, trace=True)
+    torch.cuda.synchronize()
+    ref = oracle.kmeans_lut16(w_bits, 64, rounds)
+    assert np.array_equal(bits(pw.aux), ref["lut"])
+    assert np.array_equal(ex["codes"].cpu().numpy(), ref["codes"])
+    assert np.array_equal(pw.packed.cpu().numpy(), oracle.pack(ref["codes"]))
+    tr = ex["trace"].cpu().numpy().astype(np.float64)
+    assert np.allclose(tr, ref["trace"], rtol=1e-6, atol=1e-30)
+
+
+@pytest.mark.parametrize("heavy", [False, True])
+def test_kmeans16_bit_exact(wq, heavy):
+    w = workloads.lut16_weight(64, 2048, heavy_tail=heavy)
+    _check_kmeans(wq, w)
+
+
+def test_kmeans16_edge_blocks(wq):
+    rng = np.random.default_rng(3)
+    w = workloads.lut16_weight(4, 256, heavy_tail=True, index=5)
+    w[0, :64] = 0x3C00                                  # all equal
+    vals = workloads.f64_to_bf16_bits(np.sort(rng.standard_normal(16)) * 0.01)
+    w[1, :64] = np.repeat(vals, 4)[rng.permutation(64)]  # 16 distinct values x 4
+    w[2, :64] = 0                                        # all zero
+    w[3, :64:2] = 0x8000                                 # zeros of both signs
+    for rounds in (25, 0, 3):
+        _check_kmeans(wq, w, rounds)
+
+
+def test_kmeans16_full_size_sampled(wq):
+    """The 8192x28672 LUT16 workload (Student-t) quantised on the GPU; 16 sampled rows
+    (7168 blocks) compared with the oracle bit for bit."""
+    w = workloads.lut16_weight(8192, 28672, heavy_tail=True)
+    pw, ex = wq.quantize_lloyd(to_dev_bits(w), wq.LLOYD_KMEANS16, 25)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(4).choice(8192, 16, replace=False))
+    ref = oracle.kmeans_lut16(w[rows], 64, 25)
+    assert np.array_equal(bits(pw.aux)[rows], ref["lut"])
+    assert np.array_equal(pw.packed.cpu().numpy()[rows], oracle.pack(ref["codes"]))

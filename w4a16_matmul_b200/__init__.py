@@ -4,7 +4,7 @@ matmul on B200.
 Every function marshals torch CUDA tensors into the C ABI and calls one entry point of
 libwq.so; all arithmetic runs in the library's CUDA kernels. There is no CPU or
 PyTorch fallback: importing the package fails if libwq.so has not been built
-(``python -m w4a16_matmul_b200.build``), and every call fails if the tensors are not on
+(``python w4a16_matmul_b200/build.py``), and every call fails if the tensors are not on
 a CUDA device. PyTorch supplies device memory and the current stream only.
 """
 from __future__ import annotations
@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libwq.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "wq.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m w4a16_matmul_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python w4a16_matmul_b200/build.py` "
                       "(nvcc, sm_100a). There is no fallback implementation.")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -59,6 +59,7 @@ _SIG = {
     "wq_gemm_workspace_bytes": ([_WP, _i64], _sz),
     "wq_gemm_w4a16": ([_WP, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
     "wq_debug_fail_next_launches": ([_i32], None),
+    "wq_device_error": ([ctypes.POINTER(_i32)], _i32),
 }
 for _name, (_args, _res) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -85,6 +86,15 @@ def _check(status: int) -> None:
 
 def last_error() -> str:
     return (_lib.wq_last_error() or b"").decode()
+
+
+def device_error() -> int:
+    """Reads and clears the device error word (nonzero: a bounded GPU wait expired)."""
+    code = _i32(0)
+    st = _lib.wq_device_error(ctypes.byref(code))
+    if st not in (WQ_OK, WQ_ETIMEOUT):
+        _check(st)
+    return code.value
 
 
 def version() -> int:

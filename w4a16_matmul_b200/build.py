@@ -1,6 +1,9 @@
 """Build libwq.so (the CUDA kernels and the C ABI of include/wq.h) in-tree, for sm_100a.
 
-    python -m w4a16_matmul_b200.build [--force] [--verbose]
+    python w4a16_matmul_b200/build.py [--force] [--verbose]
+
+(run by path, or loaded with load_build_module(): importing the package itself loads the
+library this script produces, so the build never goes through the package import)
 
 Each csrc/*.cu is compiled to an object under _build/ when it (or any header) is newer than
 its object, then all objects are linked into w4a16_matmul_b200/libwq.so with the CUDA

@@ -139,6 +139,15 @@ int32_t wq_version(void) { return 100; }
 
 void wq_debug_fail_next_launches(int32_t count) { g_fail_next.store(count > 0 ? count : 0); }
 
+wq_status wq_device_error(int32_t* code) {
+    g_last_error[0] = 0;
+    if (!code) return fail(WQ_EINVAL, "code is NULL");
+    wq_status st = read_device_error(code);
+    if (st) return st;
+    if (*code != 0) return fail(WQ_ETIMEOUT, "a bounded device wait expired (code %d)", *code);
+    return WQ_OK;
+}
+
 wq_status wq_quantize_dyadic(const uint16_t* w, int64_t n, int64_t k, int32_t group,
                              uint16_t* scale, uint8_t* codes, uint8_t* packed, wq_stream stream) {
     g_last_error[0] = 0;

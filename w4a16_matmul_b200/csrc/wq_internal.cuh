@@ -53,6 +53,9 @@ size_t gemm_workspace_bytes(const wq_weight& w, int64_t m);
 wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
                       size_t ws_bytes, cudaStream_t s);
 
+// Reads and clears the device error word written by expired bounded waits.
+wq_status read_device_error(int32_t* code);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
