@@ -287,27 +287,21 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
         pk, sc, xb, yb = sweep_bytes(mats, b)
         out[f"sweep_batch{b}"] = {"ms_per_step": round(ms, 4), "GB/s": round((pk + sc) / ms / 1e6, 1),
                                   "frac_hbm": round((pk + sc + xb + yb) / ms / 1e6 / peaks["hbm_gbs"], 4)}
-    # dyadic quantisation of the whole stack (bf16 -> scale + packed), HBM-bound
+    # dyadic quantisation of one layer (bf16 -> scale + packed), HBM-bound
     try:
-        n_w = sum(n * k for _, _, n, k, _ in mats[:7])
-        wts = [torch.randn((n, k), device=dev).mul_(0.02).to(torch.bfloat16) for _, _, n, k, _ in mats[:7]]
-        outs = [(torch.empty((n, k // 64), dtype=torch.bfloat16, device=dev),
-                 torch.empty((n, k // 2), dtype=torch.uint8, device=dev)) for _, _, n, k, _ in mats[:7]]
-        import ctypes
+        layer = mats[:7]
+        n_w = sum(n * k for _, _, n, k, _ in layer)
+        wts = [torch.randn((n, k), device=dev).mul_(0.02).to(torch.bfloat16) for _, _, n, k, _ in layer]
 
         def q():
-            for w, (s, p) in zip(wts, outs):
-                st = wq._lib.wq_quantize_dyadic(ctypes.c_void_p(w.data_ptr()), w.shape[0], w.shape[1], 64,
-                                                ctypes.c_void_p(s.data_ptr()), None,
-                                                ctypes.c_void_p(p.data_ptr()),
-                                                ctypes.c_void_p(stream.cuda_stream))
-                assert st == 0, wq.last_error()
+            for w in wts:
+                wq.quantize_dyadic(w, 64)
         ms = max_over_ranks(time_region(torch, stream, q, steps, warm, barrier))
         byts = n_w * (2 + 0.5 + 2 / 64)
-        out["quantize_dyadic_layer"] = {"Gweights/s": round(n_w / ms / 1e6, 2),
-                                        "GB/s": round(byts / ms / 1e6, 1),
-                                        "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
-        # dense reconstruction of the same layer
+        out["quantize_dyadic_layer"] = {"Gweights/s": round(n_w / ms / 1e6, 2), "GB/s": round(byts / ms / 1e6, 1),
+                                        "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
+                                        "launches_per_step": 7}
+
         def dq():
             for pw in packed[:7]:
                 wq.dequant(pw)
@@ -315,9 +309,94 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
         byts = n_w * (0.5 + 2 / 64 + 2)
         out["dequant_layer"] = {"GB/s": round(byts / ms / 1e6, 1),
                                 "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
-        del wts, outs
+        del wts
     except Exception as e:
         out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
+    if args.extras in ("gemm", "all"):
+        out["prefill_gemm"] = bench_gemm(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks)
+    if args.extras in ("producers", "all"):
+        out.update(bench_producers(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks))
+    return out
+
+
+def bench_gemm(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks):
+    """Prefill W4A16 GEMM on both weight shapes and every m of the prefill workload, with
+    the unfused "materialised" comparison line (dequant once + a cuBLAS bf16 GEMM)."""
+    res = {}
+    steps, warm = max(args.steps, 5), 3
+    for n, k in workloads.PREFILL_SHAPES:
+        wb = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 0 if n == 4096 else 1)
+        w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
+        pw, _ = wq.quantize_dyadic(w, 64)
+        del w
+        wdeq = wq.dequant(pw)
+        for m in workloads.PREFILL_M:
+            try:
+                x = torch.randn((m, k), device=dev).to(torch.bfloat16)
+                y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+                need = wq.gemm_workspace_bytes(pw, m)
+                ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+                ms = max_over_ranks(time_region(torch, stream, lambda: wq.gemm(pw, x, out=y, workspace=ws),
+                                                steps, warm, barrier))
+                fl = 2.0 * m * n * k
+                byts = n * k * (0.5 + 2 / 64) + 2 * m * k + 2 * m * n
+                ms_mat = max_over_ranks(time_region(torch, stream, lambda: torch.matmul(x, wdeq.t()),
+                                                    steps, warm, barrier))
+                res[f"{n}x{k}_m{m}"] = {
+                    "TFLOP/s": round(fl / ms / 1e9, 1), "frac_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4),
+                    "GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
+                    "us": round(ms * 1e3, 2), "split_k_workspace_bytes": need,
+                    "cublas_bf16_materialized_TFLOP/s": round(fl / ms_mat / 1e9, 1)}
+            except Exception as e:
+                res[f"{n}x{k}_m{m}"] = {"error": repr(e)[:200]}
+        del wdeq, pw
+    return res
+
+
+def bench_producers(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks):
+    """Lloyd g32 (a 16-matrix sample of the 224-matrix workload), 16-centroid k-means on the
+    8192x28672 LUT16 workload, and the LUT16 GEMV at batch 1/8/16."""
+    out = {}
+    try:
+        nm = 16
+        with ThreadPoolExecutor(8) as ex:
+            hw = list(ex.map(lambda i: workloads.laplace_rowscaled_weight(2048, 2048, index=i), range(nm)))
+        ws = [torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).to(dev) for h in hw]
+
+        def lloyd():
+            for w in ws:
+                wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)
+        ms = max_over_ranks(time_region(torch, stream, lloyd, 2, 1, barrier))
+        n_w = nm * 2048 * 2048
+        out["lloyd_g32"] = {"Gweights/s": round(n_w / ms / 1e6, 3), "ms_per_matrix": round(ms / nm, 3),
+                            "sample": f"{nm} of the 224 matrices 2048x2048",
+                            "extrapolated_224_s": round(ms / nm * 224 / 1e3, 3)}
+        del ws
+    except Exception as e:
+        out["lloyd_g32"] = {"error": repr(e)[:200]}
+    try:
+        n, k = workloads.LUT16_SHAPE
+        hb = workloads.lut16_weight(n, k, heavy_tail=True)
+        w = torch.from_numpy(hb.view(np.int16)).view(torch.bfloat16).to(dev)
+        del hb
+        holder = {}
+
+        def km():
+            holder["pw"], _ = wq.quantize_lloyd(w, wq.LLOYD_KMEANS16, 25)
+        ms = max_over_ranks(time_region(torch, stream, km, 1, 1, barrier))
+        out["kmeans16"] = {"Gweights/s": round(n * k / ms / 1e6, 3), "ms": round(ms, 2)}
+        pw = holder["pw"]
+        del w
+        for b in (1, 8, 16):
+            x = torch.randn((b, k), device=dev).to(torch.bfloat16)
+            y = torch.empty((b, n), dtype=torch.bfloat16, device=dev)
+            ms = max_over_ranks(time_region(torch, stream, lambda: wq.gemv(pw, x, out=y), 20, 3, barrier))
+            byts = n * k * (0.5 + 0.5)
+            out[f"lut16_gemv_b{b}"] = {"GB/s": round(byts / ms / 1e6, 1), "us": round(ms * 1e3, 2),
+                                       "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
+                                       "packed_only_GB/s": round(n * k * 0.5 / ms / 1e6, 1)}
+    except Exception as e:
+        out["kmeans16"] = {"error": repr(e)[:200]}
     return out
 
 
@@ -408,6 +487,8 @@ def main():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--extras", default="all", choices=["sweep", "gemm", "producers", "all"],
+                    help="which secondary rows to time after the headline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import workloads
-from _util import bits, f32, to_dev, to_dev_bits
+from _util import bits, f32, matmul_tolerance, to_dev, to_dev_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +27,7 @@ def _check(y, y_ref, bound, rows=None):
     if rows is not None:
         y = y[:, rows]
     err = np.abs(y - y_ref)
-    ok = err <= TOL * bound
+    ok = err <= matmul_tolerance(y_ref, bound, TOL)
     assert ok.all(), f"max err/bound {np.max(err / np.maximum(bound, 1e-300)):.3g}"
     return float(np.max(err / np.maximum(bound, 1e-300)))
 

@@ -228,20 +228,19 @@ __device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&ac
     }
 }
 
+// A step needs the fp32 path when one of its scales is nonzero but below 2^-123: then
+// step = scale/8 is not a normal bf16 and the bf16 multiply could lose bits.
 template <int KIND, int R>
 __device__ __forceinline__ bool step_has_tiny(const Step<KIND, R>& st) {
     if (KIND == kLut16) return false;
-    bool t = false;
+    uint32_t m = 0xFFFFFFFFu;
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const uint32_t e = (st.aux[r][h][j] >> 7) & 0xFF;   // bf16 exponent field
-                t |= (st.aux[r][h][j] & 0x7FFF) != 0 && e < 27;      // 0 < scale < 2^-100
-            }
-    return t;
+            for (int j = 0; j < 2; ++j) m = min(m, (st.aux[r][h][j] & 0x7FFFu) - 1u);   // 0 -> huge
+    return m < 0x01FFu;
 }
 
 template <int KIND, int NB, int R, int WK, int MAXP>
@@ -277,18 +276,22 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     const bool xa_live = g < B, xb_live = NB == 2 && (g + 8 < B);
 
     if (row0 < N) {
-        Step<KIND, R> cur, nxt;
-        int s = wk;
-        if (s < steps) load_step<KIND, R>(cur, pb, row0, g, s * 256 + t * 64, N, K);
-        for (; s < steps; s += WK) {
-            const int sn = s + WK;
-            if (sn < steps) load_step<KIND, R>(nxt, pb, row0, g, sn * 256 + t * 64, N, K);
+        // two register buffers in ping-pong: the next step's bytes load while this one computes
+        Step<KIND, R> b0, b1;
+        auto run_step = [&](const Step<KIND, R>& st, int s) {
             const int kk = s * 256 + t * 64;
-            if (__builtin_expect(__any_sync(0xFFFFFFFFu, step_has_tiny<KIND, R>(cur)), 0))
-                compute_step<KIND, NB, R, true>(cur, acc, xg, xg8, xa_live, xb_live, kk, K);
+            if (__builtin_expect(__any_sync(0xFFFFFFFFu, step_has_tiny<KIND, R>(st)), 0))
+                compute_step<KIND, NB, R, true>(st, acc, xg, xg8, xa_live, xb_live, kk, K);
             else
-                compute_step<KIND, NB, R, false>(cur, acc, xg, xg8, xa_live, xb_live, kk, K);
-            cur = nxt;
+                compute_step<KIND, NB, R, false>(st, acc, xg, xg8, xa_live, xb_live, kk, K);
+        };
+        if (wk < steps) load_step<KIND, R>(b0, pb, row0, g, wk * 256 + t * 64, N, K);
+        for (int s = wk; s < steps; s += 2 * WK) {
+            if (s + WK < steps) load_step<KIND, R>(b1, pb, row0, g, (s + WK) * 256 + t * 64, N, K);
+            run_step(b0, s);
+            if (s + WK >= steps) break;
+            if (s + 2 * WK < steps) load_step<KIND, R>(b0, pb, row0, g, (s + 2 * WK) * 256 + t * 64, N, K);
+            run_step(b1, s + WK);
         }
     }
 
@@ -335,7 +338,7 @@ wq_status run(const GemvParams<MAXP>& prm, int tiles, cudaStream_t s) {
 
 template <int KIND, int NB, int MAXP>
 wq_status pick_split(GemvParams<MAXP>& prm, const GemvProblem* probs, int count, int64_t rows16,
-                     cudaStream_t s) {
+                     int batch, cudaStream_t s) {
     // Full-K warps (no reduction) when the launch has at least ~6 warps of 32 rows per SM;
     // otherwise 16-row warps, and K split over 2 or 4 warps of a CTA for small launches.
     const int64_t sms = sm_count();
@@ -348,11 +351,11 @@ wq_status pick_split(GemvParams<MAXP>& prm, const GemvProblem* probs, int count,
         prm.tile_start[count] = tiles;
         return tiles;
     };
-#ifndef WQ_GEMV_BIG_R
-#define WQ_GEMV_BIG_R 2     // rows per warp / 16 for large launches (build-time tuning)
-#endif
-    constexpr int BIGR = (KIND == kLut16) ? 1 : WQ_GEMV_BIG_R;
-    if (rows16 >= 12 * sms * BIGR) return run<KIND, NB, BIGR, 1, MAXP>(prm, tiles_for(64 * BIGR), s);
+    // 32-row warps pay off once the activation fragment is shared by more batch rows
+    // (measured: 16-row warps win at batch <= 4, 32-row warps at batch 5..16)
+    constexpr int BIGR = (KIND == kLut16) ? 1 : 2;
+    if (BIGR == 2 && batch > 4 && rows16 >= 12 * sms * 2)
+        return run<KIND, NB, BIGR, 1, MAXP>(prm, tiles_for(64 * BIGR), s);
     if (rows16 >= 8 * sms) return run<KIND, NB, 1, 1, MAXP>(prm, tiles_for(64), s);
     if (rows16 >= 2 * sms) return run<KIND, NB, 1, 2, MAXP>(prm, tiles_for(32), s);
     return run<KIND, NB, 1, 4, MAXP>(prm, tiles_for(16), s);
@@ -369,13 +372,13 @@ wq_status launch_impl(int fmt, int group, const GemvProblem* probs, int count, i
     const bool two = batch > 8;
     const int kind = (fmt == WQ_FMT_LUT16) ? kLut16 : (group == 64 ? kDyadic64 : kDyadic32);
     if (kind == kLut16)
-        return two ? pick_split<kLut16, 2, MAXP>(prm, probs, count, rows16, s)
-                   : pick_split<kLut16, 1, MAXP>(prm, probs, count, rows16, s);
+        return two ? pick_split<kLut16, 2, MAXP>(prm, probs, count, rows16, batch, s)
+                   : pick_split<kLut16, 1, MAXP>(prm, probs, count, rows16, batch, s);
     if (kind == kDyadic64)
-        return two ? pick_split<kDyadic64, 2, MAXP>(prm, probs, count, rows16, s)
-                   : pick_split<kDyadic64, 1, MAXP>(prm, probs, count, rows16, s);
-    return two ? pick_split<kDyadic32, 2, MAXP>(prm, probs, count, rows16, s)
-               : pick_split<kDyadic32, 1, MAXP>(prm, probs, count, rows16, s);
+        return two ? pick_split<kDyadic64, 2, MAXP>(prm, probs, count, rows16, batch, s)
+                   : pick_split<kDyadic64, 1, MAXP>(prm, probs, count, rows16, batch, s);
+    return two ? pick_split<kDyadic32, 2, MAXP>(prm, probs, count, rows16, batch, s)
+               : pick_split<kDyadic32, 1, MAXP>(prm, probs, count, rows16, batch, s);
 }
 
 }  // namespace
