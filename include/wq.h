@@ -205,6 +205,29 @@ wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16
  * from the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_OK otherwise. */
 wq_status wq_device_error(int32_t* code);
 
+/* The GEMM above without a caller workspace, for callers that cannot allocate device
+ * memory: e.g. an inference server whose caching allocator owns the whole device memory
+ * budget and forbids any other cudaMalloc, a plugin that may only use the buffers its host
+ * framework hands it, or a latency-critical path that must not pay cudaMalloc's implicit
+ * device synchronisation. The pages describe no such entry point; it exists only for them.
+ * When m is small and K is split across CTAs, the fp32 partial sums go to a scratch array
+ * that the library allocates statically (a file-scope device array of
+ * WQ_GEMM_STATIC_SCRATCH_BYTES); every GPU that loads libwq holds that array until the
+ * process exits. This entry point itself allocates and frees nothing.
+ *   - Same arguments, layout, tolerance and results as wq_gemm_w4a16.
+ *   - A problem whose scratch need (wq_gemm_workspace_bytes) exceeds
+ *     WQ_GEMM_STATIC_SCRATCH_BYTES is rejected with WQ_EINVAL; use wq_gemm_w4a16 with a
+ *     workspace for it.
+ *   - All calls share the one array, which keeps the last call's contents (every call
+ *     writes all the scratch it reads, so nothing has to start at zero). Calls whose GPU
+ *     work overlaps (e.g. on two streams) race on it: serialise them.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) once and caches it; make that first call before any stream
+ *     capture. */
+#define WQ_GEMM_STATIC_SCRATCH_BYTES (16u << 20)
+wq_status wq_gemm_w4a16_static(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y,
+                               wq_stream stream);
+
 /* ------------------------------------------------------------------------------------ */
 /* Failure injection (host side only)                                                    */
 /* ------------------------------------------------------------------------------------ */

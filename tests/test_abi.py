@@ -12,7 +12,7 @@ def test_library_exports_every_header_function(wq):
     expected = {"wq_status_string", "wq_last_error", "wq_version", "wq_quantize_dyadic",
                 "wq_quantize_lloyd", "wq_pack", "wq_unpack", "wq_dequant", "wq_gemv_w4a16",
                 "wq_gemv_w4a16_grouped", "wq_gemm_workspace_bytes", "wq_gemm_w4a16",
-                "wq_debug_fail_next_launches", "wq_device_error"}
+                "wq_debug_fail_next_launches", "wq_device_error", "wq_gemm_w4a16_static"}
     assert expected <= set(names), set(names) ^ expected
     for n in names:
         assert hasattr(wq._lib, n), n

@@ -58,6 +58,7 @@ _SIG = {
     "wq_gemv_w4a16_grouped": ([_WP, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i32, _i32, _vp], _i32),
     "wq_gemm_workspace_bytes": ([_WP, _i64], _sz),
     "wq_gemm_w4a16": ([_WP, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
+    "wq_gemm_w4a16_static": ([_WP, _vp, _i64, _vp, _vp], _i32),
     "wq_debug_fail_next_launches": ([_i32], None),
     "wq_device_error": ([ctypes.POINTER(_i32)], _i32),
 }
