@@ -84,3 +84,21 @@ def test_gemm_full_size_sampled(wq, shape, m):
     y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x_bits[ms], rows=rows)
     got = f32(y)[np.ix_(ms, rows)]
     assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
+
+
+def test_gemm_one_hot_every_scale_regime(wq):
+    """The GEMM's in-smem reconstruction across every scale regime (see the GEMV test of the
+    same name): one-hot activations reproduce the dequantised column exactly."""
+    regimes = [0x0001, 0x0031, 0x007F, 0x0080, 0x00FF, 0x3D4C, 0x3F80, 0x3FFF, 0x7C00, 0x7D80,
+               0x7E55, 0x7F7F, 0x0000]
+    n, k = 16 * len(regimes), 256
+    g = np.random.default_rng(14)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    scale = np.repeat(np.array(regimes, np.uint16), 16)[:, None].repeat(k // 64, 1)
+    packed = oracle.pack(codes)
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(packed), to_dev_bits(scale))
+    wd = oracle.bf16_to_f64(oracle.dequant(oracle.DYADIC4, packed, scale, 64))
+    x = np.zeros((k, k))
+    x[np.arange(k), np.arange(k)] = 1.0
+    y = f32(wq.gemm(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
+    assert np.array_equal(y, wd.T)

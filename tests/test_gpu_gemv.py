@@ -149,3 +149,28 @@ def test_gemv_lut16_matches_oracle(wq):
     wd = oracle.fp16_to_f64(oracle.dequant(oracle.LUT16, packed, lut, 64))
     for i, c in enumerate([0, 65, 1023]):
         assert np.array_equal(y[i], oracle.bf16_to_f64(oracle.f64_to_bf16(wd[:, c])))
+
+
+SCALE_REGIMES = [0x0001, 0x0031, 0x007F, 0x0080, 0x00FF, 0x3D4C, 0x3F80, 0x3FFF, 0x7C00, 0x7D80,
+                 0x7E55, 0x7F7F, 0x0000]
+
+
+@pytest.mark.parametrize("group", [64, 32])
+def test_gemv_one_hot_every_scale_regime(wq, group):
+    """Every scale regime (subnormal, smallest normal, typical, 2^121, >= 2^124 where the
+    fp32 path takes over, the largest bf16, zero): one-hot activations reproduce the
+    dequantised column exactly, so the in-register reconstruction is bit-exact."""
+    n, k = 16 * len(SCALE_REGIMES), 256
+    g = np.random.default_rng(13)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    scale = np.repeat(np.array(SCALE_REGIMES, np.uint16), 16)[:, None].repeat(k // group, 1)
+    packed = oracle.pack(codes)
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, group, n, k, to_dev(packed), to_dev_bits(scale))
+    wd = oracle.bf16_to_f64(oracle.dequant(oracle.DYADIC4, packed, scale, group))
+    cols = np.arange(0, k, 17)
+    for lo in range(0, len(cols), 16):
+        cc = cols[lo:lo + 16]
+        x = np.zeros((len(cc), k))
+        x[np.arange(len(cc)), cc] = 1.0
+        y = f32(wq.gemv(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
+        assert np.array_equal(y, wd[:, cc].T)

@@ -115,20 +115,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
         : "r"(taddr));
 }
 
-// bf16 of the 8 codes of one packed word, in column order: (c0,c1), (c2,c3), (c4,c5), (c6,c7).
-__device__ __forceinline__ uint4 dyadic_row8(uint32_t w, uint32_t step2) {
-    const uint32_t kMagic = 0x43004300u, kNeg136 = 0xC308C308u, kOne = 0x3F803F80u, kNegZero = 0x80008000u;
-    uint32_t p0 = (w & 0x000F000Fu) | kMagic;             // (c0, c4)
-    uint32_t p1 = ((w >> 4) & 0x000F000Fu) | kMagic;      // (c1, c5)
-    uint32_t p2 = ((w >> 8) & 0x000F000Fu) | kMagic;      // (c2, c6)
-    uint32_t p3 = ((w >> 12) & 0x000F000Fu) | kMagic;     // (c3, c7)
-    p0 = bf16x2_fma(bf16x2_fma(p0, kOne, kNeg136), step2, kNegZero);
-    p1 = bf16x2_fma(bf16x2_fma(p1, kOne, kNeg136), step2, kNegZero);
-    p2 = bf16x2_fma(bf16x2_fma(p2, kOne, kNeg136), step2, kNegZero);
-    p3 = bf16x2_fma(bf16x2_fma(p3, kOne, kNeg136), step2, kNegZero);
+// bf16 of the 8 codes of one packed word, in column order: (c0,c1), (c2,c3), (c4,c5),
+// (c6,c7), each bf16(step * (idx - 8)) rounded once. A bf16 pattern below 0x0100 is worth
+// exactly pattern * 2^-133 (subnormals and the first normal binade share that spacing), so
+// masked nibble pairs need no shift; two FMAs then form scale * (idx - 8) / 8 exactly and
+// round it once. cs / cn = (16 * scale, -scale) as bf16 pairs.
+__device__ __forceinline__ uint4 dyadic_row8(uint32_t w, uint32_t cs, uint32_t cn) {
+    const uint32_t kP126 = 0x7E807E80u, kP122 = 0x7C807C80u, kNegZero = 0x80008000u;
+    const uint32_t t = w >> 8;
+    const uint32_t p0 = bf16x2_fma(bf16x2_fma(w & 0x000F000Fu, kP126, kNegZero), cs, cn);   // (c0, c4)
+    const uint32_t p1 = bf16x2_fma(bf16x2_fma(w & 0x00F000F0u, kP122, kNegZero), cs, cn);   // (c1, c5)
+    const uint32_t p2 = bf16x2_fma(bf16x2_fma(t & 0x000F000Fu, kP126, kNegZero), cs, cn);   // (c2, c6)
+    const uint32_t p3 = bf16x2_fma(bf16x2_fma(t & 0x00F000F0u, kP122, kNegZero), cs, cn);   // (c3, c7)
     return make_uint4(prmt(p0, p1, 0x5410u), prmt(p2, p3, 0x5410u), prmt(p0, p1, 0x7632u),
                       prmt(p2, p3, 0x7632u));
 }
+// The same in fp32, for scales of 2^124 and above (16 * scale would overflow bf16).
 __device__ __forceinline__ uint4 dyadic_row8_f32(uint32_t w, float step) {
     float v[8];
 #pragma unroll
@@ -274,15 +276,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 const uint4 q0 = pk[0], q1 = pk[1];
                 const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
                 uint8_t* arow = stage_a(s) + i * 128;
-                const float f0 = bf16_bits_to_float(sc0), f1 = bf16_bits_to_float(sc1);
-                const bool tiny = (f0 != 0.f && f0 < 0x1p-100f) || (f1 != 0.f && f1 < 0x1p-100f);
-                const uint32_t st0 = bf16x2_fma(prmt(sc0, 0, 0x1010u), 0x3E003E00u, 0x80008000u);
-                const uint32_t st1 = bf16x2_fma(prmt(sc1, 0, 0x1010u), 0x3E003E00u, 0x80008000u);
+                const bool huge = ((sc0 & 0x7FFFu) >= 0x7D80u) || ((sc1 & 0x7FFFu) >= 0x7D80u);
+                const uint32_t s20 = prmt(sc0, 0, 0x1010u), s21 = prmt(sc1, 0, 0x1010u);
+                const uint32_t cs0 = bf16x2_fma(s20, 0x41804180u, 0x80008000u), cn0 = s20 ^ 0x80008000u;
+                const uint32_t cs1 = bf16x2_fma(s21, 0x41804180u, 0x80008000u), cn1 = s21 ^ 0x80008000u;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const bool second = (G == 32) && c >= 4;
-                    const uint4 v = tiny ? dyadic_row8_f32(wv[c], (second ? f1 : f0) * 0.125f)
-                                         : dyadic_row8(wv[c], second ? st1 : st0);
+                    const uint4 v = huge ? dyadic_row8_f32(wv[c], bf16_bits_to_float(second ? sc1 : sc0) * 0.125f)
+                                         : dyadic_row8(wv[c], second ? cs1 : cs0, second ? cn1 : cn0);
                     *(uint4*)(arow + ((c ^ (i & 7)) << 4)) = v;
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -41,22 +41,27 @@ struct GemvParams {
     GemvProblem prob[MAXP];
 };
 
-// bf16 pairs of the 8 codes of one packed word, dyadic: pair j = (code j, code j+4),
-// element with the lower code index in the low half.
-__device__ __forceinline__ void dyadic_pairs(uint32_t w, uint32_t step2, uint32_t (&p)[4]) {
-    const uint32_t kMagic = 0x43004300u;      // bf16 128.0 twice
-    const uint32_t kNeg136 = 0xC308C308u;     // bf16 -136.0 twice
-    const uint32_t kOne = 0x3F803F80u;        // bf16 1.0 twice
-    const uint32_t kNegZero = 0x80008000u;    // -0.0: keeps bf16(0 * -8) = -0.0
-    p[0] = (w & 0x000F000Fu) | kMagic;
-    p[1] = ((w >> 4) & 0x000F000Fu) | kMagic;
-    p[2] = ((w >> 8) & 0x000F000Fu) | kMagic;
-    p[3] = ((w >> 12) & 0x000F000Fu) | kMagic;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) p[j] = bf16x2_fma(bf16x2_fma(p[j], kOne, kNeg136), step2, kNegZero);
+// bf16 pairs of the 8 codes of one packed word, dyadic: pair j = (code j, code j+4), the
+// lower code index in the low half, each bf16(step * (idx - 8)) rounded once.
+//
+// A bf16 bit pattern below 0x0100 is worth exactly (pattern) * 2^-133: the subnormals and
+// the first normal binade share that spacing. So (w & 0x000F000F) is the pair (idx0, idx4)
+// times 2^-133 and (w & 0x00F000F0) is (idx1, idx5) times 2^-129, with no shift; w >> 8 gives
+// the other two pairs the same way. One FMA by 2^126 (resp. 2^122) brings them to idx * 2^-7
+// exactly, and fma(idx * 2^-7, 16 * scale, -scale) = scale * (idx - 8) / 8 is formed exactly
+// and rounded once. cs = (16 * scale) pair, cn = (-scale) pair.
+__device__ __forceinline__ void dyadic_pairs(uint32_t w, uint32_t cs, uint32_t cn, uint32_t (&p)[4]) {
+    const uint32_t kP126 = 0x7E807E80u;       // bf16 2^126 twice
+    const uint32_t kP122 = 0x7C807C80u;       // bf16 2^122 twice
+    const uint32_t kNegZero = 0x80008000u;
+    const uint32_t t = w >> 8;
+    p[0] = bf16x2_fma(bf16x2_fma(w & 0x000F000Fu, kP126, kNegZero), cs, cn);
+    p[1] = bf16x2_fma(bf16x2_fma(w & 0x00F000F0u, kP122, kNegZero), cs, cn);
+    p[2] = bf16x2_fma(bf16x2_fma(t & 0x000F000Fu, kP126, kNegZero), cs, cn);
+    p[3] = bf16x2_fma(bf16x2_fma(t & 0x00F000F0u, kP122, kNegZero), cs, cn);
 }
 
-// Same pairs computed in fp32 (for tiny scales).
+// Same pairs computed in fp32 (for scales whose 16x overflows bf16).
 __device__ __forceinline__ void dyadic_pairs_f32(uint32_t w, float step, uint32_t (&p)[4]) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -66,9 +71,11 @@ __device__ __forceinline__ void dyadic_pairs_f32(uint32_t w, float step, uint32_
     }
 }
 
-// step = scale / 8 as a bf16 pair (exact for scale >= 2^-123).
-__device__ __forceinline__ uint32_t step_pair(uint32_t scale_bits) {
-    return bf16x2_fma(prmt(scale_bits, 0, 0x1010u), 0x3E003E00u, 0x80008000u);
+// (16 * scale, -scale) as bf16 pairs (exact for every finite scale below 2^124).
+__device__ __forceinline__ void scale_pairs(uint32_t scale_bits, uint32_t& cs, uint32_t& cn) {
+    const uint32_t s2 = prmt(scale_bits, 0, 0x1010u);
+    cs = bf16x2_fma(s2, 0x41804180u, 0x80008000u);     // x 16.0
+    cn = s2 ^ 0x80008000u;
 }
 
 // LUT16 lookup of 4 codes (nibbles of the low 16 bits of s) in a 16-entry fp16 table held
@@ -102,17 +109,17 @@ struct Step {
     uint32_t aux[R][2][KIND == kLut16 ? 8 : 2];   // dyadic: bf16 scales; LUT16: table words
 };
 
-template <int KIND, int R>
+template <int KIND, int R, bool FULL>
 __device__ __forceinline__ void load_step(Step<KIND, R>& st, const GemvProblem& pb, int row0, int g,
                                           int kk, int N, int K) {
-    const bool h0 = kk < K, h1 = kk + 32 < K;
+    const bool h0 = FULL || kk < K, h1 = FULL || kk + 32 < K;
     const size_t row_bytes = (size_t)K / 2;
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int row = row0 + 16 * r + 8 * h + g;
-            const bool rl = row < N;
+            const bool rl = FULL || row < N;
             const uint8_t* wp = pb.packed + (size_t)row * row_bytes + kk / 2;
             const uint4 fill = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
             const uint4 a = (rl && h0) ? ldg_nc_v4(wp) : fill;
@@ -145,13 +152,15 @@ __device__ __forceinline__ void load_step(Step<KIND, R>& st, const GemvProblem& 
         }
 }
 
-// One 256-column step: 8 words per row, 2 (or 4) mma per word pair.
-template <int KIND, int NB, int R, bool SLOW>
+// One 256-column step: 8 words per row, 2 (or 4) mma per word pair. FULL: the step lies
+// inside K, so every activation load is in range; lanes whose batch column is unused load
+// some valid row (those output columns are computed but never stored).
+template <int KIND, int NB, int R, bool SLOW, bool FULL>
 __device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&acc)[R][NB][4],
                                              const uint16_t* xg, const uint16_t* xg8, bool xa_live,
-                                             bool xb_live, int kk, int K) {
+                                             bool xb_live, int kk, int K, uint4 (&xr)[2]) {
     const bool h0 = kk < K, h1 = kk + 32 < K;
-    uint32_t stp[R][2][2];
+    uint32_t cs[R][2][2], cn[R][2][2];
     float fst[R][2][2];
     uint32_t plo[R][2][4], phi[R][2][4];
 #pragma unroll
@@ -167,19 +176,31 @@ __device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&ac
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    stp[r][h][j] = step_pair(st.aux[r][h][j]);
+                for (int j = 0; j < (KIND == kDyadic32 ? 2 : 1); ++j) {
                     if (SLOW) fst[r][h][j] = bf16_bits_to_float(st.aux[r][h][j]) * 0.125f;
+                    else scale_pairs(st.aux[r][h][j], cs[r][h][j], cn[r][h][j]);
                 }
             }
         }
 #pragma unroll
     for (int sub = 0; sub < 8; ++sub) {
         const int kx = kk + 8 * sub;
-        const bool xv = (sub < 4) ? h0 : h1;
-        uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
-        if (xa_live && xv) xa = ldg_v4(xg + kx);
-        if (NB == 2 && xb_live && xv) xb = ldg_v4(xg8 + kx);
+        uint4 xa, xb;
+        if (FULL) {
+            // lanes of unused batch columns keep stale registers: their columns are never stored
+            ldg_v4_if(xr[0], xg + kx, xa_live);
+            xa = xr[0];
+            if (NB == 2) {
+                ldg_v4_if(xr[1], xg8 + kx, xb_live);
+                xb = xr[1];
+            }
+        } else {
+            const bool xv = (sub < 4) ? h0 : h1;
+            xa = make_uint4(0, 0, 0, 0);
+            xb = xa;
+            if (xa_live && xv) xa = ldg_v4(xg + kx);
+            if (NB == 2 && xb_live && xv) xb = ldg_v4(xg8 + kx);
+        }
         uint32_t b[NB][4];                              // B fragments of the two mma
         if (KIND == kLut16) {
             b[0][0] = bf16x2_to_f16x2(xa.x); b[0][1] = bf16x2_to_f16x2(xa.y);
@@ -215,8 +236,8 @@ __device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&ac
                     dyadic_pairs_f32(st.w[r][0][sub], fst[r][0][hs], q0);
                     dyadic_pairs_f32(st.w[r][1][sub], fst[r][1][hs], q1);
                 } else {
-                    dyadic_pairs(st.w[r][0][sub], stp[r][0][hs], q0);
-                    dyadic_pairs(st.w[r][1][sub], stp[r][1][hs], q1);
+                    dyadic_pairs(st.w[r][0][sub], cs[r][0][hs], cn[r][0][hs], q0);
+                    dyadic_pairs(st.w[r][1][sub], cs[r][1][hs], cn[r][1][hs], q1);
                 }
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb) {
@@ -228,19 +249,18 @@ __device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&ac
     }
 }
 
-// A step needs the fp32 path when one of its scales is nonzero but below 2^-123: then
-// step = scale/8 is not a normal bf16 and the bf16 multiply could lose bits.
+// A step needs the fp32 path when 16 * scale would overflow bf16 (scale >= 2^124).
 template <int KIND, int R>
-__device__ __forceinline__ bool step_has_tiny(const Step<KIND, R>& st) {
+__device__ __forceinline__ bool step_needs_slow(const Step<KIND, R>& st) {
     if (KIND == kLut16) return false;
-    uint32_t m = 0xFFFFFFFFu;
+    uint32_t m = 0;
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) m = min(m, (st.aux[r][h][j] & 0x7FFFu) - 1u);   // 0 -> huge
-    return m < 0x01FFu;
+            for (int j = 0; j < 2; ++j) m = max(m, st.aux[r][h][j] & 0x7FFFu);
+    return m >= 0x7D80u;
 }
 
 template <int KIND, int NB, int R, int WK, int MAXP>
@@ -271,26 +291,56 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) acc[r][nb][0] = acc[r][nb][1] = acc[r][nb][2] = acc[r][nb][3] = 0.f;
 
-    const uint16_t* xg = pb.x + (size_t)g * K;
-    const uint16_t* xg8 = pb.x + (size_t)(g + 8) * K;
     const bool xa_live = g < B, xb_live = NB == 2 && (g + 8 < B);
+    // lanes whose batch column is unused read row 0 (their outputs are never stored)
+    const uint16_t* xg = pb.x + (size_t)(xa_live ? g : 0) * K;
+    const uint16_t* xg8 = pb.x + (size_t)(xb_live ? g + 8 : 0) * K;
 
+    if (row0 < N && wk == 0 && lane == 0) {
+        // The warp's rows are contiguous in memory: ask the L2 for all of them now, so the
+        // register loads below see L2 latency rather than DRAM latency.
+        const int rows = min(16 * R, N - row0);
+        const size_t row_bytes = (size_t)K / 2;
+        prefetch_l2_bulk(pb.packed + (size_t)row0 * row_bytes, (uint32_t)(rows * row_bytes));
+        if (KIND == kLut16) {
+            const size_t lb = (size_t)(K / 64) * 32;                  // fp16 [16] per block
+            prefetch_l2_bulk((const uint8_t*)pb.aux + (size_t)row0 * lb, (uint32_t)(rows * lb));
+        } else {
+            // scales: the 16-byte-aligned interior of this warp's rows
+            const size_t sb = (size_t)(K / (KIND == kDyadic64 ? 64 : 32)) * 2;
+            const uintptr_t a0 = (uintptr_t)pb.aux + (size_t)row0 * sb;
+            const uintptr_t a1 = a0 + (size_t)rows * sb;
+            const uintptr_t b0 = (a0 + 15) & ~(uintptr_t)15, b1 = a1 & ~(uintptr_t)15;
+            if (b1 > b0) prefetch_l2_bulk((const void*)b0, (uint32_t)(b1 - b0));
+        }
+    }
     if (row0 < N) {
-        // two register buffers in ping-pong: the next step's bytes load while this one computes
-        Step<KIND, R> b0, b1;
+        // FULL steps (all rows of the warp and all 256 columns in range) run without
+        // predicates; only a ragged last step or a ragged last row block take the checks
+        const bool rows_full = row0 + 16 * R <= N;
+        const int full_steps = rows_full ? (K >> 8) : 0;
+        auto load = [&](Step<KIND, R>& st, int s) {
+            if (s < full_steps) load_step<KIND, R, true>(st, pb, row0, g, s * 256 + t * 64, N, K);
+            else load_step<KIND, R, false>(st, pb, row0, g, s * 256 + t * 64, N, K);
+        };
+        uint4 xr[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
         auto run_step = [&](const Step<KIND, R>& st, int s) {
             const int kk = s * 256 + t * 64;
-            if (__builtin_expect(__any_sync(0xFFFFFFFFu, step_has_tiny<KIND, R>(st)), 0))
-                compute_step<KIND, NB, R, true>(st, acc, xg, xg8, xa_live, xb_live, kk, K);
+            if (__builtin_expect(__any_sync(0xFFFFFFFFu, step_needs_slow<KIND, R>(st)), 0))
+                compute_step<KIND, NB, R, true, false>(st, acc, xg, xg8, xa_live, xb_live, kk, K, xr);
+            else if (s < (K >> 8))
+                compute_step<KIND, NB, R, false, true>(st, acc, xg, xg8, xa_live, xb_live, kk, K, xr);
             else
-                compute_step<KIND, NB, R, false>(st, acc, xg, xg8, xa_live, xb_live, kk, K);
+                compute_step<KIND, NB, R, false, false>(st, acc, xg, xg8, xa_live, xb_live, kk, K, xr);
         };
-        if (wk < steps) load_step<KIND, R>(b0, pb, row0, g, wk * 256 + t * 64, N, K);
+        // two register buffers in ping-pong: the next step's bytes load while this one computes
+        Step<KIND, R> b0, b1;
+        if (wk < steps) load(b0, wk);
         for (int s = wk; s < steps; s += 2 * WK) {
-            if (s + WK < steps) load_step<KIND, R>(b1, pb, row0, g, (s + WK) * 256 + t * 64, N, K);
+            if (s + WK < steps) load(b1, s + WK);
             run_step(b0, s);
             if (s + WK >= steps) break;
-            if (s + 2 * WK < steps) load_step<KIND, R>(b0, pb, row0, g, (s + 2 * WK) * 256 + t * 64, N, K);
+            if (s + 2 * WK < steps) load(b0, s + 2 * WK);
             run_step(b1, s + WK);
         }
     }

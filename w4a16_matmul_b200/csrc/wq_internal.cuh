@@ -105,6 +105,20 @@ __device__ __forceinline__ uint4 ldg_v4(const void* p) {
     return v;
 }
 
+// Asks the L2 to fetch [p, p + bytes) from memory ahead of use (a hint; p and bytes must be
+// multiples of 16 and the range must lie inside one allocation).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Predicated 128-bit load: when `pred` is 0 the registers keep their previous contents
+// (no zero fill, no extra moves).
+__device__ __forceinline__ void ldg_v4_if(uint4& v, const void* p, uint32_t pred) {
+    asm volatile(
+        "{ .reg .pred q; setp.ne.b32 q, %5, 0; @q ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4]; }"
+        : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w) : "l"(p), "r"(pred));
+}
+
 __device__ __forceinline__ uint32_t ldg_u16(const void* p) {
     unsigned short v;
     asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
