@@ -4,25 +4,33 @@
 // and "K-Means量化技术…" §2.2 (LUT16: a 16-entry centroid table per block of 64), fused into
 // the product instead of written out as a dense matrix.
 //
-// Design (HBM-bound: 0.53 B per dyadic weight, 1 B per LUT16 weight; the limit to beat is
-// the instruction issue rate of the in-register reconstruction):
+// Design (HBM-bound: 0.53 B per dyadic weight, 1 B per LUT16 weight; what stands between
+// the kernel and the memory roof is the instruction count and latency of the in-register
+// reconstruction):
 //   * A warp owns 16*R rows of one problem. Lane (g = lane/4, t = lane%4) streams rows g
 //     and g+8 of every 16-row block: per 256-column step, 32 contiguous bytes of each
 //     (64 codes: one dyadic g64 group, two g32 groups, or one LUT16 block) with two
 //     128-bit non-allocating loads; a quad of lanes covers 128 contiguous bytes of a row.
 //     The next step's bytes are loaded while the current step computes.
+//   * The CTA stages its activations once per K chunk into shared memory, already in the
+//     order of the mma B fragment, so one 128-bit shared load per 8 columns replaces the
+//     global load and the byte permutes of every warp (the activations are read from L2
+//     once per CTA instead of once per warp).
 //   * The product runs on the warp-level tensor-core path (mma m16n8k16, fp32
 //     accumulate): the reconstructed weights are the A operand (16 rows x 16 columns, no
 //     padding), the activations the B operand (batch columns 0..7, and 8..15 in a second
-//     mma when batch > 8). Issuing one mma per 256 weights keeps the per-weight cost at
-//     the nibble-to-bf16 conversion, which CUDA-core FMAs could not match at batch > 1.
-//   * Dyadic reconstruction is exact: a nibble pair is OR-ed into the mantissa of the bf16
-//     value 128 (giving 128 + idx, exact), minus 136 (exact), times step in one bf16 FMA
-//     (one rounding, to nearest even) -- the same bits wq_dequant writes. Groups whose
-//     scale is below 2^-100 (step not representable as a normal bf16) take an fp32 path.
+//     mma when batch > 8).
+//   * Dyadic reconstruction is exact and costs one bf16x2 FMA per weight pair. The nibble
+//     pairs are masked straight out of the packed word, which makes them bf16 numbers
+//     idx * 2^-133 (or idx * 2^-129); one FMA with (scale * 2^66, -scale * 2^-64) forms
+//     2^-64 * step * (idx - 8) and rounds it once, i.e. 2^-64 times the bf16 weight that
+//     wq_dequant writes. The staged activations carry the compensating 2^64, so every
+//     product, and hence the fp32 sum, is the one of the unscaled operands. Steps whose
+//     scales fall outside [2^-59, 2^62), or chunks whose activations reach 2^64, take an
+//     exact fp32 path with unscaled activations.
 //   * The k order inside one mma is a permutation of the physical columns (word nibbles
-//     pair up as (0,4), (1,5), (2,6), (3,7)); the activation fragment is permuted the same
-//     way with byte permutes, so the contraction is unchanged.
+//     pair up as (0,4), (1,5), (2,6), (3,7)); the staged activations follow it, so the
+//     contraction is unchanged.
 //   * When a launch has too few rows to fill the GPU, WK warps of a CTA split K and meet
 //     in shared memory at the end; otherwise every warp covers the full K and no
 //     reduction exists. One launch, no workspace, either way.
@@ -32,36 +40,30 @@ namespace wq {
 namespace {
 
 constexpr int kMaxProblems = WQ_GEMV_MAX_GROUPED;
+#ifndef WQ_GEMV_DEPTH
+#define WQ_GEMV_DEPTH 2
+#endif
+#ifndef WQ_GEMV_MIN_CTAS_NB1
+#define WQ_GEMV_MIN_CTAS_NB1 (WQ_GEMV_DEPTH >= 4 ? 4 : WQ_GEMV_DEPTH == 3 ? 5 : 6)
+#endif
+#ifndef WQ_GEMV_MIN_CTAS_NB2
+#define WQ_GEMV_MIN_CTAS_NB2 4
+#endif
+#ifndef WQ_GEMV_R2_MIN_BATCH
+#define WQ_GEMV_R2_MIN_BATCH 4       // 32-row warps above this batch (large launches)
+#endif
 
 template <int MAXP>
 struct GemvParams {
     int count;
     int batch;
+    int chunk_steps;              // 256-column steps per staged activation chunk
     int tile_start[MAXP + 1];     // prefix sum of row tiles per problem
     GemvProblem prob[MAXP];
 };
 
-// bf16 pairs of the 8 codes of one packed word, dyadic: pair j = (code j, code j+4), the
-// lower code index in the low half, each bf16(step * (idx - 8)) rounded once.
-//
-// A bf16 bit pattern below 0x0100 is worth exactly (pattern) * 2^-133: the subnormals and
-// the first normal binade share that spacing. So (w & 0x000F000F) is the pair (idx0, idx4)
-// times 2^-133 and (w & 0x00F000F0) is (idx1, idx5) times 2^-129, with no shift; w >> 8 gives
-// the other two pairs the same way. One FMA by 2^126 (resp. 2^122) brings them to idx * 2^-7
-// exactly, and fma(idx * 2^-7, 16 * scale, -scale) = scale * (idx - 8) / 8 is formed exactly
-// and rounded once. cs = (16 * scale) pair, cn = (-scale) pair.
-__device__ __forceinline__ void dyadic_pairs(uint32_t w, uint32_t cs, uint32_t cn, uint32_t (&p)[4]) {
-    const uint32_t kP126 = 0x7E807E80u;       // bf16 2^126 twice
-    const uint32_t kP122 = 0x7C807C80u;       // bf16 2^122 twice
-    const uint32_t kNegZero = 0x80008000u;
-    const uint32_t t = w >> 8;
-    p[0] = bf16x2_fma(bf16x2_fma(w & 0x000F000Fu, kP126, kNegZero), cs, cn);
-    p[1] = bf16x2_fma(bf16x2_fma(w & 0x00F000F0u, kP122, kNegZero), cs, cn);
-    p[2] = bf16x2_fma(bf16x2_fma(t & 0x000F000Fu, kP126, kNegZero), cs, cn);
-    p[3] = bf16x2_fma(bf16x2_fma(t & 0x00F000F0u, kP122, kNegZero), cs, cn);
-}
-
-// Same pairs computed in fp32 (for scales whose 16x overflows bf16).
+// bf16 pairs of the 8 codes of one packed word, dyadic, computed in fp32 (exact for every
+// scale) and rounded once: pair j = (code j, code j+4), the lower code index in the low half.
 __device__ __forceinline__ void dyadic_pairs_f32(uint32_t w, float step, uint32_t (&p)[4]) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -71,11 +73,34 @@ __device__ __forceinline__ void dyadic_pairs_f32(uint32_t w, float step, uint32_
     }
 }
 
-// (16 * scale, -scale) as bf16 pairs (exact for every finite scale below 2^124).
-__device__ __forceinline__ void scale_pairs(uint32_t scale_bits, uint32_t& cs, uint32_t& cn) {
+// Staged-activation scale and the range of scales the one-FMA reconstruction covers.
+// With e = 64: the weights come out times 2^-64 and stay normal for scale >= 2^-59 (biased
+// exponent 68); scale * 2^66 stays finite for scale < 2^62 (biased exponent <= 188);
+// activations times 2^64 stay finite for |x| < 2^64 (bf16 magnitude bits < 0x5F80).
+constexpr uint32_t kXScalePair = 0x5F805F80u;    // bf16 2^64 twice
+constexpr uint32_t kScaleExpLo = 68, kScaleExpHi = 188;
+
+// (scale * 2^66, scale * 2^62, -scale * 2^-64) as bf16 pairs, by adding to the exponent
+// field (exact: the range check keeps every result a normal number).
+__device__ __forceinline__ void scaled_consts(uint32_t scale_bits, uint32_t& c1, uint32_t& c2,
+                                              uint32_t& d) {
     const uint32_t s2 = prmt(scale_bits, 0, 0x1010u);
-    cs = bf16x2_fma(s2, 0x41804180u, 0x80008000u);     // x 16.0
-    cn = s2 ^ 0x80008000u;
+    c1 = s2 + 0x21002100u;
+    c2 = s2 + 0x1F001F00u;
+    d = (s2 - 0x20002000u) ^ 0x80008000u;
+}
+
+// Pairs of 2^-64 * bf16(step * (idx - 8)): (w & 0x000F000F) is (idx0, idx4) * 2^-133 and
+// (w & 0x00F000F0) is (idx1, idx5) * 2^-129 as bf16 numbers; times scale * 2^66 (resp.
+// 2^62) they are exactly idx * step * 2^-64, and adding -8 * step * 2^-64 in the same FMA
+// rounds once.
+__device__ __forceinline__ void dyadic_pairs_scaled(uint32_t w, uint32_t c1, uint32_t c2,
+                                                    uint32_t d, uint32_t (&p)[4]) {
+    const uint32_t t = w >> 8;
+    p[0] = bf16x2_fma(w & 0x000F000Fu, c1, d);
+    p[1] = bf16x2_fma(w & 0x00F000F0u, c2, d);
+    p[2] = bf16x2_fma(t & 0x000F000Fu, c1, d);
+    p[3] = bf16x2_fma(t & 0x00F000F0u, c2, d);
 }
 
 // LUT16 lookup of 4 codes (nibbles of the low 16 bits of s) in a 16-entry fp16 table held
@@ -137,8 +162,10 @@ __device__ __forceinline__ void load_step(Step<KIND, R>& st, const GemvProblem& 
                 st.aux[r][h][0] = la.x; st.aux[r][h][1] = la.y; st.aux[r][h][2] = la.z; st.aux[r][h][3] = la.w;
                 st.aux[r][h][4] = lb.x; st.aux[r][h][5] = lb.y; st.aux[r][h][6] = lb.z; st.aux[r][h][7] = lb.w;
             } else {
+                // rows or groups outside the matrix get scale 1.0 (their codes are 8, so their
+                // weights are 0) which keeps the step on the one-FMA path
                 const uint16_t* sp = (const uint16_t*)pb.aux;
-                uint32_t s0 = 0, s1 = 0;
+                uint32_t s0 = 0x3F80u, s1 = 0x3F80u;
                 if (KIND == kDyadic64) {
                     if (rl && h0) s0 = ldg_u16(sp + (size_t)row * (K / 64) + kk / 64);
                     s1 = s0;
@@ -152,16 +179,15 @@ __device__ __forceinline__ void load_step(Step<KIND, R>& st, const GemvProblem& 
         }
 }
 
-// One 256-column step: 8 words per row, 2 (or 4) mma per word pair. FULL: the step lies
-// inside K, so every activation load is in range; lanes whose batch column is unused load
-// some valid row (those output columns are computed but never stored).
-template <int KIND, int NB, int R, bool SLOW, bool FULL>
-__device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&acc)[R][NB][4],
-                                             const uint16_t* xg, const uint16_t* xg8, bool xa_live,
-                                             bool xb_live, int kk, int K, uint4 (&xr)[2]) {
-    const bool h0 = kk < K, h1 = kk + 32 < K;
-    uint32_t cs[R][2][2], cn[R][2][2];
-    float fst[R][2][2];
+// One 256-column step from the staged activations: 8 words per row, 2 (or 4) mma per word
+// pair. xs0 / xs1: this lane's 16-byte slot of the step in the staged rows of batch
+// columns g and g + 8 (lanes of unused batch columns read some staged row; their outputs
+// are never stored).
+template <int KIND, int NB, int R>
+__device__ __forceinline__ void compute_step_staged(const Step<KIND, R>& st, float (&acc)[R][NB][4],
+                                                    const uint8_t* xs0, const uint8_t* xs1) {
+    constexpr int J = (KIND == kDyadic32) ? 2 : 1;
+    uint32_t c1[R][2][J], c2[R][2][J], dd[R][2][J];
     uint32_t plo[R][2][4], phi[R][2][4];
 #pragma unroll
     for (int r = 0; r < R; ++r)
@@ -176,45 +202,18 @@ __device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&ac
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < (KIND == kDyadic32 ? 2 : 1); ++j) {
-                    if (SLOW) fst[r][h][j] = bf16_bits_to_float(st.aux[r][h][j]) * 0.125f;
-                    else scale_pairs(st.aux[r][h][j], cs[r][h][j], cn[r][h][j]);
-                }
+                for (int j = 0; j < J; ++j) scaled_consts(st.aux[r][h][j], c1[r][h][j], c2[r][h][j], dd[r][h][j]);
             }
         }
 #pragma unroll
     for (int sub = 0; sub < 8; ++sub) {
-        const int kx = kk + 8 * sub;
-        uint4 xa, xb;
-        if (FULL) {
-            // lanes of unused batch columns keep stale registers: their columns are never stored
-            ldg_v4_if(xr[0], xg + kx, xa_live);
-            xa = xr[0];
+        uint32_t b[NB][4];
+        {
+            const uint4 xa = *reinterpret_cast<const uint4*>(xs0 + 64 * sub);
+            b[0][0] = xa.x; b[0][1] = xa.y; b[0][2] = xa.z; b[0][3] = xa.w;
             if (NB == 2) {
-                ldg_v4_if(xr[1], xg8 + kx, xb_live);
-                xb = xr[1];
-            }
-        } else {
-            const bool xv = (sub < 4) ? h0 : h1;
-            xa = make_uint4(0, 0, 0, 0);
-            xb = xa;
-            if (xa_live && xv) xa = ldg_v4(xg + kx);
-            if (NB == 2 && xb_live && xv) xb = ldg_v4(xg8 + kx);
-        }
-        uint32_t b[NB][4];                              // B fragments of the two mma
-        if (KIND == kLut16) {
-            b[0][0] = bf16x2_to_f16x2(xa.x); b[0][1] = bf16x2_to_f16x2(xa.y);
-            b[0][2] = bf16x2_to_f16x2(xa.z); b[0][3] = bf16x2_to_f16x2(xa.w);
-            if (NB == 2) {
-                b[NB - 1][0] = bf16x2_to_f16x2(xb.x); b[NB - 1][1] = bf16x2_to_f16x2(xb.y);
-                b[NB - 1][2] = bf16x2_to_f16x2(xb.z); b[NB - 1][3] = bf16x2_to_f16x2(xb.w);
-            }
-        } else {
-            b[0][0] = prmt(xa.x, xa.z, 0x5410u); b[0][1] = prmt(xa.x, xa.z, 0x7632u);
-            b[0][2] = prmt(xa.y, xa.w, 0x5410u); b[0][3] = prmt(xa.y, xa.w, 0x7632u);
-            if (NB == 2) {
-                b[NB - 1][0] = prmt(xb.x, xb.z, 0x5410u); b[NB - 1][1] = prmt(xb.x, xb.z, 0x7632u);
-                b[NB - 1][2] = prmt(xb.y, xb.w, 0x5410u); b[NB - 1][3] = prmt(xb.y, xb.w, 0x7632u);
+                const uint4 xb = *reinterpret_cast<const uint4*>(xs1 + 64 * sub);
+                b[NB - 1][0] = xb.x; b[NB - 1][1] = xb.y; b[NB - 1][2] = xb.z; b[NB - 1][3] = xb.w;
             }
         }
 #pragma unroll
@@ -231,14 +230,9 @@ __device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&ac
                     mma_f16_16816(acc[r][nb], q0[2], q1[2], q0[3], q1[3], b[nb][2], b[nb][3]);
                 }
             } else {
-                const int hs = (KIND == kDyadic32 && sub >= 4) ? 1 : 0;
-                if (SLOW) {
-                    dyadic_pairs_f32(st.w[r][0][sub], fst[r][0][hs], q0);
-                    dyadic_pairs_f32(st.w[r][1][sub], fst[r][1][hs], q1);
-                } else {
-                    dyadic_pairs(st.w[r][0][sub], cs[r][0][hs], cn[r][0][hs], q0);
-                    dyadic_pairs(st.w[r][1][sub], cs[r][1][hs], cn[r][1][hs], q1);
-                }
+                const int hs = (J == 2 && sub >= 4) ? 1 : 0;
+                dyadic_pairs_scaled(st.w[r][0][sub], c1[r][0][hs], c2[r][0][hs], dd[r][0][hs], q0);
+                dyadic_pairs_scaled(st.w[r][1][sub], c1[r][1][hs], c2[r][1][hs], dd[r][1][hs], q1);
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb) {
                     mma_bf16_16816(acc[r][nb], q0[0], q1[0], q0[1], q1[1], b[nb][0], b[nb][1]);
@@ -249,22 +243,142 @@ __device__ __forceinline__ void compute_step(const Step<KIND, R>& st, float (&ac
     }
 }
 
-// A step needs the fp32 path when 16 * scale would overflow bf16 (scale >= 2^124).
+// The exact fallback for a dyadic step the one-FMA form does not cover (a scale outside
+// [2^-59, 2^62) or staged activations that would overflow): weights formed in fp32 (exact
+// for every finite scale) and rounded once, activations read unscaled from global memory.
+// It reloads the step's bytes itself, one word per row and sub-step, so that it needs few
+// registers beyond those the hot loop holds.
+template <int KIND, int NB, int R>
+__device__ __forceinline__ void compute_step_exact(const GemvProblem& pb, int row0, int g, int kk, int N,
+                                                   int K, int B, float (&acc)[R][NB][4]) {
+    const int group = (KIND == kDyadic32) ? 32 : 64;
+    const bool xa_live = g < B, xb_live = NB == 2 && (g + 8 < B);
+    const uint16_t* xg = pb.x + (size_t)(xa_live ? g : 0) * K;
+    const uint16_t* xg8 = pb.x + (size_t)(xb_live ? g + 8 : 0) * K;
+    const size_t row_bytes = (size_t)K / 2;
+    const uint16_t* sp = (const uint16_t*)pb.aux;
+#pragma unroll 1
+    for (int sub = 0; sub < 8; ++sub) {
+        const int kx = kk + 8 * sub;
+        const bool xv = kx < K;
+        uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
+        if (xa_live && xv) xa = ldg_v4(xg + kx);
+        if (NB == 2 && xb_live && xv) xb = ldg_v4(xg8 + kx);
+        uint32_t b[NB][4];
+        b[0][0] = prmt(xa.x, xa.z, 0x5410u); b[0][1] = prmt(xa.x, xa.z, 0x7632u);
+        b[0][2] = prmt(xa.y, xa.w, 0x5410u); b[0][3] = prmt(xa.y, xa.w, 0x7632u);
+        if (NB == 2) {
+            b[NB - 1][0] = prmt(xb.x, xb.z, 0x5410u); b[NB - 1][1] = prmt(xb.x, xb.z, 0x7632u);
+            b[NB - 1][2] = prmt(xb.y, xb.w, 0x5410u); b[NB - 1][3] = prmt(xb.y, xb.w, 0x7632u);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            uint32_t q[2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = row0 + 16 * r + 8 * h + g;
+                uint32_t w = 0x88888888u, sc = 0;
+                if (row < N && xv) {
+                    w = ldg_u32(pb.packed + (size_t)row * row_bytes + kx / 2);
+                    sc = ldg_u16(sp + (size_t)row * (K / group) + kx / group);
+                }
+                dyadic_pairs_f32(w, bf16_bits_to_float(sc) * 0.125f, q[h]);
+            }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                mma_bf16_16816(acc[r][nb], q[0][0], q[1][0], q[0][1], q[1][1], b[nb][0], b[nb][1]);
+                mma_bf16_16816(acc[r][nb], q[0][2], q[1][2], q[0][3], q[1][3], b[nb][2], b[nb][3]);
+            }
+        }
+    }
+}
+
+// True when every scale of the step lies in [2^-59, 2^62) (biased exponent 68..188), the
+// range the one-FMA reconstruction covers.
 template <int KIND, int R>
-__device__ __forceinline__ bool step_needs_slow(const Step<KIND, R>& st) {
-    if (KIND == kLut16) return false;
-    uint32_t m = 0;
+__device__ __forceinline__ bool step_scales_in_range(const Step<KIND, R>& st) {
+    if (KIND == kLut16) return true;
+    bool ok = true;
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) m = max(m, st.aux[r][h][j] & 0x7FFFu);
-    return m >= 0x7D80u;
+            for (int j = 0; j < (KIND == kDyadic32 ? 2 : 1); ++j) {
+                const uint32_t e = (st.aux[r][h][j] >> 7) & 0xFFu;
+                ok = ok && (e - kScaleExpLo <= kScaleExpHi - kScaleExpLo);
+            }
+    return ok;
+}
+
+// Staged activations: batch row b at byte b * rs (rs = 512 * chunk_steps + 64, so the
+// eight rows one 128-bit shared load phase touches start on distinct banks); inside a row,
+// step s of the chunk at 512 * s, sub-step u at 64 * u, quad position t at 16 * t: the
+// 8 columns 256 * s + 64 * t + 8 * u .. +7 in B-fragment order. Dyadic: bf16 times 2^64,
+// columns paired (0,4), (1,5), (2,6), (3,7); LUT16: fp16 in natural order. Columns at or
+// beyond K are zero. Stages steps [c0, c0 + ns) of all B rows with the whole CTA; returns
+// (dyadic) whether some staged |x| reaches 2^64 or is not finite.
+template <int KIND>
+__device__ __forceinline__ bool stage_x(uint8_t* xs, const uint16_t* x, int B, int K, int c0,
+                                        int ns, int rs) {
+    const int per_row = ns * 32;                 // 16-byte blocks of 8 columns
+    const int total = B * per_row;
+    uint32_t bad = 0;
+    constexpr int U = 4;                         // loads in flight per thread
+    for (int base = threadIdx.x; base < total; base += 128 * U) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + 128 * u;
+            v[u] = make_uint4(0, 0, 0, 0);
+            if (i < total) {
+                const int b = i / per_row, j = i - b * per_row;
+                const int col = c0 * 256 + 8 * j;
+                if (col < K) v[u] = ldg_v4(x + (size_t)b * K + col);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + 128 * u;
+            if (i >= total) break;
+            const int b = i / per_row, j = i - b * per_row;
+            uint4 f;
+            if (KIND == kLut16) {
+                f.x = bf16x2_to_f16x2(v[u].x); f.y = bf16x2_to_f16x2(v[u].y);
+                f.z = bf16x2_to_f16x2(v[u].z); f.w = bf16x2_to_f16x2(v[u].w);
+            } else {
+                // a half of magnitude bits m >= 0x5F80 (|x| >= 2^64, inf, NaN) carries into
+                // bit 15 of that half when 0x2080 is added
+                const uint32_t m = ((v[u].x & 0x7FFF7FFFu) + 0x20802080u) | ((v[u].y & 0x7FFF7FFFu) + 0x20802080u) |
+                                   ((v[u].z & 0x7FFF7FFFu) + 0x20802080u) | ((v[u].w & 0x7FFF7FFFu) + 0x20802080u);
+                bad |= m & 0x80008000u;
+                const uint32_t kNegZero = 0x80008000u;
+                f.x = bf16x2_fma(prmt(v[u].x, v[u].z, 0x5410u), kXScalePair, kNegZero);
+                f.y = bf16x2_fma(prmt(v[u].x, v[u].z, 0x7632u), kXScalePair, kNegZero);
+                f.z = bf16x2_fma(prmt(v[u].y, v[u].w, 0x5410u), kXScalePair, kNegZero);
+                f.w = bf16x2_fma(prmt(v[u].y, v[u].w, 0x7632u), kXScalePair, kNegZero);
+            }
+            *reinterpret_cast<uint4*>(xs + b * rs + (j >> 5) * 512 + (j & 7) * 64 + ((j >> 3) & 3) * 16) = f;
+        }
+    }
+    return bad != 0;
+}
+
+// Steps of weight bytes held in registers per warp (D - 1 of them in flight): the bytes in
+// flight per SM, warps x (D - 1) x 2 KB, set the bandwidth a latency-bound stream reaches,
+// and deeper buffers buy them at fewer registers than more warps would.
+constexpr int depth(int kind, int nb, int r) {
+    return (kind != kLut16 && nb == 1 && r == 1) ? WQ_GEMV_DEPTH : 2;
+}
+
+// Resident CTAs per SM the register budget of a dyadic 16-row kernel aims at; the other
+// variants take what they need.
+constexpr int min_ctas(int kind, int nb, int r) {
+    return (kind != kLut16 && r == 1) ? (nb == 1 ? WQ_GEMV_MIN_CTAS_NB1 : WQ_GEMV_MIN_CTAS_NB2) : 1;
 }
 
 template <int KIND, int NB, int R, int WK, int MAXP>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, min_ctas(KIND, NB, R))
 gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     constexpr int WR = 4 / WK;                       // warps with distinct rows per CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -291,57 +405,49 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) acc[r][nb][0] = acc[r][nb][1] = acc[r][nb][2] = acc[r][nb][3] = 0.f;
 
-    const bool xa_live = g < B, xb_live = NB == 2 && (g + 8 < B);
-    // lanes whose batch column is unused read row 0 (their outputs are never stored)
-    const uint16_t* xg = pb.x + (size_t)(xa_live ? g : 0) * K;
-    const uint16_t* xg8 = pb.x + (size_t)(xb_live ? g + 8 : 0) * K;
-
-    if (row0 < N && wk == 0 && lane == 0) {
-        // The warp's rows are contiguous in memory: ask the L2 for all of them now, so the
-        // register loads below see L2 latency rather than DRAM latency.
-        const int rows = min(16 * R, N - row0);
-        const size_t row_bytes = (size_t)K / 2;
-        prefetch_l2_bulk(pb.packed + (size_t)row0 * row_bytes, (uint32_t)(rows * row_bytes));
-        if (KIND == kLut16) {
-            const size_t lb = (size_t)(K / 64) * 32;                  // fp16 [16] per block
-            prefetch_l2_bulk((const uint8_t*)pb.aux + (size_t)row0 * lb, (uint32_t)(rows * lb));
-        } else {
-            // scales: the 16-byte-aligned interior of this warp's rows
-            const size_t sb = (size_t)(K / (KIND == kDyadic64 ? 64 : 32)) * 2;
-            const uintptr_t a0 = (uintptr_t)pb.aux + (size_t)row0 * sb;
-            const uintptr_t a1 = a0 + (size_t)rows * sb;
-            const uintptr_t b0 = (a0 + 15) & ~(uintptr_t)15, b1 = a1 & ~(uintptr_t)15;
-            if (b1 > b0) prefetch_l2_bulk((const void*)b0, (uint32_t)(b1 - b0));
-        }
+    extern __shared__ __align__(16) uint8_t xs[];
+    const int cs = prm.chunk_steps, rs = 512 * cs + 64;
+    const uint8_t* xs0 = xs + min(g, B - 1) * rs + 16 * t;
+    const uint8_t* xs1 = xs + min(g + 8, B - 1) * rs + 16 * t;
+    const bool live = row0 < N;
+    // FULL loads (all rows of the warp and all 256 columns in range) run without
+    // predicates; only a ragged last step or a ragged last row block take the checks
+    const int full_steps = (row0 + 16 * R <= N) ? (K >> 8) : 0;
+    auto load = [&](Step<KIND, R>& st, int s) {
+        if (s < full_steps) load_step<KIND, R, true>(st, pb, row0, g, s * 256 + t * 64, N, K);
+        else load_step<KIND, R, false>(st, pb, row0, g, s * 256 + t * 64, N, K);
+    };
+    auto run_step = [&](const Step<KIND, R>& st, int s, int c0, bool xbad) {
+        if (KIND == kLut16 || (!xbad && __all_sync(0xFFFFFFFFu, step_scales_in_range<KIND, R>(st))))
+            compute_step_staged<KIND, NB, R>(st, acc, xs0 + 512 * (s - c0), xs1 + 512 * (s - c0));
+        else
+            compute_step_exact<KIND, NB, R>(pb, row0, g, s * 256 + t * 64, N, K, B, acc);
+    };
+    // D register buffers in rotation: the bytes of D - 1 steps are in flight while one step
+    // computes, and the first D - 1 steps' loads are issued before the activations are
+    // staged. A chunk holds a whole multiple of D * WK steps, so every chunk starts at
+    // buffer 0 (step j of this warp lives in buffer j % D).
+    constexpr int D = depth(KIND, NB, R);
+    Step<KIND, R> buf[D];
+    if (live) {
+#pragma unroll
+        for (int i = 0; i < D - 1; ++i)
+            if (wk + i * WK < steps) load(buf[i], wk + i * WK);
     }
-    if (row0 < N) {
-        // FULL steps (all rows of the warp and all 256 columns in range) run without
-        // predicates; only a ragged last step or a ragged last row block take the checks
-        const bool rows_full = row0 + 16 * R <= N;
-        const int full_steps = rows_full ? (K >> 8) : 0;
-        auto load = [&](Step<KIND, R>& st, int s) {
-            if (s < full_steps) load_step<KIND, R, true>(st, pb, row0, g, s * 256 + t * 64, N, K);
-            else load_step<KIND, R, false>(st, pb, row0, g, s * 256 + t * 64, N, K);
-        };
-        uint4 xr[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        auto run_step = [&](const Step<KIND, R>& st, int s) {
-            const int kk = s * 256 + t * 64;
-            if (__builtin_expect(__any_sync(0xFFFFFFFFu, step_needs_slow<KIND, R>(st)), 0))
-                compute_step<KIND, NB, R, true, false>(st, acc, xg, xg8, xa_live, xb_live, kk, K, xr);
-            else if (s < (K >> 8))
-                compute_step<KIND, NB, R, false, true>(st, acc, xg, xg8, xa_live, xb_live, kk, K, xr);
-            else
-                compute_step<KIND, NB, R, false, false>(st, acc, xg, xg8, xa_live, xb_live, kk, K, xr);
-        };
-        // two register buffers in ping-pong: the next step's bytes load while this one computes
-        Step<KIND, R> b0, b1;
-        if (wk < steps) load(b0, wk);
-        for (int s = wk; s < steps; s += 2 * WK) {
-            if (s + WK < steps) load(b1, s + WK);
-            run_step(b0, s);
-            if (s + WK >= steps) break;
-            if (s + 2 * WK < steps) load(b0, s + 2 * WK);
-            run_step(b1, s + WK);
+    for (int c0 = 0; c0 < steps; c0 += cs) {
+        if (c0 > 0) __syncthreads();               // every warp is done with the last chunk
+        const int ns = min(cs, steps - c0);
+        const bool xbad = __syncthreads_or(stage_x<KIND>(xs, pb.x, B, K, c0, ns, rs)) != 0;
+        if (!live) continue;
+        const int cend = c0 + ns;
+        for (int s0 = c0 + wk; s0 < cend; s0 += D * WK) {
+#pragma unroll
+            for (int i = 0; i < D; ++i) {
+                const int s = s0 + i * WK;
+                if (s >= cend) break;
+                if (s + (D - 1) * WK < steps) load(buf[(i + D - 1) % D], s + (D - 1) * WK);
+                run_step(buf[i], s, c0, xbad);
+            }
         }
     }
 
@@ -380,9 +486,30 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
             }
 }
 
+// Staged activations per CTA: at most this many bytes (a chunk of 256-column steps of all
+// batch rows); K is walked in chunks when batch * K does not fit.
+constexpr int kXStageBudget = 32 * 1024;
+
 template <int KIND, int NB, int R, int WK, int MAXP>
-wq_status run(const GemvParams<MAXP>& prm, int tiles, cudaStream_t s) {
-    gemv_kernel<KIND, NB, R, WK, MAXP><<<tiles, 128, 0, s>>>(prm);
+wq_status run(GemvParams<MAXP>& prm, const GemvProblem* probs, int tiles, cudaStream_t s) {
+    constexpr int unit = depth(KIND, NB, R) * WK;   // chunks are whole multiples of this
+    int max_steps = 1;
+    for (int i = 0; i < prm.count; ++i) max_steps = max(max_steps, (probs[i].k + 255) / 256);
+    int cs = max(1, (kXStageBudget / prm.batch - 64) / 512);
+    cs = max(unit, cs - cs % unit);
+    prm.chunk_steps = min(cs, max_steps);
+    const size_t smem = (size_t)prm.batch * (512 * prm.chunk_steps + 64);
+    if (smem > 48 * 1024) {
+        // small launches with many batch rows: a chunk of D * WK steps may pass 48 KB
+        static bool raised = false;
+        if (!raised) {
+            if (cudaFuncSetAttribute(gemv_kernel<KIND, NB, R, WK, MAXP>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) != cudaSuccess)
+                return check_launch("gemv shared memory");
+            raised = true;
+        }
+    }
+    gemv_kernel<KIND, NB, R, WK, MAXP><<<tiles, 128, smem, s>>>(prm);
     return check_launch("gemv");
 }
 
@@ -404,11 +531,11 @@ wq_status pick_split(GemvParams<MAXP>& prm, const GemvProblem* probs, int count,
     // 32-row warps pay off once the activation fragment is shared by more batch rows
     // (measured: 16-row warps win at batch <= 4, 32-row warps at batch 5..16)
     constexpr int BIGR = (KIND == kLut16) ? 1 : 2;
-    if (BIGR == 2 && batch > 4 && rows16 >= 12 * sms * 2)
-        return run<KIND, NB, BIGR, 1, MAXP>(prm, tiles_for(64 * BIGR), s);
-    if (rows16 >= 8 * sms) return run<KIND, NB, 1, 1, MAXP>(prm, tiles_for(64), s);
-    if (rows16 >= 2 * sms) return run<KIND, NB, 1, 2, MAXP>(prm, tiles_for(32), s);
-    return run<KIND, NB, 1, 4, MAXP>(prm, tiles_for(16), s);
+    if (BIGR == 2 && batch > WQ_GEMV_R2_MIN_BATCH && rows16 >= 12 * sms * 2)
+        return run<KIND, NB, BIGR, 1, MAXP>(prm, probs, tiles_for(64 * BIGR), s);
+    if (rows16 >= 8 * sms) return run<KIND, NB, 1, 1, MAXP>(prm, probs, tiles_for(64), s);
+    if (rows16 >= 2 * sms) return run<KIND, NB, 1, 2, MAXP>(prm, probs, tiles_for(32), s);
+    return run<KIND, NB, 1, 4, MAXP>(prm, probs, tiles_for(16), s);
 }
 
 template <int MAXP>
