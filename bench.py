@@ -124,10 +124,19 @@ def build_sweep(wq, torch, dev, batch):
         packed.append(pw)
         del w
     xs_host = [workloads.activations(batch, k, workloads.DECODE_SWEEP, idx) for _, _, _, k, idx in mats]
-    xs = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in xs_host]
-    ys = [torch.empty((batch, n), dtype=torch.bfloat16, device=dev) for _, _, n, _, _ in mats]
+    # every x (and y) is a view into one flat buffer, so that a step's inputs arrive in one
+    # host-to-device copy and its outputs leave in one (each view starts 64-byte aligned:
+    # batch * k * 2 bytes with k a multiple of 32)
+    xflat = torch.from_numpy(np.concatenate([x.reshape(-1) for x in xs_host]).view(np.int16)).view(torch.bfloat16).to(dev)
+    yflat = torch.empty(sum(batch * n for _, _, n, _, _ in mats), dtype=torch.bfloat16, device=dev)
+    xs, ys, xo, yo = [], [], 0, 0
+    for _, _, n, k, _ in mats:
+        xs.append(xflat[xo:xo + batch * k].view(batch, k))
+        ys.append(yflat[yo:yo + batch * n].view(batch, n))
+        xo += batch * k
+        yo += batch * n
     torch.cuda.synchronize(dev)
-    return mats, packed, xs_host, xs, ys
+    return mats, packed, xs_host, xs, ys, xflat, yflat
 
 
 def sweep_bytes(mats, batch):
@@ -190,7 +199,7 @@ def run_ours(args):
         return float(t.item())
 
     B = args.batch
-    mats, packed, xs_host, xs, ys = build_sweep(wq, torch, dev, B)
+    mats, packed, xs_host, xs, ys, xflat, yflat = build_sweep(wq, torch, dev, B)
     stream = torch.cuda.current_stream(dev)
     run = wq.GroupedGemv(packed, xs, ys)
     pk_b, sc_b, x_b, y_b = sweep_bytes(mats, B)
@@ -198,24 +207,29 @@ def run_ours(args):
     algo_bytes = pk_b + sc_b + x_b + y_b
 
     clocks = ClockSampler(local)
-    # ---- headline: device-resident, one grouped launch per step ------------------------
+    # ---- headline: device-resident, one grouped launch per step, replayed from a CUDA graph
+    # (the launch is captured once; a replay costs the host a few microseconds, so the
+    # timed region holds the kernel and not the argument checks of the C ABI call) --------
+    graph = torch.cuda.CUDAGraph()
+    run()                                    # first call outside capture (one-time setup)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        run()
     clocks.start()
-    ms = time_region(torch, stream, run, args.steps, args.warmup, barrier)
+    ms = time_region(torch, stream, graph.replay, args.steps, args.warmup, barrier)
     clk = clocks.stop()
     ms = max_over_ranks(ms)
     value = world * weight_bytes / (ms * 1e-3) / 1e9
     achieved = algo_bytes / (ms * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers ---------------------------
-    xs_pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in xs_host]
-    ys_pin = [torch.empty(y.shape, dtype=torch.bfloat16).pin_memory() for y in ys]
+    x_pin = xflat.cpu().pin_memory()
+    y_pin = torch.empty(yflat.shape, dtype=torch.bfloat16).pin_memory()
 
     def e2e_step():
-        for xp, xd in zip(xs_pin, xs):
-            xd.copy_(xp, non_blocking=True)
-        run()
-        for yp, yd in zip(ys_pin, ys):
-            yp.copy_(yd, non_blocking=True)
+        xflat.copy_(x_pin, non_blocking=True)       # this step's activations, host -> device
+        run()                                       # the public API call (prepared plan)
+        y_pin.copy_(yflat, non_blocking=True)       # this step's outputs, device -> host
 
     ms_e2e = max_over_ranks(time_region(torch, stream, e2e_step, args.steps, args.warmup, barrier))
     e2e = {"value": round(world * weight_bytes / (ms_e2e * 1e-3) / 1e9, 2), "unit": UNIT,

@@ -186,6 +186,27 @@ wq_status wq_gemv_w4a16_grouped(const wq_weight* ws, const uint16_t* const* xs,
                                 uint16_t* const* ys, int32_t count, int32_t batch,
                                 wq_stream stream);
 
+/* A prepared grouped GEMV ("plan"), for a launch repeated over the same buffers, such as
+ * every decode step of a model. The pages describe no such object; it exists because the
+ * argument checks of wq_gemv_w4a16_grouped (one driver query per pointer) cost about as
+ * much host time as a decode sweep's kernel takes on the GPU.
+ *   - wq_gemv_plan_create checks the arguments exactly as wq_gemv_w4a16_grouped does,
+ *     chooses the kernel variant and its grid once, and keeps the device pointers. On
+ *     failure *plan is NULL and nothing is kept.
+ *   - wq_gemv_plan_launch enqueues that one kernel on `stream`: a few microseconds of host
+ *     time, no argument checks, no allocation, allowed during stream capture. It computes
+ *     what wq_gemv_w4a16_grouped would with the buffers' contents when the kernel runs.
+ *   - The plan is host memory the library allocates: the one exception to "the library
+ *     allocates nothing and keeps no pointer". wq_gemv_plan_destroy frees it (NULL is a
+ *     no-op). The buffers must stay allocated while the plan is used; launches may come
+ *     from several threads, but no launch may run during or after destroy. */
+typedef struct wq_gemv_plan_s* wq_gemv_plan;
+wq_status wq_gemv_plan_create(const wq_weight* ws, const uint16_t* const* xs,
+                              uint16_t* const* ys, int32_t count, int32_t batch,
+                              wq_gemv_plan* plan);
+wq_status wq_gemv_plan_launch(wq_gemv_plan plan, wq_stream stream);
+void wq_gemv_plan_destroy(wq_gemv_plan plan);
+
 /* Bytes of device workspace wq_gemm_w4a16 needs for this weight and m (0 if none). */
 size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
 

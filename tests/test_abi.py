@@ -12,7 +12,8 @@ def test_library_exports_every_header_function(wq):
     expected = {"wq_status_string", "wq_last_error", "wq_version", "wq_quantize_dyadic",
                 "wq_quantize_lloyd", "wq_pack", "wq_unpack", "wq_dequant", "wq_gemv_w4a16",
                 "wq_gemv_w4a16_grouped", "wq_gemm_workspace_bytes", "wq_gemm_w4a16",
-                "wq_debug_fail_next_launches", "wq_device_error", "wq_gemm_w4a16_static"}
+                "wq_debug_fail_next_launches", "wq_device_error", "wq_gemm_w4a16_static",
+                "wq_gemv_plan_create", "wq_gemv_plan_launch", "wq_gemv_plan_destroy"}
     assert expected <= set(names), set(names) ^ expected
     for n in names:
         assert hasattr(wq._lib, n), n
@@ -48,6 +49,24 @@ def test_shape_and_group_checks_fail_before_any_cuda_call(wq):
     prm = wq.WqLloydParams(0, 100)
     assert lib.wq_quantize_lloyd(p, 4, 64, ctypes.byref(prm), p, p, p, None, None, None) == wq.WQ_EINVAL
     assert lib.wq_gemv_w4a16_grouped(None, None, None, 1, 1, None) == wq.WQ_EINVAL
+
+
+def test_gemv_plan_rejects_bad_arguments_and_keeps_nothing(wq):
+    lib = wq._lib
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    plan = ctypes.c_void_p(1234)
+    d = wq.WqWeight(wq.FMT_DYADIC4, 64, 4, 64, p.value, p.value)
+    arr = (ctypes.c_void_p * 1)(p.value)
+    assert lib.wq_gemv_plan_create(None, None, None, 1, 1, ctypes.byref(plan)) == wq.WQ_EINVAL
+    assert plan.value is None                            # NULL on failure
+    assert lib.wq_gemv_plan_create(ctypes.byref(d), arr, arr, 1, 0, ctypes.byref(plan)) == wq.WQ_EINVAL
+    assert lib.wq_gemv_plan_create(ctypes.byref(d), arr, arr, 1, 1, None) == wq.WQ_EINVAL
+    # host memory is not accepted as a device buffer
+    assert lib.wq_gemv_plan_create(ctypes.byref(d), arr, arr, 1, 1, ctypes.byref(plan)) == wq.WQ_EINVAL
+    assert plan.value is None
+    assert lib.wq_gemv_plan_launch(None, None) == wq.WQ_EINVAL
+    lib.wq_gemv_plan_destroy(None)                       # a no-op
 
 
 def test_misaligned_and_host_pointers_are_rejected(wq):

@@ -174,3 +174,51 @@ def test_gemv_one_hot_every_scale_regime(wq, group):
         x[np.arange(len(cc)), cc] = 1.0
         y = f32(wq.gemv(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
         assert np.array_equal(y, wd[:, cc].T)
+
+
+@pytest.mark.parametrize("batch", [1, 5, 16])
+def test_gemv_plan_matches_grouped_call_and_reads_current_inputs(wq, batch):
+    """A prepared plan launches the kernel the grouped call would (bit-identical output),
+    and reads whatever its bound x buffers hold when it runs."""
+    shapes = [(2048, 2048), (300, 1088), (5632, 2048), (2048, 5632)]
+    ws, packs, xs, ys = [], [], [], []
+    for i, (n, k) in enumerate(shapes):
+        pw, packed, s = _dyadic_weight(wq, n, k, 64, 200 + i)
+        ws.append(pw)
+        packs.append((packed, s))
+        xs.append(to_dev_bits(workloads.activations(batch, k, workloads.DECODE_SWEEP, 300 + i)))
+        ys.append(torch.empty((batch, n), dtype=torch.bfloat16, device="cuda"))
+    plan = wq.GroupedGemv(ws, xs, ys)
+    plan()
+    ref = wq.gemv_grouped(ws, xs)
+    for y, r in zip(ys, ref):
+        assert torch.equal(y, r)
+    # new activations written into the bound buffers: the next launch sees them
+    rng = np.random.default_rng(5)
+    new_bits = []
+    for x, (n, k) in zip(xs, shapes):
+        nb = workloads.activations(batch, k, workloads.DECODE_SWEEP, 400 + n)
+        x.copy_(to_dev_bits(nb))
+        new_bits.append(nb)
+    plan()
+    torch.cuda.synchronize()
+    for (packed, s), nb, y in zip(packs, new_bits, ys):
+        rows = rng.choice(packed.shape[0], 48, replace=False)
+        y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, nb, rows=rows)
+        _check(y, y_ref, bound, rows)
+    plan.close()
+    plan.close()                                         # idempotent
+
+
+def test_gemv_plan_replays_in_a_cuda_graph(wq):
+    pw, packed, s = _dyadic_weight(wq, 1024, 2048, 64, 31)
+    x = to_dev_bits(workloads.activations(1, 2048, workloads.DECODE_SWEEP, 31))
+    y = torch.empty((1, 1024), dtype=torch.bfloat16, device="cuda")
+    plan = wq.GroupedGemv([pw], [x], [y])
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        plan()
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, wq.gemv(pw, x))

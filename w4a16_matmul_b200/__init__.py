@@ -56,6 +56,10 @@ _SIG = {
     "wq_dequant": ([_WP, _vp, _vp], _i32),
     "wq_gemv_w4a16": ([_WP, _vp, _i32, _vp, _vp], _i32),
     "wq_gemv_w4a16_grouped": ([_WP, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i32, _i32, _vp], _i32),
+    "wq_gemv_plan_create": ([_WP, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i32, _i32,
+                             ctypes.POINTER(_vp)], _i32),
+    "wq_gemv_plan_launch": ([_vp, _vp], _i32),
+    "wq_gemv_plan_destroy": ([_vp], None),
     "wq_gemm_workspace_bytes": ([_WP, _i64], _sz),
     "wq_gemm_w4a16": ([_WP, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
     "wq_gemm_w4a16_static": ([_WP, _vp, _i64, _vp, _vp], _i32),
@@ -246,19 +250,38 @@ def gemv_grouped(ws: list[PackedWeight], xs: list[torch.Tensor],
 
 
 class GroupedGemv:
-    """A prepared grouped GEMV: descriptor arrays are built once, each call only launches."""
+    """A prepared grouped GEMV (wq_gemv_plan): the arguments are checked and the kernel is
+    chosen once, at construction; each call only enqueues the kernel, on the current stream
+    (or `stream`), reading whatever the bound x buffers hold by then. The tensors are kept
+    alive for the plan's lifetime."""
 
     def __init__(self, ws: list[PackedWeight], xs: list[torch.Tensor], ys: list[torch.Tensor]):
+        if not (len(ws) == len(xs) == len(ys)):
+            raise ValueError("ws, xs and ys must have the same length")
+        for x in xs:
+            _cuda(x, torch.bfloat16, "x")
+        for y in ys:
+            _cuda(y, torch.bfloat16, "y")
         self.cnt = len(ws)
         self.batch = xs[0].shape[0]
         self._keep = (ws, xs, ys)
-        self.arr = (WqWeight * self.cnt)(*[w.desc() for w in ws])
-        self.xp = (_vp * self.cnt)(*[x.data_ptr() for x in xs])
-        self.yp = (_vp * self.cnt)(*[y.data_ptr() for y in ys])
+        arr = (WqWeight * self.cnt)(*[w.desc() for w in ws])
+        xp = (_vp * self.cnt)(*[x.data_ptr() for x in xs])
+        yp = (_vp * self.cnt)(*[y.data_ptr() for y in ys])
+        self._plan = _vp(None)
+        _check(_lib.wq_gemv_plan_create(arr, xp, yp, self.cnt, self.batch, ctypes.byref(self._plan)))
 
     def __call__(self, stream=None) -> None:
         s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
-        _check(_lib.wq_gemv_w4a16_grouped(self.arr, self.xp, self.yp, self.cnt, self.batch, s))
+        _check(_lib.wq_gemv_plan_launch(self._plan, s))
+
+    def close(self) -> None:
+        if getattr(self, "_plan", None) and self._plan.value:
+            _lib.wq_gemv_plan_destroy(self._plan)
+            self._plan = _vp(None)
+
+    def __del__(self):
+        self.close()
 
 
 def gemm_workspace_bytes(w: PackedWeight, m: int) -> int:

@@ -220,15 +220,17 @@ wq_status wq_dequant(const wq_weight* w, uint16_t* out, wq_stream stream) {
     return launch_dequant(*w, out, (cudaStream_t)stream);
 }
 
-wq_status wq_gemv_w4a16_grouped(const wq_weight* ws, const uint16_t* const* xs,
-                                uint16_t* const* ys, int32_t count, int32_t batch,
-                                wq_stream stream) {
-    g_last_error[0] = 0;
+}  // extern "C"
+
+namespace {
+
+// The checks of a grouped GEMV call; fills probs[0..count).
+wq_status check_grouped(const wq_weight* ws, const uint16_t* const* xs, uint16_t* const* ys,
+                        int32_t count, int32_t batch, GemvProblem* probs) {
     if (!ws || !xs || !ys) return fail(WQ_EINVAL, "ws, xs and ys must be non-NULL host arrays");
     if (count < 1 || count > WQ_GEMV_MAX_GROUPED)
         return fail(WQ_EINVAL, "count=%d outside 1..%d", count, WQ_GEMV_MAX_GROUPED);
     if (batch < 1 || batch > 16) return fail(WQ_EINVAL, "batch=%d outside 1..16", batch);
-    GemvProblem probs[WQ_GEMV_MAX_GROUPED];
     for (int i = 0; i < count; ++i) {
         wq_status st = check_weight(&ws[i]);
         if (st) return st;
@@ -240,8 +242,47 @@ wq_status wq_gemv_w4a16_grouped(const wq_weight* ws, const uint16_t* const* xs,
         if ((st = check_ptr(ys[i], "y", false))) return st;
         probs[i] = GemvProblem{ws[i].packed, ws[i].aux, xs[i], ys[i], (int32_t)ws[i].n, (int32_t)ws[i].k};
     }
+    return WQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+wq_status wq_gemv_plan_create(const wq_weight* ws, const uint16_t* const* xs, uint16_t* const* ys,
+                              int32_t count, int32_t batch, wq_gemv_plan* plan) {
+    g_last_error[0] = 0;
+    if (!plan) return fail(WQ_EINVAL, "plan must be a non-NULL host pointer");
+    *plan = nullptr;
+    GemvProblem probs[WQ_GEMV_MAX_GROUPED];
+    wq_status st = check_grouped(ws, xs, ys, count, batch, probs);
+    if (st) return st;
+    void* p = nullptr;
+    if ((st = gemv_plan_build(ws[0].fmt, ws[0].group, probs, count, batch, &p))) return st;
+    *plan = reinterpret_cast<wq_gemv_plan>(p);
+    return WQ_OK;
+}
+
+wq_status wq_gemv_plan_launch(wq_gemv_plan plan, wq_stream stream) {
+    g_last_error[0] = 0;
+    if (!plan) return fail(WQ_EINVAL, "plan is NULL");
     wq_status st = check_injected();
     if (st) return st;
+    return gemv_plan_launch(plan, (cudaStream_t)stream);
+}
+
+void wq_gemv_plan_destroy(wq_gemv_plan plan) {
+    if (plan) gemv_plan_free(plan);
+}
+
+wq_status wq_gemv_w4a16_grouped(const wq_weight* ws, const uint16_t* const* xs,
+                                uint16_t* const* ys, int32_t count, int32_t batch,
+                                wq_stream stream) {
+    g_last_error[0] = 0;
+    GemvProblem probs[WQ_GEMV_MAX_GROUPED];
+    wq_status st = check_grouped(ws, xs, ys, count, batch, probs);
+    if (st) return st;
+    if ((st = check_injected())) return st;
     return launch_gemv(ws[0].fmt, ws[0].group, probs, count, batch, (cudaStream_t)stream);
 }
 

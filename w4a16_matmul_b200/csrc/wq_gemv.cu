@@ -34,6 +34,8 @@
 //   * When a launch has too few rows to fill the GPU, WK warps of a CTA split K and meet
 //     in shared memory at the end; otherwise every warp covers the full K and no
 //     reduction exists. One launch, no workspace, either way.
+#include <new>
+
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -49,8 +51,11 @@ constexpr int kMaxProblems = WQ_GEMV_MAX_GROUPED;
 #ifndef WQ_GEMV_MIN_CTAS_NB2
 #define WQ_GEMV_MIN_CTAS_NB2 4
 #endif
+#ifndef WQ_GEMV_L2HINT
+#define WQ_GEMV_L2HINT 2             // weight loads: 0 plain, 1 L2::128B, 2 L2::256B sector prefetch
+#endif
 #ifndef WQ_GEMV_R2_MIN_BATCH
-#define WQ_GEMV_R2_MIN_BATCH 4       // 32-row warps above this batch (large launches)
+#define WQ_GEMV_R2_MIN_BATCH 8       // 32-row warps above this batch (large launches)
 #endif
 
 template <int MAXP>
@@ -134,6 +139,21 @@ struct Step {
     uint32_t aux[R][2][KIND == kLut16 ? 8 : 2];   // dyadic: bf16 scales; LUT16: table words
 };
 
+// A 128-bit weight load that does not allocate in L1.
+__device__ __forceinline__ uint4 ldg_w(const void* p) {
+    uint4 v;
+#if WQ_GEMV_L2HINT == 2
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+#elif WQ_GEMV_L2HINT == 1
+    asm volatile("ld.global.nc.L1::no_allocate.L2::128B.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+#else
+    v = ldg_nc_v4(p);
+#endif
+    return v;
+}
+
 template <int KIND, int R, bool FULL>
 __device__ __forceinline__ void load_step(Step<KIND, R>& st, const GemvProblem& pb, int row0, int g,
                                           int kk, int N, int K) {
@@ -147,8 +167,8 @@ __device__ __forceinline__ void load_step(Step<KIND, R>& st, const GemvProblem& 
             const bool rl = FULL || row < N;
             const uint8_t* wp = pb.packed + (size_t)row * row_bytes + kk / 2;
             const uint4 fill = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-            const uint4 a = (rl && h0) ? ldg_nc_v4(wp) : fill;
-            const uint4 b = (rl && h1) ? ldg_nc_v4(wp + 16) : fill;
+            const uint4 a = (rl && h0) ? ldg_w(wp) : fill;
+            const uint4 b = (rl && h1) ? ldg_w(wp + 16) : fill;
             st.w[r][h][0] = a.x; st.w[r][h][1] = a.y; st.w[r][h][2] = a.z; st.w[r][h][3] = a.w;
             st.w[r][h][4] = b.x; st.w[r][h][5] = b.y; st.w[r][h][6] = b.z; st.w[r][h][7] = b.w;
             if (KIND == kLut16) {
@@ -490,35 +510,43 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
 // batch rows); K is walked in chunks when batch * K does not fit.
 constexpr int kXStageBudget = 32 * 1024;
 
+// A launch chosen and parameterised once: the kernel variant, its grid and shared memory.
+template <int MAXP>
+struct Prepared {
+    void (*kern)(GemvParams<MAXP>);
+    GemvParams<MAXP> prm;
+    int tiles;
+    size_t smem;
+};
+
 template <int KIND, int NB, int R, int WK, int MAXP>
-wq_status run(GemvParams<MAXP>& prm, const GemvProblem* probs, int tiles, cudaStream_t s) {
+wq_status prepare_variant(Prepared<MAXP>& pr, const GemvProblem* probs, int tiles) {
     constexpr int unit = depth(KIND, NB, R) * WK;   // chunks are whole multiples of this
+    GemvParams<MAXP>& prm = pr.prm;
     int max_steps = 1;
     for (int i = 0; i < prm.count; ++i) max_steps = max(max_steps, (probs[i].k + 255) / 256);
     int cs = max(1, (kXStageBudget / prm.batch - 64) / 512);
     cs = max(unit, cs - cs % unit);
     prm.chunk_steps = min(cs, max_steps);
-    const size_t smem = (size_t)prm.batch * (512 * prm.chunk_steps + 64);
-    if (smem > 48 * 1024) {
+    pr.smem = (size_t)prm.batch * (512 * prm.chunk_steps + 64);
+    pr.kern = gemv_kernel<KIND, NB, R, WK, MAXP>;
+    pr.tiles = tiles;
+    if (pr.smem > 48 * 1024) {
         // small launches with many batch rows: a chunk of D * WK steps may pass 48 KB
-        static bool raised = false;
-        if (!raised) {
-            if (cudaFuncSetAttribute(gemv_kernel<KIND, NB, R, WK, MAXP>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) != cudaSuccess)
-                return check_launch("gemv shared memory");
-            raised = true;
-        }
+        if (cudaFuncSetAttribute(pr.kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) !=
+            cudaSuccess)
+            return check_launch("gemv shared memory");
     }
-    gemv_kernel<KIND, NB, R, WK, MAXP><<<tiles, 128, smem, s>>>(prm);
-    return check_launch("gemv");
+    return WQ_OK;
 }
 
 template <int KIND, int NB, int MAXP>
-wq_status pick_split(GemvParams<MAXP>& prm, const GemvProblem* probs, int count, int64_t rows16,
-                     int batch, cudaStream_t s) {
-    // Full-K warps (no reduction) when the launch has at least ~6 warps of 32 rows per SM;
-    // otherwise 16-row warps, and K split over 2 or 4 warps of a CTA for small launches.
+wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, int64_t rows16,
+                     int batch) {
+    // Full-K warps (no reduction) when the launch has at least ~8 warps of rows per SM;
+    // otherwise K split over 2 or 4 warps of a CTA for small launches.
     const int64_t sms = sm_count();
+    GemvParams<MAXP>& prm = pr.prm;
     auto tiles_for = [&](int rows_per_cta) {
         int tiles = 0;
         for (int i = 0; i < count; ++i) {
@@ -529,33 +557,58 @@ wq_status pick_split(GemvParams<MAXP>& prm, const GemvProblem* probs, int count,
         return tiles;
     };
     // 32-row warps pay off once the activation fragment is shared by more batch rows
-    // (measured: 16-row warps win at batch <= 4, 32-row warps at batch 5..16)
+    // (measured on the decode sweep: 16-row warps win up to batch 8, 32-row warps at 9..16)
     constexpr int BIGR = (KIND == kLut16) ? 1 : 2;
     if (BIGR == 2 && batch > WQ_GEMV_R2_MIN_BATCH && rows16 >= 12 * sms * 2)
-        return run<KIND, NB, BIGR, 1, MAXP>(prm, probs, tiles_for(64 * BIGR), s);
-    if (rows16 >= 8 * sms) return run<KIND, NB, 1, 1, MAXP>(prm, probs, tiles_for(64), s);
-    if (rows16 >= 2 * sms) return run<KIND, NB, 1, 2, MAXP>(prm, probs, tiles_for(32), s);
-    return run<KIND, NB, 1, 4, MAXP>(prm, probs, tiles_for(16), s);
+        return prepare_variant<KIND, NB, BIGR, 1, MAXP>(pr, probs, tiles_for(64 * BIGR));
+    if (rows16 >= 8 * sms) return prepare_variant<KIND, NB, 1, 1, MAXP>(pr, probs, tiles_for(64));
+    if (rows16 >= 2 * sms) return prepare_variant<KIND, NB, 1, 2, MAXP>(pr, probs, tiles_for(32));
+    return prepare_variant<KIND, NB, 1, 4, MAXP>(pr, probs, tiles_for(16));
 }
 
 template <int MAXP>
-wq_status launch_impl(int fmt, int group, const GemvProblem* probs, int count, int batch,
-                      cudaStream_t s) {
-    GemvParams<MAXP> prm;
+wq_status prepare(int fmt, int group, const GemvProblem* probs, int count, int batch,
+                  Prepared<MAXP>& pr) {
+    if (count < 1 || count > MAXP) return fail(WQ_EINVAL, "count=%d outside 1..%d", count, MAXP);
+    GemvParams<MAXP>& prm = pr.prm;
     prm.count = count;
     prm.batch = batch;
+    // Longest rows first (stable by K, descending): the grid is dispatched roughly in order,
+    // so the last wave holds the shortest CTAs and the tail of the launch stays short.
+    GemvProblem sorted[MAXP];
+    for (int i = 0; i < count; ++i) {
+        int j = i;
+        while (j > 0 && sorted[j - 1].k < probs[i].k) { sorted[j] = sorted[j - 1]; --j; }
+        sorted[j] = probs[i];
+    }
+    probs = sorted;
     int64_t rows16 = 0;
     for (int i = 0; i < count; ++i) { prm.prob[i] = probs[i]; rows16 += (probs[i].n + 15) / 16; }
     const bool two = batch > 8;
     const int kind = (fmt == WQ_FMT_LUT16) ? kLut16 : (group == 64 ? kDyadic64 : kDyadic32);
     if (kind == kLut16)
-        return two ? pick_split<kLut16, 2, MAXP>(prm, probs, count, rows16, batch, s)
-                   : pick_split<kLut16, 1, MAXP>(prm, probs, count, rows16, batch, s);
+        return two ? pick_split<kLut16, 2, MAXP>(pr, probs, count, rows16, batch)
+                   : pick_split<kLut16, 1, MAXP>(pr, probs, count, rows16, batch);
     if (kind == kDyadic64)
-        return two ? pick_split<kDyadic64, 2, MAXP>(prm, probs, count, rows16, batch, s)
-                   : pick_split<kDyadic64, 1, MAXP>(prm, probs, count, rows16, batch, s);
-    return two ? pick_split<kDyadic32, 2, MAXP>(prm, probs, count, rows16, batch, s)
-               : pick_split<kDyadic32, 1, MAXP>(prm, probs, count, rows16, batch, s);
+        return two ? pick_split<kDyadic64, 2, MAXP>(pr, probs, count, rows16, batch)
+                   : pick_split<kDyadic64, 1, MAXP>(pr, probs, count, rows16, batch);
+    return two ? pick_split<kDyadic32, 2, MAXP>(pr, probs, count, rows16, batch)
+               : pick_split<kDyadic32, 1, MAXP>(pr, probs, count, rows16, batch);
+}
+
+template <int MAXP>
+wq_status launch_prepared(const Prepared<MAXP>& pr, cudaStream_t s) {
+    pr.kern<<<pr.tiles, 128, pr.smem, s>>>(pr.prm);
+    return check_launch("gemv");
+}
+
+template <int MAXP>
+wq_status launch_impl(int fmt, int group, const GemvProblem* probs, int count, int batch,
+                      cudaStream_t s) {
+    Prepared<MAXP> pr;
+    wq_status st = prepare<MAXP>(fmt, group, probs, count, batch, pr);
+    if (st != WQ_OK) return st;
+    return launch_prepared(pr, s);
 }
 
 }  // namespace
@@ -565,5 +618,21 @@ wq_status launch_gemv(int fmt, int group, const GemvProblem* probs, int count, i
     if (count == 1) return launch_impl<1>(fmt, group, probs, count, batch, s);
     return launch_impl<kMaxProblems>(fmt, group, probs, count, batch, s);
 }
+
+wq_status gemv_plan_build(int fmt, int group, const GemvProblem* probs, int count, int batch,
+                          void** plan) {
+    auto* pr = new (std::nothrow) Prepared<kMaxProblems>;
+    if (!pr) return fail(WQ_EINVAL, "out of host memory for the GEMV plan");
+    wq_status st = prepare<kMaxProblems>(fmt, group, probs, count, batch, *pr);
+    if (st != WQ_OK) { delete pr; return st; }
+    *plan = pr;
+    return WQ_OK;
+}
+
+wq_status gemv_plan_launch(const void* plan, cudaStream_t s) {
+    return launch_prepared(*static_cast<const Prepared<kMaxProblems>*>(plan), s);
+}
+
+void gemv_plan_free(void* plan) { delete static_cast<Prepared<kMaxProblems>*>(plan); }
 
 }  // namespace wq

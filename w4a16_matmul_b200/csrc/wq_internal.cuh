@@ -43,6 +43,13 @@ struct GemvProblem {
 wq_status launch_gemv(int fmt, int group, const GemvProblem* probs, int count, int batch,
                       cudaStream_t s);
 
+// A prepared grouped GEMV (kernel variant, grid and parameters chosen once): built on the
+// host heap, launched any number of times, freed by gemv_plan_free.
+wq_status gemv_plan_build(int fmt, int group, const GemvProblem* probs, int count, int batch,
+                          void** plan);
+wq_status gemv_plan_launch(const void* plan, cudaStream_t s);
+void gemv_plan_free(void* plan);
+
 wq_status launch_lloyd_g32(const uint16_t* w, int64_t n, int64_t k, int rounds, uint8_t* codes,
                            uint8_t* packed, float* levels, uint8_t* params, float* trace,
                            cudaStream_t s);
