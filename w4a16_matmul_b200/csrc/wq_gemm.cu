@@ -9,13 +9,18 @@
 //   warp 0     TMA producer: per 64-column stage, the activation tile [BN x 64] bf16
 //              (128-byte swizzle) and the packed weight tile [128 x 32 bytes];
 //   warp 1     allocates tensor memory, and one lane issues tcgen05.mma (kind::f16,
-//              bf16 x bf16 -> fp32 in TMEM, M=128, N=BN, K=16 x 4 per stage) and commits
-//              each stage back to the producers;
-//   warps 2-5  reconstruct the weight tile: thread i owns weight row i, turns its 64
-//              codes into bf16 exactly as wq_dequant does, and writes them into the
-//              K-major 128-byte-swizzled layout the MMA descriptor reads; afterwards they
-//              drain the accumulator with tcgen05.ld and store bf16 (or fp32 partial sums
-//              when K is split across CTAs, reduced by a second small kernel).
+//              bf16 x bf16 -> fp32 in TMEM, M=128, N=BN, K=16 x 4 per stage) with the
+//              weight operand A read from tensor memory and the activations B from shared
+//              memory, and commits each stage back to the producer;
+//   warps 2-5  reconstruct the weight tile: the thread of tensor-memory lane i owns weight
+//              row i, turns its 64 codes into bf16 exactly as wq_dequant does and stores
+//              them into that lane's 32-column slot of the stage (tcgen05.st); afterwards
+//              they drain the accumulator with tcgen05.ld and store bf16 (or fp32 partial
+//              sums when K is split across CTAs, reduced by a second small kernel).
+// Keeping the reconstructed operand in tensor memory leaves shared memory to the TMA tiles
+// alone: no bf16 tile is written to and read back from shared memory, whose bandwidth the
+// MMA's activation reads and the TMA writes already share, and the freed space holds six
+// pipeline stages.
 // Every wait on an mbarrier is bounded; a wait that expires records an error word on the
 // device (see wq_device_error) and the CTA skips the rest of its work, still releasing its
 // tensor memory.
@@ -34,8 +39,6 @@ namespace {
 
 constexpr int BM = 128;            // weight rows per CTA (MMA M)
 constexpr int BK = 64;             // columns per stage: one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
-constexpr int kThreads = 192;
 constexpr uint64_t kWaitNs = 2000000000ull;   // a wait longer than 2 s is declared dead
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -58,18 +61,26 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+#ifndef WQ_GEMM_SUSPEND_NS
+#define WQ_GEMM_SUSPEND_NS 20000
+#endif
+#ifndef WQ_GEMM_BIG_SLOTS
+#define WQ_GEMM_BIG_SLOTS 0
+#endif
 // Bounded wait for the completion of phase `parity`: gives up after about two seconds of
-// wall time (checked every 64 polls) and returns false.
+// wall time and returns false. Each try_wait may suspend the thread for up to
+// WQ_GEMM_SUSPEND_NS nanoseconds (it wakes as soon as the phase completes), so a waiting
+// warp does not spin on the issue slots the reconstruction warps need.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
     const uint32_t a = smem_u32(b);
     uint64_t deadline = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t done;
         asm volatile(
-            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-            : "=r"(done) : "r"(a), "r"(parity) : "memory");
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+            : "=r"(done) : "r"(a), "r"(parity), "r"((uint32_t)WQ_GEMM_SUSPEND_NS) : "memory");
         if (done) return true;
-        if ((i & 63) == 0) {
+        if ((i & 7) == 0) {
             const uint64_t now = global_ns();
             if (deadline == 0) deadline = now + kWaitNs;
             else if (now > deadline) return false;
@@ -93,13 +104,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
-        ::"r"(tmem_d), "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
-}
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(smem_u32(bar)) : "memory");
@@ -139,15 +143,83 @@ __device__ __forceinline__ uint4 dyadic_row8_f32(uint32_t w, float step) {
                       pack_bf16x2(v[6], v[7]));
 }
 
+// Pipeline depths per activation-tile width. Shared-memory stages (the [BN x 64] bf16
+// activation tile and the [128 x 32 B] packed tile each) hold the bytes in flight: as many
+// as 216 KB hold, up to 16. Tensor-memory slots (32 columns each, the reconstructed
+// weights of one stage) only need to cover reconstruction-to-MMA latency; for BN <= 64 the
+// allocation stays at 256 columns so that two CTAs can share an SM.
 template <int BN>
 struct Smem {
-    static constexpr int A_BYTES = BM * BK * 2;          // 16 KB bf16 weight tile
-    static constexpr int B_BYTES = BN * BK * 2;          // activation tile
+    static constexpr int B_BYTES = BN * BK * 2;          // activation tile (128-byte swizzle)
     static constexpr int P_BYTES = BM * BK / 2;          // 4 KB packed weight tile
-    static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
-    static constexpr int BARS = 3 * STAGES + 1;
+    static constexpr int STAGE = B_BYTES + P_BYTES;      // a multiple of 1024
+    static constexpr int STAGES = (216 * 1024 / STAGE) < 16 ? (216 * 1024 / STAGE) : 16;
+    static constexpr int BARS = 2 * STAGES + 2 * 8 + 1;
     static constexpr int TOTAL = STAGES * STAGE + BARS * 8 + 16 + 1024;   // + alignment slack
+    // tensor memory: the fp32 accumulator [128 lanes x BN columns], then SLOTS 32-column
+    // slots for reconstructed bf16 weight tiles (64 values of a row per lane, two per 32-bit
+    // column, lower k in the low half)
+    static constexpr uint32_t ACC_COLS = BN < 32 ? 32 : BN;
+    // BN >= 128: one slot per stage (the rings coincide, and the producer's wait for a free
+    // stage already orders slot reuse); BN <= 64: six slots under a 16-stage ring
+    static constexpr int SLOTS = BN <= 64 ? (int)((256 - ACC_COLS) / 32 < 6 ? (256 - ACC_COLS) / 32 : 6)
+                                          : (WQ_GEMM_BIG_SLOTS ? 8 : (STAGES < 8 ? STAGES : 8));
+    static constexpr bool COUPLED = SLOTS == STAGES;
+    static constexpr uint32_t USED_COLS = ACC_COLS + 32 * SLOTS;
+    static constexpr uint32_t TMEM_COLS = USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
+                                        : USED_COLS <= 256 ? 256 : 512;
 };
+
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
+        ::"r"(tmem_d), "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate));
+}
+
+// Stores 32 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+          "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+          "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+          "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+          "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+#ifndef WQ_GEMM_RW
+#define WQ_GEMM_RW 4
+#endif
+// Reconstruction warps per tensor-memory lane group: RW warps share each 32-lane group, each
+// filling 8 / RW of the row's eight packed words per stage (more warps hide more latency).
+constexpr int RW = WQ_GEMM_RW;
+constexpr int kThreads = 64 + 128 * RW;
+
+// Stores 32 / RW consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st_part(uint32_t taddr, const uint32_t* v) {
+    if constexpr (RW == 1) {
+        tmem_st32(taddr, *reinterpret_cast<const uint32_t(*)[32]>(v));
+    } else if constexpr (RW == 2) {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+            "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+            ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+              "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+              "r"(v[15])
+            : "memory");
+    } else {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+            ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+              "r"(v[7])
+            : "memory");
+    }
+}
 
 template <int BN, int G, bool PARTIAL>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -155,12 +227,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             const uint16_t* __restrict__ scale, void* __restrict__ out, int M, int N, int K,
             int kt_per_split) {
     using S = Smem<BN>;
+    constexpr int STAGES = S::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t* full_tma = (uint64_t*)(smem + STAGES * S::STAGE);
-    uint64_t* full_w = full_tma + STAGES;
-    uint64_t* empty = full_w + STAGES;
-    uint64_t* acc_full = empty + STAGES;
+    constexpr int SLOTS = S::SLOTS;
+    uint64_t* full_tma = (uint64_t*)(smem + STAGES * S::STAGE);   // stage landed (TMA bytes)
+    uint64_t* empty = full_tma + STAGES;                            // stage consumed (MMA done)
+    uint64_t* full_w = empty + STAGES;                              // slot reconstructed
+    uint64_t* slot_free = full_w + 8;                               // slot read by its MMAs
+    uint64_t* acc_full = slot_free + 8;
     uint32_t* s_tmem = (uint32_t*)(acc_full + 1);
     int* s_abort = (int*)(s_tmem + 1);
 
@@ -170,13 +245,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     const int kt0 = blockIdx.z * kt_per_split;
     const int kt1 = min(KT, kt0 + kt_per_split);
     const int nk = kt1 - kt0;
-    constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_tma[s], 1);
-            mbar_init(&full_w[s], 4);
             mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < SLOTS; ++a) {
+            mbar_init(&full_w[a], 4 * RW);
+            mbar_init(&slot_free[a], 1);
         }
         mbar_init(acc_full, 1);
         *s_abort = 0;
@@ -185,7 +262,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(s_tmem)), "r"(kTmemCols));
+                     ::"r"(smem_u32(s_tmem)), "r"(S::TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
         asm volatile("tcgen05.fence::before_thread_sync;");
     }
@@ -193,9 +270,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     asm volatile("tcgen05.fence::after_thread_sync;");
     const uint32_t tmem = *s_tmem;
 
-    auto stage_a = [&](int s) { return smem + s * S::STAGE; };
-    auto stage_b = [&](int s) { return smem + s * S::STAGE + S::A_BYTES; };
-    auto stage_p = [&](int s) { return smem + s * S::STAGE + S::A_BYTES + S::B_BYTES; };
+    auto stage_b = [&](int s) { return smem + s * S::STAGE; };
+    auto stage_p = [&](int s) { return smem + s * S::STAGE + S::B_BYTES; };
     auto dead = [&](int code) {
         *(volatile int*)s_abort = 1;
         atomicCAS(&g_device_error, 0, code);
@@ -216,35 +292,40 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+        // ---------------- MMA issuer: A (weights) from tensor memory, B from shared ------
         if (lane == 0) {
             constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
                                        ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-            bool ok = true;
             for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (i / STAGES) & 1;
-                if (*(volatile int*)s_abort) { ok = false; break; }
-                if (!mbar_wait(&full_w[s], ph)) { dead(2); ok = false; break; }
+                const int s = i % STAGES, a = i % SLOTS;
+                if (*(volatile int*)s_abort) break;
+                // the slot is reconstructed, which also means the stage's tiles have landed
+                if (!mbar_wait(&full_w[a], (i / SLOTS) & 1)) { dead(2); break; }
                 asm volatile("tcgen05.fence::after_thread_sync;");
-                const uint64_t da = sw128_desc(smem_u32(stage_a(s)));
                 const uint64_t db = sw128_desc(smem_u32(stage_b(s)));
+                const uint32_t ta = tmem + S::ACC_COLS + 32u * (uint32_t)a;
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)   // 32 bytes of K per MMA: +2 in descriptor units
-                    umma_f16(tmem, da + 2 * k, db + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
-                umma_commit(&empty[s]);
+                for (int k = 0; k < BK / 16; ++k)   // 16 values of K: 8 A columns, +2 in B descriptor units
+                    umma_f16_ts(tmem, ta + 8u * (uint32_t)k, db + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
+                umma_commit(&empty[s]);           // fire once these MMAs have read the stage ...
+                if constexpr (!S::COUPLED) umma_commit(&slot_free[a]);   // ... and the slot
             }
             // commit (not a plain arrive) even after an abort: it fires only once every MMA
             // issued so far has finished, so tensor memory is never freed under a running MMA
-            (void)ok;
             umma_commit(acc_full);
         }
     } else {
-        // ---------------- reconstruction, then epilogue ----------------
-        const int i = threadIdx.x - 64;                  // weight row within the tile
+        // ---------------- reconstruction into tensor memory, then epilogue ----------------
+        // a warp may touch only the tensor-memory lanes 32 * (warp % 4) .. + 31: thread
+        // (warp, lane) owns weight row 32 * (warp % 4) + lane of the tile, and of that row's
+        // eight packed words per stage the words [part * WPT, part * WPT + WPT)
+        constexpr int WPT = 8 / RW;
+        const int q = warp & 3, part = (warp - 2) >> 2;
+        const int i = 32 * q + lane;
         const int n = n0 + i;
         const bool row_ok = n < N;
         const uint16_t* srow = scale + (size_t)(row_ok ? n : 0) * (K / G);
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         // the per-group scales of this row, loaded kPre stages ahead (a ring of registers)
         constexpr int kPre = 4;
         uint32_t ring0[kPre], ring1[kPre];
@@ -262,7 +343,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             for (int u = 0; u < kPre; ++u) {
                 const int it = base + u;
                 if (it >= nk) break;
-                const int s = it % STAGES;
+                const int s = it % STAGES, a = it % SLOTS;
                 const uint32_t ph = (it / STAGES) & 1;
                 // every exit below is taken by the whole warp (it ends in __syncwarp)
                 if (__any_sync(0xFFFFFFFFu, *(volatile int*)s_abort != 0)) { live = false; break; }
@@ -271,49 +352,71 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     ring0[u] = ldg_u16(srow + (kt0 + it + kPre) * BK / G);
                     ring1[u] = (G == 32) ? ldg_u16(srow + (kt0 + it + kPre) * BK / G + 1) : ring0[u];
                 }
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full_tma[s], ph))) { dead(3); live = false; break; }
-                const uint4* pk = (const uint4*)(stage_p(s) + i * 32);
-                const uint4 q0 = pk[0], q1 = pk[1];
-                const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-                uint8_t* arow = stage_a(s) + i * 128;
+                // the packed tile has landed, and the MMAs that last read this tensor-memory
+                // slot (iteration it - SLOTS) have completed
+                // (with coupled rings the first implies the second: the TMA for this
+                // iteration was issued only after the stage's previous MMAs completed)
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full_tma[s], ph) &&
+                                             (S::COUPLED || it < SLOTS ||
+                                              mbar_wait(&slot_free[a], ((it / SLOTS) & 1) ^ 1)))) {
+                    dead(3); live = false; break;
+                }
+                uint32_t wv[WPT];
+                {
+                    const uint32_t* pk = (const uint32_t*)(stage_p(s) + i * 32 + part * WPT * 4);
+                    if constexpr (WPT >= 4) {
+#pragma unroll
+                        for (int c = 0; c < WPT; c += 4) {
+                            const uint4 t4 = *(const uint4*)(pk + c);
+                            wv[c] = t4.x; wv[c + 1] = t4.y; wv[c + 2] = t4.z; wv[c + 3] = t4.w;
+                        }
+                    } else {
+                        const uint2 t2 = *(const uint2*)pk;
+                        wv[0] = t2.x; wv[1] = t2.y;
+                    }
+                }
                 const bool huge = ((sc0 & 0x7FFFu) >= 0x7D80u) || ((sc1 & 0x7FFFu) >= 0x7D80u);
                 const uint32_t s20 = prmt(sc0, 0, 0x1010u), s21 = prmt(sc1, 0, 0x1010u);
                 const uint32_t cs0 = bf16x2_fma(s20, 0x41804180u, 0x80008000u), cn0 = s20 ^ 0x80008000u;
                 const uint32_t cs1 = bf16x2_fma(s21, 0x41804180u, 0x80008000u), cn1 = s21 ^ 0x80008000u;
+                uint32_t v[4 * WPT];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const bool second = (G == 32) && c >= 4;
-                    const uint4 v = huge ? dyadic_row8_f32(wv[c], bf16_bits_to_float(second ? sc1 : sc0) * 0.125f)
+                for (int c = 0; c < WPT; ++c) {
+                    const bool second = (G == 32) && (part * WPT + c) >= 4;
+                    const uint4 r = huge ? dyadic_row8_f32(wv[c], bf16_bits_to_float(second ? sc1 : sc0) * 0.125f)
                                          : dyadic_row8(wv[c], second ? cs1 : cs0, second ? cn1 : cn0);
-                    *(uint4*)(arow + ((c ^ (i & 7)) << 4)) = v;
+                    v[4 * c] = r.x; v[4 * c + 1] = r.y; v[4 * c + 2] = r.z; v[4 * c + 3] = r.w;
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tmem_st_part(lane_base + S::ACC_COLS + 32u * (uint32_t)a + (uint32_t)(part * 4 * WPT), v);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full_w[s]);
+                if (lane == 0) mbar_arrive(&full_w[a]);
             }
         }
-        // ---- epilogue: TMEM lanes 32*(warp%4).. hold weight rows, columns = activation rows
+        // ---- epilogue: TMEM lane 32q + lane holds weight row n, columns = activation rows
         // tcgen05.ld is warp-collective: the decision to drain is taken per warp
         const bool drain = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0)) &&
                            !__any_sync(0xFFFFFFFFu, *(volatile int*)s_abort != 0);
         if (drain) {
             asm volatile("tcgen05.fence::after_thread_sync;");
-            const int q = warp & 3;
-            const int nrow = n0 + 32 * q + lane;
+            // the RW warps of a lane group split the accumulator's columns
+            constexpr int CPP = (BN / RW) < 16 ? 16 : BN / RW;
+            const int cbeg = part * CPP, cend = min(BN, cbeg + CPP);
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = cbeg; c0 < cend; c0 += 16) {
                 uint32_t v[16];
-                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+                tmem_ld16(lane_base + (uint32_t)c0, v);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                if (nrow < N) {
+                if (row_ok) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int m = m0 + c0 + j;
                         if (m < M) {
                             if (PARTIAL)
-                                ((float*)out)[((size_t)blockIdx.z * M + m) * N + nrow] = __uint_as_float(v[j]);
+                                ((float*)out)[((size_t)blockIdx.z * M + m) * N + n] = __uint_as_float(v[j]);
                             else
-                                ((uint16_t*)out)[(size_t)m * N + nrow] =
+                                ((uint16_t*)out)[(size_t)m * N + n] =
                                     (uint16_t)float_to_bf16_bits(__uint_as_float(v[j]));
                         }
                     }
@@ -327,7 +430,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     __syncthreads();
     if (warp == 1) {
         asm volatile("tcgen05.fence::after_thread_sync;");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS));
     }
 }
 
@@ -386,13 +489,18 @@ wq_status launch_bn(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp,
                     void* out, int M, int N, int K, cudaStream_t s) {
     const int smem = Smem<BN>::TOTAL;
     const dim3 grid(p.grid_n, p.grid_m, p.splits);
+    // the shared-memory opt-in is set once per kernel variant (a function attribute holds
+    // for the process; the flags are per variant and only ever go from false to true)
+    static bool raised[2] = {false, false};
     if (p.splits > 1) {
         auto k = gemm_kernel<BN, G, true>;
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (!raised[1] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
+            raised[1] = true;
         k<<<grid, kThreads, smem, s>>>(tx, tp, scale, out, M, N, K, p.kt_per_split);
     } else {
         auto k = gemm_kernel<BN, G, false>;
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (!raised[0] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
+            raised[0] = true;
         k<<<grid, kThreads, smem, s>>>(tx, tp, scale, out, M, N, K, p.kt_per_split);
     }
     return check_launch("gemm");
