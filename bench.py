@@ -151,6 +151,18 @@ def sweep_bytes(mats, batch):
 # our arm
 # ---------------------------------------------------------------------------------------
 
+def graph_of(torch, fn):
+    """fn's launches captured once in a CUDA graph (after one eager call for any one-time
+    setup); replaying it keeps per-call host work (argument checks, allocation) out of a
+    timed region that is meant to hold the kernels."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
 def time_region(torch, stream, fn, steps, warmup, barrier):
     for _ in range(warmup):
         fn()
@@ -310,7 +322,9 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
         def q():
             for w in wts:
                 wq.quantize_dyadic(w, 64)
-        ms = max_over_ranks(time_region(torch, stream, q, steps, warm, barrier))
+
+        gq = graph_of(torch, q)
+        ms = max_over_ranks(time_region(torch, stream, gq.replay, steps, warm, barrier))
         byts = n_w * (2 + 0.5 + 2 / 64)
         out["quantize_dyadic_layer"] = {"Gweights/s": round(n_w / ms / 1e6, 2), "GB/s": round(byts / ms / 1e6, 1),
                                         "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
@@ -319,11 +333,12 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
         def dq():
             for pw in packed[:7]:
                 wq.dequant(pw)
-        ms = max_over_ranks(time_region(torch, stream, dq, steps, warm, barrier))
+        gdq = graph_of(torch, dq)
+        ms = max_over_ranks(time_region(torch, stream, gdq.replay, steps, warm, barrier))
         byts = n_w * (0.5 + 2 / 64 + 2)
         out["dequant_layer"] = {"GB/s": round(byts / ms / 1e6, 1),
                                 "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
-        del wts
+        del wts, gq, gdq
     except Exception as e:
         out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
     if args.extras in ("gemm", "all"):
@@ -350,12 +365,14 @@ def bench_gemm(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks):
                 y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
                 need = wq.gemm_workspace_bytes(pw, m)
                 ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-                ms = max_over_ranks(time_region(torch, stream, lambda: wq.gemm(pw, x, out=y, workspace=ws),
-                                                steps, warm, barrier))
+                g = graph_of(torch, lambda: wq.gemm(pw, x, out=y, workspace=ws))
+                ms = max_over_ranks(time_region(torch, stream, g.replay, steps, warm, barrier))
                 fl = 2.0 * m * n * k
                 byts = n * k * (0.5 + 2 / 64) + 2 * m * k + 2 * m * n
-                ms_mat = max_over_ranks(time_region(torch, stream, lambda: torch.matmul(x, wdeq.t()),
-                                                    steps, warm, barrier))
+                ym = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+                gm = graph_of(torch, lambda: torch.matmul(x, wdeq.t(), out=ym))
+                ms_mat = max_over_ranks(time_region(torch, stream, gm.replay, steps, warm, barrier))
+                del g, gm
                 res[f"{n}x{k}_m{m}"] = {
                     "TFLOP/s": round(fl / ms / 1e9, 1), "frac_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4),
                     "GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
@@ -404,7 +421,9 @@ def bench_producers(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks
         for b in (1, 8, 16):
             x = torch.randn((b, k), device=dev).to(torch.bfloat16)
             y = torch.empty((b, n), dtype=torch.bfloat16, device=dev)
-            ms = max_over_ranks(time_region(torch, stream, lambda: wq.gemv(pw, x, out=y), 20, 3, barrier))
+            g = graph_of(torch, lambda: wq.gemv(pw, x, out=y))
+            ms = max_over_ranks(time_region(torch, stream, g.replay, 20, 3, barrier))
+            del g
             byts = n * k * (0.5 + 0.5)
             out[f"lut16_gemv_b{b}"] = {"GB/s": round(byts / ms / 1e6, 1), "us": round(ms * 1e3, 2),
                                        "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
@@ -493,6 +512,55 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_target(args):
+    """A few launches of one kernel on one shape and nothing else, for ncu captures:
+    --profile gemm --shape N,K,M (prefill GEMM), quantize --shape N,K, dequant --shape N,K,
+    lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd). Random packed codes and
+    scales (timing does not depend on the values); inputs stay on the device."""
+    import torch
+    import __graft_entry__
+    __graft_entry__._build_module().build()
+    import w4a16_matmul_b200 as wq
+    dev = torch.device("cuda")
+    dims = [int(v) for v in args.shape.split(",")]
+    n, k = dims[0], dims[1]
+    gen = torch.Generator(device=dev).manual_seed(0)
+    packed = torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=dev, generator=gen)
+    scale = (torch.rand((n, k // 64), device=dev, generator=gen) * 0.09 + 0.01).to(torch.bfloat16)
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, packed, scale)
+    if args.profile == "gemm":
+        m = dims[2]
+        x = torch.randn((m, k), device=dev, generator=gen).to(torch.bfloat16)
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, wq.gemm_workspace_bytes(pw, m)), dtype=torch.uint8, device=dev)
+        fn = lambda: wq.gemm(pw, x, out=y, workspace=ws)
+    elif args.profile == "quantize":
+        w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+        fn = lambda: wq.quantize_dyadic(w, 64)
+    elif args.profile == "dequant":
+        out = torch.empty((n, k), dtype=torch.bfloat16, device=dev)
+        fn = lambda: wq.dequant(pw, out=out)
+    elif args.profile == "lut16":
+        b = dims[2]
+        lut = (torch.randn((n, k // 64, 16), device=dev, generator=gen) * 0.01).to(torch.float16)
+        pl = wq.PackedWeight(wq.FMT_LUT16, 64, n, k, packed, lut)
+        x = torch.randn((b, k), device=dev, generator=gen).to(torch.bfloat16)
+        y = torch.empty((b, n), dtype=torch.bfloat16, device=dev)
+        fn = lambda: wq.gemv(pl, x, out=y)
+    elif args.profile == "lloyd":
+        w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+        fn = lambda: wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)
+    else:
+        raise SystemExit(f"unknown --profile {args.profile}")
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    code = wq.device_error()
+    if code:
+        raise SystemExit(f"device error {code}")
+    print(json.dumps({"profile": args.profile, "shape": dims, "ok": True}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -506,7 +574,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--profile", default=None,
+                    help="run a few launches of one kernel for an ncu capture (see run_profile_target)")
+    ap.add_argument("--shape", default="4096,11008,4096")
     args = ap.parse_args()
+    if args.profile:
+        run_profile_target(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -171,7 +171,8 @@ wq_status wq_dequant(const wq_weight* w, uint16_t* out, wq_stream stream);
  *   x      bf16 [batch, k].
  *   batch  1..16.
  *   y      out bf16 [batch, n].
- * Within |y - y_ref| <= 2e-3 * sum_c |Wdeq[r, c]| * |x[b, c]| of the exact product y_ref.
+ * Within |y - y_ref| <= 2e-3 * sum_c |Wdeq[r, c]| * |x[b, c]| + half a bf16 ulp of y_ref of
+ * the exact product y_ref (the half ulp is the bf16 output rounding itself).
  * Needs no workspace; one kernel launch. */
 wq_status wq_gemv_w4a16(const wq_weight* w, const uint16_t* x, int32_t batch, uint16_t* y,
                         wq_stream stream);

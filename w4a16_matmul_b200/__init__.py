@@ -205,10 +205,15 @@ def unpack(packed: torch.Tensor) -> torch.Tensor:
     return out
 
 
-def dequant(w: PackedWeight) -> torch.Tensor:
-    """Dense reconstruction: bf16 [n, k] (fp16 [n, k] for LUT16)."""
+def dequant(w: PackedWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Dense reconstruction: bf16 [n, k] (fp16 [n, k] for LUT16), into `out` if given."""
     dt = torch.float16 if w.fmt == FMT_LUT16 else torch.bfloat16
-    out = torch.empty((w.n, w.k), dtype=dt, device=w.packed.device)
+    if out is None:
+        out = torch.empty((w.n, w.k), dtype=dt, device=w.packed.device)
+    else:
+        _cuda(out, dt, "out")
+        if tuple(out.shape) != (w.n, w.k):
+            raise ValueError(f"out must be [{w.n}, {w.k}]")
     d = w.desc()
     _check(_lib.wq_dequant(ctypes.byref(d), _ptr(out), _stream(w.packed)))
     return out

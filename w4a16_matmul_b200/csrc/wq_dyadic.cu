@@ -33,67 +33,86 @@ int stream_grid(int64_t items, int per_sm_blocks = 8) {
 // comparison against the midpoint below (a bf16 times an odd integer <= 17 over 16, exact
 // in fp32).
 // ---------------------------------------------------------------------------------------
+// One warp-contiguous block of 32 chunks (8 weights each) per unrolled step u: each thread
+// issues its U 128-bit loads before it computes, so U loads per thread are in flight.
+template <int G>
+__device__ __forceinline__ void quantize_chunk(uint4 v, bool live, int64_t c, int64_t k,
+                                               int64_t chunks_per_row, uint16_t* __restrict__ scale,
+                                               uint2* __restrict__ codes, uint32_t* __restrict__ packed) {
+    constexpr int LANES = G / 8;                 // threads per group (8 or 4)
+    uint32_t h[8] = {v.x & 0xFFFF, v.x >> 16, v.y & 0xFFFF, v.y >> 16,
+                     v.z & 0xFFFF, v.z >> 16, v.w & 0xFFFF, v.w >> 16};
+    float f[8];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        f[i] = bf16_bits_to_float(h[i]);
+        amax = fmaxf(amax, fabsf(f[i]));
+    }
+#pragma unroll
+    for (int off = 1; off < LANES; off <<= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+
+    uint32_t idx[8];
+    if (amax == 0.f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) idx[i] = 0;            // every code ties
+    } else {
+        // keep 16/s and 17*s/16 finite for tiny and huge scales: rescale w and s by a
+        // power of two (exact; a weight that underflows is far below the smallest step)
+        const float ps = amax < 0x1p-96f ? 0x1p32f : (amax > 0x1p96f ? 0x1p-32f : 1.0f);
+        const float s = amax * ps;
+        const float c16 = 16.0f * __frcp_rn(s);
+        const float s16 = s * 0.0625f;
+        const float two_s16 = 2.0f * s16, m17 = -17.0f * s16;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float ws = f[i] * ps;
+            int cnt = (__float2int_ru(ws * c16) + 16) >> 1;
+            cnt = min(max(cnt, 0), 15);
+            // exact midpoint below code cnt: (2 cnt - 17) * s/16
+            const float mlo = fmaf((float)cnt, two_s16, m17);
+            if (cnt > 0 && !(ws > mlo)) cnt -= 1;
+            idx[i] = (uint32_t)cnt;
+        }
+    }
+    if (live) {
+        const uint32_t p = idx[0] | idx[1] << 4 | idx[2] << 8 | idx[3] << 12 |
+                           idx[4] << 16 | idx[5] << 20 | idx[6] << 24 | idx[7] << 28;
+        if (packed) packed[c] = p;
+        if (codes)
+            codes[c] = make_uint2(idx[0] | idx[1] << 8 | idx[2] << 16 | idx[3] << 24,
+                                  idx[4] | idx[5] << 8 | idx[6] << 16 | idx[7] << 24);
+        if ((threadIdx.x & (LANES - 1)) == 0) {
+            const int64_t row = c / chunks_per_row;
+            const int64_t col = (c - row * chunks_per_row) * 8;
+            scale[row * (k / G) + col / G] = (uint16_t)float_to_bf16_bits(amax);
+        }
+    }
+}
+
 template <int G>
 __global__ void __launch_bounds__(kThreads)
 quantize_dyadic_kernel(const uint4* __restrict__ w, int64_t n_chunks, int64_t k,
                        uint16_t* __restrict__ scale, uint2* __restrict__ codes,
                        uint32_t* __restrict__ packed) {
-    constexpr int LANES = G / 8;                 // threads per group (8 or 4)
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    constexpr int U = 4;
     const int64_t chunks_per_row = k / 8;
-    for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); c0 < n_chunks;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x * U;
+    const int lane = threadIdx.x & 31;
+    // a warp covers U consecutive blocks of 32 chunks; groups never straddle n_chunks
+    for (int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31)) * U; c0 < n_chunks;
          c0 += stride) {
-        const int64_t c = c0 + (threadIdx.x & 31);
-        const bool live = c < n_chunks;          // groups never straddle n_chunks
-        uint4 v = live ? ldg_nc_v4(w + c) : make_uint4(0, 0, 0, 0);
-        uint32_t h[8] = {v.x & 0xFFFF, v.x >> 16, v.y & 0xFFFF, v.y >> 16,
-                         v.z & 0xFFFF, v.z >> 16, v.w & 0xFFFF, v.w >> 16};
-        float f[8];
-        float amax = 0.f;
+        uint4 v[U];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            f[i] = bf16_bits_to_float(h[i]);
-            amax = fmaxf(amax, fabsf(f[i]));
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = c0 + 32 * u + lane;
+            v[u] = c < n_chunks ? ldg_nc_v4(w + c) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int off = 1; off < LANES; off <<= 1)
-            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-
-        uint32_t idx[8];
-        if (amax == 0.f) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) idx[i] = 0;            // every code ties
-        } else {
-            // keep 16/s and 17*s/16 finite for tiny and huge scales: rescale w and s by a
-            // power of two (exact; a weight that underflows is far below the smallest step)
-            const float ps = amax < 0x1p-96f ? 0x1p32f : (amax > 0x1p96f ? 0x1p-32f : 1.0f);
-            const float s = amax * ps;
-            const float c16 = 16.0f * __frcp_rn(s);
-            const float s16 = s * 0.0625f;
-            const float two_s16 = 2.0f * s16, m17 = -17.0f * s16;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float ws = f[i] * ps;
-                int cnt = (__float2int_ru(ws * c16) + 16) >> 1;
-                cnt = min(max(cnt, 0), 15);
-                // exact midpoint below code cnt: (2 cnt - 17) * s/16
-                const float mlo = fmaf((float)cnt, two_s16, m17);
-                if (cnt > 0 && !(ws > mlo)) cnt -= 1;
-                idx[i] = (uint32_t)cnt;
-            }
-        }
-        if (live) {
-            const uint32_t p = idx[0] | idx[1] << 4 | idx[2] << 8 | idx[3] << 12 |
-                               idx[4] << 16 | idx[5] << 20 | idx[6] << 24 | idx[7] << 28;
-            if (packed) packed[c] = p;
-            if (codes)
-                codes[c] = make_uint2(idx[0] | idx[1] << 8 | idx[2] << 16 | idx[3] << 24,
-                                      idx[4] | idx[5] << 8 | idx[6] << 16 | idx[7] << 24);
-            if ((threadIdx.x & (LANES - 1)) == 0) {
-                const int64_t row = c / chunks_per_row;
-                const int64_t col = (c - row * chunks_per_row) * 8;
-                scale[row * (k / G) + col / G] = (uint16_t)float_to_bf16_bits(amax);
-            }
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = c0 + 32 * u + lane;
+            quantize_chunk<G>(v[u], c < n_chunks, c, k, chunks_per_row, scale, codes, packed);
         }
     }
 }
@@ -142,22 +161,45 @@ unpack_kernel(const uint2* __restrict__ packed, int64_t n16, uint4* __restrict__
 // DYADIC4: bf16(step * (idx - 8)), step = scale / 8. The product is exact in fp32 (an
 // 8-bit significand times an integer of magnitude <= 8, scaled by 2^-3), so the bf16
 // conversion is the one and only rounding.
+// One thread: 4 packed words (32 codes, which lie in one group: groups are 32 or 64 columns
+// and the words are 16-byte aligned within a row) -> 64 bytes.
 __global__ void __launch_bounds__(kThreads)
-dequant_dyadic_kernel(const uint32_t* __restrict__ packed, const uint16_t* __restrict__ scale,
-                      int64_t n_words, int64_t k, int group, uint4* __restrict__ out) {
-    const int64_t words_per_row = k / 8;
+dequant_dyadic_kernel(const uint4* __restrict__ packed, const uint16_t* __restrict__ scale,
+                      int64_t n_quads, int64_t k, int group, uint4* __restrict__ out) {
+    const int64_t quads_per_row = k / 32;
     const int64_t groups_per_row = k / group;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_words;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const uint32_t p = packed[i];
-        const int64_t row = i / words_per_row;
-        const int64_t col = (i - row * words_per_row) * 8;
-        const float step = bf16_bits_to_float(ldg_u16(scale + row * groups_per_row + col / group)) * 0.125f;
-        float v[8];
+    constexpr int U = 2;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n_quads; i0 += stride * U) {
+        uint4 p[U];
+        uint32_t sc[U];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = step * (float)((int)((p >> (4 * j)) & 15) - 8);
-        out[i] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            p[u] = make_uint4(0, 0, 0, 0);
+            sc[u] = 0;
+            if (i < n_quads) {
+                p[u] = ldg_nc_v4(packed + i);
+                const int64_t row = i / quads_per_row;
+                const int64_t col = (i - row * quads_per_row) * 32;
+                sc[u] = ldg_u16(scale + row * groups_per_row + col / group);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i >= n_quads) break;
+            const float step = bf16_bits_to_float(sc[u]) * 0.125f;
+            const uint32_t wv[4] = {p[u].x, p[u].y, p[u].z, p[u].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = step * (float)((int)((wv[q] >> (4 * j)) & 15) - 8);
+                out[4 * i + q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+            }
+        }
     }
 }
 
@@ -214,7 +256,7 @@ wq_status launch_quantize_dyadic(const uint16_t* w, int64_t n, int64_t k, int gr
                                  uint16_t* scale, uint8_t* codes, uint8_t* packed,
                                  cudaStream_t s) {
     const int64_t chunks = n * k / 8;
-    const int grid = stream_grid(chunks);
+    const int grid = stream_grid((chunks + 3) / 4);
     if (group == 64)
         quantize_dyadic_kernel<64><<<grid, kThreads, 0, s>>>((const uint4*)w, chunks, k, scale,
                                                              (uint2*)codes, (uint32_t*)packed);
@@ -239,10 +281,11 @@ wq_status launch_unpack(const uint8_t* packed, int64_t n, int64_t k, uint8_t* co
 wq_status launch_dequant(const wq_weight& w, uint16_t* out, cudaStream_t s) {
     const int64_t n_words = w.n * w.k / 8;
     const int grid = stream_grid(n_words);
-    if (w.fmt == WQ_FMT_DYADIC4)
-        dequant_dyadic_kernel<<<grid, kThreads, 0, s>>>((const uint32_t*)w.packed,
-                                                        (const uint16_t*)w.aux, n_words, w.k,
-                                                        w.group, (uint4*)out);
+    if (w.fmt == WQ_FMT_DYADIC4) {
+        const int64_t n_quads = n_words / 4;          // k is a multiple of 32
+        dequant_dyadic_kernel<<<stream_grid(n_quads), kThreads, 0, s>>>(
+            (const uint4*)w.packed, (const uint16_t*)w.aux, n_quads, w.k, w.group, (uint4*)out);
+    }
     else if (w.fmt == WQ_FMT_LLOYD8S)
         dequant_lloyd_kernel<<<grid, kThreads, 0, s>>>((const uint32_t*)w.packed,
                                                        (const float4*)w.aux, n_words, (uint4*)out);
