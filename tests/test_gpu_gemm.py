@@ -27,7 +27,7 @@ def _check(y, y_ref, bound):
     assert np.all(err <= matmul_tolerance(y_ref, bound, TOL)), f"max err/bound {ratio.max():.3g}"
 
 
-@pytest.mark.parametrize("m", [1, 16, 17, 100, 128, 129, 256, 300])
+@pytest.mark.parametrize("m", [1, 8, 9, 16, 17, 33, 64, 100, 128, 129, 256, 300])
 @pytest.mark.parametrize("n,k,group", [(128, 256, 64), (200, 320, 64), (13, 64, 64), (256, 1024, 32)])
 def test_gemm_matches_oracle(wq, m, n, k, group):
     pw, packed, s = _weight(wq, n, k, group, m * 7 + n + k)
@@ -55,8 +55,9 @@ def test_gemm_one_hot_and_zero_codes_exact(wq):
 
 def test_gemm_split_k_uses_workspace(wq):
     pw, packed, s = _weight(wq, 1024, 8192, 64, 5)
-    assert wq.gemm_workspace_bytes(pw, 16) > 0            # small m splits K
-    x_bits = workloads.activations(16, 8192, workloads.PREFILL, 5)
+    assert wq.gemm_workspace_bytes(pw, 8) == 0            # m <= 8 runs on the GEMV kernel
+    assert wq.gemm_workspace_bytes(pw, 48) > 0            # small m splits K
+    x_bits = workloads.activations(48, 8192, workloads.PREFILL, 5)
     y = wq.gemm(pw, to_dev_bits(x_bits))
     rows = np.arange(0, 1024, 7)
     y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x_bits, rows=rows)

@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 
 
 def test_static_scratch_gemm_matches_workspace_gemm(wq):
-    n, k, m = 1024, 8192, 16                  # small m: K is split, so the scratch is used
+    n, k, m = 1024, 8192, 48                  # small m: K is split, so the scratch is used
     w_bits = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 21)
     s, c = oracle.dyadic_quantize(w_bits, 64)
     packed = oracle.pack(c)

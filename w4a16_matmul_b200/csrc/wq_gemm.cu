@@ -71,7 +71,9 @@ __device__ __forceinline__ uint64_t global_ns() {
 // wall time and returns false. Each try_wait may suspend the thread for up to
 // WQ_GEMM_SUSPEND_NS nanoseconds (it wakes as soon as the phase completes), so a waiting
 // warp does not spin on the issue slots the reconstruction warps need.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+// `abort` (shared memory) is polled only while the wait spins, so that a CTA whose other
+// role gave up stops waiting at once instead of timing out wait by wait.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, const int* abort = nullptr) {
     const uint32_t a = smem_u32(b);
     uint64_t deadline = 0;
     for (uint32_t i = 0;; ++i) {
@@ -81,6 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
             : "=r"(done) : "r"(a), "r"(parity), "r"((uint32_t)WQ_GEMM_SUSPEND_NS) : "memory");
         if (done) return true;
         if ((i & 7) == 0) {
+            if (abort && *(volatile const int*)abort) return false;
             const uint64_t now = global_ns();
             if (deadline == 0) deadline = now + kWaitNs;
             else if (now > deadline) return false;
@@ -195,12 +198,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 #ifndef WQ_GEMM_RW
 #define WQ_GEMM_RW 4
 #endif
+#ifndef WQ_GEMM_RW_NARROW
+#define WQ_GEMM_RW_NARROW 2
+#endif
 // Reconstruction warps per tensor-memory lane group: RW warps share each 32-lane group, each
-// filling 8 / RW of the row's eight packed words per stage (more warps hide more latency).
-constexpr int RW = WQ_GEMM_RW;
-constexpr int kThreads = 64 + 128 * RW;
+// filling 8 / RW of the row's eight packed words per stage (more warps hide more latency;
+// fewer repeat less per-stage bookkeeping).
+constexpr int rw_for(int bn) { return bn >= 128 ? WQ_GEMM_RW : WQ_GEMM_RW_NARROW; }
+constexpr int threads_for(int bn) { return 64 + 128 * rw_for(bn); }
 
 // Stores 32 / RW consecutive 32-bit columns of this thread's tensor-memory lane.
+template <int RW>
 __device__ __forceinline__ void tmem_st_part(uint32_t taddr, const uint32_t* v) {
     if constexpr (RW == 1) {
         tmem_st32(taddr, *reinterpret_cast<const uint32_t(*)[32]>(v));
@@ -222,12 +230,13 @@ __device__ __forceinline__ void tmem_st_part(uint32_t taddr, const uint32_t* v) 
 }
 
 template <int BN, int G, bool PARTIAL>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for(BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
             const uint16_t* __restrict__ scale, void* __restrict__ out, int M, int N, int K,
             int kt_per_split) {
     using S = Smem<BN>;
     constexpr int STAGES = S::STAGES;
+    constexpr int RW = rw_for(BN);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     constexpr int SLOTS = S::SLOTS;
@@ -280,11 +289,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (i / STAGES) & 1;
-                if (*(volatile int*)s_abort) break;
-                if (!mbar_wait(&empty[s], ph ^ 1)) { dead(1); break; }
+            int s = 0;
+            uint32_t ph = 0;
+            for (int i = 0; i < nk; ++i, s = (s + 1 == STAGES) ? 0 : s + 1, ph ^= (s == 0)) {
+                if (!mbar_wait(&empty[s], ph ^ 1, s_abort)) { dead(1); break; }
                 mbar_expect_tx(&full_tma[s], S::B_BYTES + S::P_BYTES);
                 const int kt = kt0 + i;
                 tma_load_2d(stage_b(s), &tmap_x, kt * BK, m0, &full_tma[s]);
@@ -296,11 +304,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         if (lane == 0) {
             constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
                                        ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+            int s = 0, a = 0;
+            uint32_t aph = 0;
             for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES, a = i % SLOTS;
-                if (*(volatile int*)s_abort) break;
                 // the slot is reconstructed, which also means the stage's tiles have landed
-                if (!mbar_wait(&full_w[a], (i / SLOTS) & 1)) { dead(2); break; }
+                if (!mbar_wait(&full_w[a], aph, s_abort)) { dead(2); break; }
                 asm volatile("tcgen05.fence::after_thread_sync;");
                 const uint64_t db = sw128_desc(smem_u32(stage_b(s)));
                 const uint32_t ta = tmem + S::ACC_COLS + 32u * (uint32_t)a;
@@ -309,6 +317,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     umma_f16_ts(tmem, ta + 8u * (uint32_t)k, db + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
                 umma_commit(&empty[s]);           // fire once these MMAs have read the stage ...
                 if constexpr (!S::COUPLED) umma_commit(&slot_free[a]);   // ... and the slot
+                if (++s == STAGES) s = 0;
+                if (++a == SLOTS) { a = 0; aph ^= 1; }
             }
             // commit (not a plain arrive) even after an abort: it fires only once every MMA
             // issued so far has finished, so tensor memory is never freed under a running MMA
@@ -338,27 +348,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             }
         }
         bool live = true;
+        int s = 0, a = 0;                                  // stage and slot of iteration it
+        uint32_t ph = 0, aph = 0;                          // their phase parities
         for (int base = 0; base < nk && live; base += kPre) {
 #pragma unroll
             for (int u = 0; u < kPre; ++u) {
                 const int it = base + u;
                 if (it >= nk) break;
-                const int s = it % STAGES, a = it % SLOTS;
-                const uint32_t ph = (it / STAGES) & 1;
-                // every exit below is taken by the whole warp (it ends in __syncwarp)
-                if (__any_sync(0xFFFFFFFFu, *(volatile int*)s_abort != 0)) { live = false; break; }
                 const uint32_t sc0 = ring0[u], sc1 = ring1[u];
                 if (row_ok && it + kPre < nk) {
                     ring0[u] = ldg_u16(srow + (kt0 + it + kPre) * BK / G);
                     ring1[u] = (G == 32) ? ldg_u16(srow + (kt0 + it + kPre) * BK / G + 1) : ring0[u];
                 }
                 // the packed tile has landed, and the MMAs that last read this tensor-memory
-                // slot (iteration it - SLOTS) have completed
-                // (with coupled rings the first implies the second: the TMA for this
-                // iteration was issued only after the stage's previous MMAs completed)
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full_tma[s], ph) &&
+                // slot (iteration it - SLOTS) have completed (with coupled rings the first
+                // implies the second: the TMA for this iteration was issued only after the
+                // stage's previous MMAs completed). Every exit is taken by the whole warp.
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full_tma[s], ph, s_abort) &&
                                              (S::COUPLED || it < SLOTS ||
-                                              mbar_wait(&slot_free[a], ((it / SLOTS) & 1) ^ 1)))) {
+                                              mbar_wait(&slot_free[a], aph ^ 1, s_abort)))) {
                     dead(3); live = false; break;
                 }
                 uint32_t wv[WPT];
@@ -387,12 +395,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                                          : dyadic_row8(wv[c], second ? cs1 : cs0, second ? cn1 : cn0);
                     v[4 * c] = r.x; v[4 * c + 1] = r.y; v[4 * c + 2] = r.z; v[4 * c + 3] = r.w;
                 }
-                tmem_st_part(lane_base + S::ACC_COLS + 32u * (uint32_t)a + (uint32_t)(part * 4 * WPT), v);
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full_w[a]);
+                // the previous iteration's store has had this iteration's loads and arithmetic
+                // to complete: wait for it now and release that slot to the MMA, then issue
+                // this one (one tensor-memory store in flight per warp)
+                if (it > 0) {
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full_w[a == 0 ? SLOTS - 1 : a - 1]);
+                }
+                tmem_st_part<RW>(lane_base + S::ACC_COLS + 32u * (uint32_t)a + (uint32_t)(part * 4 * WPT), v);
+                if (++s == STAGES) { s = 0; ph ^= 1; }
+                if (++a == SLOTS) { a = 0; aph ^= 1; }
             }
+        }
+        // release the last slot written (also after an abort: the MMA thread has stopped
+        // waiting by then, and an extra arrival on a slot barrier is harmless)
+        if (nk > 0) {
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (live && lane == 0) mbar_arrive(&full_w[a == 0 ? SLOTS - 1 : a - 1]);
         }
         // ---- epilogue: TMEM lane 32q + lane holds weight row n, columns = activation rows
         // tcgen05.ld is warp-collective: the decision to drain is taken per warp
@@ -470,15 +493,35 @@ struct Plan {
 
 Plan plan_for(int64_t M, int64_t N, int64_t K) {
     Plan p;
-    p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    const int sms = sm_count();
     p.grid_n = (int)((N + BM - 1) / BM);
+    // The widest activation tile the MMA takes once m allows it: every activation-row tile
+    // reconstructs the same weights again, and reconstruction (not the tensor pipe) is what
+    // narrower tiles run out of (measured: BN 128 / 192 at 0.5-0.9x of BN 256 throughput even
+    // where they leave fewer SMs idle in the last wave).
+    p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
     p.grid_m = (int)((M + p.bn - 1) / p.bn);
     const int KT = (int)(K / BK);
     const int64_t tiles = (int64_t)p.grid_n * p.grid_m;
-    const int sms = sm_count();
     int splits = 1;
-    // split K while the grid is below one wave and every split keeps >= 16 stages
-    while (tiles * splits * 2 <= sms && KT / (splits * 2) >= 16) splits *= 2;
+    if (p.bn >= 128) {
+        // wide tiles (one CTA per SM): split in powers of two while the grid stays within
+        // one round and every split keeps >= 16 stages
+        while (tiles * splits * 2 <= sms && KT / (splits * 2) >= 16) splits *= 2;
+    } else {
+        // narrow tiles (256 tensor-memory columns, at most ~100 KB of shared memory) fit two
+        // CTAs per SM. A grid of equal CTAs takes ceil(CTAs / slots) rounds of (stages per
+        // CTA + about 4 stages of prologue and epilogue); take the split count with the
+        // fewest, keeping >= 8 stages per split
+        const int64_t slots = 2 * (int64_t)sms;
+        int64_t best = -1;
+        for (int sp = 1; sp <= 32 && (sp == 1 || KT / sp >= 8); ++sp) {
+            const int64_t per = (KT + sp - 1) / sp;
+            const int64_t used = (KT + per - 1) / per;           // splits that get work
+            const int64_t cost = ((tiles * used + slots - 1) / slots) * (per + 4);
+            if (best < 0 || cost < best) { best = cost; splits = (int)used; }
+        }
+    }
     p.kt_per_split = (KT + splits - 1) / splits;
     p.splits = (KT + p.kt_per_split - 1) / p.kt_per_split;
     return p;
@@ -496,19 +539,28 @@ wq_status launch_bn(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp,
         auto k = gemm_kernel<BN, G, true>;
         if (!raised[1] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[1] = true;
-        k<<<grid, kThreads, smem, s>>>(tx, tp, scale, out, M, N, K, p.kt_per_split);
+        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, scale, out, M, N, K, p.kt_per_split);
     } else {
         auto k = gemm_kernel<BN, G, false>;
         if (!raised[0] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[0] = true;
-        k<<<grid, kThreads, smem, s>>>(tx, tp, scale, out, M, N, K, p.kt_per_split);
+        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, scale, out, M, N, K, p.kt_per_split);
     }
     return check_launch("gemm");
 }
 
 }  // namespace
 
+// Up to this many activation rows the product is decode-shaped: the GEMV kernel (weights
+// rebuilt in registers, mma.sync, no TMA/TMEM pipeline) runs it faster than the
+// tensor-memory pipeline, whose per-stage bookkeeping dominates when BN is this small
+// (measured on 4096x11008: 13.8 us against about 23 us at m = 1; at m = 16 the GEMV's second
+// batch fragment makes it the slower one). This is the kernel choice by batch size of
+// "K-Means量化技术…" §4.1.
+constexpr int64_t kGemvMaxRows = 8;
+
 size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
+    if (m <= kGemvMaxRows) return 0;
     const Plan p = plan_for(m, w.n, w.k);
     return p.splits > 1 ? (size_t)p.splits * (size_t)m * (size_t)w.n * sizeof(float) : 0;
 }
@@ -516,6 +568,10 @@ size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
 wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
                       size_t ws_bytes, cudaStream_t s) {
     const int M = (int)m, N = (int)w.n, K = (int)w.k;
+    if (m <= kGemvMaxRows) {
+        const GemvProblem prob{w.packed, w.aux, x, y, N, K};
+        return launch_gemv(w.fmt, w.group, &prob, 1, M, s);
+    }
     const Plan p = plan_for(M, N, K);
     auto enc = encode_fn();
     if (!enc) return fail(WQ_ECUDA, "cuTensorMapEncodeTiled is unavailable from the driver");

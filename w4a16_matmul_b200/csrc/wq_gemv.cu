@@ -393,8 +393,15 @@ constexpr int depth(int kind, int nb, int r) {
 
 // Resident CTAs per SM the register budget of a dyadic 16-row kernel aims at; the other
 // variants take what they need.
+#ifndef WQ_GEMV_R2_CAP
+#define WQ_GEMV_R2_CAP 4
+#endif
+#ifndef WQ_GEMV_LUT_CAP
+#define WQ_GEMV_LUT_CAP 1
+#endif
 constexpr int min_ctas(int kind, int nb, int r) {
-    return (kind != kLut16 && r == 1) ? (nb == 1 ? WQ_GEMV_MIN_CTAS_NB1 : WQ_GEMV_MIN_CTAS_NB2) : 1;
+    return kind == kLut16 ? WQ_GEMV_LUT_CAP
+         : r == 1 ? (nb == 1 ? WQ_GEMV_MIN_CTAS_NB1 : WQ_GEMV_MIN_CTAS_NB2) : WQ_GEMV_R2_CAP;
 }
 
 template <int KIND, int NB, int R, int WK, int MAXP>
