@@ -339,6 +339,31 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
         out["dequant_layer"] = {"GB/s": round(byts / ms / 1e6, 1),
                                 "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
         del wts, gq, gdq
+        # the same two kernels on one large matrix (the 8192 x 28672 weight of the LUT16
+        # workload, N(0, 0.02^2) here): one launch streams ~0.6 GB, so the number is the
+        # kernel's own bandwidth rather than launch gaps between small matrices
+        n_l, k_l = workloads.LUT16_SHAPE
+        wl = (torch.randn((n_l, k_l), device=dev) * 0.02).to(torch.bfloat16)
+        hold = {}
+
+        def ql():
+            hold["pw"], _ = wq.quantize_dyadic(wl, 64)
+        gql = graph_of(torch, ql)
+        ms = max_over_ranks(time_region(torch, stream, gql.replay, steps, warm, barrier))
+        nw = n_l * k_l
+        byts = nw * (2 + 0.5 + 2 / 64)
+        out["quantize_dyadic_large"] = {"shape": [n_l, k_l], "Gweights/s": round(nw / ms / 1e6, 2),
+                                        "GB/s": round(byts / ms / 1e6, 1),
+                                        "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4), "us": round(ms * 1e3, 1)}
+        pwl = hold["pw"]
+        del wl
+        dl = torch.empty((n_l, k_l), dtype=torch.bfloat16, device=dev)
+        gdl = graph_of(torch, lambda: wq.dequant(pwl, out=dl))
+        ms = max_over_ranks(time_region(torch, stream, gdl.replay, steps, warm, barrier))
+        byts = nw * (0.5 + 2 / 64 + 2)
+        out["dequant_large"] = {"shape": [n_l, k_l], "GB/s": round(byts / ms / 1e6, 1),
+                                "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4), "us": round(ms * 1e3, 1)}
+        del gql, gdl, dl, pwl, hold
     except Exception as e:
         out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
     if args.extras in ("gemm", "all"):

@@ -35,36 +35,71 @@ int stream_grid(int64_t items, int per_sm_blocks = 8) {
 // ---------------------------------------------------------------------------------------
 // One warp-contiguous block of 32 chunks (8 weights each) per unrolled step u: each thread
 // issues its U 128-bit loads before it computes, so U loads per thread are in flight.
-template <int G>
-__device__ __forceinline__ void quantize_chunk(uint4 v, bool live, int64_t c, int64_t k,
-                                               int64_t chunks_per_row, uint16_t* __restrict__ scale,
+// 1/x from the special-function unit (relative error below 2^-22 for normal x).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+template <int G, typename I>
+__device__ __forceinline__ void quantize_chunk(uint4 v, bool live, I c, uint16_t* __restrict__ scale,
                                                uint2* __restrict__ codes, uint32_t* __restrict__ packed) {
     constexpr int LANES = G / 8;                 // threads per group (8 or 4)
-    uint32_t h[8] = {v.x & 0xFFFF, v.x >> 16, v.y & 0xFFFF, v.y >> 16,
-                     v.z & 0xFFFF, v.z >> 16, v.w & 0xFFFF, v.w >> 16};
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
     float f[8];
-    float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        f[i] = bf16_bits_to_float(h[i]);
-        amax = fmaxf(amax, fabsf(f[i]));
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(wv[i] << 16);
+        f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
     }
+    // group absmax: |w| pairs by clearing the sign bits, a packed bf16 max over the chunk,
+    // then the two halves and the group's lanes
+    uint32_t m2;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m2) : "r"(v.x & 0x7FFF7FFFu), "r"(v.y & 0x7FFF7FFFu));
+    uint32_t m3;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m3) : "r"(v.z & 0x7FFF7FFFu), "r"(v.w & 0x7FFF7FFFu));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m2) : "r"(m2), "r"(m3));
+    float amax = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
 #pragma unroll
     for (int off = 1; off < LANES; off <<= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
 
-    uint32_t idx[8];
+    uint32_t p;
     if (amax == 0.f) {
+        p = 0;                                   // every code ties: code 0
+    } else if (amax >= 0x1p-96f && amax <= 0x1p96f) {
+        // idx = #{j in 1..15 : w > m_j}, m_j = (2j - 17) s / 16, is ceil(u) - 1 (at most 15)
+        // with u = 8 w / s + 8.5 (w > m_j <=> u > j; u >= 0.5 as |w| <= s). u is formed with
+        // the hardware reciprocal (relative error below 2^-22) and one FMA: |error| < 2^-18,
+        // while a u that is not an integer is at least 2^-17 from one (w and s being bf16);
+        // ceil is an add of 2^23 rounded upward. Only an exact midpoint (u an integer) can come out one too high;
+        // the exact comparison against the midpoint below corrects it (for idx 0 that
+        // midpoint, -17 s / 16, is below every weight, so no check is needed).
+        const float c8 = 8.0f * rcp_approx(amax);
+        const float s8 = amax * 0.125f, m17 = -17.0f * amax * 0.0625f;
+        float cf[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) idx[i] = 0;            // every code ties
+        for (int i = 0; i < 8; ++i) {
+            const float u = fmaf(f[i], c8, 8.5f);
+            float x = fminf(__fadd_ru(u, 8388608.0f) - 8388609.0f, 15.0f);   // ceil(u) - 1
+            const float mlo = fmaf(x, s8, m17);                                // exact midpoint
+            cf[i] = (f[i] > mlo) ? x : x - 1.0f;
+        }
+        // nibbles packed with exact float arithmetic: 2^23 + sum cf_i 16^i (< 2^24) holds the
+        // 16-bit half of the packed word in its low mantissa bits
+        const float lo = fmaf(cf[3], 4096.0f, fmaf(cf[2], 256.0f, fmaf(cf[1], 16.0f, cf[0] + 8388608.0f)));
+        const float hi = fmaf(cf[7], 4096.0f, fmaf(cf[6], 256.0f, fmaf(cf[5], 16.0f, cf[4] + 8388608.0f)));
+        p = prmt(__float_as_uint(lo), __float_as_uint(hi), 0x5410u);
     } else {
-        // keep 16/s and 17*s/16 finite for tiny and huge scales: rescale w and s by a
-        // power of two (exact; a weight that underflows is far below the smallest step)
-        const float ps = amax < 0x1p-96f ? 0x1p32f : (amax > 0x1p96f ? 0x1p-32f : 1.0f);
+        // keep 16/s and 17*s/16 finite for tiny and huge scales: rescale w and s by a power
+        // of two (exact; a weight that underflows is far below the smallest step)
+        const float ps = amax < 0x1p-96f ? 0x1p32f : 0x1p-32f;
         const float s = amax * ps;
         const float c16 = 16.0f * __frcp_rn(s);
         const float s16 = s * 0.0625f;
         const float two_s16 = 2.0f * s16, m17 = -17.0f * s16;
+        p = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float ws = f[i] * ps;
@@ -73,46 +108,42 @@ __device__ __forceinline__ void quantize_chunk(uint4 v, bool live, int64_t c, in
             // exact midpoint below code cnt: (2 cnt - 17) * s/16
             const float mlo = fmaf((float)cnt, two_s16, m17);
             if (cnt > 0 && !(ws > mlo)) cnt -= 1;
-            idx[i] = (uint32_t)cnt;
+            p |= (uint32_t)cnt << (4 * i);
         }
     }
     if (live) {
-        const uint32_t p = idx[0] | idx[1] << 4 | idx[2] << 8 | idx[3] << 12 |
-                           idx[4] << 16 | idx[5] << 20 | idx[6] << 24 | idx[7] << 28;
         if (packed) packed[c] = p;
-        if (codes)
-            codes[c] = make_uint2(idx[0] | idx[1] << 8 | idx[2] << 16 | idx[3] << 24,
-                                  idx[4] | idx[5] << 8 | idx[6] << 16 | idx[7] << 24);
-        if ((threadIdx.x & (LANES - 1)) == 0) {
-            const int64_t row = c / chunks_per_row;
-            const int64_t col = (c - row * chunks_per_row) * 8;
-            scale[row * (k / G) + col / G] = (uint16_t)float_to_bf16_bits(amax);
+        if (codes) {
+            // nibbles -> bytes: c0 c1 c2 c3 | c4 c5 c6 c7
+            const uint32_t e = p & 0x0F0F0F0Fu, o = (p >> 4) & 0x0F0F0F0Fu;
+            codes[c] = make_uint2(prmt(e, o, 0x5140u), prmt(e, o, 0x7362u));
         }
+        // the scale array [n, k/G] tiles the rows exactly, so group (row, col/G) is number
+        // c / LANES in row-major order
+        if ((threadIdx.x & (LANES - 1)) == 0) scale[c / LANES] = (uint16_t)float_to_bf16_bits(amax);
     }
 }
 
-template <int G>
+// I: the chunk index type (uint32_t when every chunk index fits, else uint64_t).
+template <int G, typename I>
 __global__ void __launch_bounds__(kThreads)
-quantize_dyadic_kernel(const uint4* __restrict__ w, int64_t n_chunks, int64_t k,
-                       uint16_t* __restrict__ scale, uint2* __restrict__ codes,
-                       uint32_t* __restrict__ packed) {
+quantize_dyadic_kernel(const uint4* __restrict__ w, I n_chunks, uint16_t* __restrict__ scale,
+                       uint2* __restrict__ codes, uint32_t* __restrict__ packed) {
     constexpr int U = 4;
-    const int64_t chunks_per_row = k / 8;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x * U;
-    const int lane = threadIdx.x & 31;
+    const I stride = (I)gridDim.x * blockDim.x * U;
+    const I lane = threadIdx.x & 31;
     // a warp covers U consecutive blocks of 32 chunks; groups never straddle n_chunks
-    for (int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31)) * U; c0 < n_chunks;
-         c0 += stride) {
+    for (I c0 = ((I)blockIdx.x * blockDim.x + (threadIdx.x & ~31u)) * U; c0 < n_chunks; c0 += stride) {
         uint4 v[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t c = c0 + 32 * u + lane;
+            const I c = c0 + 32 * u + lane;
             v[u] = c < n_chunks ? ldg_nc_v4(w + c) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t c = c0 + 32 * u + lane;
-            quantize_chunk<G>(v[u], c < n_chunks, c, k, chunks_per_row, scale, codes, packed);
+            const I c = c0 + 32 * u + lane;
+            quantize_chunk<G, I>(v[u], c < n_chunks, c, scale, codes, packed);
         }
     }
 }
@@ -168,7 +199,7 @@ dequant_dyadic_kernel(const uint4* __restrict__ packed, const uint16_t* __restri
                       int64_t n_quads, int64_t k, int group, uint4* __restrict__ out) {
     const int64_t quads_per_row = k / 32;
     const int64_t groups_per_row = k / group;
-    constexpr int U = 2;
+    constexpr int U = 4;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n_quads; i0 += stride * U) {
         uint4 p[U];
@@ -196,8 +227,8 @@ dequant_dyadic_kernel(const uint4* __restrict__ packed, const uint16_t* __restri
                 float v[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) v[j] = step * (float)((int)((wv[q] >> (4 * j)) & 15) - 8);
-                out[4 * i + q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                stg_cs_v4(out + 4 * i + q, make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                      pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7])));
             }
         }
     }
@@ -257,12 +288,17 @@ wq_status launch_quantize_dyadic(const uint16_t* w, int64_t n, int64_t k, int gr
                                  cudaStream_t s) {
     const int64_t chunks = n * k / 8;
     const int grid = stream_grid((chunks + 3) / 4);
-    if (group == 64)
-        quantize_dyadic_kernel<64><<<grid, kThreads, 0, s>>>((const uint4*)w, chunks, k, scale,
-                                                             (uint2*)codes, (uint32_t*)packed);
-    else
-        quantize_dyadic_kernel<32><<<grid, kThreads, 0, s>>>((const uint4*)w, chunks, k, scale,
-                                                             (uint2*)codes, (uint32_t*)packed);
+    // 32-bit chunk indices while c0 + stride stays below 2^32
+    const bool narrow = chunks + (int64_t)grid * kThreads * 4 < (int64_t)1 << 32;
+#define WQ_QUANT(G, I)                                                                          \
+    quantize_dyadic_kernel<G, I><<<grid, kThreads, 0, s>>>((const uint4*)w, (I)chunks, scale,   \
+                                                          (uint2*)codes, (uint32_t*)packed)
+    if (group == 64) {
+        if (narrow) WQ_QUANT(64, uint32_t); else WQ_QUANT(64, uint64_t);
+    } else {
+        if (narrow) WQ_QUANT(32, uint32_t); else WQ_QUANT(32, uint64_t);
+    }
+#undef WQ_QUANT
     return check_launch("quantize_dyadic");
 }
 

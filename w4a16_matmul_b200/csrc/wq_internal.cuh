@@ -126,6 +126,14 @@ __device__ __forceinline__ void ldg_v4_if(uint4& v, const void* p, uint32_t pred
         : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w) : "l"(p), "r"(pred));
 }
 
+// 128-bit store with the streaming (evict-first) cache hint: output written once and not
+// read again by this kernel.
+__device__ __forceinline__ void stg_cs_v4(void* p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t ldg_u32(const void* p) {
     uint32_t v;
     asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
