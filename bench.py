@@ -419,15 +419,29 @@ def bench_producers(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks
             hw = list(ex.map(lambda i: workloads.laplace_rowscaled_weight(2048, 2048, index=i), range(nm)))
         ws = [torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).to(dev) for h in hw]
 
+        made = []
+
         def lloyd():
+            made.clear()
             for w in ws:
-                wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)
+                made.append(wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)[0])
         ms = max_over_ranks(time_region(torch, stream, lloyd, 2, 1, barrier))
         n_w = nm * 2048 * 2048
         out["lloyd_g32"] = {"Gweights/s": round(n_w / ms / 1e6, 3), "ms_per_matrix": round(ms / nm, 3),
                             "sample": f"{nm} of the 224 matrices 2048x2048",
                             "extrapolated_224_s": round(ms / nm * 224 / 1e3, 3)}
         del ws
+        # the fused LLOYD8S consumer: one grouped GEMV over those matrices, batch 1 (codes
+        # 0.5 B + fp32 levels 1 B per weight)
+        xs_l = [torch.randn((1, 2048), device=dev).to(torch.bfloat16) for _ in made]
+        ys_l = [torch.empty((1, 2048), dtype=torch.bfloat16, device=dev) for _ in made]
+        run_l = wq.GroupedGemv(made, xs_l, ys_l)
+        g = graph_of(torch, run_l)
+        ms = max_over_ranks(time_region(torch, stream, g.replay, 20, 3, barrier))
+        byts = n_w * 1.5 + len(made) * 2048 * 4
+        out["lloyd8s_gemv_b1"] = {"matrices": len(made), "GB/s": round(byts / ms / 1e6, 1), "us": round(ms * 1e3, 2),
+                                  "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
+        del g, run_l, made
     except Exception as e:
         out["lloyd_g32"] = {"error": repr(e)[:200]}
     try:

@@ -222,3 +222,58 @@ def test_gemv_plan_replays_in_a_cuda_graph(wq):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(y, wq.gemv(pw, x))
+
+
+def _lloyd_weight(wq, n, k, seed, signed_levels=False):
+    """Random LLOYD8S weights: codes 0..15 (level index | sign << 3) and 8 fp32 levels per
+    group of 32 (sorted magnitudes, as the producer makes them; optionally of either sign,
+    which the format allows)."""
+    g = np.random.default_rng(seed)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    levels = np.sort(np.abs(g.standard_normal((n, k // 32, 8))) * 0.02, -1).astype(np.float32)
+    if signed_levels:
+        levels *= np.where(g.random(levels.shape) < 0.5, -1.0, 1.0).astype(np.float32)
+    packed = oracle.pack(codes)
+    pw = wq.PackedWeight(wq.FMT_LLOYD8S, 32, n, k, to_dev(packed), torch.from_numpy(levels).cuda())
+    return pw, packed, levels
+
+
+@pytest.mark.parametrize("batch", [1, 3, 8, 9, 16])
+@pytest.mark.parametrize("n,k", [(16, 32), (37, 1088), (300, 2048), (24, 2144)])
+def test_gemv_lloyd8s_matches_oracle(wq, n, k, batch):
+    """The fused LLOYD8S consumer ("int4-g32+warm" §5.2: 8-level codebook plus sign bit held
+    in registers) against the oracle's product of its bf16(+/-level) reconstruction."""
+    pw, packed, levels = _lloyd_weight(wq, n, k, n + k + batch)
+    x_bits = workloads.activations(batch, k, workloads.DECODE_SWEEP, n + batch)
+    y = wq.gemv(pw, to_dev_bits(x_bits))
+    y_ref, bound = oracle.matmul_rows(oracle.LLOYD8S, packed, levels, 32, x_bits)
+    _check(y, y_ref, bound)
+
+
+def test_gemv_lloyd8s_one_hot_reproduces_dequant_exactly(wq):
+    n, k = 48, 256
+    pw, packed, levels = _lloyd_weight(wq, n, k, 7, signed_levels=True)
+    wd = oracle.bf16_to_f64(oracle.dequant(oracle.LLOYD8S, packed, levels, 32))
+    cols = np.arange(0, k, 5)
+    for lo in range(0, len(cols), 16):
+        cc = cols[lo:lo + 16]
+        x = np.zeros((len(cc), k))
+        x[np.arange(len(cc)), cc] = 1.0
+        y = f32(wq.gemv(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
+        assert np.array_equal(y, wd[:, cc].T)
+
+
+def test_gemv_lloyd8s_on_the_gpu_producers_output(wq):
+    """The g32 Lloyd producer's packed codes and levels, consumed by the fused GEMV and by the
+    oracle (sampled rows), on one Lloyd-workload matrix."""
+    w_bits = workloads.laplace_rowscaled_weight(512, 2048, index=3)
+    pw, _ = wq.quantize_lloyd(to_dev_bits(w_bits), wq.LLOYD_G32_WARM, 25)
+    packed = pw.packed.cpu().numpy()
+    levels = pw.aux.cpu().numpy()
+    rng = np.random.default_rng(8)
+    rows = rng.choice(512, 64, replace=False)
+    for batch in (1, 16):
+        x_bits = workloads.activations(batch, 2048, workloads.DECODE_SWEEP, 40 + batch)
+        y = wq.gemv(pw, to_dev_bits(x_bits))
+        y_ref, bound = oracle.matmul_rows(oracle.LLOYD8S, packed, levels, 32, x_bits, rows=rows)
+        _check(y, y_ref, bound, rows)

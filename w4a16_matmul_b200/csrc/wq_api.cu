@@ -236,8 +236,6 @@ wq_status check_grouped(const wq_weight* ws, const uint16_t* const* xs, uint16_t
         if (st) return st;
         if (ws[i].fmt != ws[0].fmt || ws[i].group != ws[0].group)
             return fail(WQ_EINVAL, "problem %d: all grouped weights must share format and group", i);
-        if (ws[i].fmt == WQ_FMT_LLOYD8S)
-            return fail(WQ_EUNSUPPORTED, "GEMV of LLOYD8S weights is not implemented; use wq_dequant");
         if ((st = check_ptr(xs[i], "x", false))) return st;
         if ((st = check_ptr(ys[i], "y", false))) return st;
         probs[i] = GemvProblem{ws[i].packed, ws[i].aux, xs[i], ys[i], (int32_t)ws[i].n, (int32_t)ws[i].k};

@@ -1,8 +1,9 @@
 // wq_gemv.cu -- W4A16 GEMV for decode: y[b, r] = sum_c Wdeq[r, c] x[b, c], b < batch <= 16.
 //
 // Reconstruction follows "MiniCPM5-1B 验证: 6× 压缩…" §2.2/§2.5 (dyadic: bf16(step*(idx-8)))
-// and "K-Means量化技术…" §2.2 (LUT16: a 16-entry centroid table per block of 64), fused into
-// the product instead of written out as a dense matrix.
+// "K-Means量化技术…" §2.2 (LUT16: a 16-entry centroid table per block of 64) and
+// "int4-g32+warm 裸量化…" §5.2 (LLOYD8S: bf16(±level) from a group's 8 levels, the codebook
+// held in registers), fused into the product instead of written out as a dense matrix.
 //
 // Design (HBM-bound: 0.53 B per dyadic weight, 1 B per LUT16 weight; what stands between
 // the kernel and the memory roof is the instruction count and latency of the in-register
@@ -121,6 +122,21 @@ __device__ __forceinline__ void lut16_lookup4(uint32_t s, const uint32_t* lo, co
     p23 = prmt(l, h, 0x7362u);
 }
 
+// LLOYD8S lookup of 4 codes (nibbles of the low 16 bits of s; code = level index q in bits
+// 0-2, sign in bit 3) in an 8-entry bf16 table of one group held as byte planes: lo[0..1] /
+// hi[0..1] hold the low / high bytes of bf16(level[0..7]). The sign bit of each code flips
+// the sign bit of the high byte (bf16(-v) = -bf16(v): rounding to nearest even is
+// symmetric). Returns the bf16 pairs (code0, code1) and (code2, code3).
+__device__ __forceinline__ void lloyd8_lookup4(uint32_t s, const uint32_t* lo, const uint32_t* hi,
+                                               uint32_t& p01, uint32_t& p23) {
+    const uint32_t s7 = s & 0x7777u;                                     // level index
+    const uint32_t sg = prmt(0x00000000u, 0x80808080u, (s >> 1) & 0x4444u);   // 0x80 where signed
+    const uint32_t l = prmt(lo[0], lo[1], s7);
+    const uint32_t h = prmt(hi[0], hi[1], s7) ^ sg;
+    p01 = prmt(l, h, 0x5140u);
+    p23 = prmt(l, h, 0x7362u);
+}
+
 // bf16x2 -> fp16x2 (round to nearest even; exact for |x| in [2^-14, 65504]).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
@@ -129,14 +145,15 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     return r;
 }
 
-enum Kind { kDyadic64 = 0, kDyadic32 = 1, kLut16 = 2 };
+enum Kind { kDyadic64 = 0, kDyadic32 = 1, kLut16 = 2, kLloyd8 = 3 };
 
 // Per-lane state of one 256-column step for R 16-row blocks: the 32 bytes of rows g and
 // g+8 of each block, and their per-group parameters.
 template <int KIND, int R>
 struct Step {
     uint32_t w[R][2][8];
-    uint32_t aux[R][2][KIND == kLut16 ? 8 : 2];   // dyadic: bf16 scales; LUT16: table words
+    // dyadic: bf16 scales; LUT16: table words; LLOYD8S: the fp32 levels of two groups
+    uint32_t aux[R][2][KIND == kLut16 ? 8 : KIND == kLloyd8 ? 16 : 2];
 };
 
 // A 128-bit weight load that does not allocate in L1.
@@ -171,7 +188,20 @@ __device__ __forceinline__ void load_step(Step<KIND, R>& st, const GemvProblem& 
             const uint4 b = (rl && h1) ? ldg_w(wp + 16) : fill;
             st.w[r][h][0] = a.x; st.w[r][h][1] = a.y; st.w[r][h][2] = a.z; st.w[r][h][3] = a.w;
             st.w[r][h][4] = b.x; st.w[r][h][5] = b.y; st.w[r][h][6] = b.z; st.w[r][h][7] = b.w;
-            if (KIND == kLut16) {
+            if (KIND == kLloyd8) {
+                // the 8 fp32 levels of groups kk/32 and kk/32 + 1 (64 contiguous bytes)
+                const uint4* lp = (const uint4*)((const float*)pb.aux + ((size_t)row * (K / 32) + kk / 32) * 8);
+                uint4 l[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) l[q] = make_uint4(0, 0, 0, 0);
+                if (rl && h0) { l[0] = ldg_nc_v4(lp); l[1] = ldg_nc_v4(lp + 1); }
+                if (rl && h1) { l[2] = ldg_nc_v4(lp + 2); l[3] = ldg_nc_v4(lp + 3); }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    st.aux[r][h][4 * q] = l[q].x; st.aux[r][h][4 * q + 1] = l[q].y;
+                    st.aux[r][h][4 * q + 2] = l[q].z; st.aux[r][h][4 * q + 3] = l[q].w;
+                }
+            } else if (KIND == kLut16) {
                 uint4 la = make_uint4(0, 0, 0, 0), lb = la;
                 if (rl && h0) {
                     const uint4* lp = (const uint4*)((const uint16_t*)pb.aux + ((size_t)row * (K / 64) + kk / 64) * 16);
@@ -213,7 +243,22 @@ __device__ __forceinline__ void compute_step_staged(const Step<KIND, R>& st, flo
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            if (KIND == kLut16) {
+            if (KIND == kLloyd8) {
+                // bf16(level) of both groups, split into byte planes: plo/phi[2j..2j+1] for
+                // group j (one rounding per level, to nearest even)
+                const uint32_t* L = st.aux[r][h];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t b01 = pack_bf16x2(__uint_as_float(L[8 * j]), __uint_as_float(L[8 * j + 1]));
+                    const uint32_t b23 = pack_bf16x2(__uint_as_float(L[8 * j + 2]), __uint_as_float(L[8 * j + 3]));
+                    const uint32_t b45 = pack_bf16x2(__uint_as_float(L[8 * j + 4]), __uint_as_float(L[8 * j + 5]));
+                    const uint32_t b67 = pack_bf16x2(__uint_as_float(L[8 * j + 6]), __uint_as_float(L[8 * j + 7]));
+                    plo[r][h][2 * j] = prmt(b01, b23, 0x6420u);
+                    plo[r][h][2 * j + 1] = prmt(b45, b67, 0x6420u);
+                    phi[r][h][2 * j] = prmt(b01, b23, 0x7531u);
+                    phi[r][h][2 * j + 1] = prmt(b45, b67, 0x7531u);
+                }
+            } else if (KIND == kLut16) {
                 const uint32_t* L = st.aux[r][h];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -239,7 +284,18 @@ __device__ __forceinline__ void compute_step_staged(const Step<KIND, R>& st, flo
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             uint32_t q0[4], q1[4];                      // rows g and g+8
-            if (KIND == kLut16) {
+            if (KIND == kLloyd8) {
+                const int j = sub < 4 ? 0 : 2;          // words 0-3: first group, 4-7: second
+                lloyd8_lookup4(st.w[r][0][sub], plo[r][0] + j, phi[r][0] + j, q0[0], q0[1]);
+                lloyd8_lookup4(st.w[r][0][sub] >> 16, plo[r][0] + j, phi[r][0] + j, q0[2], q0[3]);
+                lloyd8_lookup4(st.w[r][1][sub], plo[r][1] + j, phi[r][1] + j, q1[0], q1[1]);
+                lloyd8_lookup4(st.w[r][1][sub] >> 16, plo[r][1] + j, phi[r][1] + j, q1[2], q1[3]);
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    mma_bf16_16816(acc[r][nb], q0[0], q1[0], q0[1], q1[1], b[nb][0], b[nb][1]);
+                    mma_bf16_16816(acc[r][nb], q0[2], q1[2], q0[3], q1[3], b[nb][2], b[nb][3]);
+                }
+            } else if (KIND == kLut16) {
                 lut16_lookup4(st.w[r][0][sub], plo[r][0], phi[r][0], q0[0], q0[1]);
                 lut16_lookup4(st.w[r][0][sub] >> 16, plo[r][0], phi[r][0], q0[2], q0[3]);
                 lut16_lookup4(st.w[r][1][sub], plo[r][1], phi[r][1], q1[0], q1[1]);
@@ -317,7 +373,7 @@ __device__ __forceinline__ void compute_step_exact(const GemvProblem& pb, int ro
 // range the one-FMA reconstruction covers.
 template <int KIND, int R>
 __device__ __forceinline__ bool step_scales_in_range(const Step<KIND, R>& st) {
-    if (KIND == kLut16) return true;
+    if (KIND == kLut16 || KIND == kLloyd8) return true;
     bool ok = true;
 #pragma unroll
     for (int r = 0; r < R; ++r)
@@ -366,6 +422,8 @@ __device__ __forceinline__ bool stage_x(uint8_t* xs, const uint16_t* x, int B, i
             if (KIND == kLut16) {
                 f.x = bf16x2_to_f16x2(v[u].x); f.y = bf16x2_to_f16x2(v[u].y);
                 f.z = bf16x2_to_f16x2(v[u].z); f.w = bf16x2_to_f16x2(v[u].w);
+            } else if (KIND == kLloyd8) {
+                f = v[u];                               // bf16 in natural order
             } else {
                 // a half of magnitude bits m >= 0x5F80 (|x| >= 2^64, inf, NaN) carries into
                 // bit 15 of that half when 0x2080 is added
@@ -388,7 +446,7 @@ __device__ __forceinline__ bool stage_x(uint8_t* xs, const uint16_t* x, int B, i
 // flight per SM, warps x (D - 1) x 2 KB, set the bandwidth a latency-bound stream reaches,
 // and deeper buffers buy them at fewer registers than more warps would.
 constexpr int depth(int kind, int nb, int r) {
-    return (kind != kLut16 && nb == 1 && r == 1) ? WQ_GEMV_DEPTH : 2;
+    return (kind < kLut16 && nb == 1 && r == 1) ? WQ_GEMV_DEPTH : 2;
 }
 
 // Resident CTAs per SM the register budget of a dyadic 16-row kernel aims at; the other
@@ -400,7 +458,7 @@ constexpr int depth(int kind, int nb, int r) {
 #define WQ_GEMV_LUT_CAP 1
 #endif
 constexpr int min_ctas(int kind, int nb, int r) {
-    return kind == kLut16 ? WQ_GEMV_LUT_CAP
+    return kind >= kLut16 ? WQ_GEMV_LUT_CAP
          : r == 1 ? (nb == 1 ? WQ_GEMV_MIN_CTAS_NB1 : WQ_GEMV_MIN_CTAS_NB2) : WQ_GEMV_R2_CAP;
 }
 
@@ -445,7 +503,7 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
         else load_step<KIND, R, false>(st, pb, row0, g, s * 256 + t * 64, N, K);
     };
     auto run_step = [&](const Step<KIND, R>& st, int s, int c0, bool xbad) {
-        if (KIND == kLut16 || (!xbad && __all_sync(0xFFFFFFFFu, step_scales_in_range<KIND, R>(st))))
+        if (KIND >= kLut16 || (!xbad && __all_sync(0xFFFFFFFFu, step_scales_in_range<KIND, R>(st))))
             compute_step_staged<KIND, NB, R>(st, acc, xs0 + 512 * (s - c0), xs1 + 512 * (s - c0));
         else
             compute_step_exact<KIND, NB, R>(pb, row0, g, s * 256 + t * 64, N, K, B, acc);
@@ -565,7 +623,7 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
     };
     // 32-row warps pay off once the activation fragment is shared by more batch rows
     // (measured on the decode sweep: 16-row warps win up to batch 8, 32-row warps at 9..16)
-    constexpr int BIGR = (KIND == kLut16) ? 1 : 2;
+    constexpr int BIGR = (KIND >= kLut16) ? 1 : 2;
     if (BIGR == 2 && batch > WQ_GEMV_R2_MIN_BATCH && rows16 >= 12 * sms * 2)
         return prepare_variant<KIND, NB, BIGR, 1, MAXP>(pr, probs, tiles_for(64 * BIGR));
     if (rows16 >= 8 * sms) return prepare_variant<KIND, NB, 1, 1, MAXP>(pr, probs, tiles_for(64));
@@ -592,10 +650,14 @@ wq_status prepare(int fmt, int group, const GemvProblem* probs, int count, int b
     int64_t rows16 = 0;
     for (int i = 0; i < count; ++i) { prm.prob[i] = probs[i]; rows16 += (probs[i].n + 15) / 16; }
     const bool two = batch > 8;
-    const int kind = (fmt == WQ_FMT_LUT16) ? kLut16 : (group == 64 ? kDyadic64 : kDyadic32);
+    const int kind = (fmt == WQ_FMT_LUT16) ? kLut16 : (fmt == WQ_FMT_LLOYD8S) ? kLloyd8
+                   : (group == 64 ? kDyadic64 : kDyadic32);
     if (kind == kLut16)
         return two ? pick_split<kLut16, 2, MAXP>(pr, probs, count, rows16, batch)
                    : pick_split<kLut16, 1, MAXP>(pr, probs, count, rows16, batch);
+    if (kind == kLloyd8)
+        return two ? pick_split<kLloyd8, 2, MAXP>(pr, probs, count, rows16, batch)
+                   : pick_split<kLloyd8, 1, MAXP>(pr, probs, count, rows16, batch);
     if (kind == kDyadic64)
         return two ? pick_split<kDyadic64, 2, MAXP>(pr, probs, count, rows16, batch)
                    : pick_split<kDyadic64, 1, MAXP>(pr, probs, count, rows16, batch);
