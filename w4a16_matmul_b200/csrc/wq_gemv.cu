@@ -394,18 +394,18 @@ __device__ __forceinline__ bool step_scales_in_range(const Step<KIND, R>& st) {
 // columns paired (0,4), (1,5), (2,6), (3,7); LUT16: fp16 in natural order. Columns at or
 // beyond K are zero. Stages steps [c0, c0 + ns) of all B rows with the whole CTA; returns
 // (dyadic) whether some staged |x| reaches 2^64 or is not finite.
-template <int KIND>
+template <int KIND, int THREADS>
 __device__ __forceinline__ bool stage_x(uint8_t* xs, const uint16_t* x, int B, int K, int c0,
                                         int ns, int rs) {
     const int per_row = ns * 32;                 // 16-byte blocks of 8 columns
     const int total = B * per_row;
     uint32_t bad = 0;
     constexpr int U = 4;                         // loads in flight per thread
-    for (int base = threadIdx.x; base < total; base += 128 * U) {
+    for (int base = threadIdx.x; base < total; base += THREADS * U) {
         uint4 v[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int i = base + 128 * u;
+            const int i = base + THREADS * u;
             v[u] = make_uint4(0, 0, 0, 0);
             if (i < total) {
                 const int b = i / per_row, j = i - b * per_row;
@@ -415,7 +415,7 @@ __device__ __forceinline__ bool stage_x(uint8_t* xs, const uint16_t* x, int B, i
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int i = base + 128 * u;
+            const int i = base + THREADS * u;
             if (i >= total) break;
             const int b = i / per_row, j = i - b * per_row;
             uint4 f;
@@ -449,6 +449,14 @@ constexpr int depth(int kind, int nb, int r) {
     return (kind < kLut16 && nb == 1 && r == 1) ? WQ_GEMV_DEPTH : 2;
 }
 
+#ifndef WQ_GEMV_WARPS_BATCHED
+#define WQ_GEMV_WARPS_BATCHED 8
+#endif
+// Warps per CTA: full-K kernels (WK = 1) take FW row warps (a CTA stages its activations
+// once for all of them, so more warps per CTA pay once the staged batch is larger);
+// split-K kernels have 4 warps in total.
+constexpr int cta_warps(int wk, int fw) { return wk == 1 ? fw : 4; }
+
 // Resident CTAs per SM the register budget of a dyadic 16-row kernel aims at; the other
 // variants take what they need.
 #ifndef WQ_GEMV_R2_CAP
@@ -462,10 +470,13 @@ constexpr int min_ctas(int kind, int nb, int r) {
          : r == 1 ? (nb == 1 ? WQ_GEMV_MIN_CTAS_NB1 : WQ_GEMV_MIN_CTAS_NB2) : WQ_GEMV_R2_CAP;
 }
 
-template <int KIND, int NB, int R, int WK, int MAXP>
-__global__ void __launch_bounds__(128, min_ctas(KIND, NB, R))
+template <int KIND, int NB, int R, int WK, int FW, int MAXP>
+__global__ void __launch_bounds__(32 * cta_warps(WK, FW),
+                                  (min_ctas(KIND, NB, R) * 4 / cta_warps(WK, FW)) > 0
+                                      ? (min_ctas(KIND, NB, R) * 4 / cta_warps(WK, FW)) : 1)
 gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
-    constexpr int WR = 4 / WK;                       // warps with distinct rows per CTA
+    constexpr int THREADS = 32 * cta_warps(WK, FW);
+    constexpr int WR = cta_warps(WK, FW) / WK;       // warps with distinct rows per CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wr = warp % WR, wk = warp / WR;
     // ---- which problem / row tile (a tile = the 16*R*WR rows of one CTA) -----------------
@@ -522,7 +533,7 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     for (int c0 = 0; c0 < steps; c0 += cs) {
         if (c0 > 0) __syncthreads();               // every warp is done with the last chunk
         const int ns = min(cs, steps - c0);
-        const bool xbad = __syncthreads_or(stage_x<KIND>(xs, pb.x, B, K, c0, ns, rs)) != 0;
+        const bool xbad = __syncthreads_or(stage_x<KIND, THREADS>(xs, pb.x, B, K, c0, ns, rs)) != 0;
         if (!live) continue;
         const int cend = c0 + ns;
         for (int s0 = c0 + wk; s0 < cend; s0 += D * WK) {
@@ -581,10 +592,11 @@ struct Prepared {
     void (*kern)(GemvParams<MAXP>);
     GemvParams<MAXP> prm;
     int tiles;
+    int threads;
     size_t smem;
 };
 
-template <int KIND, int NB, int R, int WK, int MAXP>
+template <int KIND, int NB, int R, int WK, int FW, int MAXP>
 wq_status prepare_variant(Prepared<MAXP>& pr, const GemvProblem* probs, int tiles) {
     constexpr int unit = depth(KIND, NB, R) * WK;   // chunks are whole multiples of this
     GemvParams<MAXP>& prm = pr.prm;
@@ -594,8 +606,9 @@ wq_status prepare_variant(Prepared<MAXP>& pr, const GemvProblem* probs, int tile
     cs = max(unit, cs - cs % unit);
     prm.chunk_steps = min(cs, max_steps);
     pr.smem = (size_t)prm.batch * (512 * prm.chunk_steps + 64);
-    pr.kern = gemv_kernel<KIND, NB, R, WK, MAXP>;
+    pr.kern = gemv_kernel<KIND, NB, R, WK, FW, MAXP>;
     pr.tiles = tiles;
+    pr.threads = 32 * cta_warps(WK, FW);
     if (pr.smem > 48 * 1024) {
         // small launches with many batch rows: a chunk of D * WK steps may pass 48 KB
         if (cudaFuncSetAttribute(pr.kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) !=
@@ -624,11 +637,19 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
     // 32-row warps pay off once the activation fragment is shared by more batch rows
     // (measured on the decode sweep: 16-row warps win up to batch 8, 32-row warps at 9..16)
     constexpr int BIGR = (KIND >= kLut16) ? 1 : 2;
-    if (BIGR == 2 && batch > WQ_GEMV_R2_MIN_BATCH && rows16 >= 12 * sms * 2)
-        return prepare_variant<KIND, NB, BIGR, 1, MAXP>(pr, probs, tiles_for(64 * BIGR));
-    if (rows16 >= 8 * sms) return prepare_variant<KIND, NB, 1, 1, MAXP>(pr, probs, tiles_for(64));
-    if (rows16 >= 2 * sms) return prepare_variant<KIND, NB, 1, 2, MAXP>(pr, probs, tiles_for(32));
-    return prepare_variant<KIND, NB, 1, 4, MAXP>(pr, probs, tiles_for(16));
+    // full-K CTAs: 4 row warps at batch 1, WQ_GEMV_WARPS_BATCHED above (measured on the
+    // decode sweep: 8 warps +9 / +13 / +14 % at batch 4 / 8 / 16, neutral at batch 1)
+    if (BIGR == 2 && batch > WQ_GEMV_R2_MIN_BATCH && rows16 >= 12 * sms * 2) {
+        constexpr int FWB = WQ_GEMV_WARPS_BATCHED;
+        return prepare_variant<KIND, NB, BIGR, 1, FWB, MAXP>(pr, probs, tiles_for(16 * FWB * BIGR));
+    }
+    if (rows16 >= 8 * sms) {
+        if (batch == 1) return prepare_variant<KIND, NB, 1, 1, 4, MAXP>(pr, probs, tiles_for(64));
+        constexpr int FWB = WQ_GEMV_WARPS_BATCHED;
+        return prepare_variant<KIND, NB, 1, 1, FWB, MAXP>(pr, probs, tiles_for(16 * FWB));
+    }
+    if (rows16 >= 2 * sms) return prepare_variant<KIND, NB, 1, 2, 4, MAXP>(pr, probs, tiles_for(32));
+    return prepare_variant<KIND, NB, 1, 4, 4, MAXP>(pr, probs, tiles_for(16));
 }
 
 template <int MAXP>
@@ -667,7 +688,7 @@ wq_status prepare(int fmt, int group, const GemvProblem* probs, int count, int b
 
 template <int MAXP>
 wq_status launch_prepared(const Prepared<MAXP>& pr, cudaStream_t s) {
-    pr.kern<<<pr.tiles, 128, pr.smem, s>>>(pr.prm);
+    pr.kern<<<pr.tiles, pr.threads, pr.smem, s>>>(pr.prm);
     return check_launch("gemv");
 }
 
