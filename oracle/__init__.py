@@ -54,6 +54,7 @@ def _L():
             "orc_double_to_fp16_array": [vp, i64, vp],
             "orc_dyadic_quantize": [vp, i64, i64, i32, i64, i64, vp, vp],
             "orc_dyadic_dequant": [vp, vp, i64, i64, i32, i64, i64, vp],
+            "orc_fake_quant_ste": [vp, vp, i64, i64, i32, i64, i64, vp, vp],
             "orc_pack": [vp, i64, i64, i64, i64, vp],
             "orc_unpack": [vp, i64, i64, i64, i64, vp],
             "orc_dequant": [i32, vp, vp, i64, i64, i32, i64, i64, vp],
@@ -147,6 +148,20 @@ def dyadic_quantize(w_bits: np.ndarray, group: int = 64, threads: int | None = N
     _rows_parallel(n, lambda r0, r1: _L().orc_dyadic_quantize(_p(w), n, k, group, r0, r1,
                                                               _p(scale), _p(codes)), threads)
     return scale, codes
+
+
+def fake_quant_ste(z: np.ndarray, scale_bits: np.ndarray, group: int = 64,
+                   threads: int | None = None):
+    """[DG] §2.3 STE forward on an fp32 latent z: (q fp32 [n, k], codes uint8 [n, k]) with
+    codes the nearest of the 16 dyadic code values (lowest index on a tie) and q that value."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    scale = np.ascontiguousarray(scale_bits, dtype=np.uint16)
+    n, k = z.shape
+    q = np.empty((n, k), np.float32)
+    codes = np.empty((n, k), np.uint8)
+    _rows_parallel(n, lambda r0, r1: _L().orc_fake_quant_ste(_p(z), _p(scale), n, k, group, r0, r1,
+                                                             _p(q), _p(codes)), threads)
+    return q, codes
 
 
 def dyadic_dequant(codes: np.ndarray, scale_bits: np.ndarray, group: int = 64,

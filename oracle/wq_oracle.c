@@ -161,6 +161,38 @@ int orc_dyadic_quantize(const uint16_t* w, int64_t n, int64_t k, int32_t group,
     return 0;
 }
 
+/* STE fake quantisation, forward ([DG] §2.3 "STE"): on an fp32 latent z with the block's
+ * bf16 scale, idx = argmin_j |z - step*(j-8)| over j = 0..15 (lowest j on a tie, the same
+ * rule as the hard argmin above), step = scale/8, and the forward value is the code value
+ * q = step*(idx-8) itself (exact in fp32: an 8-bit significand times an integer of
+ * magnitude <= 8, over 8). The backward of STE is the identity and computes nothing. Every
+ * distance is exact in double (z has 24 significant bits, a code value 11). z may lie
+ * outside [-scale, scale] (the scale is a trained parameter): the argmin then picks the
+ * end code. */
+int orc_fake_quant_ste(const float* z, const uint16_t* scale, int64_t n, int64_t k, int32_t group,
+                       int64_t r0, int64_t r1, float* q, uint8_t* codes)
+{
+    (void)n;
+    if (group <= 0 || k % group != 0) return -1;
+    const int64_t ng = k / group;
+    for (int64_t r = r0; r < r1; ++r) {
+        for (int64_t c = 0; c < k; ++c) {
+            const double v = (double)z[r * k + c];
+            const double step = orc_bf16_to_double(scale[r * ng + c / group]) / 8.0;
+            if (!isfinite(v) || !isfinite(step)) return -2;
+            int best = 0;
+            double bestd = fabs(v - (0 - 8) * step);
+            for (int j = 1; j < 16; ++j) {
+                const double d = fabs(v - (j - 8) * step);
+                if (d < bestd) { bestd = d; best = j; }
+            }
+            codes[r * k + c] = (uint8_t)best;
+            q[r * k + c] = (float)((best - 8) * step);
+        }
+    }
+    return 0;
+}
+
 /* Reconstruction w = step * (idx - 8) ([DG] §2.2), stored as bf16 (one rounding). */
 int orc_dyadic_dequant(const uint8_t* codes, const uint16_t* scale, int64_t n, int64_t k,
                        int32_t group, int64_t r0, int64_t r1, uint16_t* out)
