@@ -364,6 +364,19 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
         out["dequant_large"] = {"shape": [n_l, k_l], "GB/s": round(byts / ms / 1e6, 1),
                                 "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4), "us": round(ms * 1e3, 1)}
         del gql, gdl, dl, pwl, hold
+        # STE fake quantisation forward on an fp32 latent of the same shape (4 B in, 4 B out
+        # plus 0.5 B of packed codes per element)
+        zl = torch.randn((n_l, k_l), device=dev).mul_(0.02)
+        scl = (zl.abs().reshape(n_l, k_l // 64, 64).amax(-1)).to(torch.bfloat16)
+        qo = torch.empty_like(zl)
+        po = torch.empty((n_l, k_l // 2), dtype=torch.uint8, device=dev)
+        gz = graph_of(torch, lambda: wq._check(wq._lib.wq_fake_quant_ste(
+            wq._ptr(zl), n_l, k_l, 64, wq._ptr(scl), wq._ptr(qo), None, wq._ptr(po), wq._stream(zl))))
+        ms = max_over_ranks(time_region(torch, stream, gz.replay, steps, warm, barrier))
+        byts = nw * (4 + 4 + 0.5) + nw / 64 * 2
+        out["fake_quant_ste_large"] = {"shape": [n_l, k_l], "GB/s": round(byts / ms / 1e6, 1), "us": round(ms * 1e3, 1),
+                                       "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
+        del gz, zl, scl, qo, po
     except Exception as e:
         out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
     if args.extras in ("gemm", "all"):

@@ -158,6 +158,23 @@ wq_status wq_unpack(const uint8_t* packed, int64_t n, int64_t k, uint8_t* codes,
  *   out  [n, k] 16-bit patterns. Bit-exact. */
 wq_status wq_dequant(const wq_weight* w, uint16_t* out, wq_stream stream);
 
+/* STE fake quantisation, forward ([DG] §2.3 "STE"): the forward pass of a QAT step on the
+ * fp32 latent weights z. q[r, c] = step * (idx - 8) with idx = argmin_j |z - step * (j - 8)|
+ * over j = 0..15 (lowest j on a tie, as wq_quantize_dyadic), step = scale / 8 and scale the
+ * bf16 scale of the element's group (a trained parameter, so |z| may exceed it: the argmin
+ * then picks an end code). q is the code value itself, exact in fp32. The backward pass of
+ * the straight-through estimator is the identity (dL/dz = dL/dq) and needs no call.
+ *   z       fp32 [n, k]; k % group == 0 and k % 32 == 0.
+ *   group   64 or 32.
+ *   scale   bf16 [n, k/group], finite and >= 0 (other scales give unspecified codes).
+ *   q       out fp32 [n, k].
+ *   codes   out uint8 [n, k] (idx), or NULL.
+ *   packed  out uint8 [n, k/2] (idx nibbles, as wq_pack), or NULL.
+ * Bit-exact (codes, packed bytes and q). */
+wq_status wq_fake_quant_ste(const float* z, int64_t n, int64_t k, int32_t group,
+                            const uint16_t* scale, float* q, uint8_t* codes, uint8_t* packed,
+                            wq_stream stream);
+
 /* ------------------------------------------------------------------------------------ */
 /* W4A16 consumers                                                                       */
 /* ------------------------------------------------------------------------------------ */

@@ -13,7 +13,8 @@ def test_library_exports_every_header_function(wq):
                 "wq_quantize_lloyd", "wq_pack", "wq_unpack", "wq_dequant", "wq_gemv_w4a16",
                 "wq_gemv_w4a16_grouped", "wq_gemm_workspace_bytes", "wq_gemm_w4a16",
                 "wq_debug_fail_next_launches", "wq_device_error", "wq_gemm_w4a16_static",
-                "wq_gemv_plan_create", "wq_gemv_plan_launch", "wq_gemv_plan_destroy"}
+                "wq_gemv_plan_create", "wq_gemv_plan_launch", "wq_gemv_plan_destroy",
+                "wq_fake_quant_ste"}
     assert expected <= set(names), set(names) ^ expected
     for n in names:
         assert hasattr(wq._lib, n), n
@@ -49,6 +50,8 @@ def test_shape_and_group_checks_fail_before_any_cuda_call(wq):
     prm = wq.WqLloydParams(0, 100)
     assert lib.wq_quantize_lloyd(p, 4, 64, ctypes.byref(prm), p, p, p, None, None, None) == wq.WQ_EINVAL
     assert lib.wq_gemv_w4a16_grouped(None, None, None, 1, 1, None) == wq.WQ_EINVAL
+    assert lib.wq_fake_quant_ste(p, 4, 64, 16, p, p, None, None, None) == wq.WQ_EUNSUPPORTED
+    assert lib.wq_fake_quant_ste(p, 4, 96, 64, p, p, None, None, None) == wq.WQ_EINVAL
 
 
 def test_gemv_plan_rejects_bad_arguments_and_keeps_nothing(wq):

@@ -52,6 +52,7 @@ _SIG = {
     "wq_quantize_lloyd": ([_vp, _i64, _i64, ctypes.POINTER(WqLloydParams), _vp, _vp, _vp, _vp,
                            _vp, _vp], _i32),
     "wq_pack": ([_vp, _i64, _i64, _vp, _vp], _i32),
+    "wq_fake_quant_ste": ([_vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp], _i32),
     "wq_unpack": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "wq_dequant": ([_WP, _vp, _vp], _i32),
     "wq_gemv_w4a16": ([_WP, _vp, _i32, _vp, _vp], _i32),
@@ -160,6 +161,22 @@ def quantize_dyadic(w: torch.Tensor, group: int = 64, codes: bool = False, packe
     _check(_lib.wq_quantize_dyadic(_ptr(w), n, k, group, _ptr(scale), _ptr(c), _ptr(p), _stream(w)))
     pw = PackedWeight(FMT_DYADIC4, group, n, k, p, scale) if packed else None
     return pw, c
+
+
+def fake_quant_ste(z: torch.Tensor, scale: torch.Tensor, group: int = 64, codes: bool = False,
+                   packed: bool = False):
+    """STE forward on an fp32 latent z [n, k] with bf16 scales [n, k/group]: returns
+    (q fp32 [n, k], codes uint8 [n, k] | None, packed uint8 [n, k/2] | None). The backward of
+    the straight-through estimator is the identity."""
+    _cuda(z, torch.float32, "z")
+    _cuda(scale, torch.bfloat16, "scale")
+    n, k = z.shape
+    q = torch.empty_like(z)
+    c = torch.empty((n, k), dtype=torch.uint8, device=z.device) if codes else None
+    p = torch.empty((n, k // 2), dtype=torch.uint8, device=z.device) if packed else None
+    _check(_lib.wq_fake_quant_ste(_ptr(z), n, k, group, _ptr(scale), _ptr(q), _ptr(c), _ptr(p),
+                                  _stream(z)))
+    return q, c, p
 
 
 def quantize_lloyd(w: torch.Tensor, mode: int = LLOYD_G32_WARM, rounds: int = 25,

@@ -247,6 +247,23 @@ wq_status check_grouped(const wq_weight* ws, const uint16_t* const* xs, uint16_t
 
 extern "C" {
 
+wq_status wq_fake_quant_ste(const float* z, int64_t n, int64_t k, int32_t group,
+                            const uint16_t* scale, float* q, uint8_t* codes, uint8_t* packed,
+                            wq_stream stream) {
+    g_last_error[0] = 0;
+    if (group != 64 && group != 32)
+        return fail(WQ_EUNSUPPORTED, "fake quantisation group must be 64 or 32 (got %d)", group);
+    wq_status st = check_shape(n, k, group);
+    if (st) return st;
+    if ((st = check_ptr(z, "z", false))) return st;
+    if ((st = check_ptr(scale, "scale", false))) return st;
+    if ((st = check_ptr(q, "q", false))) return st;
+    if ((st = check_ptr(codes, "codes", true))) return st;
+    if ((st = check_ptr(packed, "packed", true))) return st;
+    if ((st = check_injected())) return st;
+    return launch_fake_quant_ste(z, n, k, group, scale, q, codes, packed, (cudaStream_t)stream);
+}
+
 wq_status wq_gemv_plan_create(const wq_weight* ws, const uint16_t* const* xs, uint16_t* const* ys,
                               int32_t count, int32_t batch, wq_gemv_plan* plan) {
     g_last_error[0] = 0;
