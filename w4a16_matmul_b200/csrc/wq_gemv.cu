@@ -229,6 +229,51 @@ __device__ __forceinline__ void load_step(Step<KIND, R>& st, const GemvProblem& 
         }
 }
 
+// This lane's weight and scale pointers at step 0, for the rows g and g + 8 of each 16-row
+// block (computed once per warp; a FULL dyadic step only adds its offset).
+template <int KIND, int R>
+struct LaneRows {
+    const uint8_t* w[R][2];
+    const uint16_t* sc[R][2];
+};
+
+template <int KIND, int R>
+__device__ __forceinline__ LaneRows<KIND, R> lane_rows(const GemvProblem& pb, int row0, int g, int t,
+                                                       int N, int K) {
+    LaneRows<KIND, R> lr;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int row = min(row0 + 16 * r + 8 * h + g, N - 1);   // only FULL steps use these
+            lr.w[r][h] = pb.packed + (size_t)row * (K / 2) + 32 * t;
+            lr.sc[r][h] = (const uint16_t*)pb.aux + (KIND == kDyadic32 ? (size_t)row * (K / 32) + 2 * t
+                                                                      : (size_t)row * (K / 64) + t);
+        }
+    return lr;
+}
+
+// A FULL dyadic step (every row and column in range) from the precomputed pointers.
+template <int KIND, int R>
+__device__ __forceinline__ void load_step_full(Step<KIND, R>& st, const LaneRows<KIND, R>& lr, int s) {
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint8_t* wp = lr.w[r][h] + 128 * s;
+            const uint4 a = ldg_w(wp), b = ldg_w(wp + 16);
+            st.w[r][h][0] = a.x; st.w[r][h][1] = a.y; st.w[r][h][2] = a.z; st.w[r][h][3] = a.w;
+            st.w[r][h][4] = b.x; st.w[r][h][5] = b.y; st.w[r][h][6] = b.z; st.w[r][h][7] = b.w;
+            if (KIND == kDyadic64) {
+                st.aux[r][h][0] = ldg_u16(lr.sc[r][h] + 4 * s);
+                st.aux[r][h][1] = st.aux[r][h][0];
+            } else {
+                st.aux[r][h][0] = ldg_u16(lr.sc[r][h] + 8 * s);
+                st.aux[r][h][1] = ldg_u16(lr.sc[r][h] + 8 * s + 1);
+            }
+        }
+}
+
 // One 256-column step from the staged activations: 8 words per row, 2 (or 4) mma per word
 // pair. xs0 / xs1: this lane's 16-byte slot of the step in the staged rows of batch
 // columns g and g + 8 (lanes of unused batch columns read some staged row; their outputs
@@ -509,8 +554,12 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     // FULL loads (all rows of the warp and all 256 columns in range) run without
     // predicates; only a ragged last step or a ragged last row block take the checks
     const int full_steps = (row0 + 16 * R <= N) ? (K >> 8) : 0;
+    // (16-row warps only: the pointers cost the 32-row kernel registers it does not have)
+    constexpr bool kFastLoad = KIND == kDyadic64 && R == 1;
+    const LaneRows<KIND, R> lr = lane_rows<KIND, R>(pb, row0, g, t, N, K);
     auto load = [&](Step<KIND, R>& st, int s) {
-        if (s < full_steps) load_step<KIND, R, true>(st, pb, row0, g, s * 256 + t * 64, N, K);
+        if (kFastLoad && s < full_steps) load_step_full<KIND, R>(st, lr, s);
+        else if (s < full_steps) load_step<KIND, R, true>(st, pb, row0, g, s * 256 + t * 64, N, K);
         else load_step<KIND, R, false>(st, pb, row0, g, s * 256 + t * 64, N, K);
     };
     auto run_step = [&](const Step<KIND, R>& st, int s, int c0, bool xbad) {
