@@ -419,6 +419,26 @@ def bench_gemm(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks):
             except Exception as e:
                 res[f"{n}x{k}_m{m}"] = {"error": repr(e)[:200]}
         del wdeq, pw
+    # the fused LLOYD8S consumer on the same GEMM (g32 codes plus fp32 levels; random codes
+    # and sorted levels: the timing does not depend on the values)
+    try:
+        n, k = workloads.PREFILL_SHAPES[0]
+        gen = torch.Generator(device=dev).manual_seed(5)
+        codes = torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=dev, generator=gen)
+        levels = torch.sort(torch.rand((n, k // 32, 8), device=dev, generator=gen) * 0.05, dim=-1).values
+        pl = wq.PackedWeight(wq.FMT_LLOYD8S, 32, n, k, codes, levels.contiguous())
+        for m in (512, 4096):
+            x = torch.randn((m, k), device=dev).to(torch.bfloat16)
+            y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(max(wq.gemm_workspace_bytes(pl, m), 16), dtype=torch.uint8, device=dev)
+            g = graph_of(torch, lambda: wq.gemm(pl, x, out=y, workspace=ws))
+            ms = max_over_ranks(time_region(torch, stream, g.replay, steps, warm, barrier))
+            fl = 2.0 * m * n * k
+            res[f"lloyd8s_{n}x{k}_m{m}"] = {"TFLOP/s": round(fl / ms / 1e9, 1), "us": round(ms * 1e3, 2),
+                                            "frac_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
+            del g
+    except Exception as e:
+        res["lloyd8s"] = {"error": repr(e)[:200]}
     return res
 
 

@@ -103,3 +103,41 @@ def test_gemm_one_hot_every_scale_regime(wq):
     x[np.arange(k), np.arange(k)] = 1.0
     y = f32(wq.gemm(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
     assert np.array_equal(y, wd.T)
+
+
+def _lloyd(wq, n, k, seed, signed_levels=False):
+    g = np.random.default_rng(seed)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    levels = np.sort(np.abs(g.standard_normal((n, k // 32, 8))) * 0.02, -1).astype(np.float32)
+    if signed_levels:
+        levels *= np.where(g.random(levels.shape) < 0.5, -1.0, 1.0).astype(np.float32)
+    packed = oracle.pack(codes)
+    pw = wq.PackedWeight(wq.FMT_LLOYD8S, 32, n, k, to_dev(packed), torch.from_numpy(levels).cuda())
+    return pw, packed, levels
+
+
+@pytest.mark.parametrize("m", [1, 8, 9, 48, 128, 200, 256, 300])
+@pytest.mark.parametrize("n,k", [(128, 256), (200, 320), (256, 1024)])
+def test_gemm_lloyd8s_matches_oracle(wq, m, n, k):
+    """The fused LLOYD8S consumer on the tensor-memory GEMM ("int4-g32+warm" §5.2): the
+    group's 8 levels arrive by TMA with each stage and are rebuilt into a bf16 codebook."""
+    if k % 64:
+        pytest.skip("the GEMM needs k % 64 == 0")
+    pw, packed, levels = _lloyd(wq, n, k, m * 3 + n + k)
+    x_bits = workloads.activations(m, k, workloads.PREFILL, n + m)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul_rows(oracle.LLOYD8S, packed, levels, 32, x_bits)
+    _check(y, y_ref, bound)
+    assert wq.device_error() == 0
+
+
+def test_gemm_lloyd8s_one_hot_exact(wq):
+    n, k = 256, 512
+    pw, packed, levels = _lloyd(wq, n, k, 17, signed_levels=True)
+    wd = oracle.bf16_to_f64(oracle.dequant(oracle.LLOYD8S, packed, levels, 32))
+    cols = np.arange(0, k, 3)
+    x = np.zeros((len(cols), k))
+    x[np.arange(len(cols)), cols] = 1.0
+    y = f32(wq.gemm(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
+    assert np.array_equal(y, wd[:, cols].T)

@@ -151,11 +151,12 @@ __device__ __forceinline__ uint4 dyadic_row8_f32(uint32_t w, float step) {
 // as 216 KB hold, up to 16. Tensor-memory slots (32 columns each, the reconstructed
 // weights of one stage) only need to cover reconstruction-to-MMA latency; for BN <= 64 the
 // allocation stays at 256 columns so that two CTAs can share an SM.
-template <int BN>
+template <int BN, bool LL = false>
 struct Smem {
     static constexpr int B_BYTES = BN * BK * 2;          // activation tile (128-byte swizzle)
     static constexpr int P_BYTES = BM * BK / 2;          // 4 KB packed weight tile
-    static constexpr int STAGE = B_BYTES + P_BYTES;      // a multiple of 1024
+    static constexpr int L_BYTES = LL ? BM * 64 : 0;     // LLOYD8S: the 2 groups' fp32 levels
+    static constexpr int STAGE = B_BYTES + P_BYTES + L_BYTES;   // a multiple of 1024
     static constexpr int STAGES = (216 * 1024 / STAGE) < 16 ? (216 * 1024 / STAGE) : 16;
     static constexpr int BARS = 2 * STAGES + 2 * 8 + 1;
     static constexpr int TOTAL = STAGES * STAGE + BARS * 8 + 16 + 1024;   // + alignment slack
@@ -229,12 +230,14 @@ __device__ __forceinline__ void tmem_st_part(uint32_t taddr, const uint32_t* v) 
     }
 }
 
-template <int BN, int G, bool PARTIAL>
+// LL: LLOYD8S weights (groups of 32, 8 fp32 levels each, loaded per stage by TMA through
+// tmap_l; `scale` unused); otherwise DYADIC4 with group G.
+template <int BN, int G, bool PARTIAL, bool LL>
 __global__ void __launch_bounds__(threads_for(BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
-            const uint16_t* __restrict__ scale, void* __restrict__ out, int M, int N, int K,
-            int kt_per_split) {
-    using S = Smem<BN>;
+            const __grid_constant__ CUtensorMap tmap_l, const uint16_t* __restrict__ scale,
+            void* __restrict__ out, int M, int N, int K, int kt_per_split) {
+    using S = Smem<BN, LL>;
     constexpr int STAGES = S::STAGES;
     constexpr int RW = rw_for(BN);
     extern __shared__ uint8_t smem_raw[];
@@ -281,6 +284,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 
     auto stage_b = [&](int s) { return smem + s * S::STAGE; };
     auto stage_p = [&](int s) { return smem + s * S::STAGE + S::B_BYTES; };
+    auto stage_l = [&](int s) { return smem + s * S::STAGE + S::B_BYTES + S::P_BYTES; };
     auto dead = [&](int code) {
         *(volatile int*)s_abort = 1;
         atomicCAS(&g_device_error, 0, code);
@@ -293,10 +297,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             uint32_t ph = 0;
             for (int i = 0; i < nk; ++i, s = (s + 1 == STAGES) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!mbar_wait(&empty[s], ph ^ 1, s_abort)) { dead(1); break; }
-                mbar_expect_tx(&full_tma[s], S::B_BYTES + S::P_BYTES);
+                mbar_expect_tx(&full_tma[s], S::B_BYTES + S::P_BYTES + S::L_BYTES);
                 const int kt = kt0 + i;
                 tma_load_2d(stage_b(s), &tmap_x, kt * BK, m0, &full_tma[s]);
                 tma_load_2d(stage_p(s), &tmap_p, kt * (BK / 2), n0, &full_tma[s]);
+                if (LL) tma_load_2d(stage_l(s), &tmap_l, kt * 16, n0, &full_tma[s]);
             }
         }
     } else if (warp == 1) {
@@ -342,7 +347,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 #pragma unroll
         for (int u = 0; u < kPre; ++u) {
             ring0[u] = ring1[u] = 0;
-            if (row_ok && u < nk) {
+            if (!LL && row_ok && u < nk) {
                 ring0[u] = ldg_u16(srow + (kt0 + u) * BK / G);
                 ring1[u] = (G == 32) ? ldg_u16(srow + (kt0 + u) * BK / G + 1) : ring0[u];
             }
@@ -356,7 +361,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 const int it = base + u;
                 if (it >= nk) break;
                 const uint32_t sc0 = ring0[u], sc1 = ring1[u];
-                if (row_ok && it + kPre < nk) {
+                if (!LL && row_ok && it + kPre < nk) {
                     ring0[u] = ldg_u16(srow + (kt0 + it + kPre) * BK / G);
                     ring1[u] = (G == 32) ? ldg_u16(srow + (kt0 + it + kPre) * BK / G + 1) : ring0[u];
                 }
@@ -383,17 +388,41 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                         wv[0] = t2.x; wv[1] = t2.y;
                     }
                 }
-                const bool huge = ((sc0 & 0x7FFFu) >= 0x7D80u) || ((sc1 & 0x7FFFu) >= 0x7D80u);
-                const uint32_t s20 = prmt(sc0, 0, 0x1010u), s21 = prmt(sc1, 0, 0x1010u);
-                const uint32_t cs0 = bf16x2_fma(s20, 0x41804180u, 0x80008000u), cn0 = s20 ^ 0x80008000u;
-                const uint32_t cs1 = bf16x2_fma(s21, 0x41804180u, 0x80008000u), cn1 = s21 ^ 0x80008000u;
                 uint32_t v[4 * WPT];
+                if constexpr (LL) {
+                    // bf16(level) byte planes of the group(s) this thread's words lie in
+                    // (words 0-3: group 0, 4-7: group 1), then one permute per plane and a
+                    // sign flip per code, as the GEMV's register codebook does
+                    constexpr int NG = WPT > 4 ? 2 : 1;
+                    uint32_t plo[NG][2], phi[NG][2];
 #pragma unroll
-                for (int c = 0; c < WPT; ++c) {
-                    const bool second = (G == 32) && (part * WPT + c) >= 4;
-                    const uint4 r = huge ? dyadic_row8_f32(wv[c], bf16_bits_to_float(second ? sc1 : sc0) * 0.125f)
-                                         : dyadic_row8(wv[c], second ? cs1 : cs0, second ? cn1 : cn0);
-                    v[4 * c] = r.x; v[4 * c + 1] = r.y; v[4 * c + 2] = r.z; v[4 * c + 3] = r.w;
+                    for (int gi = 0; gi < NG; ++gi) {
+                        const int grp = NG == 2 ? gi : (part * WPT) >> 2;
+                        const float4* lv = (const float4*)(stage_l(s) + i * 64 + grp * 32);
+                        const float4 l0 = lv[0], l1 = lv[1];
+                        const uint32_t b01 = pack_bf16x2(l0.x, l0.y), b23 = pack_bf16x2(l0.z, l0.w);
+                        const uint32_t b45 = pack_bf16x2(l1.x, l1.y), b67 = pack_bf16x2(l1.z, l1.w);
+                        plo[gi][0] = prmt(b01, b23, 0x6420u); plo[gi][1] = prmt(b45, b67, 0x6420u);
+                        phi[gi][0] = prmt(b01, b23, 0x7531u); phi[gi][1] = prmt(b45, b67, 0x7531u);
+                    }
+#pragma unroll
+                    for (int c = 0; c < WPT; ++c) {
+                        const int gi = NG == 2 ? (c >> 2) : 0;
+                        lloyd8_lookup4(wv[c], plo[gi], phi[gi], v[4 * c], v[4 * c + 1]);
+                        lloyd8_lookup4(wv[c] >> 16, plo[gi], phi[gi], v[4 * c + 2], v[4 * c + 3]);
+                    }
+                } else {
+                    const bool huge = ((sc0 & 0x7FFFu) >= 0x7D80u) || ((sc1 & 0x7FFFu) >= 0x7D80u);
+                    const uint32_t s20 = prmt(sc0, 0, 0x1010u), s21 = prmt(sc1, 0, 0x1010u);
+                    const uint32_t cs0 = bf16x2_fma(s20, 0x41804180u, 0x80008000u), cn0 = s20 ^ 0x80008000u;
+                    const uint32_t cs1 = bf16x2_fma(s21, 0x41804180u, 0x80008000u), cn1 = s21 ^ 0x80008000u;
+#pragma unroll
+                    for (int c = 0; c < WPT; ++c) {
+                        const bool second = (G == 32) && (part * WPT + c) >= 4;
+                        const uint4 r = huge ? dyadic_row8_f32(wv[c], bf16_bits_to_float(second ? sc1 : sc0) * 0.125f)
+                                             : dyadic_row8(wv[c], second ? cs1 : cs0, second ? cn1 : cn0);
+                        v[4 * c] = r.x; v[4 * c + 1] = r.y; v[4 * c + 2] = r.z; v[4 * c + 3] = r.w;
+                    }
                 }
                 // the previous iteration's store has had this iteration's loads and arithmetic
                 // to complete: wait for it now and release that slot to the MMA, then issue
@@ -527,24 +556,24 @@ Plan plan_for(int64_t M, int64_t N, int64_t K) {
     return p;
 }
 
-template <int BN, int G>
-wq_status launch_bn(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp, const uint16_t* scale,
-                    void* out, int M, int N, int K, cudaStream_t s) {
-    const int smem = Smem<BN>::TOTAL;
+template <int BN, int G, bool LL>
+wq_status launch_bn(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMap& tl,
+                    const uint16_t* scale, void* out, int M, int N, int K, cudaStream_t s) {
+    const int smem = Smem<BN, LL>::TOTAL;
     const dim3 grid(p.grid_n, p.grid_m, p.splits);
     // the shared-memory opt-in is set once per kernel variant (a function attribute holds
     // for the process; the flags are per variant and only ever go from false to true)
     static bool raised[2] = {false, false};
     if (p.splits > 1) {
-        auto k = gemm_kernel<BN, G, true>;
+        auto k = gemm_kernel<BN, G, true, LL>;
         if (!raised[1] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[1] = true;
-        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, scale, out, M, N, K, p.kt_per_split);
+        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, p.kt_per_split);
     } else {
-        auto k = gemm_kernel<BN, G, false>;
+        auto k = gemm_kernel<BN, G, false, LL>;
         if (!raised[0] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[0] = true;
-        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, scale, out, M, N, K, p.kt_per_split);
+        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, p.kt_per_split);
     }
     return check_launch("gemm");
 }
@@ -596,14 +625,27 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(WQ_ECUDA, "tensor map for packed weights failed (%d)", (int)r);
     }
+    CUtensorMap tl = tp;                   // unused by DYADIC4 launches
+    if (w.fmt == WQ_FMT_LLOYD8S) {
+        // levels [N, K/32, 8] fp32 as a 2D [N, K/4] array; a stage's 2 groups are 16 floats
+        cuuint64_t dims[2] = {(cuuint64_t)K / 4, (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)K};
+        cuuint32_t box[2] = {16, (cuuint32_t)BM};
+        cuuint32_t es[2] = {1, 1};
+        CUresult r = enc(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void*)w.aux, dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(WQ_ECUDA, "tensor map for LLOYD8S levels failed (%d)", (int)r);
+    }
     void* out = p.splits > 1 ? ws : (void*)y;
     if (p.splits > 1 && (ws == nullptr || ws_bytes < gemm_workspace_bytes(w, m)))
         return fail(WQ_EINVAL, "workspace too small");
     const uint16_t* sc = (const uint16_t*)w.aux;
     wq_status st;
 #define WQ_BN(BNV)                                                                                  \
-    st = (w.group == 64) ? launch_bn<BNV, 64>(p, tx, tp, sc, out, M, N, K, s)                     \
-                         : launch_bn<BNV, 32>(p, tx, tp, sc, out, M, N, K, s)
+    st = (w.fmt == WQ_FMT_LLOYD8S) ? launch_bn<BNV, 32, true>(p, tx, tp, tl, sc, out, M, N, K, s)    \
+       : (w.group == 64)           ? launch_bn<BNV, 64, false>(p, tx, tp, tl, sc, out, M, N, K, s)   \
+                                   : launch_bn<BNV, 32, false>(p, tx, tp, tl, sc, out, M, N, K, s)
     switch (p.bn) {
         case 16: WQ_BN(16); break;
         case 32: WQ_BN(32); break;

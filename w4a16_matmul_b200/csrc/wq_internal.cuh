@@ -149,6 +149,21 @@ __device__ __forceinline__ uint32_t ldg_u16(const void* p) {
     return v;
 }
 
+// LLOYD8S lookup of 4 codes (nibbles of the low 16 bits of s; code = level index q in bits
+// 0-2, sign in bit 3) in an 8-entry bf16 table of one group held as byte planes: lo[0..1] /
+// hi[0..1] hold the low / high bytes of bf16(level[0..7]). The sign bit of each code flips
+// the sign bit of the high byte (bf16(-v) = -bf16(v): rounding to nearest even is
+// symmetric). Returns the bf16 pairs (code0, code1) and (code2, code3).
+__device__ __forceinline__ void lloyd8_lookup4(uint32_t s, const uint32_t* lo, const uint32_t* hi,
+                                               uint32_t& p01, uint32_t& p23) {
+    const uint32_t s7 = s & 0x7777u;                                     // level index
+    const uint32_t sg = prmt(0x00000000u, 0x80808080u, (s >> 1) & 0x4444u);   // 0x80 where signed
+    const uint32_t l = prmt(lo[0], lo[1], s7);
+    const uint32_t h = prmt(hi[0], hi[1], s7) ^ sg;
+    p01 = prmt(l, h, 0x5140u);
+    p23 = prmt(l, h, 0x7362u);
+}
+
 // D += A * B on the legacy warp-level tensor-core path, m16n8k16, bf16 in, fp32 accumulate.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
