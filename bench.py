@@ -180,6 +180,24 @@ def time_region(torch, stream, fn, steps, warmup, barrier):
     return t0.elapsed_time(t1) / steps
 
 
+def max_over_ranks_fn(torch, dist, world: int, device):
+    """The timing reduction every multi-GPU number goes through: the max of a per-rank value
+    over all ranks (an all-reduce on `device`: the GPU under NCCL, the CPU under gloo)."""
+    def reduce(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return reduce
+
+
+def replica_value(world: int, bytes_per_rank: int, max_ms: float) -> float:
+    """Weak scaling over independent replicas: every rank streams the same per-rank bytes, and
+    the whole job's rate is all ranks' bytes over the slowest rank's time (GB/s)."""
+    return world * bytes_per_rank / (max_ms * 1e-3) / 1e9
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -203,12 +221,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    max_over_ranks = max_over_ranks_fn(torch, dist, world, dev)
 
     B = args.batch
     mats, packed, xs_host, xs, ys, xflat, yflat = build_sweep(wq, torch, dev, B)
@@ -231,7 +244,7 @@ def run_ours(args):
     ms = time_region(torch, stream, graph.replay, args.steps, args.warmup, barrier)
     clk = clocks.stop()
     ms = max_over_ranks(ms)
-    value = world * weight_bytes / (ms * 1e-3) / 1e9
+    value = replica_value(world, weight_bytes, ms)
     achieved = algo_bytes / (ms * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers ---------------------------
@@ -244,7 +257,7 @@ def run_ours(args):
         y_pin.copy_(yflat, non_blocking=True)       # this step's outputs, device -> host
 
     ms_e2e = max_over_ranks(time_region(torch, stream, e2e_step, args.steps, args.warmup, barrier))
-    e2e = {"value": round(world * weight_bytes / (ms_e2e * 1e-3) / 1e9, 2), "unit": UNIT,
+    e2e = {"value": round(replica_value(world, weight_bytes, ms_e2e), 2), "unit": UNIT,
            "h2d_bytes_per_step": x_b, "d2h_bytes_per_step": y_b, "ms_per_step": round(ms_e2e, 4)}
 
     extras = {}
