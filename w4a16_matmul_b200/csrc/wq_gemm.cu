@@ -38,7 +38,8 @@ __device__ int g_device_error;     // 0, or the code of the first expired device
 namespace {
 
 constexpr int BM = 128;            // weight rows per CTA (MMA M)
-constexpr int BK = 64;             // columns per stage: one 128-byte swizzle row of bf16
+// Columns per stage, KB: 64 (one 128-byte swizzle row of bf16) or 128 (two such tiles, used
+// when K % 128 == 0: twice the reconstruction work per stage for the same bookkeeping).
 constexpr uint64_t kWaitNs = 2000000000ull;   // a wait longer than 2 s is declared dead
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -151,11 +152,11 @@ __device__ __forceinline__ uint4 dyadic_row8_f32(uint32_t w, float step) {
 // as 216 KB hold, up to 16. Tensor-memory slots (32 columns each, the reconstructed
 // weights of one stage) only need to cover reconstruction-to-MMA latency; for BN <= 64 the
 // allocation stays at 256 columns so that two CTAs can share an SM.
-template <int BN, bool LL = false>
+template <int BN, bool LL = false, int KB = 64>
 struct Smem {
-    static constexpr int B_BYTES = BN * BK * 2;          // activation tile (128-byte swizzle)
-    static constexpr int P_BYTES = BM * BK / 2;          // 4 KB packed weight tile
-    static constexpr int L_BYTES = LL ? BM * 64 : 0;     // LLOYD8S: the 2 groups' fp32 levels
+    static constexpr int B_BYTES = BN * KB * 2;          // KB/64 activation tiles (128-byte swizzle)
+    static constexpr int P_BYTES = BM * KB / 2;          // packed weight tile
+    static constexpr int L_BYTES = LL ? BM * KB : 0;     // LLOYD8S: the stage's groups' fp32 levels
     static constexpr int STAGE = B_BYTES + P_BYTES + L_BYTES;   // a multiple of 1024
     static constexpr int STAGES = (216 * 1024 / STAGE) < 16 ? (216 * 1024 / STAGE) : 16;
     static constexpr int BARS = 2 * STAGES + 2 * 8 + 1;
@@ -164,12 +165,15 @@ struct Smem {
     // slots for reconstructed bf16 weight tiles (64 values of a row per lane, two per 32-bit
     // column, lower k in the low half)
     static constexpr uint32_t ACC_COLS = BN < 32 ? 32 : BN;
-    // BN >= 128: one slot per stage (the rings coincide, and the producer's wait for a free
-    // stage already orders slot reuse); BN <= 64: six slots under a 16-stage ring
-    static constexpr int SLOTS = BN <= 64 ? (int)((256 - ACC_COLS) / 32 < 6 ? (256 - ACC_COLS) / 32 : 6)
-                                          : (WQ_GEMM_BIG_SLOTS ? 8 : (STAGES < 8 ? STAGES : 8));
+    static constexpr int SLOT_COLS = KB / 2;              // bf16 pairs of one stage's row
+    // BN >= 128: one slot per stage where tensor memory holds them (the rings coincide, and
+    // the producer's wait for a free stage already orders slot reuse); BN <= 64: up to six
+    // slots under a deep ring, within 256 columns
+    static constexpr int NARROW_SLOTS = (int)((256 - ACC_COLS) / SLOT_COLS) < 6 ? (int)((256 - ACC_COLS) / SLOT_COLS) : 6;
+    static constexpr int WIDE_FIT = (int)((512 - ACC_COLS) / SLOT_COLS) < 8 ? (int)((512 - ACC_COLS) / SLOT_COLS) : 8;
+    static constexpr int SLOTS = BN <= 64 ? NARROW_SLOTS : (STAGES < WIDE_FIT ? STAGES : WIDE_FIT);
     static constexpr bool COUPLED = SLOTS == STAGES;
-    static constexpr uint32_t USED_COLS = ACC_COLS + 32 * SLOTS;
+    static constexpr uint32_t USED_COLS = ACC_COLS + SLOT_COLS * SLOTS;
     static constexpr uint32_t TMEM_COLS = USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
                                         : USED_COLS <= 256 ? 256 : 512;
 };
@@ -203,17 +207,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 #define WQ_GEMM_RW_NARROW 2
 #endif
 // Reconstruction warps per tensor-memory lane group: RW warps share each 32-lane group, each
-// filling 8 / RW of the row's eight packed words per stage (more warps hide more latency;
-// fewer repeat less per-stage bookkeeping).
+// filling 1 / RW of the row's packed words per stage (more warps hide more latency; fewer
+// repeat less per-stage bookkeeping).
 constexpr int rw_for(int bn) { return bn >= 128 ? WQ_GEMM_RW : WQ_GEMM_RW_NARROW; }
 constexpr int threads_for(int bn) { return 64 + 128 * rw_for(bn); }
 
-// Stores 32 / RW consecutive 32-bit columns of this thread's tensor-memory lane.
-template <int RW>
+// Stores NC (8, 16 or 32) consecutive 32-bit columns of this thread's tensor-memory lane.
+template <int NC>
 __device__ __forceinline__ void tmem_st_part(uint32_t taddr, const uint32_t* v) {
-    if constexpr (RW == 1) {
+    static_assert(NC == 8 || NC == 16 || NC == 32, "8, 16 or 32 columns");
+    if constexpr (NC == 32) {
         tmem_st32(taddr, *reinterpret_cast<const uint32_t(*)[32]>(v));
-    } else if constexpr (RW == 2) {
+    } else if constexpr (NC == 16) {
         asm volatile(
             "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
             "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
@@ -232,12 +237,12 @@ __device__ __forceinline__ void tmem_st_part(uint32_t taddr, const uint32_t* v) 
 
 // LL: LLOYD8S weights (groups of 32, 8 fp32 levels each, loaded per stage by TMA through
 // tmap_l; `scale` unused); otherwise DYADIC4 with group G.
-template <int BN, int G, bool PARTIAL, bool LL>
+template <int BN, int G, bool PARTIAL, bool LL, int KB>
 __global__ void __launch_bounds__(threads_for(BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
             const __grid_constant__ CUtensorMap tmap_l, const uint16_t* __restrict__ scale,
             void* __restrict__ out, int M, int N, int K, int kt_per_split) {
-    using S = Smem<BN, LL>;
+    using S = Smem<BN, LL, KB>;
     constexpr int STAGES = S::STAGES;
     constexpr int RW = rw_for(BN);
     extern __shared__ uint8_t smem_raw[];
@@ -253,7 +258,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * BM, m0 = blockIdx.y * BN;
-    const int KT = K / BK;
+    const int KT = K / KB;
     const int kt0 = blockIdx.z * kt_per_split;
     const int kt1 = min(KT, kt0 + kt_per_split);
     const int nk = kt1 - kt0;
@@ -299,9 +304,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 if (!mbar_wait(&empty[s], ph ^ 1, s_abort)) { dead(1); break; }
                 mbar_expect_tx(&full_tma[s], S::B_BYTES + S::P_BYTES + S::L_BYTES);
                 const int kt = kt0 + i;
-                tma_load_2d(stage_b(s), &tmap_x, kt * BK, m0, &full_tma[s]);
-                tma_load_2d(stage_p(s), &tmap_p, kt * (BK / 2), n0, &full_tma[s]);
-                if (LL) tma_load_2d(stage_l(s), &tmap_l, kt * 16, n0, &full_tma[s]);
+#pragma unroll
+                for (int j = 0; j < KB / 64; ++j)
+                    tma_load_2d(stage_b(s) + j * BN * 128, &tmap_x, kt * KB + 64 * j, m0, &full_tma[s]);
+                tma_load_2d(stage_p(s), &tmap_p, kt * (KB / 2), n0, &full_tma[s]);
+                if (LL) tma_load_2d(stage_l(s), &tmap_l, kt * (KB / 4), n0, &full_tma[s]);
             }
         }
     } else if (warp == 1) {
@@ -315,11 +322,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 // the slot is reconstructed, which also means the stage's tiles have landed
                 if (!mbar_wait(&full_w[a], aph, s_abort)) { dead(2); break; }
                 asm volatile("tcgen05.fence::after_thread_sync;");
-                const uint64_t db = sw128_desc(smem_u32(stage_b(s)));
-                const uint32_t ta = tmem + S::ACC_COLS + 32u * (uint32_t)a;
+                const uint32_t ta = tmem + S::ACC_COLS + (uint32_t)(S::SLOT_COLS * a);
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)   // 16 values of K: 8 A columns, +2 in B descriptor units
-                    umma_f16_ts(tmem, ta + 8u * (uint32_t)k, db + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
+                for (int k = 0; k < KB / 16; ++k) {  // 16 values of K: 8 A columns, +2 in B descriptor units
+                    const uint64_t db = sw128_desc(smem_u32(stage_b(s) + (k / 4) * BN * 128));
+                    umma_f16_ts(tmem, ta + 8u * (uint32_t)k, db + 2 * (k % 4), idesc, (i > 0 || k > 0) ? 1u : 0u);
+                }
                 umma_commit(&empty[s]);           // fire once these MMAs have read the stage ...
                 if constexpr (!S::COUPLED) umma_commit(&slot_free[a]);   // ... and the slot
                 if (++s == STAGES) s = 0;
@@ -333,23 +341,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         // ---------------- reconstruction into tensor memory, then epilogue ----------------
         // a warp may touch only the tensor-memory lanes 32 * (warp % 4) .. + 31: thread
         // (warp, lane) owns weight row 32 * (warp % 4) + lane of the tile, and of that row's
-        // eight packed words per stage the words [part * WPT, part * WPT + WPT)
-        constexpr int WPT = 8 / RW;
+        // KB / 8 packed words per stage the words [part * WPT, part * WPT + WPT), columns
+        // colbase .. colbase + 8 WPT - 1 of the stage
+        constexpr int WPT = (KB / 8) / RW;
+        // a thread's columns span one group, or two g32 groups (then aligned to them)
+        constexpr bool SPAN2 = !LL && WPT * 8 > G;
+        static_assert(WPT * 8 <= 2 * G || LL, "at most two scale groups per thread and stage");
         const int q = warp & 3, part = (warp - 2) >> 2;
+        const int colbase = part * WPT * 8;
         const int i = 32 * q + lane;
         const int n = n0 + i;
         const bool row_ok = n < N;
-        const uint16_t* srow = scale + (size_t)(row_ok ? n : 0) * (K / G);
+        const uint16_t* srow = scale + (size_t)(row_ok ? n : 0) * (K / G) + colbase / G;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        // the per-group scales of this row, loaded kPre stages ahead (a ring of registers)
+        // the scales of this thread's group(s), loaded kPre stages ahead (a ring of registers)
         constexpr int kPre = 4;
         uint32_t ring0[kPre], ring1[kPre];
 #pragma unroll
         for (int u = 0; u < kPre; ++u) {
             ring0[u] = ring1[u] = 0;
             if (!LL && row_ok && u < nk) {
-                ring0[u] = ldg_u16(srow + (kt0 + u) * BK / G);
-                ring1[u] = (G == 32) ? ldg_u16(srow + (kt0 + u) * BK / G + 1) : ring0[u];
+                ring0[u] = ldg_u16(srow + (kt0 + u) * (KB / G));
+                ring1[u] = SPAN2 ? ldg_u16(srow + (kt0 + u) * (KB / G) + 1) : ring0[u];
             }
         }
         bool live = true;
@@ -362,8 +375,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 if (it >= nk) break;
                 const uint32_t sc0 = ring0[u], sc1 = ring1[u];
                 if (!LL && row_ok && it + kPre < nk) {
-                    ring0[u] = ldg_u16(srow + (kt0 + it + kPre) * BK / G);
-                    ring1[u] = (G == 32) ? ldg_u16(srow + (kt0 + it + kPre) * BK / G + 1) : ring0[u];
+                    ring0[u] = ldg_u16(srow + (kt0 + it + kPre) * (KB / G));
+                    ring1[u] = SPAN2 ? ldg_u16(srow + (kt0 + it + kPre) * (KB / G) + 1) : ring0[u];
                 }
                 // the packed tile has landed, and the MMAs that last read this tensor-memory
                 // slot (iteration it - SLOTS) have completed (with coupled rings the first
@@ -376,7 +389,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 }
                 uint32_t wv[WPT];
                 {
-                    const uint32_t* pk = (const uint32_t*)(stage_p(s) + i * 32 + part * WPT * 4);
+                    const uint32_t* pk = (const uint32_t*)(stage_p(s) + i * (KB / 2) + colbase / 2);
                     if constexpr (WPT >= 4) {
 #pragma unroll
                         for (int c = 0; c < WPT; c += 4) {
@@ -390,15 +403,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 }
                 uint32_t v[4 * WPT];
                 if constexpr (LL) {
-                    // bf16(level) byte planes of the group(s) this thread's words lie in
-                    // (words 0-3: group 0, 4-7: group 1), then one permute per plane and a
-                    // sign flip per code, as the GEMV's register codebook does
-                    constexpr int NG = WPT > 4 ? 2 : 1;
+                    // bf16(level) byte planes of the group(s) this thread's words lie in (4
+                    // words per group of 32), then one permute per plane and a sign flip per
+                    // code, as the GEMV's register codebook does
+                    constexpr int NG = (WPT + 3) / 4;
                     uint32_t plo[NG][2], phi[NG][2];
 #pragma unroll
                     for (int gi = 0; gi < NG; ++gi) {
-                        const int grp = NG == 2 ? gi : (part * WPT) >> 2;
-                        const float4* lv = (const float4*)(stage_l(s) + i * 64 + grp * 32);
+                        const int grp = colbase / 32 + gi;
+                        const float4* lv = (const float4*)(stage_l(s) + i * KB + grp * 32);
                         const float4 l0 = lv[0], l1 = lv[1];
                         const uint32_t b01 = pack_bf16x2(l0.x, l0.y), b23 = pack_bf16x2(l0.z, l0.w);
                         const uint32_t b45 = pack_bf16x2(l1.x, l1.y), b67 = pack_bf16x2(l1.z, l1.w);
@@ -407,7 +420,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     }
 #pragma unroll
                     for (int c = 0; c < WPT; ++c) {
-                        const int gi = NG == 2 ? (c >> 2) : 0;
+                        const int gi = c >> 2;
                         lloyd8_lookup4(wv[c], plo[gi], phi[gi], v[4 * c], v[4 * c + 1]);
                         lloyd8_lookup4(wv[c] >> 16, plo[gi], phi[gi], v[4 * c + 2], v[4 * c + 3]);
                     }
@@ -418,7 +431,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     const uint32_t cs1 = bf16x2_fma(s21, 0x41804180u, 0x80008000u), cn1 = s21 ^ 0x80008000u;
 #pragma unroll
                     for (int c = 0; c < WPT; ++c) {
-                        const bool second = (G == 32) && (part * WPT + c) >= 4;
+                        const bool second = SPAN2 && 8 * c >= G;
                         const uint4 r = huge ? dyadic_row8_f32(wv[c], bf16_bits_to_float(second ? sc1 : sc0) * 0.125f)
                                              : dyadic_row8(wv[c], second ? cs1 : cs0, second ? cn1 : cn0);
                         v[4 * c] = r.x; v[4 * c + 1] = r.y; v[4 * c + 2] = r.z; v[4 * c + 3] = r.w;
@@ -433,7 +446,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&full_w[a == 0 ? SLOTS - 1 : a - 1]);
                 }
-                tmem_st_part<RW>(lane_base + S::ACC_COLS + 32u * (uint32_t)a + (uint32_t)(part * 4 * WPT), v);
+                tmem_st_part<4 * WPT>(lane_base + S::ACC_COLS + (uint32_t)(S::SLOT_COLS * a + 4 * WPT * part), v);
                 if (++s == STAGES) { s = 0; ph ^= 1; }
                 if (++a == SLOTS) { a = 0; aph ^= 1; }
             }
@@ -517,37 +530,49 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 struct Plan {
-    int bn, splits, kt_per_split, grid_n, grid_m;
+    int bn, kb, splits, kt_per_split, grid_n, grid_m;
 };
 
-Plan plan_for(int64_t M, int64_t N, int64_t K) {
+#ifndef WQ_GEMM_KB128
+#define WQ_GEMM_KB128 1
+#endif
+
+Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt) {
     Plan p;
     const int sms = sm_count();
+    p.kb = 64;
     p.grid_n = (int)((N + BM - 1) / BM);
     // The widest activation tile the MMA takes once m allows it: every activation-row tile
     // reconstructs the same weights again, and reconstruction (not the tensor pipe) is what
     // narrower tiles run out of (measured: BN 128 / 192 at 0.5-0.9x of BN 256 throughput even
     // where they leave fewer SMs idle in the last wave).
     p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    // 128-column stages for 128-wide activation tiles where K allows: there they halve the
+    // per-stage bookkeeping of the reconstruction, which this m is bound by (measured 1.4x at
+    // m = 128); the 256-wide tiles keep 64-column stages, whose finer ring overlaps better
+    // (measured 1.1x), and LLOYD8S keeps 64 (its level tiles would double too)
+    if (WQ_GEMM_KB128 && p.bn == 128 && K % 128 == 0 && fmt != WQ_FMT_LLOYD8S) p.kb = 128;
     p.grid_m = (int)((M + p.bn - 1) / p.bn);
-    const int KT = (int)(K / BK);
+    const int KT = (int)(K / p.kb);
     const int64_t tiles = (int64_t)p.grid_n * p.grid_m;
+    const int min_wide = 1024 / p.kb, min_narrow = 512 / p.kb;   // stages per split, at least
     int splits = 1;
     if (p.bn >= 128) {
         // wide tiles (one CTA per SM): split in powers of two while the grid stays within
-        // one round and every split keeps >= 16 stages
-        while (tiles * splits * 2 <= sms && KT / (splits * 2) >= 16) splits *= 2;
+        // one round and every split keeps >= 1024 columns
+        while (tiles * splits * 2 <= sms && KT / (splits * 2) >= min_wide) splits *= 2;
     } else {
         // narrow tiles (256 tensor-memory columns, at most ~100 KB of shared memory) fit two
         // CTAs per SM. A grid of equal CTAs takes ceil(CTAs / slots) rounds of (stages per
-        // CTA + about 4 stages of prologue and epilogue); take the split count with the
-        // fewest, keeping >= 8 stages per split
+        // CTA + a prologue and epilogue of about 256 columns' worth); take the split count
+        // with the fewest, keeping >= 512 columns per split
         const int64_t slots = 2 * (int64_t)sms;
+        const int64_t fixed = 256 / p.kb;
         int64_t best = -1;
-        for (int sp = 1; sp <= 32 && (sp == 1 || KT / sp >= 8); ++sp) {
+        for (int sp = 1; sp <= 32 && (sp == 1 || KT / sp >= min_narrow); ++sp) {
             const int64_t per = (KT + sp - 1) / sp;
             const int64_t used = (KT + per - 1) / per;           // splits that get work
-            const int64_t cost = ((tiles * used + slots - 1) / slots) * (per + 4);
+            const int64_t cost = ((tiles * used + slots - 1) / slots) * (per + fixed);
             if (best < 0 || cost < best) { best = cost; splits = (int)used; }
         }
     }
@@ -556,21 +581,21 @@ Plan plan_for(int64_t M, int64_t N, int64_t K) {
     return p;
 }
 
-template <int BN, int G, bool LL>
+template <int BN, int G, bool LL, int KB>
 wq_status launch_bn(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMap& tl,
                     const uint16_t* scale, void* out, int M, int N, int K, cudaStream_t s) {
-    const int smem = Smem<BN, LL>::TOTAL;
+    const int smem = Smem<BN, LL, KB>::TOTAL;
     const dim3 grid(p.grid_n, p.grid_m, p.splits);
     // the shared-memory opt-in is set once per kernel variant (a function attribute holds
     // for the process; the flags are per variant and only ever go from false to true)
     static bool raised[2] = {false, false};
     if (p.splits > 1) {
-        auto k = gemm_kernel<BN, G, true, LL>;
+        auto k = gemm_kernel<BN, G, true, LL, KB>;
         if (!raised[1] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[1] = true;
         k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, p.kt_per_split);
     } else {
-        auto k = gemm_kernel<BN, G, false, LL>;
+        auto k = gemm_kernel<BN, G, false, LL, KB>;
         if (!raised[0] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[0] = true;
         k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, p.kt_per_split);
@@ -590,7 +615,7 @@ constexpr int64_t kGemvMaxRows = 8;
 
 size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
     if (m <= kGemvMaxRows) return 0;
-    const Plan p = plan_for(m, w.n, w.k);
+    const Plan p = plan_for(m, w.n, w.k, w.fmt);
     return p.splits > 1 ? (size_t)p.splits * (size_t)m * (size_t)w.n * sizeof(float) : 0;
 }
 
@@ -601,14 +626,14 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
         const GemvProblem prob{w.packed, w.aux, x, y, N, K};
         return launch_gemv(w.fmt, w.group, &prob, 1, M, s);
     }
-    const Plan p = plan_for(M, N, K);
+    const Plan p = plan_for(M, N, K, w.fmt);
     auto enc = encode_fn();
     if (!enc) return fail(WQ_ECUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
     CUtensorMap tx, tp;
     {
         cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
         cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)p.bn};
+        cuuint32_t box[2] = {64, (cuuint32_t)p.bn};        // one 128-byte swizzle row wide
         cuuint32_t es[2] = {1, 1};
         CUresult r = enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)x, dims, strides, box, es,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -618,7 +643,7 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
     {
         cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)N};
         cuuint64_t strides[1] = {(cuuint64_t)K / 2};
-        cuuint32_t box[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)BM};
+        cuuint32_t box[2] = {(cuuint32_t)(p.kb / 2), (cuuint32_t)BM};
         cuuint32_t es[2] = {1, 1};
         CUresult r = enc(&tp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)w.packed, dims, strides, box, es,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -630,7 +655,7 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
         // levels [N, K/32, 8] fp32 as a 2D [N, K/4] array; a stage's 2 groups are 16 floats
         cuuint64_t dims[2] = {(cuuint64_t)K / 4, (cuuint64_t)N};
         cuuint64_t strides[1] = {(cuuint64_t)K};
-        cuuint32_t box[2] = {16, (cuuint32_t)BM};
+        cuuint32_t box[2] = {(cuuint32_t)(p.kb / 4), (cuuint32_t)BM};
         cuuint32_t es[2] = {1, 1};
         CUresult r = enc(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void*)w.aux, dims, strides, box, es,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -642,16 +667,18 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
         return fail(WQ_EINVAL, "workspace too small");
     const uint16_t* sc = (const uint16_t*)w.aux;
     wq_status st;
-#define WQ_BN(BNV)                                                                                  \
-    st = (w.fmt == WQ_FMT_LLOYD8S) ? launch_bn<BNV, 32, true>(p, tx, tp, tl, sc, out, M, N, K, s)    \
-       : (w.group == 64)           ? launch_bn<BNV, 64, false>(p, tx, tp, tl, sc, out, M, N, K, s)   \
-                                   : launch_bn<BNV, 32, false>(p, tx, tp, tl, sc, out, M, N, K, s)
+#define WQ_BN(BNV, KBV)                                                                                 \
+    st = (w.fmt == WQ_FMT_LLOYD8S) ? launch_bn<BNV, 32, true, 64>(p, tx, tp, tl, sc, out, M, N, K, s)    \
+       : (w.group == 64) ? launch_bn<BNV, 64, false, KBV>(p, tx, tp, tl, sc, out, M, N, K, s)            \
+                         : launch_bn<BNV, 32, false, KBV>(p, tx, tp, tl, sc, out, M, N, K, s)
     switch (p.bn) {
-        case 16: WQ_BN(16); break;
-        case 32: WQ_BN(32); break;
-        case 64: WQ_BN(64); break;
-        case 128: WQ_BN(128); break;
-        default: WQ_BN(256); break;
+        case 16: WQ_BN(16, 64); break;
+        case 32: WQ_BN(32, 64); break;
+        case 64: WQ_BN(64, 64); break;
+        case 128:
+            if (p.kb == 128) { WQ_BN(128, 128); } else { WQ_BN(128, 64); }
+            break;
+        default: WQ_BN(256, 64); break;
     }
 #undef WQ_BN
     if (st != WQ_OK || p.splits == 1) return st;
