@@ -533,6 +533,9 @@ struct Plan {
     int bn, kb, splits, kt_per_split, grid_n, grid_m;
 };
 
+#ifndef WQ_GEMM_BN128_MAX
+#define WQ_GEMM_BN128_MAX 128
+#endif
 #ifndef WQ_GEMM_KB128
 #define WQ_GEMM_KB128 1
 #endif
@@ -546,7 +549,7 @@ Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt) {
     // reconstructs the same weights again, and reconstruction (not the tensor pipe) is what
     // narrower tiles run out of (measured: BN 128 / 192 at 0.5-0.9x of BN 256 throughput even
     // where they leave fewer SMs idle in the last wave).
-    p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= WQ_GEMM_BN128_MAX ? 128 : 256;
     // 128-column stages for 128-wide activation tiles where K allows: there they halve the
     // per-stage bookkeeping of the reconstruction, which this m is bound by (measured 1.4x at
     // m = 128); the 256-wide tiles keep 64-column stages, whose finer ring overlaps better
