@@ -277,3 +277,21 @@ def test_gemv_lloyd8s_on_the_gpu_producers_output(wq):
         y = wq.gemv(pw, to_dev_bits(x_bits))
         y_ref, bound = oracle.matmul_rows(oracle.LLOYD8S, packed, levels, 32, x_bits, rows=rows)
         _check(y, y_ref, bound, rows)
+
+
+@pytest.mark.parametrize("n,k", [(4096, 4096), (4100, 4160)])
+@pytest.mark.parametrize("batch", [1, 3, 16])
+def test_gemv_cluster_split_k_matches_oracle(wq, n, k, batch):
+    """Single launches of >= 16 M weights with too few rows to fill the GPU split K across a
+    thread-block cluster (partial sums reduced through distributed shared memory); ragged
+    rows and a ragged last step included. Sampled rows against the oracle."""
+    g = np.random.default_rng(n + k + batch)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    scale = workloads.f64_to_bf16_bits(g.uniform(0.005, 0.05, (n, k // 64)))
+    packed = oracle.pack(codes)
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(packed), to_dev_bits(scale))
+    x_bits = workloads.activations(batch, k, workloads.DECODE_SWEEP, batch)
+    y = wq.gemv(pw, to_dev_bits(x_bits))
+    rows = np.concatenate([g.choice(n, 96, replace=False), np.arange(n - 8, n)])
+    y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, scale, 64, x_bits, rows=rows)
+    _check(y, y_ref, bound, rows)

@@ -35,6 +35,7 @@
 //   * When a launch has too few rows to fill the GPU, WK warps of a CTA split K and meet
 //     in shared memory at the end; otherwise every warp covers the full K and no
 //     reduction exists. One launch, no workspace, either way.
+#include <cooperative_groups.h>
 #include <new>
 
 #include "wq_internal.cuh"
@@ -479,6 +480,9 @@ constexpr int depth(int kind, int nb, int r) {
     return (kind < kLut16 && nb == 1 && r == 1) ? WQ_GEMV_DEPTH : 2;
 }
 
+#ifndef WQ_GEMV_CLUSTER
+#define WQ_GEMV_CLUSTER 1             // small launches split K across a thread-block cluster
+#endif
 #ifndef WQ_GEMV_WARPS_BATCHED
 #define WQ_GEMV_WARPS_BATCHED 8
 #endif
@@ -500,30 +504,40 @@ constexpr int min_ctas(int kind, int nb, int r) {
          : r == 1 ? (nb == 1 ? WQ_GEMV_MIN_CTAS_NB1 : WQ_GEMV_MIN_CTAS_NB2) : WQ_GEMV_R2_CAP;
 }
 
-template <int KIND, int NB, int R, int WK, int FW, int MAXP>
+// CL > 1: a thread-block cluster of CL CTAs shares each row tile, CTA rank c taking a
+// contiguous slice of the K steps; the partial sums meet in rank 0's shared memory over the
+// cluster (distributed shared memory), between two cluster barriers.
+template <int KIND, int NB, int R, int WK, int FW, int MAXP, int CL>
 __global__ void __launch_bounds__(32 * cta_warps(WK, FW),
                                   (min_ctas(KIND, NB, R) * 4 / cta_warps(WK, FW)) > 0
                                       ? (min_ctas(KIND, NB, R) * 4 / cta_warps(WK, FW)) : 1)
 gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
+    static_assert(CL == 1 || WK == 1, "a cluster splits K across CTAs, not within one");
     constexpr int THREADS = 32 * cta_warps(WK, FW);
     constexpr int WR = cta_warps(WK, FW) / WK;       // warps with distinct rows per CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wr = warp % WR, wk = warp / WR;
+    const int tb = (int)blockIdx.x / CL;             // row tile (clusters are CL consecutive CTAs)
+    const int crank = (int)blockIdx.x % CL;
     // ---- which problem / row tile (a tile = the 16*R*WR rows of one CTA) -----------------
     int p = 0;
     if (MAXP > 1) {
         int lo = 0, hi = prm.count - 1;
-        while (lo < hi) {                      // last p with tile_start[p] <= blockIdx.x
+        while (lo < hi) {                      // last p with tile_start[p] <= tb
             const int mid = (lo + hi + 1) >> 1;
-            if (prm.tile_start[mid] <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+            if (prm.tile_start[mid] <= tb) lo = mid; else hi = mid - 1;
         }
         p = lo;
     }
     const GemvProblem& pb = prm.prob[p];
     const int N = pb.n, K = pb.k, B = prm.batch;
-    const int row0 = ((int)blockIdx.x - prm.tile_start[p]) * (16 * R * WR) + wr * 16 * R;
+    const int row0 = (tb - prm.tile_start[p]) * (16 * R * WR) + wr * 16 * R;
     const int g = lane >> 2, t = lane & 3;
-    const int steps = (K + 255) >> 8;
+    const int all_steps = (K + 255) >> 8;
+    // this CTA's steps: [s_lo, steps)
+    const int per = (all_steps + CL - 1) / CL;
+    const int s_lo = min(all_steps, crank * per);
+    const int steps = min(all_steps, s_lo + per);
 
     float acc[R][NB][4];
 #pragma unroll
@@ -562,10 +576,10 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     if (live) {
 #pragma unroll
         for (int i = 0; i < D - 1; ++i)
-            if (wk + i * WK < steps) load(buf[i], wk + i * WK);
+            if (s_lo + wk + i * WK < steps) load(buf[i], s_lo + wk + i * WK);
     }
-    for (int c0 = 0; c0 < steps; c0 += cs) {
-        if (c0 > 0) __syncthreads();               // every warp is done with the last chunk
+    for (int c0 = s_lo; c0 < steps; c0 += cs) {
+        if (c0 > s_lo) __syncthreads();            // every warp is done with the last chunk
         const int ns = min(cs, steps - c0);
         const bool xbad = __syncthreads_or(stage_x<KIND, THREADS>(xs, pb.x, B, K, c0, ns, rs)) != 0;
         if (!live) continue;
@@ -582,6 +596,33 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     }
 
     // ---- output: fragment (lane, nb, j): row = g + 8*(j>>1), batch = 8*nb + 2t + (j&1) ----
+    if constexpr (CL > 1) {
+        __shared__ float cred[WR][R][NB][4][32];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) cred[wr][r][nb][j][lane] = acc[r][nb][j];
+        namespace cg = cooperative_groups;
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();                          // every rank's partial sums are in place
+        if (crank == 0) {
+#pragma unroll 1
+            for (int q = 1; q < CL; ++q) {
+                const float* rem = cluster.map_shared_rank(&cred[0][0][0][0][0], q);
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            acc[r][nb][j] += rem[(((wr * R + r) * NB + nb) * 4 + j) * 32 + lane];
+            }
+        }
+        cluster.sync();                          // rank 0 is done reading the others
+        if (crank != 0) return;
+    }
     if (WK > 1) {
         __shared__ float red[WK > 1 ? WK : 1][WR][R][NB][4][32];
 #pragma unroll
@@ -625,12 +666,13 @@ template <int MAXP>
 struct Prepared {
     void (*kern)(GemvParams<MAXP>);
     GemvParams<MAXP> prm;
-    int tiles;
+    int tiles;                   // row tiles; the grid has tiles * cl CTAs
+    int cl;                      // cluster size (CTAs splitting one tile's K)
     int threads;
     size_t smem;
 };
 
-template <int KIND, int NB, int R, int WK, int FW, int MAXP>
+template <int KIND, int NB, int R, int WK, int FW, int MAXP, int CL = 1>
 wq_status prepare_variant(Prepared<MAXP>& pr, const GemvProblem* probs, int tiles) {
     constexpr int unit = depth(KIND, NB, R) * WK;   // chunks are whole multiples of this
     GemvParams<MAXP>& prm = pr.prm;
@@ -640,8 +682,9 @@ wq_status prepare_variant(Prepared<MAXP>& pr, const GemvProblem* probs, int tile
     cs = max(unit, cs - cs % unit);
     prm.chunk_steps = min(cs, max_steps);
     pr.smem = (size_t)prm.batch * (512 * prm.chunk_steps + 64);
-    pr.kern = gemv_kernel<KIND, NB, R, WK, FW, MAXP>;
+    pr.kern = gemv_kernel<KIND, NB, R, WK, FW, MAXP, CL>;
     pr.tiles = tiles;
+    pr.cl = CL;
     pr.threads = 32 * cta_warps(WK, FW);
     if (pr.smem > 48 * 1024) {
         // small launches with many batch rows: a chunk of D * WK steps may pass 48 KB
@@ -682,6 +725,27 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
         constexpr int FWB = WQ_GEMV_WARPS_BATCHED;
         return prepare_variant<KIND, NB, 1, 1, FWB, MAXP>(pr, probs, tiles_for(16 * FWB));
     }
+#if WQ_GEMV_CLUSTER
+    {
+        // too few rows to fill the GPU: a cluster of CL CTAs per 64-row tile splits K (each
+        // CTA at least 2 steps), sized for about 24 resident warps per SM
+        // (only for launches of >= 16 M weights: below that the cluster launch costs more
+        // than it saves; measured 5.0 -> 6.3 us on a 2048 x 2048 matrix)
+        int max_steps = 1;
+        int64_t weights = 0;
+        for (int i = 0; i < count; ++i) {
+            max_steps = max(max_steps, (probs[i].k + 255) / 256);
+            weights += (int64_t)probs[i].n * probs[i].k;
+        }
+        const int64_t tiles64 = (rows16 + 3) / 4;
+        int64_t want = (24 * sms + 4 * tiles64 - 1) / (4 * tiles64);
+        int cl = weights < ((int64_t)1 << 24) ? 1 : want >= 8 ? 8 : want >= 4 ? 4 : want >= 2 ? 2 : 1;
+        while (cl > 1 && max_steps / cl < 2) cl >>= 1;
+        if (cl == 8) return prepare_variant<KIND, NB, 1, 1, 4, MAXP, 8>(pr, probs, tiles_for(64));
+        if (cl == 4) return prepare_variant<KIND, NB, 1, 1, 4, MAXP, 4>(pr, probs, tiles_for(64));
+        if (cl == 2) return prepare_variant<KIND, NB, 1, 1, 4, MAXP, 2>(pr, probs, tiles_for(64));
+    }
+#endif
     if (rows16 >= 2 * sms) return prepare_variant<KIND, NB, 1, 2, 4, MAXP>(pr, probs, tiles_for(32));
     return prepare_variant<KIND, NB, 1, 4, 4, MAXP>(pr, probs, tiles_for(16));
 }
@@ -722,8 +786,24 @@ wq_status prepare(int fmt, int group, const GemvProblem* probs, int count, int b
 
 template <int MAXP>
 wq_status launch_prepared(const Prepared<MAXP>& pr, cudaStream_t s) {
-    pr.kern<<<pr.tiles, pr.threads, pr.smem, s>>>(pr.prm);
-    return check_launch("gemv");
+    if (pr.cl == 1) {
+        pr.kern<<<pr.tiles, pr.threads, pr.smem, s>>>(pr.prm);
+        return check_launch("gemv");
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pr.tiles * pr.cl);
+    cfg.blockDim = dim3(pr.threads);
+    cfg.dynamicSmemBytes = pr.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pr.cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, pr.kern, pr.prm) != cudaSuccess) return check_launch("gemv (cluster)");
+    return check_launch("gemv (cluster)");
 }
 
 template <int MAXP>
