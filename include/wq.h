@@ -232,7 +232,7 @@ size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
  * "materialized" bf16 path fused): y[i, r] = sum_c Wdeq[r, c] * x[i, c] for i < m, fp32
  * accumulation in tensor memory, bf16 output. Formats DYADIC4 (group 64 or 32) and LLOYD8S
  * (the 8-level codebook plus sign of [G32] §5.2, rebuilt per stage from the group's levels). For
- * m <= 8 the decode-shaped case runs on the GEMV kernel of wq_gemv_w4a16 (the kernel
+ * m <= 12 the decode-shaped case runs on the GEMV kernel of wq_gemv_w4a16 (the kernel
  * choice by batch size of [KM] §4.1), with the same tolerance and no workspace.
  *   x      bf16 [m, k]; m >= 1; k % 64 == 0.
  *   y      out bf16 [m, n].

@@ -27,7 +27,7 @@ def _check(y, y_ref, bound):
     assert np.all(err <= matmul_tolerance(y_ref, bound, TOL)), f"max err/bound {ratio.max():.3g}"
 
 
-@pytest.mark.parametrize("m", [1, 8, 9, 16, 17, 33, 64, 100, 128, 129, 256, 300])
+@pytest.mark.parametrize("m", [1, 8, 9, 12, 13, 16, 17, 33, 64, 100, 128, 129, 256, 300])
 @pytest.mark.parametrize("n,k,group", [(128, 256, 64), (200, 320, 64), (13, 64, 64), (256, 1024, 32)])
 def test_gemm_matches_oracle(wq, m, n, k, group):
     pw, packed, s = _weight(wq, n, k, group, m * 7 + n + k)
@@ -55,7 +55,7 @@ def test_gemm_one_hot_and_zero_codes_exact(wq):
 
 def test_gemm_split_k_uses_workspace(wq):
     pw, packed, s = _weight(wq, 1024, 8192, 64, 5)
-    assert wq.gemm_workspace_bytes(pw, 8) == 0            # m <= 8 runs on the GEMV kernel
+    assert wq.gemm_workspace_bytes(pw, 12) == 0           # m <= 12 runs on the GEMV kernel
     assert wq.gemm_workspace_bytes(pw, 48) > 0            # small m splits K
     x_bits = workloads.activations(48, 8192, workloads.PREFILL, 5)
     y = wq.gemm(pw, to_dev_bits(x_bits))
@@ -116,7 +116,7 @@ def _lloyd(wq, n, k, seed, signed_levels=False):
     return pw, packed, levels
 
 
-@pytest.mark.parametrize("m", [1, 8, 9, 48, 128, 200, 256, 300])
+@pytest.mark.parametrize("m", [1, 8, 12, 13, 48, 128, 200, 256, 300])
 @pytest.mark.parametrize("n,k", [(128, 256), (200, 320), (256, 1024)])
 def test_gemm_lloyd8s_matches_oracle(wq, m, n, k):
     """The fused LLOYD8S consumer on the tensor-memory GEMM ("int4-g32+warm" §5.2): the

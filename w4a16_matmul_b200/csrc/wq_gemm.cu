@@ -610,11 +610,12 @@ wq_status launch_bn(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp,
 
 // Up to this many activation rows the product is decode-shaped: the GEMV kernel (weights
 // rebuilt in registers, mma.sync, no TMA/TMEM pipeline) runs it faster than the
-// tensor-memory pipeline, whose per-stage bookkeeping dominates when BN is this small
-// (measured on 4096x11008: 13.8 us against about 23 us at m = 1; at m = 16 the GEMV's second
-// batch fragment makes it the slower one). This is the kernel choice by batch size of
+// tensor-memory pipeline, whose per-stage bookkeeping dominates when BN is this small.
+// Measured on 4096x11008 and 11008x4096: at m = 8, 14.9 / 12.2 us against about 23 us; at
+// m = 12, 18.4 / 19.3 us against 20.9 / 22.5 us; at m = 16 the two are even, so the GEMV's
+// second batch fragment stops at 12 rows. This is the kernel choice by batch size of
 // "K-Means量化技术…" §4.1.
-constexpr int64_t kGemvMaxRows = 8;
+constexpr int64_t kGemvMaxRows = 12;
 
 size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
     if (m <= kGemvMaxRows) return 0;
