@@ -12,6 +12,7 @@ Sources, cited by key in the C file and below:
   [DG]  "MiniCPM5-1B 验证: 6× 压缩, ppl 反超 fp, 1.2GB 显存, 50ms Triton 推理"
   [KM]  "K-Means量化技术：突破LLM低比特部署瓶颈"
   [G32] "int4-g32+warm 裸量化：原理与实验报告"
+  [BX]  "同一个 1B 模型，我上了三种压缩方案：无损的、4bit 的、还有没跑通的" (BF16X)
 """
 from __future__ import annotations
 
@@ -64,6 +65,8 @@ def _L():
             "orc_lloyd_candidate": [i32, vp, vp, vp],
             "orc_lloyd_params_byte": [i32],
             "orc_lloyd_num_candidates": [],
+            "orc_bf16x_encode": [vp, i64, i64, vp, vp, vp, vp, i64, vp],
+            "orc_bf16x_decode": [vp, vp, vp, vp, i64, i64, i64, vp],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -72,6 +75,8 @@ def _L():
         lib.orc_lloyd_inverse.argtypes = [i32, ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                           ctypes.c_double]
         lib.orc_lloyd_inverse.restype = ctypes.c_double
+        lib.orc_bf16x_superblocks.argtypes = [i64, i64]
+        lib.orc_bf16x_superblocks.restype = i64
         lib.orc_storage_bytes.argtypes = [i32, ctypes.c_double, i32]
         lib.orc_storage_bytes.restype = ctypes.c_double
         lib.orc_storage_lloyd_codebook_bytes.argtypes = [ctypes.c_double, i32]
@@ -293,3 +298,36 @@ def storage_bytes(fmt: int, nweights: float, group: int) -> float:
 
 def storage_lloyd_codebook_bytes(nweights: float, group: int) -> float:
     return _L().orc_storage_lloyd_codebook_bytes(float(nweights), group)
+
+
+def bf16x_encode(w_bits: np.ndarray) -> dict:
+    """[BX] BF16X encoding of a bf16 [n, k] matrix (k % 16 == 0): dict of sm uint8 [n, k],
+    hdr uint64 [n, k/16], sb_off uint32 [S + 1], ovf uint8 [escaped]."""
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    n, k = w.shape
+    L = _L()
+    S = L.orc_bf16x_superblocks(n, k)
+    sm = np.empty((n, k), np.uint8)
+    hdr = np.empty((n, k // 16), np.uint64)
+    sb = np.empty(S + 1, np.uint32)
+    ovf = np.empty(max(n * k, 1), np.uint8)
+    cnt = np.zeros(1, np.int64)
+    rc = L.orc_bf16x_encode(_p(w), n, k, _p(sm), _p(hdr), _p(sb), _p(ovf), ovf.size, _p(cnt))
+    if rc != 0:
+        raise ValueError(f"orc_bf16x_encode: {rc}")
+    return dict(sm=sm, hdr=hdr, sb_off=sb, ovf=ovf[:int(cnt[0])].copy())
+
+
+def bf16x_decode(enc: dict, n: int, k: int) -> np.ndarray:
+    """Inverse of bf16x_encode: bf16 bits [n, k]. Raises if the index fields disagree with
+    the escape table."""
+    out = np.empty((n, k), np.uint16)
+    ovf = np.ascontiguousarray(enc["ovf"], np.uint8)
+    ovf_buf = ovf if ovf.size else np.zeros(1, np.uint8)
+    rc = _L().orc_bf16x_decode(_p(np.ascontiguousarray(enc["sm"], np.uint8)),
+                               _p(np.ascontiguousarray(enc["hdr"], np.uint64)),
+                               _p(np.ascontiguousarray(enc["sb_off"], np.uint32)), _p(ovf_buf),
+                               ovf.size, n, k, _p(out))
+    if rc != 0:
+        raise ValueError(f"orc_bf16x_decode: {rc}")
+    return out

@@ -11,6 +11,8 @@
  *         (the DyadicGumbel 4-bit article), wmrh.cn/news/898890
  *   [KM]  "K-Means量化技术：突破LLM低比特部署瓶颈", mhpn.cn/news/872954
  *   [G32] "int4-g32+warm 裸量化：原理与实验报告", 0539edu.com/news/5477008
+ *   [BX]  "同一个 1B 模型，我上了三种压缩方案：无损的、4bit 的、还有没跑通的",
+ *         bjdmk.com.cn/news/3920032, section "第一剑·完美主义：BF16X" (lossless codec)
  *
  * Conventions
  *   - W is row-major [n, k] (out x in), groups are runs of `group` consecutive
@@ -645,4 +647,98 @@ double orc_storage_bytes(int32_t fmt, double nweights, int32_t group)
 double orc_storage_lloyd_codebook_bytes(double nweights, int32_t group)
 {
     return nweights / group * 8.0 * 4.0;
+}
+
+/* ------------------------------------------------------------------------------- */
+/* [BX] BF16X: lossless bf16 block codec                                             */
+/* ------------------------------------------------------------------------------- */
+/*
+ * [BX] "第一剑·完美主义：BF16X": blocks of 16 bf16 weights share the largest exponent of
+ * the block; each weight keeps a 3-bit difference to it; the few weights too far below
+ * it go to an overflow table; decoding gives back every bit. The page fixes neither the
+ * bit layout nor what happens to sign and mantissa; the reading taken here keeps both
+ * verbatim (a lossless codec must), so:
+ *
+ *   weight j of block b (flat row-major index 16 b + j), bits h = s:1 | e:8 | m:7
+ *   E_b      = max_j e_j                       (the shared exponent field)
+ *   d_j      = E_b - e_j; stored as d_j if d_j <= 6, else 7 = "escaped"
+ *   sm[i]    = s << 7 | m                      (one byte per weight, flat order)
+ *   hdr[b]   = 64 bits: bit j of plane p (p = 0, 1, 2) at bit 16 p + j holds bit p of the
+ *              stored 3-bit field of weight j; bits 48..55 = E_b; bits 56..63 = number of
+ *              escaped weights in the earlier blocks of b's superblock
+ *   superblock = 16 consecutive blocks (256 weights); sb_off[t] = escaped weights in all
+ *              superblocks before t, sb_off[S] = total, S = ceil(blocks / 16)
+ *   ovf[]    = the exponent fields e_j of the escaped weights, in flat index order
+ *
+ * Every bf16 pattern (zeros, subnormals, Inf, NaN payloads) round-trips.
+ * The encoder below walks the weights in order with one running escape counter.
+ */
+int64_t orc_bf16x_superblocks(int64_t n, int64_t k)
+{
+    return (n * k / 16 + 15) / 16;
+}
+
+int orc_bf16x_encode(const uint16_t* w, int64_t n, int64_t k, uint8_t* sm, uint64_t* hdr,
+                     uint32_t* sb_off, uint8_t* ovf, int64_t ovf_cap, int64_t* n_ovf)
+{
+    if (n < 0 || k < 0 || k % 16 != 0) return -1;
+    int64_t nblocks = n * k / 16, escaped = 0;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        if (b % 16 == 0) sb_off[b / 16] = (uint32_t)escaped;
+        int emax = 0;
+        for (int j = 0; j < 16; ++j) {
+            int e = (w[16 * b + j] >> 7) & 0xFF;
+            if (e > emax) emax = e;
+        }
+        uint64_t h = (uint64_t)emax << 48;
+        h |= (uint64_t)(escaped - (int64_t)sb_off[b / 16]) << 56;
+        for (int j = 0; j < 16; ++j) {
+            uint16_t v = w[16 * b + j];
+            int e = (v >> 7) & 0xFF;
+            int d = emax - e;
+            int field = d <= 6 ? d : 7;
+            if (field == 7) {
+                if (escaped >= ovf_cap) return -2;
+                ovf[escaped++] = (uint8_t)e;
+            }
+            for (int p = 0; p < 3; ++p)
+                if ((field >> p) & 1) h |= (uint64_t)1 << (16 * p + j);
+            sm[16 * b + j] = (uint8_t)(((v >> 8) & 0x80) | (v & 0x7F));
+        }
+        hdr[b] = h;
+    }
+    sb_off[(nblocks + 15) / 16] = (uint32_t)escaped;
+    *n_ovf = escaped;
+    return 0;
+}
+
+/* Decoding reads the escape table with its own running counter, in flat order. The
+ * superblock offsets and per-block prefixes are redundant random-access indexes; they
+ * are checked against the counter (-3 if they disagree) and not otherwise used. */
+int orc_bf16x_decode(const uint8_t* sm, const uint64_t* hdr, const uint32_t* sb_off,
+                     const uint8_t* ovf, int64_t n_ovf, int64_t n, int64_t k, uint16_t* out)
+{
+    if (n < 0 || k < 0 || k % 16 != 0) return -1;
+    int64_t nblocks = n * k / 16, next = 0;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        uint64_t h = hdr[b];
+        if ((int64_t)sb_off[b / 16] + (int64_t)(h >> 56) != next) return -3;
+        int emax = (int)((h >> 48) & 0xFF);
+        for (int j = 0; j < 16; ++j) {
+            int field = 0;
+            for (int p = 0; p < 3; ++p) field |= (int)((h >> (16 * p + j)) & 1) << p;
+            int e;
+            if (field == 7) {
+                if (next >= n_ovf) return -2;
+                e = ovf[next++];
+            } else {
+                e = emax - field;
+                if (e < 0) return -4;
+            }
+            uint8_t c = sm[16 * b + j];
+            out[16 * b + j] = (uint16_t)(((c & 0x80) << 8) | (e << 7) | (c & 0x7F));
+        }
+    }
+    if (sb_off[(nblocks + 15) / 16] != (uint32_t)next || next != n_ovf) return -3;
+    return 0;
 }
