@@ -11,6 +11,8 @@
  *   [G32] "int4-g32+warm 裸量化：原理与实验报告": §1.2 112-candidate shape grid,
  *         §1.3 quantisation flow (candidate argmin, 25 Lloyd rounds, sign bit),
  *         §2 storage format, §5.1-5.2 offline quantisation and inference.
+ *   [BX]  "同一个 1B 模型，我上了三种压缩方案：无损的、4bit 的、还有没跑通的", section
+ *         "第一剑·完美主义：BF16X": the lossless bf16 block codec.
  *
  * Conventions shared by every entry point
  *   - Matrices are row-major. A weight W is [n, k] = (out, in); groups are runs of
@@ -48,7 +50,8 @@ typedef enum wq_status {
     WQ_EALIGN = 2,        /* pointer not 16-byte aligned */
     WQ_EUNSUPPORTED = 3,  /* valid request this build does not implement (e.g. group) */
     WQ_ECUDA = 4,         /* the CUDA runtime reported an error (launch or attribute query) */
-    WQ_ETIMEOUT = 5       /* a bounded device-side wait gave up (reserved) */
+    WQ_ETIMEOUT = 5,      /* a bounded device-side wait gave up (reserved) */
+    WQ_EDATA = 6          /* a kernel found inconsistent encoded data (wq_device_error) */
 } wq_status;
 
 /* Static description of a status code. Never NULL. */
@@ -241,11 +244,51 @@ size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
 wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y,
                         void* ws, size_t ws_bytes, wq_stream stream);
 
-/* Reads and clears the library's device-side error word. Kernels that wait on the GPU
+/* Reads and clears the library's device-side error words. Kernels that wait on the GPU
  * (the GEMM pipeline's mbarrier waits) give up after a bounded time instead of hanging and
- * record a nonzero code there; *code receives it (0 = none). Synchronous (copies one int
- * from the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_OK otherwise. */
+ * record a nonzero code; the BF16X kernels record one when an overflow-table index would
+ * pass ovf_bytes (the access is skipped). *code receives the code (0 = none). Synchronous
+ * (copies two ints from the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_EDATA
+ * for inconsistent BF16X data, WQ_OK otherwise. */
 wq_status wq_device_error(int32_t* code);
+
+/* ------------------------------------------------------------------------------------ */
+/* BF16X lossless block codec ([BX] "第一剑·完美主义：BF16X")                              */
+/* ------------------------------------------------------------------------------------ */
+/* Blocks of 16 consecutive bf16 weights (flat row-major order) share their largest
+ * exponent field E; each weight keeps a 3-bit field, E - e when that is at most 6, else 7
+ * (escaped: its exponent field goes to an overflow table); sign and mantissa are kept
+ * verbatim, so decoding gives back every bit pattern, Inf and NaN included (the one
+ * exception to "inputs must be finite"). The page fixes neither bit layout nor the mantissa
+ * storage; this library's layout, for a matrix of n*k weights (k % 32 == 0, n*k < 2^32):
+ *   sm      uint8 [n, k]: sign << 7 | mantissa, one byte per weight.
+ *   hdr     uint64 [n, k/16]: bit 16p + j = bit p of weight j's field (p = 0, 1, 2);
+ *           bits 48..55 = E; bits 56..63 = escapes in the earlier blocks of the block's
+ *           superblock (16 consecutive blocks).
+ *   sb_off  uint32 [S + 1], S = wq_bf16x_superblocks(n, k): escapes before superblock t;
+ *           sb_off[S] = total escapes.
+ *   ovf     uint8 [total]: exponent fields of the escaped weights in flat order
+ *           (ovf_bytes = its allocated size; at least 16 bytes are allocated even if empty).
+ * Storage is 12 bits per weight plus 4 bytes per 256 weights plus one byte per escape. */
+
+/* S for an [n, k] matrix, or -1 if k is not a multiple of 16 or n, k < 1. */
+int64_t wq_bf16x_superblocks(int64_t n, int64_t k);
+
+/* First encoding pass: sb_off[0..S] = the exclusive escape offsets and the total. The caller
+ * reads sb_off[S] back to size ovf, then calls wq_bf16x_encode with the same w and sb_off. */
+wq_status wq_bf16x_count(const uint16_t* w, int64_t n, int64_t k, uint32_t* sb_off, wq_stream stream);
+
+/* Second pass: writes sm, hdr and ovf. An escape index at or past ovf_bytes (an sb_off not
+ * produced by wq_bf16x_count for this w) is skipped and flagged for wq_device_error. */
+wq_status wq_bf16x_encode(const uint16_t* w, int64_t n, int64_t k, const uint32_t* sb_off,
+                          uint8_t* sm, uint64_t* hdr, uint8_t* ovf, int64_t ovf_bytes,
+                          wq_stream stream);
+
+/* out = the bf16 [n, k] matrix the encoding holds (bit-exact). Overflow reads at or past
+ * ovf_bytes are skipped (exponent 0 is used) and flagged for wq_device_error. */
+wq_status wq_bf16x_decode(const uint8_t* sm, const uint64_t* hdr, const uint32_t* sb_off,
+                          const uint8_t* ovf, int64_t ovf_bytes, int64_t n, int64_t k,
+                          uint16_t* out, wq_stream stream);
 
 /* The GEMM above without a caller workspace, for callers that cannot allocate device
  * memory: e.g. an inference server whose caching allocator owns the whole device memory

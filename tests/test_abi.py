@@ -14,14 +14,15 @@ def test_library_exports_every_header_function(wq):
                 "wq_gemv_w4a16_grouped", "wq_gemm_workspace_bytes", "wq_gemm_w4a16",
                 "wq_debug_fail_next_launches", "wq_device_error", "wq_gemm_w4a16_static",
                 "wq_gemv_plan_create", "wq_gemv_plan_launch", "wq_gemv_plan_destroy",
-                "wq_fake_quant_ste"}
+                "wq_fake_quant_ste", "wq_bf16x_superblocks", "wq_bf16x_count", "wq_bf16x_encode",
+                "wq_bf16x_decode"}
     assert expected <= set(names), set(names) ^ expected
     for n in names:
         assert hasattr(wq._lib, n), n
 
 
 def test_status_strings_and_version(wq):
-    for s in range(6):
+    for s in range(7):
         assert wq._lib.wq_status_string(s).decode().startswith("WQ_")
     assert wq._lib.wq_status_string(99).decode() == "unknown wq_status"
     assert wq.version() >= 100
@@ -52,6 +53,14 @@ def test_shape_and_group_checks_fail_before_any_cuda_call(wq):
     assert lib.wq_gemv_w4a16_grouped(None, None, None, 1, 1, None) == wq.WQ_EINVAL
     assert lib.wq_fake_quant_ste(p, 4, 64, 16, p, p, None, None, None) == wq.WQ_EUNSUPPORTED
     assert lib.wq_fake_quant_ste(p, 4, 96, 64, p, p, None, None, None) == wq.WQ_EINVAL
+    # BF16X: k % 32, n*k below 2^32, ovf_bytes >= 0
+    assert lib.wq_bf16x_superblocks(3, 96) == 2 and lib.wq_bf16x_superblocks(16, 4096) == 256
+    assert lib.wq_bf16x_superblocks(4, 40) == -1
+    assert lib.wq_bf16x_count(p, 4, 48, p, None) == wq.WQ_EINVAL
+    assert lib.wq_bf16x_count(p, 1 << 20, 1 << 12, p, None) == wq.WQ_EINVAL
+    assert "2^32" in wq.last_error()
+    assert lib.wq_bf16x_encode(p, 4, 64, p, p, p, p, -1, None) == wq.WQ_EINVAL
+    assert lib.wq_bf16x_decode(p, p, p, p, 16, 4, 80, p, None) == wq.WQ_EINVAL
 
 
 def test_gemv_plan_rejects_bad_arguments_and_keeps_nothing(wq):

@@ -27,7 +27,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 # --- constants mirrored from include/wq.h -----------------------------------------------
-WQ_OK, WQ_EINVAL, WQ_EALIGN, WQ_EUNSUPPORTED, WQ_ECUDA, WQ_ETIMEOUT = range(6)
+WQ_OK, WQ_EINVAL, WQ_EALIGN, WQ_EUNSUPPORTED, WQ_ECUDA, WQ_ETIMEOUT, WQ_EDATA = range(7)
 FMT_DYADIC4, FMT_LLOYD8S, FMT_LUT16 = 0, 1, 2
 LLOYD_G32_WARM, LLOYD_KMEANS16 = 0, 1
 GEMV_MAX_GROUPED = 192
@@ -66,6 +66,10 @@ _SIG = {
     "wq_gemm_w4a16_static": ([_WP, _vp, _i64, _vp, _vp], _i32),
     "wq_debug_fail_next_launches": ([_i32], None),
     "wq_device_error": ([ctypes.POINTER(_i32)], _i32),
+    "wq_bf16x_superblocks": ([_i64, _i64], _i64),
+    "wq_bf16x_count": ([_vp, _i64, _i64, _vp, _vp], _i32),
+    "wq_bf16x_encode": ([_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp], _i32),
+    "wq_bf16x_decode": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp], _i32),
 }
 for _name, (_args, _res) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -95,10 +99,11 @@ def last_error() -> str:
 
 
 def device_error() -> int:
-    """Reads and clears the device error word (nonzero: a bounded GPU wait expired)."""
+    """Reads and clears the device error words (nonzero: a bounded GPU wait expired, or a
+    BF16X kernel met an overflow index past its table)."""
     code = _i32(0)
     st = _lib.wq_device_error(ctypes.byref(code))
-    if st not in (WQ_OK, WQ_ETIMEOUT):
+    if st not in (WQ_OK, WQ_ETIMEOUT, WQ_EDATA):
         _check(st)
     return code.value
 
@@ -324,3 +329,67 @@ def gemm(w: PackedWeight, x: torch.Tensor, out: torch.Tensor | None = None,
     _check(_lib.wq_gemm_w4a16(ctypes.byref(d), _ptr(x), m, _ptr(y), _ptr(workspace),
                               need, _stream(x)))
     return y
+
+
+# --- BF16X lossless codec ------------------------------------------------------------------
+@dataclass
+class Bf16xWeight:
+    """A bf16 [n, k] matrix in the BF16X layout of include/wq.h. Unsigned fields are held in
+    signed tensors of the same width (hdr: int64 for uint64, sb_off: int32 for uint32)."""
+    n: int
+    k: int
+    sm: torch.Tensor        # uint8 [n, k]
+    hdr: torch.Tensor       # int64 [n, k/16]
+    sb_off: torch.Tensor    # int32 [S + 1]
+    ovf: torch.Tensor       # uint8 [max(escapes, 16)]
+    escapes: int
+
+    def nbytes(self) -> int:
+        """Bytes the encoding needs (the overflow table at its exact length)."""
+        return self.sm.numel() + 8 * self.hdr.numel() + 4 * self.sb_off.numel() + self.escapes
+
+
+def bf16x_superblocks(n: int, k: int) -> int:
+    return int(_lib.wq_bf16x_superblocks(n, k))
+
+
+def bf16x_count(w: torch.Tensor, sb_off: torch.Tensor) -> None:
+    _cuda(w, torch.bfloat16, "w")
+    n, k = w.shape
+    _check(_lib.wq_bf16x_count(_ptr(w), n, k, _ptr(sb_off), _stream(w)))
+
+
+def bf16x_encode(w: torch.Tensor) -> Bf16xWeight:
+    """Encodes a bf16 [n, k] CUDA matrix. Synchronises once, to size the overflow table."""
+    _cuda(w, torch.bfloat16, "w")
+    n, k = w.shape
+    dev = w.device
+    S = bf16x_superblocks(n, k)
+    if S < 0:
+        raise WqError(WQ_EINVAL, f"k={k} is not a multiple of 16")
+    sb = torch.empty(S + 1, dtype=torch.int32, device=dev)
+    _check(_lib.wq_bf16x_count(_ptr(w), n, k, _ptr(sb), _stream(w)))
+    total = int(sb[S].item()) & 0xFFFFFFFF
+    sm = torch.empty((n, k), dtype=torch.uint8, device=dev)
+    hdr = torch.empty((n, k // 16), dtype=torch.int64, device=dev)
+    ovf = torch.empty(max(total, 16), dtype=torch.uint8, device=dev)
+    _check(_lib.wq_bf16x_encode(_ptr(w), n, k, _ptr(sb), _ptr(sm), _ptr(hdr), _ptr(ovf), ovf.numel(),
+                                _stream(w)))
+    return Bf16xWeight(n, k, sm, hdr, sb, ovf, total)
+
+
+def bf16x_encode_into(w: torch.Tensor, b: Bf16xWeight) -> None:
+    """Both passes into an existing encoding of the same matrix (no allocation, no sync)."""
+    n, k = w.shape
+    _check(_lib.wq_bf16x_count(_ptr(w), n, k, _ptr(b.sb_off), _stream(w)))
+    _check(_lib.wq_bf16x_encode(_ptr(w), n, k, _ptr(b.sb_off), _ptr(b.sm), _ptr(b.hdr), _ptr(b.ovf),
+                                b.ovf.numel(), _stream(w)))
+
+
+def bf16x_decode(b: Bf16xWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """The bf16 [n, k] matrix the encoding holds, bit for bit."""
+    if out is None:
+        out = torch.empty((b.n, b.k), dtype=torch.bfloat16, device=b.sm.device)
+    _check(_lib.wq_bf16x_decode(_ptr(b.sm), _ptr(b.hdr), _ptr(b.sb_off), _ptr(b.ovf), b.ovf.numel(),
+                                b.n, b.k, _ptr(out), _stream(out)))
+    return out

@@ -114,6 +114,15 @@ wq_status check_weight(const wq_weight* w) {
     return WQ_OK;
 }
 
+// BF16X sizes: the usual matrix checks, and every escape index below 2^32 (sb_off is uint32)
+wq_status check_bf16x_shape(int64_t n, int64_t k) {
+    wq_status st = check_shape(n, k, 0);
+    if (st) return st;
+    if (n * k >= (1LL << 32))
+        return fail(WQ_EINVAL, "n*k=%lld must be below 2^32 (32-bit escape offsets)", (long long)(n * k));
+    return WQ_OK;
+}
+
 }  // namespace
 }  // namespace wq
 
@@ -129,6 +138,7 @@ const char* wq_status_string(int32_t s) {
         case WQ_EUNSUPPORTED: return "WQ_EUNSUPPORTED: valid request not implemented";
         case WQ_ECUDA: return "WQ_ECUDA: CUDA runtime error";
         case WQ_ETIMEOUT: return "WQ_ETIMEOUT: bounded device wait expired";
+        case WQ_EDATA: return "WQ_EDATA: the device found inconsistent encoded data";
         default: return "unknown wq_status";
     }
 }
@@ -144,8 +154,61 @@ wq_status wq_device_error(int32_t* code) {
     if (!code) return fail(WQ_EINVAL, "code is NULL");
     wq_status st = read_device_error(code);
     if (st) return st;
+    int32_t data = 0;
+    if ((st = read_bf16x_error(&data))) return st;
     if (*code != 0) return fail(WQ_ETIMEOUT, "a bounded device wait expired (code %d)", *code);
+    if (data != 0) {
+        *code = data;
+        return fail(WQ_EDATA, "BF16X overflow index past ovf_bytes (code %d)", data);
+    }
     return WQ_OK;
+}
+
+int64_t wq_bf16x_superblocks(int64_t n, int64_t k) {
+    if (n < 1 || k < 1 || k % 16 != 0) return -1;
+    return bf16x_superblocks(n, k);
+}
+
+wq_status wq_bf16x_count(const uint16_t* w, int64_t n, int64_t k, uint32_t* sb_off, wq_stream stream) {
+    g_last_error[0] = 0;
+    wq_status st = check_bf16x_shape(n, k);
+    if (st) return st;
+    if ((st = check_ptr(w, "w", false))) return st;
+    if ((st = check_ptr(sb_off, "sb_off", false))) return st;
+    if ((st = check_injected())) return st;
+    return launch_bf16x_count(w, n, k, sb_off, (cudaStream_t)stream);
+}
+
+wq_status wq_bf16x_encode(const uint16_t* w, int64_t n, int64_t k, const uint32_t* sb_off,
+                          uint8_t* sm, uint64_t* hdr, uint8_t* ovf, int64_t ovf_bytes,
+                          wq_stream stream) {
+    g_last_error[0] = 0;
+    wq_status st = check_bf16x_shape(n, k);
+    if (st) return st;
+    if (ovf_bytes < 0) return fail(WQ_EINVAL, "ovf_bytes=%lld is negative", (long long)ovf_bytes);
+    if ((st = check_ptr(w, "w", false))) return st;
+    if ((st = check_ptr(sb_off, "sb_off", false))) return st;
+    if ((st = check_ptr(sm, "sm", false))) return st;
+    if ((st = check_ptr(hdr, "hdr", false))) return st;
+    if ((st = check_ptr(ovf, "ovf", false))) return st;
+    if ((st = check_injected())) return st;
+    return launch_bf16x_encode(w, n, k, sb_off, sm, hdr, ovf, ovf_bytes, (cudaStream_t)stream);
+}
+
+wq_status wq_bf16x_decode(const uint8_t* sm, const uint64_t* hdr, const uint32_t* sb_off,
+                          const uint8_t* ovf, int64_t ovf_bytes, int64_t n, int64_t k,
+                          uint16_t* out, wq_stream stream) {
+    g_last_error[0] = 0;
+    wq_status st = check_bf16x_shape(n, k);
+    if (st) return st;
+    if (ovf_bytes < 0) return fail(WQ_EINVAL, "ovf_bytes=%lld is negative", (long long)ovf_bytes);
+    if ((st = check_ptr(sm, "sm", false))) return st;
+    if ((st = check_ptr(hdr, "hdr", false))) return st;
+    if ((st = check_ptr(sb_off, "sb_off", false))) return st;
+    if ((st = check_ptr(ovf, "ovf", false))) return st;
+    if ((st = check_ptr(out, "out", false))) return st;
+    if ((st = check_injected())) return st;
+    return launch_bf16x_decode(sm, hdr, sb_off, ovf, ovf_bytes, n, k, out, (cudaStream_t)stream);
 }
 
 wq_status wq_quantize_dyadic(const uint16_t* w, int64_t n, int64_t k, int32_t group,

@@ -66,6 +66,16 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
 // Reads and clears the device error word written by expired bounded waits.
 wq_status read_device_error(int32_t* code);
 
+// BF16X lossless codec (wq_bf16x.cu)
+int64_t bf16x_superblocks(int64_t n, int64_t k);
+wq_status launch_bf16x_count(const uint16_t* w, int64_t n, int64_t k, uint32_t* sb_off, cudaStream_t s);
+wq_status launch_bf16x_encode(const uint16_t* w, int64_t n, int64_t k, const uint32_t* sb_off,
+                              uint8_t* sm, uint64_t* hdr, uint8_t* ovf, int64_t ovf_cap, cudaStream_t s);
+wq_status launch_bf16x_decode(const uint8_t* sm, const uint64_t* hdr, const uint32_t* sb_off,
+                              const uint8_t* ovf, int64_t ovf_cap, int64_t n, int64_t k,
+                              uint16_t* out, cudaStream_t s);
+wq_status read_bf16x_error(int32_t* code);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
