@@ -389,7 +389,44 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
         byts = nw * (4 + 4 + 0.5) + nw / 64 * 2
         out["fake_quant_ste_large"] = {"shape": [n_l, k_l], "GB/s": round(byts / ms / 1e6, 1), "us": round(ms * 1e3, 1),
                                        "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
-        del gz, zl, scl, qo, po
+        del gz
+        # Gumbel-ST backward on the same latent: z, gq in; gz, gscale out (12.1 B per element),
+        # 16 softmax weights per element, tau = 1 step^2 of a typical group
+        gql = torch.randn((n_l, k_l), device=dev)
+        gzo = torch.empty_like(zl)
+        gso = torch.empty((n_l, k_l // 64), dtype=torch.float32, device=dev)
+        tau = float((scl.float().median() / 8) ** 2)
+        ggb = graph_of(torch, lambda: wq._check(wq._lib.wq_gumbel_st_backward(
+            wq._ptr(zl), n_l, k_l, 64, wq._ptr(scl), tau, wq._ptr(gql), wq._ptr(gzo), wq._ptr(gso),
+            wq._stream(zl))))
+        ms = max_over_ranks(time_region(torch, stream, ggb.replay, steps, warm, barrier))
+        byts = nw * (4 + 4 + 4) + nw / 64 * (2 + 4)
+        out["gumbel_st_backward_large"] = {"shape": [n_l, k_l], "us": round(ms * 1e3, 1),
+                                           "Gelements/s": round(nw / ms / 1e6, 2),
+                                           "GB/s": round(byts / ms / 1e6, 1),
+                                           "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
+                                           "ex2_per_element": 16}
+        del ggb, gql, gzo, gso, zl, scl, qo, po
+        # BF16X lossless codec on a bf16 matrix of the same shape (N(0, 0.02^2)): the two
+        # encoding passes (count, encode) and the decode, each a plain stream
+        wb = (torch.randn((n_l, k_l), device=dev) * 0.02).to(torch.bfloat16)
+        enc = wq.bf16x_encode(wb)
+        ge = graph_of(torch, lambda: wq.bf16x_encode_into(wb, enc))
+        ms_e = max_over_ranks(time_region(torch, stream, ge.replay, steps, warm, barrier))
+        dout = torch.empty_like(wb)
+        gd = graph_of(torch, lambda: wq.bf16x_decode(enc, out=dout))
+        ms_d = max_over_ranks(time_region(torch, stream, gd.replay, steps, warm, barrier))
+        assert torch.equal(dout.view(torch.int16), wb.view(torch.int16)), "BF16X round trip differs"
+        code_b = enc.nbytes()
+        enc_b = nw * 2 + nw * 2 + code_b             # count reads w; encode reads w, writes the code
+        dec_b = code_b + nw * 2
+        out["bf16x_large"] = {"shape": [n_l, k_l], "bits_per_weight": round(8 * code_b / nw, 3),
+                              "escapes": enc.escapes,
+                              "encode_us": round(ms_e * 1e3, 1), "encode_GB/s": round(enc_b / ms_e / 1e6, 1),
+                              "encode_frac_hbm": round(enc_b / ms_e / 1e6 / peaks["hbm_gbs"], 4),
+                              "decode_us": round(ms_d * 1e3, 1), "decode_GB/s": round(dec_b / ms_d / 1e6, 1),
+                              "decode_frac_hbm": round(dec_b / ms_d / 1e6 / peaks["hbm_gbs"], 4)}
+        del ge, gd, enc, wb, dout
     except Exception as e:
         out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
     if args.extras in ("gemm", "all"):
@@ -600,7 +637,8 @@ def run_reference(args):
 def run_profile_target(args):
     """A few launches of one kernel on one shape and nothing else, for ncu captures:
     --profile gemm --shape N,K,M (prefill GEMM), quantize --shape N,K, dequant --shape N,K,
-    lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd). Random packed codes and
+    lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd), gumbel --shape N,K
+    (Gumbel-ST backward), bf16x --shape N,K (BF16X encode + decode). Random packed codes and
     scales (timing does not depend on the values); inputs stay on the device."""
     import torch
     import __graft_entry__
@@ -632,6 +670,17 @@ def run_profile_target(args):
         x = torch.randn((b, k), device=dev, generator=gen).to(torch.bfloat16)
         y = torch.empty((b, n), dtype=torch.bfloat16, device=dev)
         fn = lambda: wq.gemv(pl, x, out=y)
+    elif args.profile == "gumbel":
+        z = torch.randn((n, k), device=dev, generator=gen) * 0.02
+        s = (z.abs().reshape(n, k // 64, 64).amax(-1) * 1.1).to(torch.bfloat16)
+        gq = torch.randn((n, k), device=dev, generator=gen)
+        tau = float((s.float().median() / 8) ** 2)
+        fn = lambda: wq.gumbel_st_backward(z, s, gq, tau, 64)
+    elif args.profile == "bf16x":
+        w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+        enc = wq.bf16x_encode(w)
+        out = torch.empty_like(w)
+        fn = lambda: (wq.bf16x_encode_into(w, enc), wq.bf16x_decode(enc, out=out))
     elif args.profile == "lloyd":
         w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
         fn = lambda: wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)

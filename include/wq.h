@@ -178,6 +178,30 @@ wq_status wq_fake_quant_ste(const float* z, int64_t n, int64_t k, int32_t group,
                             const uint16_t* scale, float* q, uint8_t* codes, uint8_t* packed,
                             wq_stream stream);
 
+/* Gumbel-ST soft assignment, backward ([DG] §2.3 "Gumbel-ST"), the page's other QAT
+ * estimator: soft = softmax(-dist / tau) . codes, hard = codes[argmin dist],
+ * q = hard + (soft - soft.detach()), with codes = step * {-8..7}, step = scale / 8 and
+ * dist_j = (z - codes_j)^2 (readings: the squared distance, no noise term since the printed
+ * softmax has none, lowest index on an argmin tie). The forward value q is hard itself,
+ * exactly what wq_fake_quant_ste returns; this call is the backward for an upstream
+ * gradient gq:
+ *   gz[r, c]     = gq[r, c] * d soft / d z
+ *   gscale[r, g] = sum over the group's c of gq[r, c] * (d hard / d scale + d soft / d scale)
+ * (the codes depend on the trained scale, so the hard term adds (idx - 8) / 8).
+ *   z       fp32 [n, k] latent; k % group == 0 and k % 32 == 0.
+ *   group   64 or 32.
+ *   scale   bf16 [n, k/group], finite and >= 0.
+ *   tau     temperature, a positive normal float (else WQ_EINVAL). scale^2 / tau must stay
+ *           below 2^120 (outputs are unspecified beyond it).
+ *   gq      fp32 [n, k] upstream gradient dL/dq, finite.
+ *   gz      out fp32 [n, k] = dL/dz.
+ *   gscale  out fp32 [n, k/group] = dL/dscale, or NULL.
+ * fp32 arithmetic: |gz - gz_ref| <= 1e-4 |gz_ref| + 2^-100 |gq| (1 + 2 step^2 / tau) and
+ * |gscale - gscale_ref| <= 1e-4 times the group's sum of |terms| of the exact derivative. */
+wq_status wq_gumbel_st_backward(const float* z, int64_t n, int64_t k, int32_t group,
+                                const uint16_t* scale, float tau, const float* gq, float* gz,
+                                float* gscale, wq_stream stream);
+
 /* ------------------------------------------------------------------------------------ */
 /* W4A16 consumers                                                                       */
 /* ------------------------------------------------------------------------------------ */

@@ -56,6 +56,8 @@ def _L():
             "orc_dyadic_quantize": [vp, i64, i64, i32, i64, i64, vp, vp],
             "orc_dyadic_dequant": [vp, vp, i64, i64, i32, i64, i64, vp],
             "orc_fake_quant_ste": [vp, vp, i64, i64, i32, i64, i64, vp, vp],
+            "orc_gumbel_st_backward": [vp, vp, vp, i64, i64, i32, ctypes.c_double, i64, i64, vp, vp,
+                                       vp, vp],
             "orc_pack": [vp, i64, i64, i64, i64, vp],
             "orc_unpack": [vp, i64, i64, i64, i64, vp],
             "orc_dequant": [i32, vp, vp, i64, i64, i32, i64, i64, vp],
@@ -167,6 +169,25 @@ def fake_quant_ste(z: np.ndarray, scale_bits: np.ndarray, group: int = 64,
     _rows_parallel(n, lambda r0, r1: _L().orc_fake_quant_ste(_p(z), _p(scale), n, k, group, r0, r1,
                                                              _p(q), _p(codes)), threads)
     return q, codes
+
+
+def gumbel_st_backward(z: np.ndarray, scale_bits: np.ndarray, gq: np.ndarray, tau: float,
+                       group: int = 64, threads: int | None = None):
+    """[DG] §2.3 Gumbel-ST (q = hard + (soft - soft.detach()), soft = softmax(-dist/tau).codes)
+    backward for the upstream gradient gq: (gz fp32 [n, k], gscale fp64 [n, k/group], gz_mag,
+    gscale_mag), the *_mag arrays being the same sums over absolute values of every term."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    gq = np.ascontiguousarray(gq, dtype=np.float32)
+    scale = np.ascontiguousarray(scale_bits, dtype=np.uint16)
+    n, k = z.shape
+    gz = np.empty((n, k), np.float32)
+    gz_mag = np.empty((n, k), np.float64)
+    gs = np.empty((n, k // group), np.float64)
+    gs_mag = np.empty((n, k // group), np.float64)
+    _rows_parallel(n, lambda r0, r1: _L().orc_gumbel_st_backward(
+        _p(z), _p(scale), _p(gq), n, k, group, float(tau), r0, r1, _p(gz), _p(gs), _p(gz_mag),
+        _p(gs_mag)), threads)
+    return gz, gs, gz_mag, gs_mag
 
 
 def dyadic_dequant(codes: np.ndarray, scale_bits: np.ndarray, group: int = 64,

@@ -195,6 +195,94 @@ int orc_fake_quant_ste(const float* z, const uint16_t* scale, int64_t n, int64_t
     return 0;
 }
 
+/* Gumbel-ST soft assignment, backward ([DG] §2.3 "Gumbel-ST"). The page's training step:
+ *   codes = step * {-8, ..., 7}, step = scale / 8     (a function of the trained scale)
+ *   soft  = softmax(-dist / tau) . codes               (soft weighting)
+ *   hard  = codes[argmin(dist)]                         (hard choice)
+ *   q     = hard + (soft - soft.detach())               (hard forward, soft backward)
+ * Readings: dist_j = (z - codes_j)^2 (the squared distance the page checkpoints as
+ * "dist2" in §2.4); the printed softmax carries no noise term, so none is added; argmin
+ * ties go to the lowest index. The forward value q is hard itself (soft - soft = 0), the
+ * STE forward above. This function gives the backward for an upstream gradient gq:
+ *   gz[i]       = gq[i] * d soft / d z
+ *   gscale[g]   = sum over the group of gq[i] * (d hard / d scale + d soft / d scale)
+ * by the chain rule written out term by term through the softmax, in double:
+ *   l_j = -dist_j / tau,  d p_j / d t = p_j * sum_i p_i (d l_j / d t - d l_i / d t)
+ *   (the softmax Jacobian p_j (delta_ji - p_i), with sum_i p_i = 1), where
+ *   d l_j / d z - d l_i / d z         = 2 (codes_j - codes_i) / tau,
+ *   d l_j / d scale - d l_i / d scale = 2 ((z - codes_j) a_j - (z - codes_i) a_i) / tau,
+ *   a_j = d codes_j / d scale = (j - 8) / 8, d hard / d scale = a_idx, d hard / d z = 0
+ *   (idx is piecewise constant in z).
+ * Each difference of two logit derivatives is formed from its closed form, in which z
+ * cancels exactly: subtracting the two large derivatives themselves loses most digits when
+ * tau is small and z lies beyond the codes. gz_mag / gscale_mag (may be NULL) receive the
+ * same sums taken over absolute values of every term, a scale for comparing a
+ * lower-precision result with these. */
+int orc_gumbel_st_backward(const float* z, const uint16_t* scale, const float* gq, int64_t n,
+                           int64_t k, int32_t group, double tau, int64_t r0, int64_t r1,
+                           float* gz, double* gscale, double* gz_mag, double* gscale_mag)
+{
+    (void)n;
+    if (group <= 0 || k % group != 0) return -1;
+    if (!(tau > 0.0) || !isfinite(tau)) return -3;
+    const int64_t ng = k / group;
+    for (int64_t r = r0; r < r1; ++r) {
+        for (int64_t g = 0; g < ng; ++g) {
+            const double s = orc_bf16_to_double(scale[r * ng + g]);
+            const double step = s / 8.0;
+            if (!isfinite(s)) return -2;
+            double codes[16], a[16];
+            for (int j = 0; j < 16; ++j) {
+                codes[j] = step * (j - 8);
+                a[j] = (j - 8) / 8.0;
+            }
+            double gs = 0.0, gs_mag = 0.0;
+            for (int64_t c = g * group; c < (g + 1) * group; ++c) {
+                const double v = (double)z[r * k + c], up = (double)gq[r * k + c];
+                if (!isfinite(v) || !isfinite(up)) return -2;
+                double dist[16], l[16], p[16];
+                int idx = 0;
+                for (int j = 0; j < 16; ++j) {
+                    dist[j] = (v - codes[j]) * (v - codes[j]);
+                    if (dist[j] < dist[idx]) idx = j;
+                    l[j] = -dist[j] / tau;
+                }
+                double lmax = l[0];
+                for (int j = 1; j < 16; ++j) lmax = l[j] > lmax ? l[j] : lmax;
+                double den = 0.0;
+                for (int j = 0; j < 16; ++j) { p[j] = exp(l[j] - lmax); den += p[j]; }
+                for (int j = 0; j < 16; ++j) p[j] /= den;
+                double dsoft_z = 0.0, dsoft_s = 0.0, mag_z = 0.0, mag_s = 0.0;
+                for (int j = 0; j < 16; ++j) {
+                    double dpz = 0.0, dps = 0.0, dpz_mag = 0.0, dps_mag = 0.0;
+                    for (int i = 0; i < 16; ++i) {
+                        const double ddz = 2.0 * (codes[j] - codes[i]) / tau;
+                        const double dds = 2.0 * ((v - codes[j]) * a[j] - (v - codes[i]) * a[i]) / tau;
+                        dpz += p[i] * ddz;
+                        dps += p[i] * dds;
+                        dpz_mag += p[i] * fabs(ddz);
+                        dps_mag += p[i] * fabs(dds);
+                    }
+                    dpz *= p[j];
+                    dps *= p[j];
+                    dsoft_z += codes[j] * dpz;
+                    dsoft_s += p[j] * a[j] + codes[j] * dps;
+                    mag_z += fabs(codes[j]) * p[j] * dpz_mag;
+                    mag_s += p[j] * fabs(a[j]) + fabs(codes[j]) * p[j] * dps_mag;
+                }
+                const double dhard_s = a[idx];
+                gz[r * k + c] = (float)(up * dsoft_z);
+                if (gz_mag) gz_mag[r * k + c] = fabs(up) * mag_z;
+                gs += up * (dhard_s + dsoft_s);
+                gs_mag += fabs(up) * (fabs(dhard_s) + mag_s);
+            }
+            if (gscale) gscale[r * ng + g] = gs;
+            if (gscale_mag) gscale_mag[r * ng + g] = gs_mag;
+        }
+    }
+    return 0;
+}
+
 /* Reconstruction w = step * (idx - 8) ([DG] §2.2), stored as bf16 (one rounding). */
 int orc_dyadic_dequant(const uint8_t* codes, const uint16_t* scale, int64_t n, int64_t k,
                        int32_t group, int64_t r0, int64_t r1, uint16_t* out)

@@ -53,6 +53,7 @@ _SIG = {
                            _vp, _vp], _i32),
     "wq_pack": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "wq_fake_quant_ste": ([_vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp], _i32),
+    "wq_gumbel_st_backward": ([_vp, _i64, _i64, _i32, _vp, ctypes.c_float, _vp, _vp, _vp, _vp], _i32),
     "wq_unpack": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "wq_dequant": ([_WP, _vp, _vp], _i32),
     "wq_gemv_w4a16": ([_WP, _vp, _i32, _vp, _vp], _i32),
@@ -182,6 +183,22 @@ def fake_quant_ste(z: torch.Tensor, scale: torch.Tensor, group: int = 64, codes:
     _check(_lib.wq_fake_quant_ste(_ptr(z), n, k, group, _ptr(scale), _ptr(q), _ptr(c), _ptr(p),
                                   _stream(z)))
     return q, c, p
+
+
+def gumbel_st_backward(z: torch.Tensor, scale: torch.Tensor, gq: torch.Tensor, tau: float,
+                       group: int = 64, scale_grad: bool = True):
+    """Gumbel-ST backward (soft = softmax(-dist/tau).codes, q = hard + (soft - soft.detach()))
+    for the upstream gradient gq: returns (gz fp32 [n, k], gscale fp32 [n, k/group] | None).
+    The forward value of Gumbel-ST is the hard code, i.e. fake_quant_ste's q."""
+    _cuda(z, torch.float32, "z")
+    _cuda(gq, torch.float32, "gq")
+    _cuda(scale, torch.bfloat16, "scale")
+    n, k = z.shape
+    gz = torch.empty_like(z)
+    gs = torch.empty((n, k // group), dtype=torch.float32, device=z.device) if scale_grad else None
+    _check(_lib.wq_gumbel_st_backward(_ptr(z), n, k, group, _ptr(scale), float(tau), _ptr(gq),
+                                      _ptr(gz), _ptr(gs), _stream(z)))
+    return gz, gs
 
 
 def quantize_lloyd(w: torch.Tensor, mode: int = LLOYD_G32_WARM, rounds: int = 25,

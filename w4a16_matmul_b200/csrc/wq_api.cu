@@ -327,6 +327,25 @@ wq_status wq_fake_quant_ste(const float* z, int64_t n, int64_t k, int32_t group,
     return launch_fake_quant_ste(z, n, k, group, scale, q, codes, packed, (cudaStream_t)stream);
 }
 
+wq_status wq_gumbel_st_backward(const float* z, int64_t n, int64_t k, int32_t group,
+                                const uint16_t* scale, float tau, const float* gq, float* gz,
+                                float* gscale, wq_stream stream) {
+    g_last_error[0] = 0;
+    if (group != 64 && group != 32)
+        return fail(WQ_EUNSUPPORTED, "Gumbel-ST group must be 64 or 32 (got %d)", group);
+    if (!(tau > 0.0f) || !(tau <= 3.0e38f) || tau < 1.17549435e-38f)
+        return fail(WQ_EINVAL, "tau must be a positive normal finite float (got %g)", (double)tau);
+    wq_status st = check_shape(n, k, group);
+    if (st) return st;
+    if ((st = check_ptr(z, "z", false))) return st;
+    if ((st = check_ptr(scale, "scale", false))) return st;
+    if ((st = check_ptr(gq, "gq", false))) return st;
+    if ((st = check_ptr(gz, "gz", false))) return st;
+    if ((st = check_ptr(gscale, "gscale", true))) return st;
+    if ((st = check_injected())) return st;
+    return launch_gumbel_st_backward(z, n, k, group, scale, tau, gq, gz, gscale, (cudaStream_t)stream);
+}
+
 wq_status wq_gemv_plan_create(const wq_weight* ws, const uint16_t* const* xs, uint16_t* const* ys,
                               int32_t count, int32_t batch, wq_gemv_plan* plan) {
     g_last_error[0] = 0;

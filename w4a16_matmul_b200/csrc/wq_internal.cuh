@@ -33,6 +33,9 @@ wq_status launch_pack(const uint8_t* codes, int64_t n, int64_t k, uint8_t* packe
 wq_status launch_fake_quant_ste(const float* z, int64_t n, int64_t k, int group,
                                 const uint16_t* scale, float* q, uint8_t* codes, uint8_t* packed,
                                 cudaStream_t s);
+wq_status launch_gumbel_st_backward(const float* z, int64_t n, int64_t k, int group,
+                                    const uint16_t* scale, float tau, const float* gq, float* gz,
+                                    float* gscale, cudaStream_t s);
 wq_status launch_unpack(const uint8_t* packed, int64_t n, int64_t k, uint8_t* codes, cudaStream_t s);
 wq_status launch_dequant(const wq_weight& w, uint16_t* out, cudaStream_t s);
 

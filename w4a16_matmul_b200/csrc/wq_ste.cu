@@ -8,6 +8,23 @@
 // argmin -> level_idx -> pack" of §2.5.
 //
 // HBM-bound stream: 4 B read, 4 B written per element (plus 1 B or 0.5 B of codes when asked).
+//
+// The same file holds the backward of the page's other estimator, Gumbel-ST (§2.3):
+// soft = softmax(-dist/tau) . codes, hard = codes[argmin dist], q = hard + (soft - soft.detach()),
+// dist_j = (z - codes_j)^2. Its forward value is hard (the STE forward above); its backward,
+// for an upstream gradient gq, is gz = gq * d soft/d z per element and, per group,
+// gscale = sum gq * (d hard/d scale + d soft/d scale) (the codes are step * (j - 8) with
+// step = scale / 8, a function of the trained scale). With p the softmax weights and
+// u_j = j - idx the code offset from the nearest code, both derivatives are moments of p:
+//   d soft/d z     = (2/tau) step^2 M2,                     M2 = sum p (u - mu)^2
+//   d soft/d scale = (mu + idx - 8)/8
+//                    + (2/tau) (step/8) ((z - 2 c_idx - 2 step mu) M2 - step M3),
+// mu = sum p u, M3 = sum p (u - mu)^3 (p normalised), c_idx = step (idx - 8). The weights
+// come from their logits relative to the nearest code, log2 p_j = u (A - B u) with
+// A = 2 (z - c_idx) step log2(e)/tau and B = step^2 log2(e)/tau, so no term is a difference
+// of two large numbers, and the central moments stay accurate in fp32 at any temperature.
+// Per element: 16 ex2 on the special-function unit and about 10 fp32 operations per code,
+// so the kernel is bound by instruction issue, not by HBM (12 B per element).
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -101,7 +118,103 @@ fake_quant_ste_kernel(const float4* __restrict__ z, const uint16_t* __restrict__
     }
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// One element of the Gumbel-ST backward (formulas at the top of this file).
+//   st2 = step^2 * log2(e) / tau (B), l2t = 2 log2(e) / tau, r2 = 2 / tau.
+__device__ __forceinline__ void gumbel_st_element(float z, float up, float s, float c8, float step,
+                                                  float m17, bool fast, float l2t, float r2,
+                                                  float& gz, float& gs) {
+    const float fi = (float)ste_index(z, s, c8, step, m17, fast);
+    const float c_idx = step * (fi - 8.0f);
+    const float e = z - c_idx;
+    const float A = e * step * l2t;
+    const float B = step * step * (0.5f * l2t);
+    float p[16];
+    float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float u = (float)j - fi;
+        p[j] = ex2_approx(u * fmaf(-B, u, A));
+        s0 += p[j];
+        s1 = fmaf(p[j], u, s1);
+    }
+    const float inv = 1.0f / s0;                     // s0 >= 1: the nearest code has weight 1
+    const float mu = s1 * inv;
+    float m2 = 0.0f, m3 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float v = ((float)j - fi) - mu;
+        const float pvv = p[j] * v * v;
+        m2 += pvv;
+        m3 = fmaf(pvv, v, m3);
+    }
+    m2 *= inv;
+    m3 *= inv;
+    gz = up * ((r2 * step) * step * m2);
+    const float cov = (step * 0.125f) * fmaf(z - 2.0f * c_idx - 2.0f * step * mu, m2, -step * m3);
+    gs = up * ((fi - 8.0f) * 0.125f + (mu + fi - 8.0f) * 0.125f + r2 * cov);
+}
+
+// One thread: 8 consecutive elements; the 8 (group 64) or 4 (group 32) threads of a group
+// sit in adjacent lanes and add their scale gradients with shuffles. The loop runs on a
+// warp-uniform index, so every lane reaches every shuffle; n8 is a multiple of the lanes
+// per group, so the idle lanes of the last trip hold whole groups.
+__global__ void __launch_bounds__(kThreads)
+gumbel_st_backward_kernel(const float4* __restrict__ z, const uint16_t* __restrict__ scale,
+                          const float4* __restrict__ gq, int64_t n8, int group, float l2t, float r2,
+                          float4* __restrict__ gz, float* __restrict__ gscale) {
+    const int lane = threadIdx.x & 31;
+    const int per_group = group / 8;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < n8; base += stride) {
+        const int64_t i = base + lane;
+        float gsum = 0.0f;
+        if (i < n8) {
+            const uint4 za = ldg_nc_v4(z + 2 * i), zb = ldg_nc_v4(z + 2 * i + 1);
+            const uint4 ga = ldg_nc_v4(gq + 2 * i), gb = ldg_nc_v4(gq + 2 * i + 1);
+            const float s = bf16_bits_to_float(ldg_u16(scale + i / per_group));
+            const bool fast = s >= 0x1p-96f && s <= 0x1p96f;
+            const float c8 = fast ? 8.0f * rcp_fast(s) : 0.0f;
+            const float step = s * 0.125f, m17 = -17.0f * s * 0.0625f;
+            const uint32_t zv[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+            const uint32_t gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            uint32_t out[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float g, gsj;
+                gumbel_st_element(__uint_as_float(zv[j]), __uint_as_float(gv[j]), s, c8, step, m17,
+                                  fast, l2t, r2, g, gsj);
+                out[j] = __float_as_uint(g);
+                gsum += gsj;
+            }
+            stg_cs_v4(gz + 2 * i, make_uint4(out[0], out[1], out[2], out[3]));
+            stg_cs_v4(gz + 2 * i + 1, make_uint4(out[4], out[5], out[6], out[7]));
+        }
+        for (int off = 1; off < per_group; off <<= 1) gsum += __shfl_xor_sync(0xffffffffu, gsum, off);
+        if (gscale && i < n8 && (lane & (per_group - 1)) == 0) gscale[i / per_group] = gsum;
+    }
+}
+
 }  // namespace
+
+wq_status launch_gumbel_st_backward(const float* z, int64_t n, int64_t k, int group,
+                                    const uint16_t* scale, float tau, const float* gq, float* gz,
+                                    float* gscale, cudaStream_t s) {
+    const int64_t n8 = n * k / 8;
+    int64_t blocks = (n8 + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    const double l2e = 1.4426950408889634;
+    gumbel_st_backward_kernel<<<(int)(blocks < 1 ? 1 : blocks), kThreads, 0, s>>>(
+        (const float4*)z, scale, (const float4*)gq, n8, group, (float)(2.0 * l2e / (double)tau),
+        (float)(2.0 / (double)tau), (float4*)gz, gscale);
+    return check_launch("gumbel_st_backward");
+}
 
 wq_status launch_fake_quant_ste(const float* z, int64_t n, int64_t k, int group,
                                 const uint16_t* scale, float* q, uint8_t* codes, uint8_t* packed,
