@@ -94,51 +94,78 @@ __device__ __forceinline__ uint32_t half_emax(const uint4 w) {
     return max(max_byte(e0), max_byte(e1));
 }
 
+// Escape offsets: an exclusive scan of the per-superblock escape counts, in place in sb_off,
+// over tiles of kTileSb superblocks, in three launches and no other memory. A superblock
+// holds at most 240 escapes (each block's largest exponent never escapes), so a count fits
+// in bits 0..7 of its entry and bits 8..31 are free until the last launch:
+//   count       entry s = count of superblock s; the last entry of each tile also holds
+//               the tile's total in bits 8..31 (at most 240 * kTileSb < 2^24);
+//   tile scan   one CTA: the exclusive offset O_t of every tile but the last goes to bits
+//               8..31 of the tile's entries 0 (O_t & 0xFFFFFF) and 1 (O_t >> 24); the last
+//               tile's offset goes to sb_off[S];
+//   tile final  one CTA per tile: entry s = O_t + the escapes of the tile's earlier
+//               superblocks; the last tile's CTA writes sb_off[S] = the total.
+// Every launch reads only entries no other CTA of the same launch writes.
+constexpr int kTileSb = 256;                     // superblocks per scan tile (>= 3)
+constexpr int kFinalThreads = kTileSb / 4;
+
 __global__ void __launch_bounds__(kThreads)
-bf16x_count_kernel(const uint4* __restrict__ w, int64_t nhalf, int64_t nsb, uint32_t* __restrict__ sb_cnt) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
-    for (int64_t s0 = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * kUnits; s0 < nsb;
-         s0 += warps * kUnits) {
-        uint4 v[kUnits];
+bf16x_count_kernel(const uint4* __restrict__ w, int64_t nhalf, int64_t nsb, uint32_t* __restrict__ sb) {
+    __shared__ uint32_t s_sum[kThreads / 32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t ntiles = (nsb + kTileSb - 1) / kTileSb;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t t0 = tile * kTileSb, t1 = min(t0 + (int64_t)kTileSb, nsb);
+        uint32_t run = 0;                                            // warp-uniform
+        for (int64_t s0 = t0 + (int64_t)wid * kUnits; s0 < t1; s0 += (kThreads / 32) * kUnits) {
+            uint4 v[kUnits];
 #pragma unroll
-        for (int u = 0; u < kUnits; ++u) {
-            const int64_t t = (s0 + u) * 32 + lane;
-            v[u] = make_uint4(0, 0, 0, 0);
-            if (t < nhalf) v[u] = ldg_nc_v4(w + t);
-        }
+            for (int u = 0; u < kUnits; ++u) {
+                const int64_t t = (s0 + u) * 32 + lane;
+                v[u] = make_uint4(0, 0, 0, 0);
+                if (s0 + u < t1 && t < nhalf) v[u] = ldg_nc_v4(w + t);
+            }
 #pragma unroll
-        for (int u = 0; u < kUnits; ++u) {
-            if (s0 + u >= nsb) break;
-            const uint32_t me = half_emax(v[u]);
-            const uint32_t E = max(me, __shfl_xor_sync(0xFFFFFFFFu, me, 1));
-            Half h;
-            encode_half(v[u], E, h);
-            const int64_t t = (s0 + u) * 32 + lane;
-            const uint32_t c = t < nhalf ? __popc(h.esc) : 0u;
-            const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, c);
-            if (lane == 0) sb_cnt[s0 + u] = total;
+            for (int u = 0; u < kUnits; ++u) {
+                if (s0 + u >= t1) break;
+                const uint32_t me = half_emax(v[u]);
+                const uint32_t E = max(me, __shfl_xor_sync(0xFFFFFFFFu, me, 1));
+                Half h;
+                encode_half(v[u], E, h);
+                const int64_t t = (s0 + u) * 32 + lane;
+                const uint32_t c = t < nhalf ? __popc(h.esc) : 0u;
+                const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, c);
+                if (lane == 0) sb[s0 + u] = total;
+                run += total;
+            }
         }
+        if (lane == 0) s_sum[wid] = run;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t tot = 0;
+#pragma unroll
+            for (int i = 0; i < kThreads / 32; ++i) tot += s_sum[i];
+            sb[t1 - 1] |= tot << 8;                                  // written before the barrier
+        }
+        __syncthreads();
     }
 }
 
-// In-place exclusive scan of sb[0..count) with sb[count] = the total; one CTA.
-constexpr int kScanThreads = 1024, kScanItems = 16;
+// One CTA, looping over the tiles 1024 at a time.
+constexpr int kTileScanThreads = 1024;
 
-__global__ void __launch_bounds__(kScanThreads) bf16x_scan_kernel(uint32_t* __restrict__ sb, int64_t count) {
-    __shared__ uint32_t s_warp[kScanThreads / 32];
+__global__ void __launch_bounds__(kTileScanThreads)
+bf16x_tile_scan_kernel(uint32_t* __restrict__ sb, int64_t nsb) {
+    __shared__ uint32_t s_warp[kTileScanThreads / 32];
     __shared__ uint32_t s_total;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t ntiles = (nsb + kTileSb - 1) / kTileSb;
     uint32_t carry = 0;
-    for (int64_t base = 0; base < count; base += (int64_t)kScanThreads * kScanItems) {
-        const int64_t i0 = base + (int64_t)tid * kScanItems;
-        uint32_t v[kScanItems], sum = 0;
-#pragma unroll
-        for (int i = 0; i < kScanItems; ++i) {
-            v[i] = (i0 + i < count) ? sb[i0 + i] : 0u;
-            sum += v[i];
-        }
-        uint32_t incl = sum;                                        // warp inclusive scan
+    for (int64_t base = 0; base < ntiles; base += kTileScanThreads) {
+        const int64_t t = base + tid;
+        // totals of the full tiles only (the last tile's total is never needed)
+        const uint32_t v = t < ntiles - 1 ? sb[(t + 1) * kTileSb - 1] >> 8 : 0u;
+        uint32_t incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
@@ -147,26 +174,77 @@ __global__ void __launch_bounds__(kScanThreads) bf16x_scan_kernel(uint32_t* __re
         if (lane == 31) s_warp[wid] = incl;
         __syncthreads();
         if (wid == 0) {
-            uint32_t ws = s_warp[lane], wi = ws;
+            const uint32_t ws = s_warp[lane];
+            uint32_t wi = ws;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
                 if (lane >= o) wi += y;
             }
-            s_warp[lane] = wi - ws;                                  // exclusive warp offsets
+            s_warp[lane] = wi - ws;
             if (lane == 31) s_total = wi;
         }
         __syncthreads();
-        uint32_t run = carry + s_warp[wid] + incl - sum;
-#pragma unroll
-        for (int i = 0; i < kScanItems; ++i) {
-            if (i0 + i < count) sb[i0 + i] = run;
-            run += v[i];
+        const uint32_t off = carry + s_warp[wid] + incl - v;
+        if (t < ntiles - 1) {
+            sb[t * kTileSb] |= (off & 0xFFFFFFu) << 8;
+            sb[t * kTileSb + 1] |= (off >> 24) << 8;
+        } else if (t == ntiles - 1) {
+            sb[nsb] = off;
         }
         carry += s_total;
-        __syncthreads();                                             // s_warp reused next tile
+        __syncthreads();
     }
-    if (tid == 0) sb[count] = carry;
+}
+
+__global__ void __launch_bounds__(kFinalThreads)
+bf16x_tile_final_kernel(uint32_t* __restrict__ sb, int64_t nsb) {
+    __shared__ uint32_t s_warp[kFinalThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t ntiles = (nsb + kTileSb - 1) / kTileSb;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t t0 = tile * kTileSb, t1 = min(t0 + (int64_t)kTileSb, nsb);
+        const bool last = t1 == nsb;
+        const uint32_t off = last ? sb[nsb] : (sb[t0] >> 8) | ((sb[t0 + 1] >> 8) << 24);
+        const int64_t i0 = t0 + 4 * tid;
+        uint32_t c[4];
+        if (i0 + 3 < t1) {
+            const uint4 q = *reinterpret_cast<const uint4*>(sb + i0);
+            c[0] = q.x; c[1] = q.y; c[2] = q.z; c[3] = q.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) c[j] = i0 + j < t1 ? sb[i0 + j] : 0u;
+        }
+        uint32_t sum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { c[j] &= 0xFFu; sum += c[j]; }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_warp[wid] = incl;
+        __syncthreads();                            // also: every thread has read `off`
+        uint32_t before = 0, tile_total = 0;
+#pragma unroll
+        for (int i = 0; i < kFinalThreads / 32; ++i) {
+            before += i < wid ? s_warp[i] : 0u;
+            tile_total += s_warp[i];
+        }
+        uint32_t run = off + before + incl - sum;
+        uint32_t o4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { o4[j] = run; run += c[j]; }
+        if (i0 + 3 < t1) {
+            *reinterpret_cast<uint4*>(sb + i0) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) if (i0 + j < t1) sb[i0 + j] = o4[j];
+        }
+        if (last && tid == 0) sb[nsb] = off + tile_total;
+        __syncthreads();                            // s_warp reused by the next tile
+    }
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -312,11 +390,16 @@ int64_t bf16x_superblocks(int64_t n, int64_t k) { return (n * k / 16 + 15) / 16;
 
 wq_status launch_bf16x_count(const uint16_t* w, int64_t n, int64_t k, uint32_t* sb_off, cudaStream_t s) {
     const int64_t nhalf = n * k / 8, nsb = bf16x_superblocks(n, k);
-    bf16x_count_kernel<<<grid_for(nsb), kThreads, 0, s>>>((const uint4*)w, nhalf, nsb, sb_off);
+    const int64_t ntiles = (nsb + kTileSb - 1) / kTileSb;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    const int grid = (int)(ntiles < cap ? ntiles : cap);
+    bf16x_count_kernel<<<grid, kThreads, 0, s>>>((const uint4*)w, nhalf, nsb, sb_off);
     wq_status st = check_launch("bf16x count");
     if (st) return st;
-    bf16x_scan_kernel<<<1, kScanThreads, 0, s>>>(sb_off, nsb);
-    return check_launch("bf16x scan");
+    bf16x_tile_scan_kernel<<<1, kTileScanThreads, 0, s>>>(sb_off, nsb);
+    if ((st = check_launch("bf16x tile scan"))) return st;
+    bf16x_tile_final_kernel<<<grid, kFinalThreads, 0, s>>>(sb_off, nsb);
+    return check_launch("bf16x tile final");
 }
 
 wq_status launch_bf16x_encode(const uint16_t* w, int64_t n, int64_t k, const uint32_t* sb_off,

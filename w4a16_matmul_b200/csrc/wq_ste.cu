@@ -23,8 +23,9 @@
 // come from their logits relative to the nearest code, log2 p_j = u (A - B u) with
 // A = 2 (z - c_idx) step log2(e)/tau and B = step^2 log2(e)/tau, so no term is a difference
 // of two large numbers, and the central moments stay accurate in fp32 at any temperature.
-// Per element: 16 ex2 on the special-function unit and about 10 fp32 operations per code,
-// so the kernel is bound by instruction issue, not by HBM (12 B per element).
+// Per element: 16 ex2 on the special-function unit and 9 fp32 operations per code, issued
+// two elements at a time as packed fp32x2 instructions; the special-function unit (16 ex2
+// per element) then bounds the kernel, not HBM (12 B per element).
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -124,40 +125,55 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return r;
 }
 
-// One element of the Gumbel-ST backward (formulas at the top of this file).
-//   st2 = step^2 * log2(e) / tau (B), l2t = 2 log2(e) / tau, r2 = 2 / tau.
-__device__ __forceinline__ void gumbel_st_element(float z, float up, float s, float c8, float step,
-                                                  float m17, bool fast, float l2t, float r2,
-                                                  float& gz, float& gs) {
-    const float fi = (float)ste_index(z, s, c8, step, m17, fast);
-    const float c_idx = step * (fi - 8.0f);
-    const float e = z - c_idx;
-    const float A = e * step * l2t;
-    const float B = step * step * (0.5f * l2t);
-    float p[16];
-    float s0 = 0.0f, s1 = 0.0f;
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// Two elements of the Gumbel-ST backward (formulas at the top of this file) on the packed
+// fp32x2 pipe. The moments are taken in one pass as raw moments about the nearest code,
+// E[u^k] = sum p u^k / sum p, and centred afterwards: u stays within [-15, 15], so the
+// centring loses at most a few bits, far inside the tolerance. Both elements share the
+// group's step.  l2t = 2 log2(e) / tau, r2 = 2 / tau.
+__device__ __forceinline__ void gumbel_st_pair(float2 z, float2 up, float s, float c8, float step,
+                                               float m17, bool fast, float l2t, float r2,
+                                               float2& gz, float2& gs) {
+    const float2 fi = make_float2((float)ste_index(z.x, s, c8, step, m17, fast),
+                                  (float)ste_index(z.y, s, c8, step, m17, fast));
+    const float2 c_idx = __fmul2_rn(f2(step), __fadd2_rn(fi, f2(-8.0f)));
+    const float2 e = __fadd2_rn(z, make_float2(-c_idx.x, -c_idx.y));
+    const float2 A = __fmul2_rn(e, f2(step * l2t));
+    const float2 nB = f2(-(step * step * (0.5f * l2t)));
+    const float2 nfi = make_float2(-fi.x, -fi.y);
+    float2 s0 = f2(0.0f), s1 = f2(0.0f), s2 = f2(0.0f), s3 = f2(0.0f);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-        const float u = (float)j - fi;
-        p[j] = ex2_approx(u * fmaf(-B, u, A));
-        s0 += p[j];
-        s1 = fmaf(p[j], u, s1);
+        const float2 u = __fadd2_rn(f2((float)j), nfi);
+        const float2 arg = __fmul2_rn(u, __ffma2_rn(nB, u, A));
+        const float2 p = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+        s0 = __fadd2_rn(s0, p);
+        const float2 pu = __fmul2_rn(p, u);
+        s1 = __fadd2_rn(s1, pu);
+        s2 = __ffma2_rn(pu, u, s2);
+        s3 = __ffma2_rn(__fmul2_rn(pu, u), u, s3);
     }
-    const float inv = 1.0f / s0;                     // s0 >= 1: the nearest code has weight 1
-    const float mu = s1 * inv;
-    float m2 = 0.0f, m3 = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const float v = ((float)j - fi) - mu;
-        const float pvv = p[j] * v * v;
-        m2 += pvv;
-        m3 = fmaf(pvv, v, m3);
-    }
-    m2 *= inv;
-    m3 *= inv;
-    gz = up * ((r2 * step) * step * m2);
-    const float cov = (step * 0.125f) * fmaf(z - 2.0f * c_idx - 2.0f * step * mu, m2, -step * m3);
-    gs = up * ((fi - 8.0f) * 0.125f + (mu + fi - 8.0f) * 0.125f + r2 * cov);
+    // s0 is in [1, 16]: the nearest code has weight 1
+    const float2 inv = make_float2(rcp_approx(s0.x), rcp_approx(s0.y));
+    const float2 mu = __fmul2_rn(s1, inv), e2 = __fmul2_rn(s2, inv), e3 = __fmul2_rn(s3, inv);
+    const float2 m2 = __ffma2_rn(make_float2(-mu.x, -mu.y), mu, e2);                // E[u^2] - mu^2
+    // E[u^3] - 3 mu E[u^2] + 2 mu^3 = E[u^3] - mu (3 E[u^2] - 2 mu^2)
+    const float2 m3 = __ffma2_rn(make_float2(-mu.x, -mu.y),
+                                 __ffma2_rn(f2(-2.0f), __fmul2_rn(mu, mu), __fmul2_rn(f2(3.0f), e2)), e3);
+    gz = __fmul2_rn(up, __fmul2_rn(f2((r2 * step) * step), m2));
+    // z - 2 c_idx - 2 step mu
+    const float2 lin = __ffma2_rn(f2(-2.0f * step), mu, __ffma2_rn(f2(-2.0f), c_idx, z));
+    const float2 cov = __fmul2_rn(f2(step * 0.125f), __ffma2_rn(lin, m2, __fmul2_rn(f2(-step), m3)));
+    // (idx - 8)/8 from the hard term plus (mu + idx - 8)/8 + (2/tau) cov from the soft one
+    const float2 hard_soft = __fmul2_rn(__fadd2_rn(__ffma2_rn(f2(2.0f), fi, f2(-16.0f)), mu), f2(0.125f));
+    gs = __fmul2_rn(up, __ffma2_rn(f2(r2), cov, hard_soft));
 }
 
 // One thread: 8 consecutive elements; the 8 (group 64) or 4 (group 32) threads of a group
@@ -181,16 +197,22 @@ gumbel_st_backward_kernel(const float4* __restrict__ z, const uint16_t* __restri
             const bool fast = s >= 0x1p-96f && s <= 0x1p96f;
             const float c8 = fast ? 8.0f * rcp_fast(s) : 0.0f;
             const float step = s * 0.125f, m17 = -17.0f * s * 0.0625f;
-            const uint32_t zv[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-            const uint32_t gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            const float2 zp[4] = {make_float2(__uint_as_float(za.x), __uint_as_float(za.y)),
+                                  make_float2(__uint_as_float(za.z), __uint_as_float(za.w)),
+                                  make_float2(__uint_as_float(zb.x), __uint_as_float(zb.y)),
+                                  make_float2(__uint_as_float(zb.z), __uint_as_float(zb.w))};
+            const float2 gp[4] = {make_float2(__uint_as_float(ga.x), __uint_as_float(ga.y)),
+                                  make_float2(__uint_as_float(ga.z), __uint_as_float(ga.w)),
+                                  make_float2(__uint_as_float(gb.x), __uint_as_float(gb.y)),
+                                  make_float2(__uint_as_float(gb.z), __uint_as_float(gb.w))};
             uint32_t out[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float g, gsj;
-                gumbel_st_element(__uint_as_float(zv[j]), __uint_as_float(gv[j]), s, c8, step, m17,
-                                  fast, l2t, r2, g, gsj);
-                out[j] = __float_as_uint(g);
-                gsum += gsj;
+            for (int j = 0; j < 4; ++j) {
+                float2 g, gsj;
+                gumbel_st_pair(zp[j], gp[j], s, c8, step, m17, fast, l2t, r2, g, gsj);
+                out[2 * j] = __float_as_uint(g.x);
+                out[2 * j + 1] = __float_as_uint(g.y);
+                gsum += gsj.x + gsj.y;
             }
             stg_cs_v4(gz + 2 * i, make_uint4(out[0], out[1], out[2], out[3]));
             stg_cs_v4(gz + 2 * i + 1, make_uint4(out[4], out[5], out[6], out[7]));
