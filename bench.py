@@ -277,7 +277,9 @@ def run_ours(args):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": None, "peak_source": peaks["source"],
+                     # dram__bytes_read.sum + dram__bytes_write.sum of one launch of this
+                     # kernel at batch 1 (profiles/gemv_decode_sweep_b1.md)
+                     "traffic": 567902976 if B == 1 else None, "peak_source": peaks["source"],
                      "algorithmic_bytes_per_launch": algo_bytes, "kernel": "gemv_kernel (grouped)"},
         "e2e": e2e,
         "gpu_launches": args.steps,
@@ -698,7 +700,7 @@ def run_profile_target(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

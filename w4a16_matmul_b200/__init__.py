@@ -320,7 +320,9 @@ class GroupedGemv:
         _check(_lib.wq_gemv_plan_launch(self._plan, s))
 
     def close(self) -> None:
-        if getattr(self, "_plan", None) and self._plan.value:
+        # at interpreter shutdown the module globals may already be gone: the process is
+        # exiting and the plan's host memory goes with it
+        if getattr(self, "_plan", None) and self._plan.value and _lib is not None:
             _lib.wq_gemv_plan_destroy(self._plan)
             self._plan = _vp(None)
 

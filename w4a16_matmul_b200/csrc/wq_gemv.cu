@@ -48,7 +48,7 @@ constexpr int kMaxProblems = WQ_GEMV_MAX_GROUPED;
 #define WQ_GEMV_DEPTH 2
 #endif
 #ifndef WQ_GEMV_MIN_CTAS_NB1
-#define WQ_GEMV_MIN_CTAS_NB1 (WQ_GEMV_DEPTH >= 4 ? 4 : WQ_GEMV_DEPTH == 3 ? 5 : 6)
+#define WQ_GEMV_MIN_CTAS_NB1 (WQ_GEMV_DEPTH >= 4 ? 4 : 5)
 #endif
 #ifndef WQ_GEMV_MIN_CTAS_NB2
 #define WQ_GEMV_MIN_CTAS_NB2 4
@@ -491,26 +491,33 @@ constexpr int depth(int kind, int nb, int r) {
 // split-K kernels have 4 warps in total.
 constexpr int cta_warps(int wk, int fw) { return wk == 1 ? fw : 4; }
 
-// Resident CTAs per SM the register budget of a dyadic 16-row kernel aims at; the other
-// variants take what they need.
+// Resident warps per SM the register budget aims at. The dyadic 16-row kernels: 4-warp
+// CTAs (batch 1) at WQ_GEMV_MIN_CTAS_NB1 CTAs (measured on the decode sweep: 5 CTAs of
+// 96 registers beat 6 of 80 by 2-3 %, the fatter budget saving more instructions than the
+// lost warps cost), 8-warp CTAs (batch 2..8) at 24 warps; the other variants take what
+// they need.
 #ifndef WQ_GEMV_R2_CAP
 #define WQ_GEMV_R2_CAP 4
 #endif
 #ifndef WQ_GEMV_LUT_CAP
 #define WQ_GEMV_LUT_CAP 1
 #endif
-constexpr int min_ctas(int kind, int nb, int r) {
-    return kind >= kLut16 ? WQ_GEMV_LUT_CAP
-         : r == 1 ? (nb == 1 ? WQ_GEMV_MIN_CTAS_NB1 : WQ_GEMV_MIN_CTAS_NB2) : WQ_GEMV_R2_CAP;
+constexpr int min_warps(int kind, int nb, int r, int warps_per_cta) {
+    return kind >= kLut16 ? 4 * WQ_GEMV_LUT_CAP
+         : r != 1 ? 4 * WQ_GEMV_R2_CAP
+         : nb != 1 ? 4 * WQ_GEMV_MIN_CTAS_NB2
+         : warps_per_cta == 4 ? 4 * WQ_GEMV_MIN_CTAS_NB1 : 24;
+}
+constexpr int min_blocks(int kind, int nb, int r, int warps_per_cta) {
+    return min_warps(kind, nb, r, warps_per_cta) / warps_per_cta > 0
+               ? min_warps(kind, nb, r, warps_per_cta) / warps_per_cta : 1;
 }
 
 // CL > 1: a thread-block cluster of CL CTAs shares each row tile, CTA rank c taking a
 // contiguous slice of the K steps; the partial sums meet in rank 0's shared memory over the
 // cluster (distributed shared memory), between two cluster barriers.
 template <int KIND, int NB, int R, int WK, int FW, int MAXP, int CL>
-__global__ void __launch_bounds__(32 * cta_warps(WK, FW),
-                                  (min_ctas(KIND, NB, R) * 4 / cta_warps(WK, FW)) > 0
-                                      ? (min_ctas(KIND, NB, R) * 4 / cta_warps(WK, FW)) : 1)
+__global__ void __launch_bounds__(32 * cta_warps(WK, FW), min_blocks(KIND, NB, R, cta_warps(WK, FW)))
 gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     static_assert(CL == 1 || WK == 1, "a cluster splits K across CTAs, not within one");
     constexpr int THREADS = 32 * cta_warps(WK, FW);
