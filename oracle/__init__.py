@@ -19,6 +19,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
+import threading
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -42,7 +43,18 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+_lib_lock = threading.Lock()
+
+
 def _L():
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lib_lock:                 # the row-parallel callers arrive from several threads
+        return _load()
+
+
+def _load():
     global _lib
     if _lib is None:
         build()
@@ -69,6 +81,10 @@ def _L():
             "orc_lloyd_num_candidates": [],
             "orc_bf16x_encode": [vp, i64, i64, vp, vp, vp, vp, i64, vp],
             "orc_bf16x_decode": [vp, vp, vp, vp, i64, i64, i64, vp],
+            "orc_wf_analyze": [vp, i64, i64, ctypes.c_double, i64, i64, vp, vp, vp],
+            "orc_wf_offsets": [vp, i64, vp],
+            "orc_wf_pack": [vp, i64, i64, vp, vp, vp, i64, i64, vp],
+            "orc_wf_dequant": [vp, vp, vp, vp, i64, i64, i64, i64, vp],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -351,4 +367,56 @@ def bf16x_decode(enc: dict, n: int, k: int) -> np.ndarray:
                                ovf.size, n, k, _p(out))
     if rc != 0:
         raise ValueError(f"orc_bf16x_decode: {rc}")
+    return out
+
+
+# --- [DG] water-filling (3/4/5-bit blocks in one index space) ------------------------------
+
+def wf_analyze(w_bits: np.ndarray, lam: float, threads: int | None = None):
+    """Per 64-weight block: (scale bf16 bits [n, k/64], width uint8 [n, k/64], dist fp64
+    [n, k/64, 3] = squared error at 3, 4, 5 bits)."""
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    n, k = w.shape
+    scale = np.empty((n, k // 64), np.uint16)
+    width = np.empty((n, k // 64), np.uint8)
+    dist = np.empty((n, k // 64, 3), np.float64)
+    _rows_parallel(n, lambda r0, r1: _L().orc_wf_analyze(_p(w), n, k, float(lam), r0, r1, _p(scale),
+                                                         _p(width), _p(dist)), threads)
+    return scale, width, dist
+
+
+def wf_offsets(width: np.ndarray) -> np.ndarray:
+    """Byte offset of every block (8 * width bytes each, row-major) and the total."""
+    wd = np.ascontiguousarray(width, dtype=np.uint8).reshape(-1)
+    off = np.empty(wd.size + 1, np.uint32)
+    rc = _L().orc_wf_offsets(_p(wd), wd.size, _p(off))
+    if rc != 0:
+        raise ValueError(f"orc_wf_offsets: {rc}")
+    return off
+
+
+def wf_pack(w_bits: np.ndarray, scale: np.ndarray, width: np.ndarray, blk_off: np.ndarray,
+            threads: int | None = None) -> np.ndarray:
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    n, k = w.shape
+    scale = np.ascontiguousarray(scale, dtype=np.uint16)
+    width = np.ascontiguousarray(width, dtype=np.uint8)
+    blk_off = np.ascontiguousarray(blk_off, dtype=np.uint32)
+    packed = np.zeros(int(blk_off[-1]), np.uint8)
+    _rows_parallel(n, lambda r0, r1: _L().orc_wf_pack(_p(w), n, k, _p(scale), _p(width), _p(blk_off),
+                                                      r0, r1, _p(packed)), threads)
+    return packed
+
+
+def wf_dequant(packed: np.ndarray, scale: np.ndarray, width: np.ndarray, blk_off: np.ndarray,
+               n: int, k: int, threads: int | None = None) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    if packed.size == 0:
+        packed = np.zeros(1, np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.uint16)
+    width = np.ascontiguousarray(width, dtype=np.uint8)
+    blk_off = np.ascontiguousarray(blk_off, dtype=np.uint32)
+    out = np.empty((n, k), np.uint16)
+    _rows_parallel(n, lambda r0, r1: _L().orc_wf_dequant(_p(packed), _p(scale), _p(width), _p(blk_off),
+                                                         n, k, r0, r1, _p(out)), threads)
     return out

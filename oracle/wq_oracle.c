@@ -830,3 +830,144 @@ int orc_bf16x_decode(const uint8_t* sm, const uint64_t* hdr, const uint32_t* sb_
     if (sb_off[(nblocks + 15) / 16] != (uint32_t)next || next != n_ovf) return -3;
     return 0;
 }
+
+/* ------------------------------------------------------------------------------- */
+/* [DG] water-filling: 3/4/5-bit dyadic blocks in one level index space             */
+/* ------------------------------------------------------------------------------- */
+/*
+ * [DG] §2.1: with half = 2^(b-1) and step = scale / half, the b-bit codebook is
+ * step * {-half, ..., half - 1}; codebooks of different b line up, so when water-filling
+ * changes one block's precision the 3/4/5-bit codes share one level index space and the
+ * codebook need not be rebuilt. [DG] §6 leaves water-filling disabled and says no more.
+ * Readings taken here (the page fixes neither the allocation rule nor the layout):
+ *   block     64 consecutive weights of a row (the §2.2 block), scale = max |w| (bf16).
+ *   codes     for b in {3, 4, 5}: idx_b = argmin_j |w - (j - half_b) * scale / half_b|
+ *             over j = 0 .. 2^b - 1, lowest j on a tie (the 4-bit rule of §2.3).
+ *   index     idx_5 = idx_b * 2^(5 - b): the same value step_5 * (idx_5 - 16).
+ *   D_b       the block's squared error sum_j (w_j - code)^2. Each difference is exact in
+ *             float and double (the code is zero, or within a factor of two of w), each
+ *             square is exact in double; the sum runs over j = 0..63 in order, in double.
+ *   width     the water level lambda (a distortion per weight, chosen by the caller):
+ *             the smallest b in {3, 4, 5} with D_b <= 64 * lambda, else 5. Blocks whose
+ *             3-bit error already lies under the water keep 3 bits; the others get bits
+ *             until their error does, up to 5 (reverse water-filling with three rates).
+ *   layout    scale bf16 [n, k/64]; width uint8 [n, k/64]; the blocks' bit streams back to
+ *             back in row-major block order, block i taking 8 * width_i bytes, its code j
+ *             in bits [b j, b j + b) counted from bit 0 of the block's first byte (for
+ *             b = 4 this is the nibble layout of §2.5); blk_off uint32 [n k/64 + 1]: the
+ *             byte offset of every block, and the total at the end.
+ */
+
+/* idx_b by a plain search over the 2^b codes (lowest index on a tie) */
+static int wf_index(double w, double scale, int b)
+{
+    const int half = 1 << (b - 1);
+    const double step = scale / half;
+    int best = 0;
+    double bestd = fabs(w - (0 - half) * step);
+    for (int j = 1; j < (1 << b); ++j) {
+        const double d = fabs(w - (j - half) * step);
+        if (d < bestd) { bestd = d; best = j; }
+    }
+    return best;
+}
+
+/* Per block: scale, the three distortions (dist may be NULL: [n, k/64, 3] for b = 3, 4, 5),
+ * the width for water level lambda, and blk_size = 8 * width bytes. */
+int orc_wf_analyze(const uint16_t* w, int64_t n, int64_t k, double lambda, int64_t r0, int64_t r1,
+                   uint16_t* scale, uint8_t* width, double* dist)
+{
+    (void)n;
+    if (k % 64 != 0) return -1;
+    if (!(lambda >= 0.0)) return -3;
+    const int64_t nb = k / 64;
+    for (int64_t r = r0; r < r1; ++r) {
+        for (int64_t g = 0; g < nb; ++g) {
+            const uint16_t* wg = w + r * k + g * 64;
+            double amax = 0.0;
+            for (int j = 0; j < 64; ++j) {
+                const double v = orc_bf16_to_double(wg[j]);
+                if (!isfinite(v)) return -2;
+                if (fabs(v) > amax) amax = fabs(v);
+            }
+            scale[r * nb + g] = orc_double_to_bf16(amax);
+            int chosen = 5;
+            for (int b = 3; b <= 5; ++b) {
+                const int half = 1 << (b - 1);
+                double D = 0.0;
+                for (int j = 0; j < 64; ++j) {
+                    const double v = orc_bf16_to_double(wg[j]);
+                    const int idx = wf_index(v, amax, b);
+                    const double e = v - (idx - half) * (amax / half);
+                    D += e * e;
+                }
+                if (dist) dist[(r * nb + g) * 3 + (b - 3)] = D;
+                if (chosen == 5 && b < 5 && D <= 64.0 * lambda) chosen = b;
+            }
+            width[r * nb + g] = (uint8_t)chosen;
+        }
+    }
+    return 0;
+}
+
+/* blk_off[0..nblocks] = exclusive prefix of 8 * width, total at the end */
+int orc_wf_offsets(const uint8_t* width, int64_t nblocks, uint32_t* blk_off)
+{
+    uint64_t off = 0;
+    for (int64_t i = 0; i < nblocks; ++i) {
+        if (width[i] < 3 || width[i] > 5) return -2;
+        blk_off[i] = (uint32_t)off;
+        off += 8u * width[i];
+        if (off >= ((uint64_t)1 << 32)) return -4;
+    }
+    blk_off[nblocks] = (uint32_t)off;
+    return 0;
+}
+
+/* The blocks' codes at their widths, bit-packed (layout above). */
+int orc_wf_pack(const uint16_t* w, int64_t n, int64_t k, const uint16_t* scale, const uint8_t* width,
+                const uint32_t* blk_off, int64_t r0, int64_t r1, uint8_t* packed)
+{
+    (void)n;
+    if (k % 64 != 0) return -1;
+    const int64_t nb = k / 64;
+    for (int64_t r = r0; r < r1; ++r)
+        for (int64_t g = 0; g < nb; ++g) {
+            const int b = width[r * nb + g];
+            if (b < 3 || b > 5) return -2;
+            const double s = orc_bf16_to_double(scale[r * nb + g]);
+            uint8_t* out = packed + blk_off[r * nb + g];
+            memset(out, 0, (size_t)(8 * b));
+            for (int j = 0; j < 64; ++j) {
+                const int idx = wf_index(orc_bf16_to_double(w[r * k + g * 64 + j]), s, b);
+                for (int t = 0; t < b; ++t)
+                    if ((idx >> t) & 1) out[(b * j + t) / 8] |= (uint8_t)(1u << ((b * j + t) % 8));
+            }
+        }
+    return 0;
+}
+
+/* Reconstruction through the 5-bit index space: idx_5 = idx_b << (5 - b),
+ * w = bf16((scale / 16) * (idx_5 - 16)). */
+int orc_wf_dequant(const uint8_t* packed, const uint16_t* scale, const uint8_t* width,
+                   const uint32_t* blk_off, int64_t n, int64_t k, int64_t r0, int64_t r1, uint16_t* out)
+{
+    (void)n;
+    if (k % 64 != 0) return -1;
+    const int64_t nb = k / 64;
+    for (int64_t r = r0; r < r1; ++r)
+        for (int64_t g = 0; g < nb; ++g) {
+            const int b = width[r * nb + g];
+            if (b < 3 || b > 5) return -2;
+            const double s = orc_bf16_to_double(scale[r * nb + g]);
+            const uint8_t* in = packed + blk_off[r * nb + g];
+            for (int j = 0; j < 64; ++j) {
+                int idx = 0;
+                for (int t = 0; t < b; ++t)
+                    idx |= ((in[(b * j + t) / 8] >> ((b * j + t) % 8)) & 1) << t;
+                const int idx5 = idx << (5 - b);
+                out[r * k + g * 64 + j] = orc_double_to_bf16(s / 16.0 * (idx5 - 16));
+            }
+        }
+    return 0;
+}

@@ -1,0 +1,154 @@
+"""Pins of the oracle's water-filling coder ("MiniCPM5-1B 验证…" §2.1: 3/4/5-bit dyadic
+codebooks in one level index space; §6: water-filling, not enabled there): a hand-worked
+block (tests/golden/wf_worked_example.txt), the nesting of the three codebooks (the
+distortion cannot grow with the width), the water-level rule itself, brute-force argmin,
+agreement of the 4-bit blocks with the dyadic 4-bit quantiser and packer, and the
+reconstruction through the 5-bit index space against the b-bit closed form."""
+import os
+
+import numpy as np
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "wf_worked_example.txt")
+
+
+def _golden():
+    out = {}
+    for line in open(GOLDEN):
+        if line.startswith("#") or not line.strip():
+            continue
+        key, *vals = line.split()
+        out[key] = [float(v) for v in vals] if key[0] in "Dl" else bytes(int(v, 16) for v in vals)
+    return out
+
+
+def _worked_block():
+    w = np.full((1, 64), 0.125)
+    w[0, 0] = -1.0
+    return workloads.f64_to_bf16_bits(w)
+
+
+def test_hand_worked_block():
+    g = _golden()
+    w = _worked_block()
+    thr = g["lambda_threshold"][0]
+    for lam, width in [(thr, 3), (np.nextafter(thr, 0.0), 4), (0.0, 4)]:
+        scale, wd, dist = oracle.wf_analyze(w, lam)
+        assert oracle.bf16_to_f64(scale)[0, 0] == 1.0
+        assert list(dist[0, 0]) == [g["D3"][0], g["D4"][0], g["D5"][0]]
+        assert wd[0, 0] == width
+        off = oracle.wf_offsets(wd)
+        assert list(off) == [0, 8 * width]
+        packed = oracle.wf_pack(w, scale, wd, off)
+        assert packed.tobytes() == g[f"bytes{width}"]
+        rec = oracle.wf_dequant(packed, scale, wd, off, 1, 64)
+        if width == 4:
+            assert np.array_equal(rec, w)                   # on the 4-bit grid: exact
+        else:                                               # 0.125 fell to code 4, i.e. +0.0
+            assert rec[0, 0] == w[0, 0] and np.all(rec[0, 1:] == 0)
+    # a forced 5-bit block (lambda < 0 is rejected, so compare the 5-bit stream through the
+    # packer with width 5 set by hand)
+    scale, _, _ = oracle.wf_analyze(w, 0.0)
+    wd5 = np.array([[5]], np.uint8)
+    off5 = oracle.wf_offsets(wd5)
+    assert oracle.wf_pack(w, scale, wd5, off5).tobytes() == g["bytes5"]
+
+
+def _rand(seed, n=16, k=512):
+    g = np.random.default_rng(seed)
+    w = g.standard_normal((n, k)) * 0.02 * g.uniform(0.2, 3.0, (n, 1))
+    w[g.random((n, k)) < 0.01] *= 20
+    return workloads.f64_to_bf16_bits(w)
+
+
+def test_distortion_cannot_grow_with_width():
+    # 3-bit codes are 4-bit codes are 5-bit codes (nested grids): D5 <= D4 <= D3 exactly
+    _, _, dist = oracle.wf_analyze(_rand(1), 0.0)
+    assert np.all(dist[..., 2] <= dist[..., 1]) and np.all(dist[..., 1] <= dist[..., 0])
+    assert np.all(dist[..., 2] < dist[..., 0])                # random data is never on the grid
+
+
+def test_water_level_rule():
+    w = _rand(2)
+    _, _, dist = oracle.wf_analyze(w, 0.0)
+    for lam in np.quantile(dist[..., 1].reshape(-1) / 64, [0.1, 0.5, 0.9]):
+        _, wd, d = oracle.wf_analyze(w, lam)
+        b = wd.astype(int)
+        assert set(np.unique(b)) <= {3, 4, 5}
+        D_at = np.take_along_axis(d, (b - 3)[..., None], axis=-1)[..., 0]
+        assert np.all((D_at <= 64 * lam) | (b == 5))           # under the water, or capped
+        below = np.take_along_axis(d, np.maximum(b - 4, 0)[..., None], axis=-1)[..., 0]
+        assert np.all((below > 64 * lam) | (b == 3))           # one bit fewer would not do
+    # very high water: everything at 3 bits; zero water: only exact blocks below 5
+    _, wd, _ = oracle.wf_analyze(w, 1e30)
+    assert np.all(wd == 3)
+    _, wd, _ = oracle.wf_analyze(w, 0.0)
+    assert np.all(wd == 5)
+
+
+def test_argmin_brute_force_and_ties():
+    # tiny blocks against numpy's argmin (first minimum = lowest index) at every width
+    g = np.random.default_rng(3)
+    w = workloads.f64_to_bf16_bits(g.standard_normal((3, 64)) * 0.05)
+    scale, _, _ = oracle.wf_analyze(w, 0.0)
+    s = oracle.bf16_to_f64(scale)
+    v = oracle.bf16_to_f64(w)
+    for b in (3, 4, 5):
+        half = 2 ** (b - 1)
+        wd = np.full((3, 1), b, np.uint8)
+        off = oracle.wf_offsets(wd)
+        packed = oracle.wf_pack(w, scale, wd, off)
+        codes = np.arange(2 ** b) - half
+        want = np.argmin(np.abs(v[..., None] - s[:, :1, None] / half * codes), axis=-1)
+        # unpack the b-bit stream by integer arithmetic on the whole block
+        for r in range(3):
+            blk = int.from_bytes(packed[off[r]:off[r + 1]].tobytes(), "little")
+            got = [(blk >> (b * j)) & (2 ** b - 1) for j in range(64)]
+            assert got == list(want[r])
+
+
+def test_four_bit_blocks_are_the_dyadic_format():
+    w = _rand(4, n=8, k=1024)
+    _, _, dist = oracle.wf_analyze(w, 0.0)
+    lam = float(np.median(dist[..., 1]) / 64)
+    scale, wd, _ = oracle.wf_analyze(w, lam)
+    off = oracle.wf_offsets(wd)
+    packed = oracle.wf_pack(w, scale, wd, off)
+    s4, c4 = oracle.dyadic_quantize(w, 64)
+    p4 = oracle.pack(c4)
+    assert np.array_equal(s4, scale)
+    rec = oracle.wf_dequant(packed, scale, wd, off, 8, 1024)
+    d4 = oracle.dyadic_dequant(c4, s4, 64)
+    n4 = 0
+    for r in range(8):
+        for g_ in range(16):
+            i = r * 16 + g_
+            if wd[r, g_] == 4:
+                n4 += 1
+                assert packed[off[i]:off[i + 1]].tobytes() == p4[r, 32 * g_:32 * g_ + 32].tobytes()
+                assert np.array_equal(rec[r, 64 * g_:64 * g_ + 64], d4[r, 64 * g_:64 * g_ + 64])
+    assert n4 > 0
+
+
+def test_reconstruction_through_the_five_bit_index_space():
+    # the 5-bit mapping idx5 = idx_b << (5 - b) must give bf16(step_b * (idx_b - half_b))
+    w = _rand(5, n=6, k=256)
+    _, _, dist = oracle.wf_analyze(w, 0.0)
+    lam = float(np.quantile(dist[..., 1], 0.4) / 64)
+    scale, wd, _ = oracle.wf_analyze(w, lam)
+    off = oracle.wf_offsets(wd)
+    packed = oracle.wf_pack(w, scale, wd, off)
+    rec = oracle.wf_dequant(packed, scale, wd, off, 6, 256)
+    s = oracle.bf16_to_f64(scale)
+    for r in range(6):
+        for g_ in range(4):
+            b = int(wd[r, g_])
+            i = r * 4 + g_
+            blk = int.from_bytes(packed[off[i]:off[i + 1]].tobytes(), "little")
+            idx = np.array([(blk >> (b * j)) & (2 ** b - 1) for j in range(64)], np.float64)
+            want = oracle.f64_to_bf16(s[r, g_] / 2 ** (b - 1) * (idx - 2 ** (b - 1)))
+            assert np.array_equal(rec[r, 64 * g_:64 * g_ + 64], want)
+    # and the storage: 8 * width bytes per block, plus a bf16 scale and a width byte
+    assert off[-1] == 8 * int(wd.astype(np.int64).sum())
