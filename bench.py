@@ -428,7 +428,37 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
                               "encode_frac_hbm": round(enc_b / ms_e / 1e6 / peaks["hbm_gbs"], 4),
                               "decode_us": round(ms_d * 1e3, 1), "decode_GB/s": round(dec_b / ms_d / 1e6, 1),
                               "decode_frac_hbm": round(dec_b / ms_d / 1e6 / peaks["hbm_gbs"], 4)}
-        del ge, gd, enc, wb, dout
+        del ge, gd, enc, dout
+        # water-filling 3/4/5-bit blocks on the same matrix, water level at the median 4-bit
+        # squared error (about 4.5 bits per weight): both producer passes (analyze with the
+        # offset scan, pack) and the dequant
+        nblk = n_l * k_l // 64
+        sc, wd, off, dd = wq.wf_analyze(wb, 0.0, dist=True)
+        lam = float(dd[..., 1].median()) / 64
+        del dd
+        pk = torch.empty(40 * nblk, dtype=torch.uint8, device=dev)
+
+        def wf_q():
+            wq._check(wq._lib.wq_quantize_wf_analyze(wq._ptr(wb), n_l, k_l, lam, wq._ptr(sc), wq._ptr(wd),
+                                                     wq._ptr(off), None, wq._stream(wb)))
+            wq._check(wq._lib.wq_quantize_wf_pack(wq._ptr(wb), n_l, k_l, wq._ptr(sc), wq._ptr(wd), wq._ptr(off),
+                                                  wq._ptr(pk), pk.numel(), wq._stream(wb)))
+        gq_ = graph_of(torch, wf_q)
+        ms_q = max_over_ranks(time_region(torch, stream, gq_.replay, steps, warm, barrier))
+        total = int(off[-1].item()) & 0xFFFFFFFF
+        dwf = torch.empty_like(wb)
+        gdw = graph_of(torch, lambda: wq._check(wq._lib.wq_dequant_wf(
+            wq._ptr(pk), pk.numel(), wq._ptr(sc), wq._ptr(wd), wq._ptr(off), n_l, k_l, wq._ptr(dwf), wq._stream(wb))))
+        ms_dq = max_over_ranks(time_region(torch, stream, gdw.replay, steps, warm, barrier))
+        side = nblk * (2 + 1 + 4)                          # scale, width, offset per block
+        dq_b = total + side + nw * 2
+        out["water_filling_large"] = {"shape": [n_l, k_l], "lambda": lam,
+                                      "bits_per_weight": round(8 * total / nw, 3),
+                                      "quantize_us": round(ms_q * 1e3, 1),
+                                      "quantize_Gweights/s": round(nw / ms_q / 1e6, 2),
+                                      "dequant_us": round(ms_dq * 1e3, 1), "dequant_GB/s": round(dq_b / ms_dq / 1e6, 1),
+                                      "dequant_frac_hbm": round(dq_b / ms_dq / 1e6 / peaks["hbm_gbs"], 4)}
+        del gq_, gdw, sc, wd, off, pk, dwf, wb
     except Exception as e:
         out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
     if args.extras in ("gemm", "all"):
@@ -640,7 +670,8 @@ def run_profile_target(args):
     """A few launches of one kernel on one shape and nothing else, for ncu captures:
     --profile gemm --shape N,K,M (prefill GEMM), quantize --shape N,K, dequant --shape N,K,
     lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd), gumbel --shape N,K
-    (Gumbel-ST backward), bf16x --shape N,K (BF16X encode + decode). Random packed codes and
+    (Gumbel-ST backward), bf16x --shape N,K (BF16X encode + decode), wf --shape N,K
+    (water-filling analyze + dequant). Random packed codes and
     scales (timing does not depend on the values); inputs stay on the device."""
     import torch
     import __graft_entry__
@@ -683,6 +714,11 @@ def run_profile_target(args):
         enc = wq.bf16x_encode(w)
         out = torch.empty_like(w)
         fn = lambda: (wq.bf16x_encode_into(w, enc), wq.bf16x_decode(enc, out=out))
+    elif args.profile == "wf":
+        w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+        q = wq.quantize_wf(w, 1e-6)
+        out = torch.empty_like(w)
+        fn = lambda: (wq.wf_analyze(w, 1e-6), wq.dequant_wf(q, out=out))
     elif args.profile == "lloyd":
         w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
         fn = lambda: wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)

@@ -314,6 +314,49 @@ wq_status wq_bf16x_decode(const uint8_t* sm, const uint64_t* hdr, const uint32_t
                           const uint8_t* ovf, int64_t ovf_bytes, int64_t n, int64_t k,
                           uint16_t* out, wq_stream stream);
 
+/* ------------------------------------------------------------------------------------ */
+/* Water-filling: 3/4/5-bit dyadic blocks in one level index space ([DG] §2.1, §6)       */
+/* ------------------------------------------------------------------------------------ */
+/* [DG] §2.1: with half = 2^(b-1) and step = scale / half the b-bit codebook is
+ * step * {-half .. half-1}; the 3/4/5-bit codebooks line up, so a block's precision can
+ * change without rebuilding the codebook: code idx_b of a b-bit block is code
+ * idx_5 = idx_b << (5 - b) of the 5-bit codebook, reconstructed as bf16((scale / 16) *
+ * (idx_5 - 16)). [DG] §6 leaves the allocation disabled; this library's reading of it:
+ *   block   64 consecutive weights of a row; scale = max |w| (bf16, exact).
+ *   codes   idx_b = argmin_j |w - (j - half) * step| over j = 0 .. 2^b - 1, lowest j on a tie.
+ *   D_b     the block's squared error sum (w - code)^2 at b bits (each term exact in double,
+ *           summed over the block's weights in order, in double).
+ *   width   the smallest b in {3, 4, 5} with D_b <= 64 * lambda (the water level lambda, a
+ *           squared error per weight), else 5. A bit budget is met by the choice of lambda
+ *           (dist lets the caller pick it).
+ *   layout  scale bf16 [n, k/64]; width uint8 [n, k/64]; packed: the blocks' bit streams back
+ *           to back in row-major block order, block i taking 8 * width_i bytes, code j in
+ *           bits [b j, b j + b) counted from bit 0 of the block's first byte (b = 4 gives the
+ *           nibble layout of wq_pack); blk_off uint32 [n k/64 + 1]: each block's byte offset,
+ *           and the total byte count at the end.
+ * k must be a multiple of 64 and n * k / 64 * 40 below 2^32. Results are bit-exact. */
+
+/* Pass 1: scale, width and blk_off for water level lambda (>= 0; +inf gives 3 bits
+ * everywhere); dist (may be NULL) receives D_3, D_4, D_5 as fp64 [n, k/64, 3]. The caller
+ * reads blk_off[n k/64] back to size packed. */
+wq_status wq_quantize_wf_analyze(const uint16_t* w, int64_t n, int64_t k, double lambda,
+                                 uint16_t* scale, uint8_t* width, uint32_t* blk_off, double* dist,
+                                 wq_stream stream);
+
+/* Pass 2: the codes at each block's width into packed (packed_bytes allocated, at least
+ * blk_off[n k/64]). A block that does not fit, or a width outside 3..5, is skipped and
+ * flagged for wq_device_error. */
+wq_status wq_quantize_wf_pack(const uint16_t* w, int64_t n, int64_t k, const uint16_t* scale,
+                              const uint8_t* width, const uint32_t* blk_off, uint8_t* packed,
+                              int64_t packed_bytes, wq_stream stream);
+
+/* out = bf16 [n, k] reconstruction through the 5-bit index space (bit-exact). A block
+ * outside packed_bytes, or a width outside 3..5, gives zeros and is flagged for
+ * wq_device_error. */
+wq_status wq_dequant_wf(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
+                        const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
+                        uint16_t* out, wq_stream stream);
+
 /* The GEMM above without a caller workspace, for callers that cannot allocate device
  * memory: e.g. an inference server whose caching allocator owns the whole device memory
  * budget and forbids any other cudaMalloc, a plugin that may only use the buffers its host

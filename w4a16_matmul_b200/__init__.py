@@ -67,6 +67,9 @@ _SIG = {
     "wq_gemm_w4a16_static": ([_WP, _vp, _i64, _vp, _vp], _i32),
     "wq_debug_fail_next_launches": ([_i32], None),
     "wq_device_error": ([ctypes.POINTER(_i32)], _i32),
+    "wq_quantize_wf_analyze": ([_vp, _i64, _i64, ctypes.c_double, _vp, _vp, _vp, _vp, _vp], _i32),
+    "wq_quantize_wf_pack": ([_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp], _i32),
+    "wq_dequant_wf": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp], _i32),
     "wq_bf16x_superblocks": ([_i64, _i64], _i64),
     "wq_bf16x_count": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "wq_bf16x_encode": ([_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp], _i32),
@@ -411,4 +414,51 @@ def bf16x_decode(b: Bf16xWeight, out: torch.Tensor | None = None) -> torch.Tenso
         out = torch.empty((b.n, b.k), dtype=torch.bfloat16, device=b.sm.device)
     _check(_lib.wq_bf16x_decode(_ptr(b.sm), _ptr(b.hdr), _ptr(b.sb_off), _ptr(b.ovf), b.ovf.numel(),
                                 b.n, b.k, _ptr(out), _stream(out)))
+    return out
+
+
+# --- water-filling 3/4/5-bit dyadic blocks --------------------------------------------------
+@dataclass
+class WfWeight:
+    """A bf16 [n, k] matrix as water-filled dyadic blocks (layout in include/wq.h). blk_off is
+    uint32 held in an int32 tensor."""
+    n: int
+    k: int
+    scale: torch.Tensor     # bf16 [n, k/64]
+    width: torch.Tensor     # uint8 [n, k/64]
+    blk_off: torch.Tensor   # int32 [n k/64 + 1]
+    packed: torch.Tensor    # uint8 [max(total, 16)]
+    total: int              # bytes of packed in use
+
+
+def wf_analyze(w: torch.Tensor, lam: float, dist: bool = False):
+    """Pass 1 of water-filling: (scale, width, blk_off, dist | None)."""
+    _cuda(w, torch.bfloat16, "w")
+    n, k = w.shape
+    dev = w.device
+    scale = torch.empty((n, k // 64), dtype=torch.bfloat16, device=dev)
+    width = torch.empty((n, k // 64), dtype=torch.uint8, device=dev)
+    off = torch.empty(n * (k // 64) + 1, dtype=torch.int32, device=dev)
+    d = torch.empty((n, k // 64, 3), dtype=torch.float64, device=dev) if dist else None
+    _check(_lib.wq_quantize_wf_analyze(_ptr(w), n, k, float(lam), _ptr(scale), _ptr(width), _ptr(off),
+                                       _ptr(d), _stream(w)))
+    return scale, width, off, d
+
+
+def quantize_wf(w: torch.Tensor, lam: float) -> WfWeight:
+    """Water-filling quantisation at water level lam. Synchronises once, to size packed."""
+    n, k = w.shape
+    scale, width, off, _ = wf_analyze(w, lam)
+    total = int(off[-1].item()) & 0xFFFFFFFF
+    packed = torch.empty(max(total, 16), dtype=torch.uint8, device=w.device)
+    _check(_lib.wq_quantize_wf_pack(_ptr(w), n, k, _ptr(scale), _ptr(width), _ptr(off), _ptr(packed),
+                                    packed.numel(), _stream(w)))
+    return WfWeight(n, k, scale, width, off, packed, total)
+
+
+def dequant_wf(q: WfWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((q.n, q.k), dtype=torch.bfloat16, device=q.packed.device)
+    _check(_lib.wq_dequant_wf(_ptr(q.packed), q.packed.numel(), _ptr(q.scale), _ptr(q.width),
+                              _ptr(q.blk_off), q.n, q.k, _ptr(out), _stream(out)))
     return out

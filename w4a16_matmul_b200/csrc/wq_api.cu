@@ -154,14 +154,78 @@ wq_status wq_device_error(int32_t* code) {
     if (!code) return fail(WQ_EINVAL, "code is NULL");
     wq_status st = read_device_error(code);
     if (st) return st;
-    int32_t data = 0;
+    int32_t data = 0, wf = 0;
     if ((st = read_bf16x_error(&data))) return st;
+    if ((st = read_wf_error(&wf))) return st;
     if (*code != 0) return fail(WQ_ETIMEOUT, "a bounded device wait expired (code %d)", *code);
     if (data != 0) {
         *code = data;
         return fail(WQ_EDATA, "BF16X overflow index past ovf_bytes (code %d)", data);
     }
+    if (wf != 0) {
+        *code = wf;
+        return fail(WQ_EDATA, "water-filling block outside packed_bytes or bad width (code %d)", wf);
+    }
     return WQ_OK;
+}
+
+// Water-filling sizes: the usual matrix checks, k a multiple of 64, and every block offset
+// (at most 40 bytes per block) below 2^32.
+static wq_status check_wf_shape(int64_t n, int64_t k) {
+    wq_status st = check_shape(n, k, 64);
+    if (st) return st;
+    if (n * (k / 64) * 40 >= (1LL << 32))
+        return fail(WQ_EINVAL, "n * k / 64 * 40 bytes must stay below 2^32 (n=%lld, k=%lld)",
+                    (long long)n, (long long)k);
+    return WQ_OK;
+}
+
+wq_status wq_quantize_wf_analyze(const uint16_t* w, int64_t n, int64_t k, double lambda,
+                                 uint16_t* scale, uint8_t* width, uint32_t* blk_off, double* dist,
+                                 wq_stream stream) {
+    g_last_error[0] = 0;
+    wq_status st = check_wf_shape(n, k);
+    if (st) return st;
+    if (!(lambda >= 0.0)) return fail(WQ_EINVAL, "lambda must be >= 0 (got %g)", lambda);
+    if ((st = check_ptr(w, "w", false))) return st;
+    if ((st = check_ptr(scale, "scale", false))) return st;
+    if ((st = check_ptr(width, "width", false))) return st;
+    if ((st = check_ptr(blk_off, "blk_off", false))) return st;
+    if ((st = check_ptr(dist, "dist", true))) return st;
+    if ((st = check_injected())) return st;
+    return launch_wf_analyze(w, n, k, lambda, scale, width, blk_off, dist, (cudaStream_t)stream);
+}
+
+wq_status wq_quantize_wf_pack(const uint16_t* w, int64_t n, int64_t k, const uint16_t* scale,
+                              const uint8_t* width, const uint32_t* blk_off, uint8_t* packed,
+                              int64_t packed_bytes, wq_stream stream) {
+    g_last_error[0] = 0;
+    wq_status st = check_wf_shape(n, k);
+    if (st) return st;
+    if (packed_bytes < 0) return fail(WQ_EINVAL, "packed_bytes must be >= 0");
+    if ((st = check_ptr(w, "w", false))) return st;
+    if ((st = check_ptr(scale, "scale", false))) return st;
+    if ((st = check_ptr(width, "width", false))) return st;
+    if ((st = check_ptr(blk_off, "blk_off", false))) return st;
+    if ((st = check_ptr(packed, "packed", false))) return st;
+    if ((st = check_injected())) return st;
+    return launch_wf_pack(w, n, k, scale, width, blk_off, packed, packed_bytes, (cudaStream_t)stream);
+}
+
+wq_status wq_dequant_wf(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
+                        const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
+                        uint16_t* out, wq_stream stream) {
+    g_last_error[0] = 0;
+    wq_status st = check_wf_shape(n, k);
+    if (st) return st;
+    if (packed_bytes < 0) return fail(WQ_EINVAL, "packed_bytes must be >= 0");
+    if ((st = check_ptr(packed, "packed", false))) return st;
+    if ((st = check_ptr(scale, "scale", false))) return st;
+    if ((st = check_ptr(width, "width", false))) return st;
+    if ((st = check_ptr(blk_off, "blk_off", false))) return st;
+    if ((st = check_ptr(out, "out", false))) return st;
+    if ((st = check_injected())) return st;
+    return launch_wf_dequant(packed, packed_bytes, scale, width, blk_off, n, k, out, (cudaStream_t)stream);
 }
 
 int64_t wq_bf16x_superblocks(int64_t n, int64_t k) {

@@ -106,7 +106,7 @@ __device__ __forceinline__ uint32_t half_emax(const uint4 w) {
 //   tile final  one CTA per tile: entry s = O_t + the escapes of the tile's earlier
 //               superblocks; the last tile's CTA writes sb_off[S] = the total.
 // Every launch reads only entries no other CTA of the same launch writes.
-constexpr int kTileSb = 256;                     // superblocks per scan tile (>= 3)
+constexpr int kTileSb = kScanTile;               // superblocks per scan tile (>= 3)
 constexpr int kFinalThreads = kTileSb / 4;
 
 __global__ void __launch_bounds__(kThreads)
@@ -396,10 +396,18 @@ wq_status launch_bf16x_count(const uint16_t* w, int64_t n, int64_t k, uint32_t* 
     bf16x_count_kernel<<<grid, kThreads, 0, s>>>((const uint4*)w, nhalf, nsb, sb_off);
     wq_status st = check_launch("bf16x count");
     if (st) return st;
-    bf16x_tile_scan_kernel<<<1, kTileScanThreads, 0, s>>>(sb_off, nsb);
-    if ((st = check_launch("bf16x tile scan"))) return st;
-    bf16x_tile_final_kernel<<<grid, kFinalThreads, 0, s>>>(sb_off, nsb);
-    return check_launch("bf16x tile final");
+    return launch_tile_scan_u8(sb_off, nsb, s);
+}
+
+wq_status launch_tile_scan_u8(uint32_t* a, int64_t count, cudaStream_t s) {
+    const int64_t ntiles = (count + kTileSb - 1) / kTileSb;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    const int grid = (int)(ntiles < cap ? ntiles : cap);
+    bf16x_tile_scan_kernel<<<1, kTileScanThreads, 0, s>>>(a, count);
+    wq_status st = check_launch("tile scan");
+    if (st) return st;
+    bf16x_tile_final_kernel<<<grid, kFinalThreads, 0, s>>>(a, count);
+    return check_launch("tile final");
 }
 
 wq_status launch_bf16x_encode(const uint16_t* w, int64_t n, int64_t k, const uint32_t* sb_off,

@@ -79,6 +79,23 @@ wq_status launch_bf16x_decode(const uint8_t* sm, const uint64_t* hdr, const uint
                               uint16_t* out, cudaStream_t s);
 wq_status read_bf16x_error(int32_t* code);
 
+// In-place exclusive scan of count 8-bit values held in the low byte of a[0..count), total
+// in a[count], for values written by a pass that also stored, in bits 8..31 of the last
+// entry of every tile of kScanTile entries, that tile's total (see wq_bf16x.cu).
+constexpr int kScanTile = 256;
+wq_status launch_tile_scan_u8(uint32_t* a, int64_t count, cudaStream_t s);
+
+// Water-filling 3/4/5-bit dyadic blocks (wq_wf.cu).
+wq_status launch_wf_analyze(const uint16_t* w, int64_t n, int64_t k, double lambda, uint16_t* scale,
+                            uint8_t* width, uint32_t* blk_off, double* dist, cudaStream_t s);
+wq_status launch_wf_pack(const uint16_t* w, int64_t n, int64_t k, const uint16_t* scale,
+                         const uint8_t* width, const uint32_t* blk_off, uint8_t* packed,
+                         int64_t packed_bytes, cudaStream_t s);
+wq_status launch_wf_dequant(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
+                            const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
+                            uint16_t* out, cudaStream_t s);
+wq_status read_wf_error(int32_t* code);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

@@ -1,0 +1,269 @@
+// wq_wf.cu -- water-filling dyadic blocks of 3, 4 or 5 bits in one level index space
+// ("MiniCPM5-1B 验证: 6× 压缩…" §2.1 dyadic codebook, §6 water-filling).
+//
+// With half = 2^(b-1) and step = scale / half the b-bit codebook is step * {-half .. half-1},
+// and the codebooks of different b line up: code idx_b of a b-bit block is code
+// idx_5 = idx_b << (5 - b) of the 5-bit codebook of the same scale, so one reconstruction,
+// bf16((scale / 16) * (idx_5 - 16)), serves every width. Per 64-weight block (the §2.2
+// block, scale = max |w|) the width is the smallest b in {3, 4, 5} whose squared error
+// D_b = sum (w - code)^2 lies at or under the water level 64 * lambda, else 5.
+//
+// Exactness: every midpoint between two codes, scale * odd / 2^b, is exact in fp32 for
+// scales in [2^-100, 2^100] (in double otherwise), so the nearest-code search is exact;
+// each error w - code is exact (the code is zero or within a factor of two of w), its
+// square is exact in double, and D_b is summed over the block's weights in order, in double
+// (one thread per block). Widths, codes and distortions are therefore bit-identical with a
+// plain double-precision evaluation.
+//
+// Layout: scale bf16 [n, k/64]; width uint8 [n, k/64]; the blocks' bit streams back to back
+// in row-major block order, block i taking 8 * width_i bytes with code j in bits
+// [b j, b j + b) from bit 0 of its first byte (b = 4 is the nibble layout of §2.5);
+// blk_off uint32 [n k/64 + 1] holds every block's byte offset and the total.
+//
+// Kernels: analyze (scale, the three distortions, width, the scan's tile totals), the shared
+// in-place tile scan of the block sizes, pack (codes at the chosen width), dequant (eight
+// threads per block: each rebuilds 8 weights from b whole bytes and stores 16 bytes, so a
+// block's 128 output bytes leave in one coalesced run).
+#include "wq_internal.cuh"
+
+namespace wq {
+namespace {
+
+constexpr int kThreads = 256;                   // one block of weights per thread
+static_assert(kThreads == kScanTile, "an analyze CTA covers one scan tile");
+constexpr int kPad = 33;                        // staged words per block (32 + 1: no bank conflicts)
+
+__device__ int g_wf_error;                      // 0, or the first inconsistent-data code
+
+__device__ __forceinline__ void report(int code) { atomicCAS(&g_wf_error, 0, code); }
+
+// Stage this warp's 32 blocks (32 x 128 bytes) into shared memory, one block per 33 words.
+__device__ __forceinline__ void stage_blocks(const uint4* __restrict__ w, int64_t nblk, int64_t first,
+                                             uint32_t* sw) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const int v = q * 32 + lane;             // 16-byte piece of the warp's 4 KB
+        const int blk = v >> 3, word = 4 * (v & 7);
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (first + blk < nblk) x = ldg_nc_v4(w + (first + blk) * 8 + (v & 7));
+        uint32_t* d = sw + blk * kPad + word;
+        d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+    }
+    __syncwarp();
+}
+
+// Largest |w| of the block as bf16 bits (the magnitude order of finite bf16 patterns).
+__device__ __forceinline__ uint32_t block_absmax(const uint32_t* b) {
+    uint32_t m = 0;
+#pragma unroll 8
+    for (int t = 0; t < 32; ++t) m = max(m, max(b[t] & 0x7FFFu, (b[t] >> 16) & 0x7FFFu));
+    return m;
+}
+
+// idx_b of w: the number of midpoints (between codes x - 1 and x, x = 1 .. 2^b - 1) below w,
+// found bit by bit (the midpoints increase with x; a tie goes to the lower code).
+__device__ __forceinline__ int index_b(float w, float s, int b, bool fast) {
+    const int half = 1 << (b - 1);
+    int idx = 0;
+    if (fast) {
+        const float inv = __int_as_float((127 - b) << 23);          // 2^-b
+        for (int bit = b - 1; bit >= 0; --bit) {
+            const int cand = idx | (1 << bit);
+            const float m = s * (float)(2 * cand - 2 * half - 1) * inv;
+            if (w > m) idx = cand;
+        }
+    } else {
+        const double sd = (double)s, wd = (double)w;
+        for (int bit = b - 1; bit >= 0; --bit) {
+            const int cand = idx | (1 << bit);
+            const double m = sd * (double)(2 * cand - 2 * half - 1) / (double)(2 * half);
+            if (wd > m) idx = cand;
+        }
+    }
+    return idx;
+}
+
+// The code value step * (idx - half) and the exact error w - code, as a double.
+__device__ __forceinline__ double error_b(float w, float s, int b, int idx, bool fast) {
+    const int half = 1 << (b - 1);
+    if (fast) {
+        const float c = s * (float)(idx - half) * __int_as_float((128 - b) << 23);   // 2^-(b-1)
+        return (double)(w - c);
+    }
+    return (double)w - (double)s * (double)(idx - half) / (double)half;
+}
+
+__global__ void __launch_bounds__(kThreads)
+wf_analyze_kernel(const uint4* __restrict__ w, int64_t nblk, double lambda64, uint16_t* __restrict__ scale,
+                  uint8_t* __restrict__ width, uint32_t* __restrict__ blk_off, double* __restrict__ dist) {
+    __shared__ uint32_t sw[kThreads / 32][32 * kPad];
+    __shared__ uint32_t s_sum[kThreads / 32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t ntiles = (nblk + kScanTile - 1) / kScanTile;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t t0 = tile * kScanTile, t1 = min(t0 + (int64_t)kScanTile, nblk);
+        const int64_t first = t0 + 32 * wid;
+        stage_blocks(w, nblk, first, sw[wid]);
+        const int64_t i = first + lane;
+        uint32_t size = 0;
+        if (i < t1) {
+            const uint32_t* b = sw[wid] + lane * kPad;
+            const uint32_t sbits = block_absmax(b);
+            const float s = bf16_bits_to_float(sbits);
+            const bool fast = s >= 0x1p-100f && s <= 0x1p100f;
+            int chosen = 5;
+            for (int bw = 3; bw <= 5; ++bw) {
+                double D = 0.0;
+                for (int t = 0; t < 32; ++t) {
+                    const float w0 = bf16_bits_to_float(b[t] & 0xFFFFu), w1 = bf16_bits_to_float(b[t] >> 16);
+                    const double e0 = error_b(w0, s, bw, index_b(w0, s, bw, fast), fast);
+                    D = fma(e0, e0, D);
+                    const double e1 = error_b(w1, s, bw, index_b(w1, s, bw, fast), fast);
+                    D = fma(e1, e1, D);
+                }
+                if (dist) dist[i * 3 + (bw - 3)] = D;
+                if (chosen == 5 && bw < 5 && D <= lambda64) chosen = bw;
+            }
+            scale[i] = (uint16_t)sbits;
+            width[i] = (uint8_t)chosen;
+            size = 8u * (uint32_t)chosen;
+            blk_off[i] = size;
+        }
+        // the tile's total into bits 8..31 of its last entry, for the scan
+        const uint32_t wsum = __reduce_add_sync(0xFFFFFFFFu, size);
+        if (lane == 0) s_sum[wid] = wsum;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t tot = 0;
+#pragma unroll
+            for (int q = 0; q < kThreads / 32; ++q) tot += s_sum[q];
+            blk_off[t1 - 1] |= tot << 8;
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+wf_pack_kernel(const uint4* __restrict__ w, int64_t nblk, const uint16_t* __restrict__ scale,
+               const uint8_t* __restrict__ width, const uint32_t* __restrict__ blk_off,
+               uint8_t* __restrict__ packed, int64_t packed_bytes) {
+    __shared__ uint32_t sw[kThreads / 32][32 * kPad];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+    for (int64_t first = ((int64_t)blockIdx.x * (kThreads / 32) + wid) * 32; first < nblk; first += warps * 32) {
+        stage_blocks(w, nblk, first, sw[wid]);
+        const int64_t i = first + lane;
+        if (i < nblk) {
+            const int bw = width[i];
+            const int64_t off = (int64_t)blk_off[i];
+            if (bw < 3 || bw > 5 || (off & 7) != 0 || off + 8 * bw > packed_bytes) {
+                report(2001);
+            } else {
+                const uint32_t* b = sw[wid] + lane * kPad;
+                const float s = bf16_bits_to_float(scale[i]);
+                const bool fast = s >= 0x1p-100f && s <= 0x1p100f;
+                unsigned long long* out = reinterpret_cast<unsigned long long*>(packed + off);
+                unsigned long long acc = 0;
+                int nbits = 0, word = 0;
+                for (int t = 0; t < 64; ++t) {
+                    const uint32_t h = (t & 1) ? (b[t >> 1] >> 16) : (b[t >> 1] & 0xFFFFu);
+                    const unsigned long long idx = (unsigned long long)index_b(bf16_bits_to_float(h), s, bw, fast);
+                    acc |= idx << nbits;
+                    nbits += bw;
+                    if (nbits >= 64) {
+                        out[word++] = acc;
+                        nbits -= 64;
+                        acc = nbits > 0 ? idx >> (bw - nbits) : 0ull;
+                    }
+                }
+            }
+        }
+        __syncwarp();                            // the staging buffer is reused next trip
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+wf_dequant_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const uint16_t* __restrict__ scale,
+                  const uint8_t* __restrict__ width, const uint32_t* __restrict__ blk_off, int64_t nblk,
+                  uint4* __restrict__ out) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gid < nblk * 8; gid += stride) {
+        const int64_t i = gid >> 3;
+        const int t = (int)(gid & 7);
+        const int bw = __ldg(width + i);
+        const int64_t off = (int64_t)ldg_u32(blk_off + i);
+        uint32_t o[4] = {0, 0, 0, 0};
+        if (bw < 3 || bw > 5 || (off & 7) != 0 || off + 8 * bw > packed_bytes) {
+            report(2000);
+        } else {
+            // this thread's 8 codes are the b bytes at off + b t (8 codes of b bits)
+            const int64_t byte0 = off + (int64_t)bw * t;
+            const int64_t w0 = byte0 & ~7ll;
+            const int sh = (int)(byte0 & 7) * 8;
+            const unsigned long long* src = reinterpret_cast<const unsigned long long*>(packed);
+            unsigned long long v = __ldg(src + (w0 >> 3)) >> sh;
+            if (sh + 8 * bw > 64) v |= __ldg(src + (w0 >> 3) + 1) << (64 - sh);
+            const float s16 = bf16_bits_to_float(ldg_u16(scale + i)) * 0.0625f;
+            const uint32_t mask = (1u << bw) - 1u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i0 = (int)(((uint32_t)(v >> (bw * 2 * j)) & mask) << (5 - bw));
+                const int i1 = (int)(((uint32_t)(v >> (bw * (2 * j + 1))) & mask) << (5 - bw));
+                o[j] = pack_bf16x2(s16 * (float)(i0 - 16), s16 * (float)(i1 - 16));
+            }
+        }
+        stg_cs_v4(out + gid, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+}
+
+int grid_cap(int64_t want) {
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (want > cap) want = cap;
+    return (int)(want < 1 ? 1 : want);
+}
+
+}  // namespace
+
+wq_status launch_wf_analyze(const uint16_t* w, int64_t n, int64_t k, double lambda, uint16_t* scale,
+                            uint8_t* width, uint32_t* blk_off, double* dist, cudaStream_t s) {
+    const int64_t nblk = n * k / 64;
+    const int64_t ntiles = (nblk + kScanTile - 1) / kScanTile;
+    wf_analyze_kernel<<<grid_cap(ntiles), kThreads, 0, s>>>((const uint4*)w, nblk, 64.0 * lambda, scale,
+                                                            width, blk_off, dist);
+    wq_status st = check_launch("wf analyze");
+    if (st) return st;
+    return launch_tile_scan_u8(blk_off, nblk, s);
+}
+
+wq_status launch_wf_pack(const uint16_t* w, int64_t n, int64_t k, const uint16_t* scale,
+                         const uint8_t* width, const uint32_t* blk_off, uint8_t* packed,
+                         int64_t packed_bytes, cudaStream_t s) {
+    const int64_t nblk = n * k / 64;
+    wf_pack_kernel<<<grid_cap((nblk + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+        (const uint4*)w, nblk, scale, width, blk_off, packed, packed_bytes);
+    return check_launch("wf pack");
+}
+
+wq_status launch_wf_dequant(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
+                            const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
+                            uint16_t* out, cudaStream_t s) {
+    const int64_t nblk = n * k / 64;
+    wf_dequant_kernel<<<grid_cap((nblk * 8 + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+        packed, packed_bytes, scale, width, blk_off, nblk, (uint4*)out);
+    return check_launch("wf dequant");
+}
+
+wq_status read_wf_error(int32_t* code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_wf_error, sizeof v);
+    if (e != cudaSuccess) return fail(WQ_ECUDA, "reading the water-filling error word: %s", cudaGetErrorString(e));
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_wf_error, &zero, sizeof zero);
+    }
+    *code = v;
+    return WQ_OK;
+}
+
+}  // namespace wq
