@@ -141,3 +141,26 @@ def test_gemm_lloyd8s_one_hot_exact(wq):
     x[np.arange(len(cols)), cols] = 1.0
     y = f32(wq.gemm(pw, to_dev_bits(workloads.f64_to_bf16_bits(x))))
     assert np.array_equal(y, wd[:, cols].T)
+
+
+def test_gemm_last_wave_split(wq):
+    """Wide tiles in whole waves plus a short tail: the tail tiles run as a second launch with
+    K split across CTAs (partial sums in the workspace). 158 weight-row tiles of 128 on a
+    148-SM B200 leave a tail of 10; rows of the tail tiles and of the first wave are
+    sampled."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    tiles = sms + 10
+    n, k, m = 128 * tiles, 4096, 256
+    pw, packed, s = _weight(wq, n, k, 64, 31)
+    assert wq.gemm_workspace_bytes(pw, m) > 0               # the tail split is planned
+    x_bits = workloads.activations(m, k, workloads.PREFILL, 31)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+    rows = np.concatenate([np.arange(0, 128 * sms, 397), np.arange(128 * sms, n, 5), [n - 1]])
+    ms = np.arange(0, m, 3)
+    y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x_bits[ms], rows=rows)
+    got = f32(y)[np.ix_(ms, rows)]
+    assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
+    # the same through the static-scratch entry point (the tail's scratch stays within it)
+    assert wq.gemm_workspace_bytes(pw, m) <= (16 << 20)

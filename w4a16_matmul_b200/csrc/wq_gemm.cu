@@ -241,7 +241,7 @@ template <int BN, int G, bool PARTIAL, bool LL, int KB>
 __global__ void __launch_bounds__(threads_for(BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
             const __grid_constant__ CUtensorMap tmap_l, const uint16_t* __restrict__ scale,
-            void* __restrict__ out, int M, int N, int K, int kt_per_split) {
+            void* __restrict__ out, int M, int N, int K, int kt_per_split, int grid_n, int tile0) {
     using S = Smem<BN, LL, KB>;
     constexpr int STAGES = S::STAGES;
     constexpr int RW = rw_for(BN);
@@ -257,9 +257,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     int* s_abort = (int*)(s_tmem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BM, m0 = blockIdx.y * BN;
+    // tile (weight-row tile fastest, the launch order the grid had as a 2D grid); a launch
+    // may cover a contiguous range of tiles starting at tile0
+    const int lin = tile0 + (int)blockIdx.x;
+    const int n0 = (lin % grid_n) * BM, m0 = (lin / grid_n) * BN;
     const int KT = K / KB;
-    const int kt0 = blockIdx.z * kt_per_split;
+    const int kt0 = blockIdx.y * kt_per_split;
     const int kt1 = min(KT, kt0 + kt_per_split);
     const int nk = kt1 - kt0;
 
@@ -478,8 +481,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     for (int j = 0; j < 16; ++j) {
                         const int m = m0 + c0 + j;
                         if (m < M) {
-                            if (PARTIAL)
-                                ((float*)out)[((size_t)blockIdx.z * M + m) * N + n] = __uint_as_float(v[j]);
+                            if (PARTIAL)                 // [split][tile of the launch][BN][BM]
+                                ((float*)out)[(((size_t)blockIdx.y * gridDim.x + blockIdx.x) * BN + c0 + j) * BM +
+                                              (n - n0)] = __uint_as_float(v[j]);
                             else
                                 ((uint16_t*)out)[(size_t)m * N + n] =
                                     (uint16_t)float_to_bf16_bits(__uint_as_float(v[j]));
@@ -499,14 +503,23 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     }
 }
 
-// y[m, n] = bf16(sum over splits of the fp32 partial sums)
-__global__ void __launch_bounds__(256)
-splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t mn, uint16_t* __restrict__ y) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mn; i += (int64_t)gridDim.x * blockDim.x) {
-        float v = 0.f;
-        for (int s = 0; s < splits; ++s) v += part[s * mn + i];
-        y[i] = (uint16_t)float_to_bf16_bits(v);
-    }
+// y[m, n] = bf16(sum over splits of the fp32 partial sums) for the ntl tiles of a partial
+// launch starting at tile0; partial sums are laid out [split][tile][bn][BM]. One CTA per
+// (tile, activation row): its 128 threads are the tile's 128 weight rows, so every load and
+// store of a warp covers 32 consecutive rows, and the split loads are independent.
+__global__ void __launch_bounds__(BM)
+splitk_reduce_kernel(const float* __restrict__ part, int splits, int ntl, int tile0, int grid_n, int bn,
+                     int M, int N, uint16_t* __restrict__ y) {
+    const int64_t plane = (int64_t)ntl * bn * BM;
+    const int lt = blockIdx.x, c = blockIdx.y, r = threadIdx.x;
+    const int lin = tile0 + lt;
+    const int n = (lin % grid_n) * BM + r, m = (lin / grid_n) * bn + c;
+    if (n >= N || m >= M) return;
+    const float* src = part + ((int64_t)lt * bn + c) * BM + r;
+    float v = 0.f;
+#pragma unroll 4
+    for (int sp = 0; sp < splits; ++sp) v += __ldg(src + sp * plane);
+    y[(size_t)m * N + n] = (uint16_t)float_to_bf16_bits(v);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -531,7 +544,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 struct Plan {
     int bn, kb, splits, kt_per_split, grid_n, grid_m;
+    // last-wave split: the first `full` tiles (whole waves) run unsplit; the remaining
+    // tiles run as a second launch with K split tail_splits ways (1: no second launch)
+    int full, tail_splits, tail_kt_per_split;
 };
+
+// Scratch the last-wave split may use (it then stays within the static scratch of
+// wq_gemm_w4a16_static).
+constexpr size_t kTailScratchBytes = (size_t)16 << 20;
 
 #ifndef WQ_GEMM_BN128_MAX
 #define WQ_GEMM_BN128_MAX 128
@@ -581,29 +601,80 @@ Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt) {
     }
     p.kt_per_split = (KT + splits - 1) / splits;
     p.splits = (KT + p.kt_per_split - 1) / p.kt_per_split;
+    // One or two whole waves of wide tiles plus a tail of at most half a wave: a single pass
+    // spends a full wave's time on the tail. Run the whole waves as they are, then the tail
+    // tiles with K split s ways (s tail CTAs per tile fit one wave: the tail then takes about
+    // 1/s of a wave), each split keeping >= 512 columns, the partial sums within
+    // kTailScratchBytes. (Measured on 11008 x 4096: m = 512, 1 wave + 24 tiles, 1.25x; with
+    // 9 waves + 44 tiles at m = 4096 the second launch and its reduction cost what the tail
+    // saves, hence the two-wave limit.)
+    p.full = (int)tiles;
+    p.tail_splits = 1;
+    p.tail_kt_per_split = KT;
+    if (p.bn >= 128 && p.splits == 1) {
+        const int64_t full = tiles / sms * sms, tail = tiles - full;
+        if (full > 0 && full <= 2 * sms && tail > 0 && 2 * tail <= sms) {
+            int64_t sp = sms / tail;
+            while (sp > 1 && KT / sp < min_narrow) --sp;
+            while (sp > 1 && (size_t)sp * tail * BM * p.bn * sizeof(float) > kTailScratchBytes) --sp;
+            if (sp > 1) {
+                p.tail_kt_per_split = (KT + (int)sp - 1) / (int)sp;
+                p.tail_splits = (KT + p.tail_kt_per_split - 1) / p.tail_kt_per_split;
+                p.full = (int)full;
+            }
+        }
+    }
     return p;
 }
 
+// One launch over tiles [tile0, tile0 + ntl) with K split `splits` ways (partial sums to
+// `out` in the [split][tile][BN][BM] layout when partial, bf16 y otherwise).
 template <int BN, int G, bool LL, int KB>
-wq_status launch_bn(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMap& tl,
+wq_status launch_bn(const Plan& p, bool partial, int tile0, int ntl, int splits, int kt_per_split,
+                    const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMap& tl,
                     const uint16_t* scale, void* out, int M, int N, int K, cudaStream_t s) {
     const int smem = Smem<BN, LL, KB>::TOTAL;
-    const dim3 grid(p.grid_n, p.grid_m, p.splits);
+    const dim3 grid(ntl, splits, 1);
     // the shared-memory opt-in is set once per kernel variant (a function attribute holds
     // for the process; the flags are per variant and only ever go from false to true)
     static bool raised[2] = {false, false};
-    if (p.splits > 1) {
+    if (partial) {
         auto k = gemm_kernel<BN, G, true, LL, KB>;
         if (!raised[1] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[1] = true;
-        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, p.kt_per_split);
+        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, kt_per_split, p.grid_n, tile0);
     } else {
         auto k = gemm_kernel<BN, G, false, LL, KB>;
         if (!raised[0] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[0] = true;
-        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, p.kt_per_split);
+        k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, kt_per_split, p.grid_n, tile0);
     }
     return check_launch("gemm");
+}
+
+// The plan's launches: one (unsplit, or split everywhere) or two (whole waves unsplit, then
+// the split tail), each split launch followed by its reduction.
+template <int BN, int G, bool LL, int KB>
+wq_status launch_plan(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMap& tl,
+                      const uint16_t* scale, uint16_t* y, void* ws, int M, int N, int K, cudaStream_t s) {
+    const int tiles = p.grid_n * p.grid_m;
+    auto reduce = [&](int splits, int tile0, int ntl) {
+        splitk_reduce_kernel<<<dim3(ntl, BN), BM, 0, s>>>((const float*)ws, splits, ntl, tile0, p.grid_n, BN, M, N, y);
+        return check_launch("gemm split-k reduce");
+    };
+    wq_status st;
+    if (p.splits > 1) {
+        if ((st = launch_bn<BN, G, LL, KB>(p, true, 0, tiles, p.splits, p.kt_per_split, tx, tp, tl, scale, ws, M, N,
+                                           K, s)))
+            return st;
+        return reduce(p.splits, 0, tiles);
+    }
+    if ((st = launch_bn<BN, G, LL, KB>(p, false, 0, p.full, 1, K / KB, tx, tp, tl, scale, y, M, N, K, s))) return st;
+    if (p.full == tiles) return WQ_OK;
+    if ((st = launch_bn<BN, G, LL, KB>(p, true, p.full, tiles - p.full, p.tail_splits, p.tail_kt_per_split, tx, tp,
+                                       tl, scale, ws, M, N, K, s)))
+        return st;
+    return reduce(p.tail_splits, p.full, tiles - p.full);
 }
 
 }  // namespace
@@ -620,7 +691,11 @@ constexpr int64_t kGemvMaxRows = 12;
 size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
     if (m <= kGemvMaxRows) return 0;
     const Plan p = plan_for(m, w.n, w.k, w.fmt);
-    return p.splits > 1 ? (size_t)p.splits * (size_t)m * (size_t)w.n * sizeof(float) : 0;
+    const size_t tile = (size_t)BM * (size_t)p.bn * sizeof(float);
+    const size_t tiles = (size_t)p.grid_n * (size_t)p.grid_m;
+    if (p.splits > 1) return (size_t)p.splits * tiles * tile;
+    if (p.full < (int)tiles) return (size_t)p.tail_splits * (tiles - (size_t)p.full) * tile;
+    return 0;
 }
 
 wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
@@ -666,15 +741,14 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(WQ_ECUDA, "tensor map for LLOYD8S levels failed (%d)", (int)r);
     }
-    void* out = p.splits > 1 ? ws : (void*)y;
-    if (p.splits > 1 && (ws == nullptr || ws_bytes < gemm_workspace_bytes(w, m)))
-        return fail(WQ_EINVAL, "workspace too small");
+    const size_t need = gemm_workspace_bytes(w, m);
+    if (need > 0 && (ws == nullptr || ws_bytes < need)) return fail(WQ_EINVAL, "workspace too small");
     const uint16_t* sc = (const uint16_t*)w.aux;
     wq_status st;
-#define WQ_BN(BNV, KBV)                                                                                 \
-    st = (w.fmt == WQ_FMT_LLOYD8S) ? launch_bn<BNV, 32, true, 64>(p, tx, tp, tl, sc, out, M, N, K, s)    \
-       : (w.group == 64) ? launch_bn<BNV, 64, false, KBV>(p, tx, tp, tl, sc, out, M, N, K, s)            \
-                         : launch_bn<BNV, 32, false, KBV>(p, tx, tp, tl, sc, out, M, N, K, s)
+#define WQ_BN(BNV, KBV)                                                                                  \
+    st = (w.fmt == WQ_FMT_LLOYD8S) ? launch_plan<BNV, 32, true, 64>(p, tx, tp, tl, sc, y, ws, M, N, K, s) \
+       : (w.group == 64) ? launch_plan<BNV, 64, false, KBV>(p, tx, tp, tl, sc, y, ws, M, N, K, s)         \
+                         : launch_plan<BNV, 32, false, KBV>(p, tx, tp, tl, sc, y, ws, M, N, K, s)
     switch (p.bn) {
         case 16: WQ_BN(16, 64); break;
         case 32: WQ_BN(32, 64); break;
@@ -685,12 +759,7 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
         default: WQ_BN(256, 64); break;
     }
 #undef WQ_BN
-    if (st != WQ_OK || p.splits == 1) return st;
-    const int64_t mn = (int64_t)M * N;
-    int grid = (int)((mn + 255) / 256);
-    if (grid > sm_count() * 8) grid = sm_count() * 8;
-    splitk_reduce_kernel<<<grid, 256, 0, s>>>((const float*)ws, p.splits, mn, y);
-    return check_launch("gemm split-k reduce");
+    return st;
 }
 
 wq_status read_device_error(int32_t* code) {
