@@ -113,10 +113,12 @@ __device__ __forceinline__ void dyadic_pairs_scaled(uint32_t w, uint32_t c1, uin
 // LUT16 lookup of 4 codes (nibbles of the low 16 bits of s) in a 16-entry fp16 table held
 // as byte planes: lo[q] / hi[q] hold the low / high bytes of entries 4q..4q+3. Returns the
 // fp16 pairs (code0, code1) and (code2, code3).
+// The byte mask (0xFF where code >= 8) comes from prmt's sign-replicate selector mode: the
+// codes' bit 3 is the top bit of a byte of s (codes 1, 3) or of s << 4 (codes 0, 2).
 __device__ __forceinline__ void lut16_lookup4(uint32_t s, const uint32_t* lo, const uint32_t* hi,
                                               uint32_t& p01, uint32_t& p23) {
     const uint32_t s7 = s & 0x7777u;                                  // index within 8 entries
-    const uint32_t m = prmt(0x00000000u, 0xFFFFFFFFu, (s >> 1) & 0x4444u);   // byte mask: code >= 8
+    const uint32_t m = prmt(s, s << 4, 0x9D8Cu);                      // byte mask: code >= 8
     const uint32_t l = (prmt(lo[0], lo[1], s7) & ~m) | (prmt(lo[2], lo[3], s7) & m);
     const uint32_t h = (prmt(hi[0], hi[1], s7) & ~m) | (prmt(hi[2], hi[3], s7) & m);
     p01 = prmt(l, h, 0x5140u);
@@ -480,6 +482,9 @@ constexpr int depth(int kind, int nb, int r) {
     return (kind < kLut16 && nb == 1 && r == 1) ? WQ_GEMV_DEPTH : 2;
 }
 
+#ifndef WQ_GEMV_CL_WARPS
+#define WQ_GEMV_CL_WARPS 24           // resident warps per SM the cluster split of small launches aims at
+#endif
 #ifndef WQ_GEMV_CLUSTER
 #define WQ_GEMV_CLUSTER 1             // small launches split K across a thread-block cluster
 #endif
@@ -499,11 +504,18 @@ constexpr int cta_warps(int wk, int fw) { return wk == 1 ? fw : 4; }
 #ifndef WQ_GEMV_R2_CAP
 #define WQ_GEMV_R2_CAP 4
 #endif
+// LUT16: 4 CTAs per SM (at most 128 registers, no spills; measured on the 8192 x 28672
+// LUT16 GEMV: 84 -> 78 / 110 -> 96 / 141 -> 118 us at batch 1 / 8 / 16 against 3 CTAs);
+// LLOYD8S keeps its full register budget (it spills at 128).
 #ifndef WQ_GEMV_LUT_CAP
-#define WQ_GEMV_LUT_CAP 1
+#define WQ_GEMV_LUT_CAP 4
+#endif
+#ifndef WQ_GEMV_LLOYD_CAP
+#define WQ_GEMV_LLOYD_CAP 1
 #endif
 constexpr int min_warps(int kind, int nb, int r, int warps_per_cta) {
-    return kind >= kLut16 ? 4 * WQ_GEMV_LUT_CAP
+    return kind == kLloyd8 ? 4 * WQ_GEMV_LLOYD_CAP
+         : kind == kLut16 ? 4 * WQ_GEMV_LUT_CAP
          : r != 1 ? 4 * WQ_GEMV_R2_CAP
          : nb != 1 ? 4 * WQ_GEMV_MIN_CTAS_NB2
          : warps_per_cta == 4 ? 4 * WQ_GEMV_MIN_CTAS_NB1 : 24;
@@ -745,7 +757,7 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
             weights += (int64_t)probs[i].n * probs[i].k;
         }
         const int64_t tiles64 = (rows16 + 3) / 4;
-        int64_t want = (24 * sms + 4 * tiles64 - 1) / (4 * tiles64);
+        int64_t want = (WQ_GEMV_CL_WARPS * sms + 4 * tiles64 - 1) / (4 * tiles64);
         int cl = weights < ((int64_t)1 << 24) ? 1 : want >= 8 ? 8 : want >= 4 ? 4 : want >= 2 ? 2 : 1;
         while (cl > 1 && max_steps / cl < 2) cl >>= 1;
         if (cl == 8) return prepare_variant<KIND, NB, 1, 1, 4, MAXP, 8>(pr, probs, tiles_for(64));

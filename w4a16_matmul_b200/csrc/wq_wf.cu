@@ -84,6 +84,22 @@ __device__ __forceinline__ int index_b(float w, float s, int b, bool fast) {
     return idx;
 }
 
+// idx_5, idx_4 and idx_3 of w from one 5-bit search. The 4-bit midpoints are the 5-bit codes
+// of odd index (s (2x - 17) / 16 = code_5(2x - 1)), and idx_5 places w against every 5-bit
+// code but code_5(idx_5) itself, so idx_4 = idx_5 / 2, plus one when idx_5 is odd (and below
+// 31) and w lies above code_5(idx_5); likewise idx_3 from idx_4 and the 4-bit codes.
+__device__ __forceinline__ void index_543(float w, float s, bool fast, int& i5, int& i4, int& i3) {
+    i5 = index_b(w, s, 5, fast);
+    if (fast) {
+        i4 = (i5 >> 1) + (((i5 & 1) && i5 < 31 && w > s * (float)(i5 - 16) * 0.0625f) ? 1 : 0);
+        i3 = (i4 >> 1) + (((i4 & 1) && i4 < 15 && w > s * (float)(i4 - 8) * 0.125f) ? 1 : 0);
+    } else {
+        const double sd = (double)s, wd = (double)w;
+        i4 = (i5 >> 1) + (((i5 & 1) && i5 < 31 && wd > sd * (double)(i5 - 16) / 16.0) ? 1 : 0);
+        i3 = (i4 >> 1) + (((i4 & 1) && i4 < 15 && wd > sd * (double)(i4 - 8) / 8.0) ? 1 : 0);
+    }
+}
+
 // The code value step * (idx - half) and the exact error w - code, as a double.
 __device__ __forceinline__ double error_b(float w, float s, int b, int idx, bool fast) {
     const int half = 1 << (b - 1);
@@ -112,19 +128,24 @@ wf_analyze_kernel(const uint4* __restrict__ w, int64_t nblk, double lambda64, ui
             const uint32_t sbits = block_absmax(b);
             const float s = bf16_bits_to_float(sbits);
             const bool fast = s >= 0x1p-100f && s <= 0x1p100f;
-            int chosen = 5;
-            for (int bw = 3; bw <= 5; ++bw) {
-                double D = 0.0;
-                for (int t = 0; t < 32; ++t) {
-                    const float w0 = bf16_bits_to_float(b[t] & 0xFFFFu), w1 = bf16_bits_to_float(b[t] >> 16);
-                    const double e0 = error_b(w0, s, bw, index_b(w0, s, bw, fast), fast);
-                    D = fma(e0, e0, D);
-                    const double e1 = error_b(w1, s, bw, index_b(w1, s, bw, fast), fast);
-                    D = fma(e1, e1, D);
-                }
-                if (dist) dist[i * 3 + (bw - 3)] = D;
-                if (chosen == 5 && bw < 5 && D <= lambda64) chosen = bw;
+            // the three sums run side by side, each over the block's weights in order
+            double D3 = 0.0, D4 = 0.0, D5 = 0.0;
+            for (int j = 0; j < 64; ++j) {
+                const float v = bf16_bits_to_float((j & 1) ? (b[j >> 1] >> 16) : (b[j >> 1] & 0xFFFFu));
+                int i5, i4, i3;
+                index_543(v, s, fast, i5, i4, i3);
+                const double e3 = error_b(v, s, 3, i3, fast), e4 = error_b(v, s, 4, i4, fast),
+                             e5 = error_b(v, s, 5, i5, fast);
+                D3 = fma(e3, e3, D3);
+                D4 = fma(e4, e4, D4);
+                D5 = fma(e5, e5, D5);
             }
+            if (dist) {
+                dist[i * 3] = D3;
+                dist[i * 3 + 1] = D4;
+                dist[i * 3 + 2] = D5;
+            }
+            const int chosen = D3 <= lambda64 ? 3 : D4 <= lambda64 ? 4 : 5;
             scale[i] = (uint16_t)sbits;
             width[i] = (uint8_t)chosen;
             size = 8u * (uint32_t)chosen;
