@@ -568,7 +568,7 @@ def bench_producers(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks
 
         def km():
             holder["pw"], _ = wq.quantize_lloyd(w, wq.LLOYD_KMEANS16, 25)
-        ms = max_over_ranks(time_region(torch, stream, km, 1, 1, barrier))
+        ms = max_over_ranks(time_region(torch, stream, km, 3, 1, barrier))
         out["kmeans16"] = {"Gweights/s": round(n * k / ms / 1e6, 3), "ms": round(ms, 2)}
         pw = holder["pw"]
         del w

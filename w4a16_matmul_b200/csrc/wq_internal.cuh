@@ -187,9 +187,11 @@ __device__ __forceinline__ uint32_t ldg_u16(const void* p) {
 __device__ __forceinline__ void lloyd8_lookup4(uint32_t s, const uint32_t* lo, const uint32_t* hi,
                                                uint32_t& p01, uint32_t& p23) {
     const uint32_t s7 = s & 0x7777u;                                     // level index
-    const uint32_t sg = prmt(0x00000000u, 0x80808080u, (s >> 1) & 0x4444u);   // 0x80 where signed
+    // 0xFF where the code's sign bit (bit 3) is set: prmt's sign-replicate selector mode on
+    // the byte whose top bit it is (s for codes 1 and 3, s << 4 for codes 0 and 2)
+    const uint32_t sg = prmt(s, s << 4, 0x9D8Cu);
     const uint32_t l = prmt(lo[0], lo[1], s7);
-    const uint32_t h = prmt(hi[0], hi[1], s7) ^ sg;
+    const uint32_t h = prmt(hi[0], hi[1], s7) ^ (sg & 0x80808080u);
     p01 = prmt(l, h, 0x5140u);
     p23 = prmt(l, h, 0x7362u);
 }
