@@ -192,44 +192,40 @@ unpack_kernel(const uint2* __restrict__ packed, int64_t n16, uint4* __restrict__
 // DYADIC4: bf16(step * (idx - 8)), step = scale / 8. The product is exact in fp32 (an
 // 8-bit significand times an integer of magnitude <= 8, scaled by 2^-3), so the bf16
 // conversion is the one and only rounding.
-// One thread: 4 packed words (32 codes, which lie in one group: groups are 32 or 64 columns
-// and the words are 16-byte aligned within a row) -> 64 bytes.
+// A warp takes 128 consecutive packed words per trip, lane l the words l, l + 32, l + 64 and
+// l + 96, so every 4-byte load covers 128 contiguous bytes and every 16-byte store 512
+// contiguous bytes of the output (four 16-byte stores per thread at a 64-byte stride ran
+// 30 % slower: each store instruction then touches 32 sectors half-way). Groups and rows are
+// contiguous in the flat packed array, so word i's scale is scale[8 i / group].
 __global__ void __launch_bounds__(kThreads)
-dequant_dyadic_kernel(const uint4* __restrict__ packed, const uint16_t* __restrict__ scale,
-                      int64_t n_quads, int64_t k, int group, uint4* __restrict__ out) {
-    const int64_t quads_per_row = k / 32;
-    const int64_t groups_per_row = k / group;
+dequant_dyadic_kernel(const uint32_t* __restrict__ packed, const uint16_t* __restrict__ scale,
+                      int64_t n_words, int gshift, uint4* __restrict__ out) {
     constexpr int U = 4;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n_quads; i0 += stride * U) {
-        uint4 p[U];
-        uint32_t sc[U];
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t base = ((int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * (32 * U);
+         base < n_words; base += warps * (32 * U)) {
+        uint32_t p[U], sc[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t i = i0 + u * stride;
-            p[u] = make_uint4(0, 0, 0, 0);
+            const int64_t i = base + 32 * u + lane;
+            p[u] = 0x88888888u;
             sc[u] = 0;
-            if (i < n_quads) {
-                p[u] = ldg_nc_v4(packed + i);
-                const int64_t row = i / quads_per_row;
-                const int64_t col = (i - row * quads_per_row) * 32;
-                sc[u] = ldg_u16(scale + row * groups_per_row + col / group);
+            if (i < n_words) {
+                p[u] = __ldg(packed + i);
+                sc[u] = ldg_u16(scale + (i >> gshift));
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t i = i0 + u * stride;
-            if (i >= n_quads) break;
+            const int64_t i = base + 32 * u + lane;
+            if (i >= n_words) break;
             const float step = bf16_bits_to_float(sc[u]) * 0.125f;
-            const uint32_t wv[4] = {p[u].x, p[u].y, p[u].z, p[u].w};
+            float v[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = step * (float)((int)((wv[q] >> (4 * j)) & 15) - 8);
-                stg_cs_v4(out + 4 * i + q, make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                                      pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7])));
-            }
+            for (int j = 0; j < 8; ++j) v[j] = step * (float)((int)((p[u] >> (4 * j)) & 15) - 8);
+            stg_cs_v4(out + i, make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7])));
         }
     }
 }
@@ -318,9 +314,8 @@ wq_status launch_dequant(const wq_weight& w, uint16_t* out, cudaStream_t s) {
     const int64_t n_words = w.n * w.k / 8;
     const int grid = stream_grid(n_words);
     if (w.fmt == WQ_FMT_DYADIC4) {
-        const int64_t n_quads = n_words / 4;          // k is a multiple of 32
-        dequant_dyadic_kernel<<<stream_grid(n_quads), kThreads, 0, s>>>(
-            (const uint4*)w.packed, (const uint16_t*)w.aux, n_quads, w.k, w.group, (uint4*)out);
+        dequant_dyadic_kernel<<<stream_grid((n_words + 3) / 4), kThreads, 0, s>>>(
+            (const uint32_t*)w.packed, (const uint16_t*)w.aux, n_words, w.group == 64 ? 3 : 2, (uint4*)out);
     }
     else if (w.fmt == WQ_FMT_LLOYD8S)
         dequant_lloyd_kernel<<<grid, kThreads, 0, s>>>((const uint32_t*)w.packed,
