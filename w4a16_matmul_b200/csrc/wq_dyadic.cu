@@ -78,19 +78,28 @@ __device__ __forceinline__ void quantize_chunk(uint4 v, bool live, I c, uint16_t
         // midpoint, -17 s / 16, is below every weight, so no check is needed).
         const float c8 = 8.0f * rcp_approx(amax);
         const float s8 = amax * 0.125f, m17 = -17.0f * amax * 0.0625f;
-        float cf[8];
+        // weights j and j + 4 side by side on the packed fp32x2 pipe (each lane of an x2
+        // instruction rounds exactly as its scalar form), so the nibble packing below also
+        // runs as pairs: (low half of the word, high half)
+        float2 cf[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float u = fmaf(f[i], c8, 8.5f);
-            float x = fminf(__fadd_ru(u, 8388608.0f) - 8388609.0f, 15.0f);   // ceil(u) - 1
-            const float mlo = fmaf(x, s8, m17);                                // exact midpoint
-            cf[i] = (f[i] > mlo) ? x : x - 1.0f;
+        for (int j = 0; j < 4; ++j) {
+            const float2 fw = make_float2(f[j], f[j + 4]);
+            const float2 u = __ffma2_rn(fw, make_float2(c8, c8), make_float2(8.5f, 8.5f));
+            float2 x = __fadd2_rn(__fadd2_ru(u, make_float2(8388608.0f, 8388608.0f)),
+                                  make_float2(-8388609.0f, -8388609.0f));               // ceil(u) - 1
+            x = make_float2(fminf(x.x, 15.0f), fminf(x.y, 15.0f));
+            const float2 mlo = __ffma2_rn(x, make_float2(s8, s8), make_float2(m17, m17));   // exact midpoint
+            const float2 xm1 = __fadd2_rn(x, make_float2(-1.0f, -1.0f));
+            cf[j] = make_float2(fw.x > mlo.x ? x.x : xm1.x, fw.y > mlo.y ? x.y : xm1.y);
         }
         // nibbles packed with exact float arithmetic: 2^23 + sum cf_i 16^i (< 2^24) holds the
-        // 16-bit half of the packed word in its low mantissa bits
-        const float lo = fmaf(cf[3], 4096.0f, fmaf(cf[2], 256.0f, fmaf(cf[1], 16.0f, cf[0] + 8388608.0f)));
-        const float hi = fmaf(cf[7], 4096.0f, fmaf(cf[6], 256.0f, fmaf(cf[5], 16.0f, cf[4] + 8388608.0f)));
-        p = prmt(__float_as_uint(lo), __float_as_uint(hi), 0x5410u);
+        // 16-bit half of the packed word in its low mantissa bits (both halves at once)
+        float2 acc = __fadd2_rn(cf[0], make_float2(8388608.0f, 8388608.0f));
+        acc = __ffma2_rn(cf[1], make_float2(16.0f, 16.0f), acc);
+        acc = __ffma2_rn(cf[2], make_float2(256.0f, 256.0f), acc);
+        acc = __ffma2_rn(cf[3], make_float2(4096.0f, 4096.0f), acc);
+        p = prmt(__float_as_uint(acc.x), __float_as_uint(acc.y), 0x5410u);
     } else {
         // keep 16/s and 17*s/16 finite for tiny and huge scales: rescale w and s by a power
         // of two (exact; a weight that underflows is far below the smallest step)
