@@ -108,3 +108,23 @@ def test_injected_launch_failure_and_device_checks(wq):
     import ctypes
     st = wq._lib.wq_unpack(ctypes.c_void_p(host.data_ptr()), 4, 64, ctypes.c_void_p(host.data_ptr()), None)
     assert st == wq.WQ_EINVAL and "device memory" in wq.last_error()
+
+
+def test_dequant_every_code_at_every_scale(wq):
+    """Dequant over all 16 codes at every finite non-negative bf16 scale (32,640 patterns,
+    one per group of 64), bit-exact against the oracle: covers the fast bf16x2 path and the
+    fp32 path for scales below 2^-120, subnormal and zero scales included."""
+    scales = np.arange(0x7F80, dtype=np.uint16)                # +0 .. max finite
+    groups = scales.size
+    k = 64 * 64
+    n = (groups + 63) // 64
+    sc = np.zeros(n * 64, np.uint16)
+    sc[:groups] = scales
+    sc = sc.reshape(n, 64)
+    codes = np.tile(np.arange(16, dtype=np.uint8), (n, k // 16))
+    codes = np.roll(codes, 3, axis=1)                         # codes 0..15 in every word position
+    packed = oracle.pack(codes)
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, torch.from_numpy(packed).cuda(), to_dev_bits(sc))
+    got = bits(wq.dequant(pw))
+    torch.cuda.synchronize()
+    assert np.array_equal(got, oracle.dequant(oracle.DYADIC4, packed, sc, 64))

@@ -229,12 +229,34 @@ dequant_dyadic_kernel(const uint32_t* __restrict__ packed, const uint16_t* __res
         for (int u = 0; u < U; ++u) {
             const int64_t i = base + 32 * u + lane;
             if (i >= n_words) break;
-            const float step = bf16_bits_to_float(sc[u]) * 0.125f;
-            float v[8];
+            uint4 o;
+            if ((sc[u] & 0x7FFFu) >= 0x0380u) {
+                // scale >= 2^-120: every nonzero step * (idx - 8) is a normal bf16. Two codes
+                // at a time: (w >> 4j) & 0x000F000F | 0x4300 in each half is the bf16 pair
+                // (128 + idx_j, 128 + idx_j+4); minus 136 gives idx - 8 exactly, and one bf16x2
+                // multiply by (step, step) (step = scale / 8: the exponent field minus 3)
+                // rounds step * (idx - 8) once, which is the definition.
+                const uint32_t st2 = prmt(sc[u] - 0x0180u, 0u, 0x1010u);
+                uint32_t q[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = step * (float)((int)((p[u] >> (4 * j)) & 15) - 8);
-            stg_cs_v4(out + i, make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7])));
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t m = ((p[u] >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
+                    const uint32_t d = bf16x2_fma(m, 0x3F803F80u, 0xC308C308u);    // idx - 8
+                    q[j] = bf16x2_fma(d, st2, 0x80008000u);                        // + (-0)
+                }
+                // q[j] = (code j, code j + 4): regroup into (0, 1) (2, 3) (4, 5) (6, 7)
+                o = make_uint4(prmt(q[0], q[1], 0x5410u), prmt(q[2], q[3], 0x5410u),
+                               prmt(q[0], q[1], 0x7632u), prmt(q[2], q[3], 0x7632u));
+            } else {
+                // tiny (or zero) scales: exact in fp32, rounded once to bf16
+                const float step = bf16_bits_to_float(sc[u]) * 0.125f;
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = step * (float)((int)((p[u] >> (4 * j)) & 15) - 8);
+                o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                               pack_bf16x2(v[6], v[7]));
+            }
+            stg_cs_v4(out + i, o);
         }
     }
 }
