@@ -24,7 +24,11 @@
 //   - a byte is >= 7 iff bit 7 of ((F & 0x7F) + 0x79) | F is set (no carry crosses bytes);
 //   - bit p of four bytes gathers into a nibble by a multiply with 0x01020408 (each bit
 //     lands on its own position, so no sums carry), and a nibble spreads back into four
-//     bytes by a multiply with 0x00204081.
+//     bytes by a multiply with 0x00204081;
+//   - the block's largest exponent field is the largest magnitude (|w| bits order like
+//     |w|) shifted down 7, from packed 16-bit max instructions; the counting pass needs no
+//     fields at all: w escapes iff |w| < (E - 6) << 7, compared two at a time in 16-bit
+//     lanes where (w | 0x8000) - T cannot borrow across the halves.
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -46,10 +50,10 @@ __device__ __forceinline__ void split4(uint32_t x, uint32_t y, uint32_t& e, uint
     e = ((hi << 1) & 0xFEFEFEFEu) | ((lo >> 7) & 0x01010101u);
 }
 
-__device__ __forceinline__ uint32_t max_byte(uint32_t v) {
-    const uint32_t a = max(v & 0xFFu, (v >> 8) & 0xFFu);
-    const uint32_t b = max((v >> 16) & 0xFFu, v >> 24);
-    return max(a, b);
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 // bit 0 of each byte -> a nibble
@@ -87,11 +91,11 @@ __device__ __forceinline__ void encode_half(const uint4 w, uint32_t E, Half& h) 
     }
 }
 
-__device__ __forceinline__ uint32_t half_emax(const uint4 w) {
-    uint32_t e0, e1, s0, s1;
-    split4(w.x, w.y, e0, s0);
-    split4(w.z, w.w, e1, s1);
-    return max(max_byte(e0), max_byte(e1));
+// The largest exponent field of 8 bf16 (the magnitude bits order like the values).
+__device__ __forceinline__ uint32_t half_emax16(const uint4 w) {
+    uint32_t m = max_u16x2(max_u16x2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                           max_u16x2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16) >> 7;
 }
 
 // Escape offsets: an exclusive scan of the per-superblock escape counts, in place in sb_off,
@@ -128,12 +132,22 @@ bf16x_count_kernel(const uint4* __restrict__ w, int64_t nhalf, int64_t nsb, uint
 #pragma unroll
             for (int u = 0; u < kUnits; ++u) {
                 if (s0 + u >= t1) break;
-                const uint32_t me = half_emax(v[u]);
-                const uint32_t E = max(me, __shfl_xor_sync(0xFFFFFFFFu, me, 1));
-                Half h;
-                encode_half(v[u], E, h);
+                // only the count: a weight escapes iff E - e >= 7, i.e. its magnitude bits
+                // |w| (15 bits, exponent field above the 7 mantissa bits) lie below
+                // T = (E - 6) << 7. The magnitudes are compared two at a time in 16-bit lanes:
+                // (w | 0x8000) - T cannot borrow across the halves, and bit 15 of each half is
+                // set iff |w| >= T.
+                const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                const uint32_t mx = half_emax16(v[u]);                  // this half's E
+                const uint32_t E = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+                uint32_t c = 0;
+                if (E >= 7) {
+                    const uint32_t T2 = ((E - 6) << 7) * 0x00010001u;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) c += __popc(~((wv[q] | 0x80008000u) - T2) & 0x80008000u);
+                }
                 const int64_t t = (s0 + u) * 32 + lane;
-                const uint32_t c = t < nhalf ? __popc(h.esc) : 0u;
+                if (t >= nhalf) c = 0;
                 const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, c);
                 if (lane == 0) sb[s0 + u] = total;
                 run += total;
@@ -267,7 +281,7 @@ bf16x_encode_kernel(const uint4* __restrict__ w, int64_t nhalf, int64_t nsb,
             const int64_t s = s0 + u;
             if (s >= nsb) break;
             const int64_t t = s * 32 + lane;
-            const uint32_t me = half_emax(v[u]);
+            const uint32_t me = half_emax16(v[u]);
             const uint32_t E = max(me, __shfl_xor_sync(0xFFFFFFFFu, me, 1));
             Half h;
             encode_half(v[u], E, h);
