@@ -295,3 +295,51 @@ def test_gemv_cluster_split_k_matches_oracle(wq, n, k, batch):
     rows = np.concatenate([g.choice(n, 96, replace=False), np.arange(n - 8, n)])
     y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, scale, 64, x_bits, rows=rows)
     _check(y, y_ref, bound, rows)
+
+
+@pytest.mark.parametrize("batch", [1, 4, 16])
+def test_full_decode_sweep_in_the_benchmarked_launch(wq, batch):
+    """All 168 matrices of the decode-sweep stack (1,056,964,608 weights) in the one grouped,
+    prepared launch the benchmark times (the full-K kernel variant that only a launch of this
+    size selects). Seeded codes and scales from the host; 6 sampled rows of every matrix,
+    plus its last row, against the oracle."""
+    mats = workloads.sweep_matrices()
+    g = np.random.default_rng(77 + batch)
+    ws, host, xs_bits = [], [], []
+    for layer, name, n, k, idx in mats:
+        packed = g.integers(0, 256, (n, k // 2), dtype=np.uint8)
+        scale = workloads.f64_to_bf16_bits(g.uniform(0.002, 0.08, (n, k // 64)))
+        ws.append(wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(packed), to_dev_bits(scale)))
+        host.append((packed, scale))
+        xs_bits.append(workloads.activations(batch, k, workloads.DECODE_SWEEP, idx))
+    xs = [to_dev_bits(x) for x in xs_bits]
+    ys = [torch.empty((batch, n), dtype=torch.bfloat16, device="cuda") for _, _, n, _, _ in mats]
+    plan = wq.GroupedGemv(ws, xs, ys)
+    plan()
+    torch.cuda.synchronize()
+    plan.close()
+    assert wq.device_error() == 0
+    for (packed, scale), x, y in zip(host, xs_bits, ys):
+        n = packed.shape[0]
+        rows = np.concatenate([g.choice(n, 6, replace=False), [n - 1]])
+        y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, scale, 64, x, rows=rows)
+        _check(y, y_ref, bound, rows)
+
+
+@pytest.mark.parametrize("batch", [1, 8, 16])
+def test_lut16_full_size_in_the_benchmarked_launch(wq, batch):
+    """The 16-centroid LUT workload at full size (8192 x 28672: K split across a cluster of
+    CTAs, the launch the benchmark times), seeded codes and sorted fp16 centroid tables from
+    the host; 64 sampled rows, plus the last row, against the oracle."""
+    n, k = workloads.LUT16_SHAPE
+    g = np.random.default_rng(91 + batch)
+    packed = g.integers(0, 256, (n, k // 2), dtype=np.uint8)
+    lut = oracle.f64_to_fp16(np.sort(g.standard_normal((n, k // 64, 16)), -1) * 0.01)
+    pw = wq.PackedWeight(wq.FMT_LUT16, 64, n, k, to_dev(packed), to_dev_bits(lut, torch.float16))
+    x_bits = workloads.activations(batch, k, workloads.LUT16, batch)
+    y = wq.gemv(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+    rows = np.concatenate([np.sort(g.choice(n, 64, replace=False)), [n - 1]])
+    y_ref, bound = oracle.matmul_rows(oracle.LUT16, packed, lut, 64, x_bits, rows=rows)
+    _check(y, y_ref, bound, rows)
