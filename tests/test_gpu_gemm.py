@@ -2,6 +2,8 @@
 reconstruction: |y - y_ref| <= 2e-3 * sum_k |Wdeq[n, k]| |x[m, k]| per element, plus exact
 special cases (one-hot activations reproduce a dequantised column; all-eight codes give
 zero) and the split-K workspace path used for small m."""
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -65,14 +67,22 @@ def test_gemm_split_k_uses_workspace(wq):
     assert np.all(err <= matmul_tolerance(y_ref, bound, TOL))
 
 
+@functools.lru_cache(maxsize=2)
+def _prefill_quantised(n, k):
+    """A prefill weight quantised by the oracle on the host (packed codes, bf16 scales)."""
+    w_bits = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 0 if n == 4096 else 1)
+    s, c = oracle.dyadic_quantize(w_bits, 64)
+    return oracle.pack(c), s
+
+
 @pytest.mark.parametrize("shape", workloads.PREFILL_SHAPES)
 @pytest.mark.parametrize("m", workloads.PREFILL_M)
 def test_gemm_full_size_sampled(wq, shape, m):
     """The prefill workload at full size: (n, k) = (4096, 11008) / (11008, 4096), every m;
     96 sampled weight rows x up to 128 sampled activation rows against the oracle."""
     n, k = shape
-    w_bits = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 0 if n == 4096 else 1)
-    pw, _ = wq.quantize_dyadic(to_dev_bits(w_bits), 64)
+    packed, s = _prefill_quantised(n, k)
+    pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(packed), to_dev_bits(s))
     x_bits = workloads.activations(m, k, workloads.PREFILL, m)
     y = wq.gemm(pw, to_dev_bits(x_bits))
     torch.cuda.synchronize()
@@ -80,8 +90,6 @@ def test_gemm_full_size_sampled(wq, shape, m):
     rng = np.random.default_rng(m + n)
     rows = np.sort(rng.choice(n, 96, replace=False))
     ms = np.sort(rng.choice(m, min(m, 128), replace=False))
-    packed = pw.packed.cpu().numpy()
-    s = pw.aux.view(torch.int16).cpu().numpy().view(np.uint16)
     y_ref, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x_bits[ms], rows=rows)
     got = f32(y)[np.ix_(ms, rows)]
     assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))

@@ -101,16 +101,17 @@ def test_grouped_gemv_equals_single_calls(wq, batch):
 
 
 def test_decode_sweep_layer_full_size_sampled(wq):
-    """One layer of the decode-sweep stack at full size, quantised on the GPU, in the
-    grouped launch the benchmark times; sampled rows of every projection against the
-    oracle, at batch 1 and 16."""
+    """One layer of the decode-sweep stack at full size, quantised by the oracle, in one
+    grouped launch; sampled rows of every projection against the oracle, at batch 1 and 16."""
     mats = [m for m in workloads.sweep_matrices(1)]
     ws, pk = [], []
     for layer, name, n, k, idx in mats:
+        # quantised by the oracle on the host: the GEMV's inputs never come from the GPU path
         w_bits = workloads.gaussian_outlier_weight(n, k, workloads.DECODE_SWEEP, idx)
-        pw, _ = wq.quantize_dyadic(to_dev_bits(w_bits), 64)
-        ws.append(pw)
-        pk.append((pw.packed.cpu().numpy(), bits(pw.aux)))
+        s, c = oracle.dyadic_quantize(w_bits, 64)
+        packed = oracle.pack(c)
+        ws.append(wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(packed), to_dev_bits(s)))
+        pk.append((packed, s))
     rng = np.random.default_rng(4)
     for batch in (1, 16):
         xb = [workloads.activations(batch, k, workloads.DECODE_SWEEP, idx) for _, _, _, k, idx in mats]
@@ -263,15 +264,16 @@ def test_gemv_lloyd8s_one_hot_reproduces_dequant_exactly(wq):
         assert np.array_equal(y, wd[:, cc].T)
 
 
-def test_gemv_lloyd8s_on_the_gpu_producers_output(wq):
-    """The g32 Lloyd producer's packed codes and levels, consumed by the fused GEMV and by the
-    oracle (sampled rows), on one Lloyd-workload matrix."""
-    w_bits = workloads.laplace_rowscaled_weight(512, 2048, index=3)
-    pw, _ = wq.quantize_lloyd(to_dev_bits(w_bits), wq.LLOYD_G32_WARM, 25)
-    packed = pw.packed.cpu().numpy()
-    levels = pw.aux.cpu().numpy()
+def test_gemv_lloyd8s_on_lloyd_quantised_weights(wq):
+    """Codes and levels of the g32 Lloyd producer (the oracle's, on the host) on rows of the
+    Lloyd workload, consumed by the fused GEMV and by the oracle (sampled rows)."""
+    w_bits = workloads.laplace_rowscaled_weight(128, 2048, index=3)
+    ref = oracle.lloyd(w_bits, 32, 25)
+    packed = oracle.pack(ref["codes"])
+    levels = ref["levels"].astype(np.float32)
+    pw = wq.PackedWeight(wq.FMT_LLOYD8S, 32, 128, 2048, to_dev(packed), torch.from_numpy(levels).cuda())
     rng = np.random.default_rng(8)
-    rows = rng.choice(512, 64, replace=False)
+    rows = rng.choice(128, 64, replace=False)
     for batch in (1, 16):
         x_bits = workloads.activations(batch, 2048, workloads.DECODE_SWEEP, 40 + batch)
         y = wq.gemv(pw, to_dev_bits(x_bits))

@@ -50,8 +50,9 @@ def _check_lloyd(wq, w_bits, rounds=25, max_mismatch_frac=1e-3):
         assert np.all(gpu_c_mse[mism] <= best[mism] * (1 + 1e-4) + 1e-12 * gmax[mism] ** 2)
         ref = forced
     assert np.array_equal(g_par, ref["params"])
-    # packed bytes agree with the codes
-    assert np.array_equal(pw.packed.cpu().numpy(), oracle.pack(g_codes))
+    # the packed bytes hold the codes (the GPU's own unpack; nothing of the GPU's goes into
+    # the oracle except the near-tie candidates above, which it validates first)
+    assert np.array_equal(wq.unpack(pw.packed).cpu().numpy(), g_codes)
     # codes exact where the nearest-level margin is not a near-tie
     clear = ref["min_margin"] > 1e-6 * gmax
     cmatch = (g_codes.reshape(n, k // 32, 32) == ref["codes"].reshape(n, k // 32, 32)).all(-1)
@@ -65,10 +66,14 @@ def _check_lloyd(wq, w_bits, rounds=25, max_mismatch_frac=1e-3):
     diff = np.abs(g_tr - tr)[clear]
     assert np.all((diff <= 1e-5 * tr[clear] + 2.0 ** -126)[inrange])
     assert np.all(np.isinf(g_tr[clear][~inrange]))
-    # dequant of the GPU's own output is exactly the oracle's reconstruction of it
-    d = wq.dequant(pw)
-    assert np.array_equal(bits(d), oracle.dequant(oracle.LLOYD8S, pw.packed.cpu().numpy(),
-                                                  pw.aux.cpu().numpy(), 32))
+    # dequant of the oracle's codes and levels (as fp32, the stored format) is exactly the
+    # oracle's reconstruction of them
+    r_packed = oracle.pack(ref["codes"])
+    r_levels = ref["levels"].astype(np.float32)
+    rw = wq.PackedWeight(wq.FMT_LLOYD8S, 32, n, k, torch.from_numpy(r_packed).cuda(),
+                         torch.from_numpy(r_levels).cuda())
+    d = wq.dequant(rw)
+    assert np.array_equal(bits(d), oracle.dequant(oracle.LLOYD8S, r_packed, r_levels, 32))
     return frac, (~clear).mean()
 
 
