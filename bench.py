@@ -248,17 +248,65 @@ def run_ours(args):
     achieved = algo_bytes / (ms * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers ---------------------------
+    # Every step copies its activations in from pinned host memory and its outputs back
+    # out, inside the timed region. The steps are independent batches, so two device buffer
+    # sets (one prepared plan each) let step i + 1's copy-in and step i - 1's copy-out run
+    # beside step i's kernel: a copy-in stream, the compute stream and a copy-out stream,
+    # ordered by events (a buffer set is refilled only after its kernel has read it, and its
+    # outputs are overwritten only after they have been copied out).
     x_pin = xflat.cpu().pin_memory()
-    y_pin = torch.empty(yflat.shape, dtype=torch.bfloat16).pin_memory()
+    y_pins = [torch.empty(yflat.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xflat2, yflat2 = torch.empty_like(xflat), torch.empty_like(yflat)
+    xs2, ys2, xo, yo = [], [], 0, 0
+    for _, _, n, k, _ in mats:
+        xs2.append(xflat2[xo:xo + B * k].view(B, k))
+        ys2.append(yflat2[yo:yo + B * n].view(B, n))
+        xo += B * k
+        yo += B * n
+    runs = [run, wq.GroupedGemv(packed, xs2, ys2)]
+    xbufs, ybufs = [xflat, xflat2], [yflat, yflat2]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        xflat.copy_(x_pin, non_blocking=True)       # this step's activations, host -> device
-        run()                                       # the public API call (prepared plan)
-        y_pin.copy_(yflat, non_blocking=True)       # this step's outputs, device -> host
+    def e2e_steps(nsteps):
+        comp, out = [None, None], [None, None]
+        for i in range(nsteps):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if comp[b] is not None:
+                    s_in.wait_event(comp[b])            # its kernel has read this buffer set
+                xbufs[b].copy_(x_pin, non_blocking=True)    # this step's activations in
+                e_in = torch.cuda.Event()
+                e_in.record(s_in)
+            stream.wait_event(e_in)
+            if out[b] is not None:
+                stream.wait_event(out[b])               # its last outputs have left
+            runs[b]()                                   # the public API call (prepared plan)
+            comp[b] = torch.cuda.Event()
+            comp[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp[b])
+                y_pins[b].copy_(ybufs[b], non_blocking=True)   # this step's outputs out
+                out[b] = torch.cuda.Event()
+                out[b].record(s_out)
+        return [e for e in out if e is not None]
 
-    ms_e2e = max_over_ranks(time_region(torch, stream, e2e_step, args.steps, args.warmup, barrier))
+    e2e_steps(max(args.warmup, 2))
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    s_in.wait_stream(stream)
+    for e in e2e_steps(args.steps):
+        stream.wait_event(e)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(t0.elapsed_time(t1) / args.steps)
     e2e = {"value": round(replica_value(world, weight_bytes, ms_e2e), 2), "unit": UNIT,
-           "h2d_bytes_per_step": x_b, "d2h_bytes_per_step": y_b, "ms_per_step": round(ms_e2e, 4)}
+           "h2d_bytes_per_step": x_b, "d2h_bytes_per_step": y_b, "ms_per_step": round(ms_e2e, 4),
+           "pipelining": "2 buffer sets: copy-in of step i+1 and copy-out of step i-1 beside step i's kernel"}
 
     extras = {}
     if not args.no_extras:
