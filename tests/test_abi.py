@@ -61,6 +61,22 @@ def test_shape_and_group_checks_fail_before_any_cuda_call(wq):
     assert "2^32" in wq.last_error()
     assert lib.wq_bf16x_encode(p, 4, 64, p, p, p, p, -1, None) == wq.WQ_EINVAL
     assert lib.wq_bf16x_decode(p, p, p, p, 16, 4, 80, p, None) == wq.WQ_EINVAL
+    # Gumbel-ST: group, temperature (positive normal finite), shapes
+    assert lib.wq_gumbel_st_backward(p, 4, 64, 16, p, 1.0, p, p, None, None) == wq.WQ_EUNSUPPORTED
+    for tau in (0.0, -1.0, float("nan"), float("inf"), 1e-39):
+        assert lib.wq_gumbel_st_backward(p, 4, 64, 64, p, tau, p, p, None, None) == wq.WQ_EINVAL
+    assert "tau" in wq.last_error()
+    assert lib.wq_gumbel_st_backward(p, 4, 96, 64, p, 1.0, p, p, None, None) == wq.WQ_EINVAL
+    assert lib.wq_gumbel_st_backward(p, 0, 64, 64, p, 1.0, p, p, None, None) == wq.WQ_EINVAL
+    # water-filling: k % 64, block offsets below 2^32, lambda >= 0, buffer sizes >= 0
+    assert lib.wq_quantize_wf_analyze(p, 4, 96, 0.0, p, p, p, None, None) == wq.WQ_EINVAL
+    assert lib.wq_quantize_wf_analyze(p, 1 << 20, 1 << 14, 0.0, p, p, p, None, None) == wq.WQ_EINVAL
+    assert "2^32" in wq.last_error()
+    assert lib.wq_quantize_wf_analyze(p, 4, 64, -1.0, p, p, p, None, None) == wq.WQ_EINVAL
+    assert lib.wq_quantize_wf_analyze(p, 4, 64, float("nan"), p, p, p, None, None) == wq.WQ_EINVAL
+    assert lib.wq_quantize_wf_pack(p, 4, 64, p, p, p, p, -1, None) == wq.WQ_EINVAL
+    assert lib.wq_dequant_wf(p, -1, p, p, p, 4, 64, p, None) == wq.WQ_EINVAL
+    assert lib.wq_dequant_wf(p, 16, p, p, p, 0, 64, p, None) == wq.WQ_EINVAL
 
 
 def test_gemv_plan_rejects_bad_arguments_and_keeps_nothing(wq):
