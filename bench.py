@@ -441,22 +441,25 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
                                        "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
         del gz
         # Gumbel-ST backward on the same latent: z, gq in; gz, gscale out (12.1 B per element),
-        # 16 softmax weights per element, tau = 1 step^2 of a typical group
+        # 16 softmax weights per element; at tau = 1.0 (mid-way through the page's 5 -> 0.3
+        # anneal: the weights spread over all codes) and at tau = step^2 of a typical group
+        # (weights concentrated near the nearest code)
         gql = torch.randn((n_l, k_l), device=dev)
         gzo = torch.empty_like(zl)
         gso = torch.empty((n_l, k_l // 64), dtype=torch.float32, device=dev)
-        tau = float((scl.float().median() / 8) ** 2)
-        ggb = graph_of(torch, lambda: wq._check(wq._lib.wq_gumbel_st_backward(
-            wq._ptr(zl), n_l, k_l, 64, wq._ptr(scl), tau, wq._ptr(gql), wq._ptr(gzo), wq._ptr(gso),
-            wq._stream(zl))))
-        ms = max_over_ranks(time_region(torch, stream, ggb.replay, steps, warm, barrier))
-        byts = nw * (4 + 4 + 4) + nw / 64 * (2 + 4)
-        out["gumbel_st_backward_large"] = {"shape": [n_l, k_l], "us": round(ms * 1e3, 1),
-                                           "Gelements/s": round(nw / ms / 1e6, 2),
-                                           "GB/s": round(byts / ms / 1e6, 1),
-                                           "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
-                                           "ex2_per_element": 16}
-        del ggb, gql, gzo, gso, zl, scl, qo, po
+        gum = {"shape": [n_l, k_l], "ex2_per_element": 16}
+        for name, tau in (("tau_1.0", 1.0), ("tau_step2", float((scl.float().median() / 8) ** 2))):
+            ggb = graph_of(torch, lambda: wq._check(wq._lib.wq_gumbel_st_backward(
+                wq._ptr(zl), n_l, k_l, 64, wq._ptr(scl), tau, wq._ptr(gql), wq._ptr(gzo), wq._ptr(gso),
+                wq._stream(zl))))
+            ms = max_over_ranks(time_region(torch, stream, ggb.replay, steps, warm, barrier))
+            byts = nw * (4 + 4 + 4) + nw / 64 * (2 + 4)
+            gum[name] = {"tau": tau, "us": round(ms * 1e3, 1), "Gelements/s": round(nw / ms / 1e6, 2),
+                         "GB/s": round(byts / ms / 1e6, 1),
+                         "frac_hbm": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4)}
+            del ggb
+        out["gumbel_st_backward_large"] = gum
+        del gql, gzo, gso, zl, scl, qo, po
         # BF16X lossless codec on a bf16 matrix of the same shape (N(0, 0.02^2)): the two
         # encoding passes (count, encode) and the decode, each a plain stream
         wb = (torch.randn((n_l, k_l), device=dev) * 0.02).to(torch.bfloat16)

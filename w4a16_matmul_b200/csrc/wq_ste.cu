@@ -145,28 +145,81 @@ __device__ __forceinline__ void gumbel_st_pair(float2 z, float2 up, float s, flo
                                   (float)ste_index(z.y, s, c8, step, m17, fast));
     const float2 c_idx = __fmul2_rn(f2(step), __fadd2_rn(fi, f2(-8.0f)));
     const float2 e = __fadd2_rn(z, make_float2(-c_idx.x, -c_idx.y));
-    const float2 A = __fmul2_rn(e, f2(step * l2t));
-    const float2 nB = f2(-(step * step * (0.5f * l2t)));
-    const float2 nfi = make_float2(-fi.x, -fi.y);
-    float2 s0 = f2(0.0f), s1 = f2(0.0f), s2 = f2(0.0f), s3 = f2(0.0f);
+    const float B = step * step * (0.5f * l2t);
+    float2 mu, m2, m3;
+    if (B > 0x1p-6f) {
+        // weights concentrated near the nearest code: logits and moments about it
+        const float2 A = __fmul2_rn(e, f2(step * l2t));
+        const float2 nB = f2(-B);
+        const float2 nfi = make_float2(-fi.x, -fi.y);
+        float2 s0 = f2(0.0f), s1 = f2(0.0f), s2 = f2(0.0f), s3 = f2(0.0f);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const float2 u = __fadd2_rn(f2((float)j), nfi);
-        const float2 arg = __fmul2_rn(u, __ffma2_rn(nB, u, A));
-        const float2 p = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
-        s0 = __fadd2_rn(s0, p);
-        const float2 pu = __fmul2_rn(p, u);
-        s1 = __fadd2_rn(s1, pu);
-        s2 = __ffma2_rn(pu, u, s2);
-        s3 = __ffma2_rn(__fmul2_rn(pu, u), u, s3);
+        for (int j = 0; j < 16; ++j) {
+            const float2 u = __fadd2_rn(f2((float)j), nfi);
+            const float2 arg = __fmul2_rn(u, __ffma2_rn(nB, u, A));
+            const float2 p = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+            s0 = __fadd2_rn(s0, p);
+            const float2 pu = __fmul2_rn(p, u);
+            s1 = __fadd2_rn(s1, pu);
+            s2 = __ffma2_rn(pu, u, s2);
+            s3 = __ffma2_rn(__fmul2_rn(pu, u), u, s3);
+        }
+        // s0 is in [1, 16]: the nearest code has weight 1
+        const float2 inv = make_float2(rcp_approx(s0.x), rcp_approx(s0.y));
+        mu = __fmul2_rn(s1, inv);
+        const float2 e2 = __fmul2_rn(s2, inv), e3 = __fmul2_rn(s3, inv);
+        m2 = __ffma2_rn(make_float2(-mu.x, -mu.y), mu, e2);                          // E[u^2] - mu^2
+        // E[u^3] - 3 mu E[u^2] + 2 mu^3 = E[u^3] - mu (3 E[u^2] - 2 mu^2)
+        m3 = __ffma2_rn(make_float2(-mu.x, -mu.y),
+                        __ffma2_rn(f2(-2.0f), __fmul2_rn(mu, mu), __fmul2_rn(f2(3.0f), e2)), e3);
+    } else {
+        // B <= 2^-6 (the page's temperatures on weight-scale latents): log2 p_j varies by at
+        // most 225 B over the 16 codes within the scale, so the weights are spread and the
+        // logits are a quadratic in the code index j (constant coefficients per element;
+        // rounding error below 1e-5 in the exponent), with the moments accumulated about the fixed centre
+        // j' = j - 7.5 (constant powers of j'; the spread distribution keeps the centring to
+        // a few lost bits). With f = z + 8 step: log2 p_j - log2 p_idx =
+        //   -B j^2 + 2 K f step j + K (e^2 - f^2),  K = log2(e) / tau,
+        // and K (e^2 - f^2) = -K step idx (e + f) without cancellation.
+        const float K = 0.5f * l2t;
+        const float2 f = __ffma2_rn(f2(8.0f), f2(step), z);
+        const float2 c1 = __fmul2_rn(f, f2(2.0f * K * step));
+        const float2 c0 = __fmul2_rn(__fmul2_rn(fi, f2(-K * step)), __fadd2_rn(e, f));
+        // The weights of consecutive codes have the ratio r_j = p_(j+1) / p_j =
+        // 2^(c1 - B (2 j + 1)), and r_(j+1) = r_j * 2^(-2 B): every 4 codes an anchor takes p
+        // and r from the special-function unit, the next 3 codes follow by multiplication
+        // (at most 3 roundings and ex2 errors each: about 1e-6 relative), so 8 ex2 per
+        // element are spent instead of 16.
+        const float rho = ex2_approx(-2.0f * B);
+        float2 s0 = f2(0.0f), s1 = f2(0.0f), s2 = f2(0.0f), s3 = f2(0.0f);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const float j0 = (float)(4 * a);
+            const float2 arg = __ffma2_rn(__ffma2_rn(f2(-B), f2(j0), c1), f2(j0), c0);
+            const float2 argr = __fadd2_rn(c1, f2(-B * (2.0f * j0 + 1.0f)));
+            float2 p = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+            float2 r = make_float2(ex2_approx(argr.x), ex2_approx(argr.y));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float jc = j0 + (float)q - 7.5f;
+                s0 = __fadd2_rn(s0, p);
+                s1 = __ffma2_rn(p, f2(jc), s1);
+                s2 = __ffma2_rn(p, f2(jc * jc), s2);
+                s3 = __ffma2_rn(p, f2(jc * jc * jc), s3);
+                if (q < 3) {
+                    p = __fmul2_rn(p, r);
+                    r = __fmul2_rn(r, f2(rho));
+                }
+            }
+        }
+        const float2 inv = make_float2(rcp_approx(s0.x), rcp_approx(s0.y));
+        const float2 mc = __fmul2_rn(s1, inv);                                      // E[j'], about 7.5
+        const float2 e2 = __fmul2_rn(s2, inv), e3 = __fmul2_rn(s3, inv);
+        m2 = __ffma2_rn(make_float2(-mc.x, -mc.y), mc, e2);
+        m3 = __ffma2_rn(make_float2(-mc.x, -mc.y),
+                        __ffma2_rn(f2(-2.0f), __fmul2_rn(mc, mc), __fmul2_rn(f2(3.0f), e2)), e3);
+        mu = __fadd2_rn(mc, __fadd2_rn(f2(7.5f), make_float2(-fi.x, -fi.y)));       // about idx
     }
-    // s0 is in [1, 16]: the nearest code has weight 1
-    const float2 inv = make_float2(rcp_approx(s0.x), rcp_approx(s0.y));
-    const float2 mu = __fmul2_rn(s1, inv), e2 = __fmul2_rn(s2, inv), e3 = __fmul2_rn(s3, inv);
-    const float2 m2 = __ffma2_rn(make_float2(-mu.x, -mu.y), mu, e2);                // E[u^2] - mu^2
-    // E[u^3] - 3 mu E[u^2] + 2 mu^3 = E[u^3] - mu (3 E[u^2] - 2 mu^2)
-    const float2 m3 = __ffma2_rn(make_float2(-mu.x, -mu.y),
-                                 __ffma2_rn(f2(-2.0f), __fmul2_rn(mu, mu), __fmul2_rn(f2(3.0f), e2)), e3);
     gz = __fmul2_rn(up, __fmul2_rn(f2((r2 * step) * step), m2));
     // z - 2 c_idx - 2 step mu
     const float2 lin = __ffma2_rn(f2(-2.0f * step), mu, __ffma2_rn(f2(-2.0f), c_idx, z));
