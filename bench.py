@@ -721,7 +721,8 @@ def run_profile_target(args):
     """A few launches of one kernel on one shape and nothing else, for ncu captures:
     --profile gemm --shape N,K,M (prefill GEMM), quantize --shape N,K, dequant --shape N,K,
     lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd), gumbel --shape N,K
-    (Gumbel-ST backward), bf16x --shape N,K (BF16X encode + decode), wf --shape N,K
+    (Gumbel-ST backward at tau = step^2; gumbel1: at tau = 1.0), ste --shape N,K (STE forward),
+    bf16x --shape N,K (BF16X encode + decode), wf --shape N,K
     (water-filling analyze + dequant). Random packed codes and
     scales (timing does not depend on the values); inputs stay on the device."""
     import torch
@@ -760,6 +761,15 @@ def run_profile_target(args):
         gq = torch.randn((n, k), device=dev, generator=gen)
         tau = float((s.float().median() / 8) ** 2)
         fn = lambda: wq.gumbel_st_backward(z, s, gq, tau, 64)
+    elif args.profile == "gumbel1":
+        z = torch.randn((n, k), device=dev, generator=gen) * 0.02
+        s = (z.abs().reshape(n, k // 64, 64).amax(-1) * 1.1).to(torch.bfloat16)
+        gq = torch.randn((n, k), device=dev, generator=gen)
+        fn = lambda: wq.gumbel_st_backward(z, s, gq, 1.0, 64)
+    elif args.profile == "ste":
+        z = torch.randn((n, k), device=dev, generator=gen) * 0.02
+        s = (z.abs().reshape(n, k // 64, 64).amax(-1)).to(torch.bfloat16)
+        fn = lambda: wq.fake_quant_ste(z, s, 64, packed=True)
     elif args.profile == "bf16x":
         w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
         enc = wq.bf16x_encode(w)
