@@ -39,28 +39,32 @@ __device__ __forceinline__ float rcp_fast(float x) {
     return r;
 }
 
-// idx for one element. idx = #{j in 1..15 : z > m_j} with m_j = (2j - 17) s / 16.
+// idx for one element, idx = #{j in 1..15 : z > m_j} with m_j = (2j - 17) s / 16.
 //   Fast path (s in [2^-96, 2^96]): every m_j is exact in fp32 (an 8-bit significand times an
 //   odd integer <= 17, over 16). u = 8 z / s + 8.5, clamped to [0, 16.5], approximates the
 //   real count boundary to better than 2^-18, so ceil(u) - 1 is the count or one off either
 //   way; one exact comparison each way settles it.
 //   Other scales: the count itself, with each midpoint formed exactly in double.
-__device__ __forceinline__ uint32_t ste_index(float z, float s, float c8, float s8, float m17,
-                                              bool fast) {
-    if (s == 0.0f) return 0;                                   // every code ties
+// The index as a float (an exact small integer): the callers form the code value from it
+// without an int-to-float conversion, and the integer code as float_as_uint(x + 2^23) & 15.
+__device__ __forceinline__ float ste_index_f(float z, float s, float c8, float s8, float m17,
+                                             bool fast) {
+    if (s == 0.0f) return 0.0f;                                // every code ties
     if (fast) {
         const float u = fminf(fmaxf(fmaf(z, c8, 8.5f), 0.0f), 16.5f);
         float x = fminf(fmaxf(__fadd_ru(u, 8388608.0f) - 8388609.0f, 0.0f), 15.0f);
         if (x > 0.0f && !(z > fmaf(x, s8, m17))) x -= 1.0f;               // z <= m_x
         else if (x < 15.0f && z > fmaf(x + 1.0f, s8, m17)) x += 1.0f;     // z > m_{x+1}
-        return __float_as_uint(x + 8388608.0f) & 15u;
+        return x;
     }
     const double sd = (double)s, zd = (double)z;
-    uint32_t n = 0;
+    float n = 0.0f;
 #pragma unroll
-    for (int j = 1; j < 16; ++j) n += zd > (double)(2 * j - 17) * sd * 0.0625 ? 1u : 0u;
+    for (int j = 1; j < 16; ++j) n += zd > (double)(2 * j - 17) * sd * 0.0625 ? 1.0f : 0.0f;
     return n;
 }
+
+__device__ __forceinline__ uint32_t index_bits(float x) { return __float_as_uint(x + 8388608.0f) & 15u; }
 
 // One thread: 8 consecutive elements (one quarter or eighth of a group), U such blocks in
 // flight, grid-stride.
@@ -99,11 +103,11 @@ fake_quant_ste_kernel(const float4* __restrict__ z, const uint16_t* __restrict__
             float qv[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                idx[j] = ste_index(zv[j], s, c8, s8, m17, fast);
+                const float xf = ste_index_f(zv[j], s, c8, s8, m17, fast);
+                idx[j] = index_bits(xf);
                 // the code value: exact in fp32 on the fast path; otherwise the double value
                 // rounded once, as the definition reads
-                qv[j] = fast ? s8 * (float)((int)idx[j] - 8)
-                             : (float)((double)s * 0.125 * (double)((int)idx[j] - 8));
+                qv[j] = fast ? s8 * (xf - 8.0f) : (float)((double)s * 0.125 * (double)(xf - 8.0f));
             }
             stg_cs_v4(q + 2 * i, make_uint4(__float_as_uint(qv[0]), __float_as_uint(qv[1]),
                                             __float_as_uint(qv[2]), __float_as_uint(qv[3])));
@@ -141,8 +145,8 @@ __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 __device__ __forceinline__ void gumbel_st_pair(float2 z, float2 up, float s, float c8, float step,
                                                float m17, bool fast, float l2t, float r2,
                                                float2& gz, float2& gs) {
-    const float2 fi = make_float2((float)ste_index(z.x, s, c8, step, m17, fast),
-                                  (float)ste_index(z.y, s, c8, step, m17, fast));
+    const float2 fi = make_float2(ste_index_f(z.x, s, c8, step, m17, fast),
+                                  ste_index_f(z.y, s, c8, step, m17, fast));
     const float2 c_idx = __fmul2_rn(f2(step), __fadd2_rn(fi, f2(-8.0f)));
     const float2 e = __fadd2_rn(z, make_float2(-c_idx.x, -c_idx.y));
     const float B = step * step * (0.5f * l2t);
