@@ -48,7 +48,7 @@ typedef enum wq_status {
     WQ_OK = 0,
     WQ_EINVAL = 1,        /* bad size, NULL or non-device pointer, bad format field */
     WQ_EALIGN = 2,        /* pointer not 16-byte aligned */
-    WQ_EUNSUPPORTED = 3,  /* valid request this build does not implement (e.g. group) */
+    WQ_EUNSUPPORTED = 3,  /* valid request this library does not implement (e.g. group) */
     WQ_ECUDA = 4,         /* the CUDA runtime reported an error (launch or attribute query) */
     WQ_ETIMEOUT = 5,      /* a bounded device-side wait gave up (reserved) */
     WQ_EDATA = 6          /* a kernel found inconsistent encoded data (wq_device_error) */
