@@ -225,13 +225,30 @@ wf_dequant_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, cons
             const unsigned long long* src = reinterpret_cast<const unsigned long long*>(packed);
             unsigned long long v = __ldg(src + (w0 >> 3)) >> sh;
             if (sh + 8 * bw > 64) v |= __ldg(src + (w0 >> 3) + 1) << (64 - sh);
-            const float s16 = bf16_bits_to_float(ldg_u16(scale + i)) * 0.0625f;
+            const uint32_t sb = ldg_u16(scale + i);
             const uint32_t mask = (1u << bw) - 1u;
+            if ((sb & 0x7FFFu) >= 0x0400u) {
+                // scale >= 2^-119: every nonzero (scale / 16) (idx_5 - 16) is a normal bf16.
+                // Two codes at a time: idx_5 | 0x4300 is the bf16 number 128 + idx_5, minus 144
+                // is idx_5 - 16 exactly, and one bf16x2 multiply by scale / 16 (the exponent
+                // field minus 4) rounds the product once, as the definition reads.
+                const uint32_t s16x2 = prmt(sb - 0x0200u, 0u, 0x1010u);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i0 = (int)(((uint32_t)(v >> (bw * 2 * j)) & mask) << (5 - bw));
-                const int i1 = (int)(((uint32_t)(v >> (bw * (2 * j + 1))) & mask) << (5 - bw));
-                o[j] = pack_bf16x2(s16 * (float)(i0 - 16), s16 * (float)(i1 - 16));
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t c0 = (uint32_t)(v >> (bw * 2 * j)) & mask;
+                    const uint32_t c1 = (uint32_t)(v >> (bw * (2 * j + 1))) & mask;
+                    const uint32_t m = ((c0 | (c1 << 16)) << (5 - bw)) | 0x43004300u;
+                    const uint32_t d = bf16x2_fma(m, 0x3F803F80u, 0xC310C310u);    // idx_5 - 16
+                    o[j] = bf16x2_fma(d, s16x2, 0x80008000u);
+                }
+            } else {
+                const float s16 = bf16_bits_to_float(sb) * 0.0625f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i0 = (int)(((uint32_t)(v >> (bw * 2 * j)) & mask) << (5 - bw));
+                    const int i1 = (int)(((uint32_t)(v >> (bw * (2 * j + 1))) & mask) << (5 - bw));
+                    o[j] = pack_bf16x2(s16 * (float)(i0 - 16), s16 * (float)(i1 - 16));
+                }
             }
         }
         stg_cs_v4(out + gid, make_uint4(o[0], o[1], o[2], o[3]));
