@@ -84,3 +84,25 @@ def test_lloyd_rows_apply_the_sign_bit():
     expect = oracle.bf16_to_f64(workloads.f64_to_bf16_bits(expect))   # fp32 -> bf16 RNE
     assert np.array_equal(wd[0, :16], expect)
     assert np.signbit(wd[0, 8])                                       # -0.0 for level 0, sign 1
+
+
+def test_codebook_formats_match_numpy_matmul_on_their_dequant():
+    # LUT16 (fp16 centroids, blocks of 64) and LLOYD8S (signed fp32 levels, groups of 32):
+    # the product equals x Wdeq^T with Wdeq from the separately pinned dequant
+    g = np.random.default_rng(21)
+    n, k = 40, 256
+    x = workloads.activations(3, k, workloads.LUT16, 2)
+    xd = oracle.bf16_to_f64(x)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    packed = oracle.pack(codes)
+    lut = oracle.f64_to_fp16(np.sort(g.standard_normal((n, k // 64, 16)), -1) * 0.01)
+    levels = np.sort(np.abs(g.standard_normal((n, k // 32, 8))) * 0.02, -1).astype(np.float32)
+    for fmt, aux, grp, decode in [(oracle.LUT16, lut, 64, oracle.fp16_to_f64),
+                                  (oracle.LLOYD8S, levels, 32, oracle.bf16_to_f64)]:
+        wd = decode(oracle.dequant(fmt, packed, aux, grp))
+        y, bound = oracle.matmul_rows(fmt, packed, aux, grp, x)
+        assert np.allclose(y, xd @ wd.T, rtol=0, atol=1e-13 * np.abs(xd).sum() * np.abs(wd).max())
+        assert np.allclose(bound, np.abs(xd) @ np.abs(wd).T, rtol=1e-13)
+        rows = np.array([n - 1, 3, 3], np.int64)
+        ys, _ = oracle.matmul_rows(fmt, packed, aux, grp, x, rows=rows)
+        assert np.array_equal(ys, y[:, rows])
