@@ -572,6 +572,26 @@ def bench_gemm(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks):
             del g
     except Exception as e:
         res["lloyd8s"] = {"error": repr(e)[:200]}
+    # the LUT16 consumer on the same GEMM (fp16 centroids, fp16 MMA; the timed region includes
+    # the activations' bf16 -> fp16 conversion into the workspace)
+    try:
+        n, k = workloads.PREFILL_SHAPES[0]
+        gen = torch.Generator(device=dev).manual_seed(6)
+        codes = torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=dev, generator=gen)
+        lut = torch.sort(torch.randn((n, k // 64, 16), device=dev, generator=gen) * 0.01, dim=-1).values
+        pu = wq.PackedWeight(wq.FMT_LUT16, 64, n, k, codes, lut.to(torch.float16).contiguous())
+        for m in (512, 4096):
+            x = torch.randn((m, k), device=dev).to(torch.bfloat16)
+            y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(max(wq.gemm_workspace_bytes(pu, m), 16), dtype=torch.uint8, device=dev)
+            g = graph_of(torch, lambda: wq.gemm(pu, x, out=y, workspace=ws))
+            ms = max_over_ranks(time_region(torch, stream, g.replay, steps, warm, barrier))
+            fl = 2.0 * m * n * k
+            res[f"lut16_{n}x{k}_m{m}"] = {"TFLOP/s": round(fl / ms / 1e9, 1), "us": round(ms * 1e3, 2),
+                                          "frac_fp16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
+            del g
+    except Exception as e:
+        res["lut16"] = {"error": repr(e)[:200]}
     return res
 
 

@@ -257,13 +257,17 @@ size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
 
 /* Prefill-side W4A16 GEMM on the tcgen05 tensor cores ([KM] §4.1 large batch; [DG] §3.2
  * "materialized" bf16 path fused): y[i, r] = sum_c Wdeq[r, c] * x[i, c] for i < m, fp32
- * accumulation in tensor memory, bf16 output. Formats DYADIC4 (group 64 or 32) and LLOYD8S
- * (the 8-level codebook plus sign of [G32] §5.2, rebuilt per stage from the group's levels). For
- * m <= 12 the decode-shaped case runs on the GEMV kernel of wq_gemv_w4a16 (the kernel
- * choice by batch size of [KM] §4.1), with the same tolerance and no workspace.
+ * accumulation in tensor memory, bf16 output. Formats DYADIC4 (group 64 or 32), LLOYD8S
+ * (the 8-level codebook plus sign of [G32] §5.2, rebuilt per stage from the group's levels)
+ * and LUT16 (the per-block-64 centroid table of [KM] §2.2, looked up per stage; the product
+ * runs in fp16 with the activations converted bf16 -> fp16 into the workspace, exact for
+ * |x| in [2^-14, 65504] as in wq_gemv_w4a16). For m <= 12 the decode-shaped case runs on the
+ * GEMV kernel of wq_gemv_w4a16 (the kernel choice by batch size of [KM] §4.1), with the same
+ * tolerance and no workspace.
  *   x      bf16 [m, k]; m >= 1; k % 64 == 0.
  *   y      out bf16 [m, n].
- *   ws     device workspace of at least wq_gemm_workspace_bytes(w, m) bytes (NULL if 0).
+ *   ws     device workspace of at least wq_gemm_workspace_bytes(w, m) bytes (NULL if 0);
+ *          for LUT16 it includes 2*m*k bytes for the fp16 activations.
  * Same tolerance as wq_gemv_w4a16. */
 wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y,
                         void* ws, size_t ws_bytes, wq_stream stream);

@@ -172,3 +172,61 @@ def test_gemm_last_wave_split(wq):
     assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
     # the same through the static-scratch entry point (the tail's scratch stays within it)
     assert wq.gemm_workspace_bytes(pw, m) <= (16 << 20)
+
+
+def _lut16(wq, n, k, seed):
+    g = np.random.default_rng(seed)
+    codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+    lut = oracle.f64_to_fp16(np.sort(g.standard_normal((n, k // 64, 16)), -1) * 0.01)
+    packed = oracle.pack(codes)
+    pw = wq.PackedWeight(wq.FMT_LUT16, 64, n, k, to_dev(packed), to_dev_bits(lut, torch.float16))
+    return pw, packed, lut
+
+
+@pytest.mark.parametrize("m", [1, 12, 13, 16, 48, 128, 200, 256, 300])
+@pytest.mark.parametrize("n,k", [(128, 256), (200, 320), (256, 1024)])
+def test_gemm_lut16_matches_oracle(wq, m, n, k):
+    """The LUT16 consumer on the tensor-memory GEMM ("K-Means量化技术…" §2.2, the large-batch
+    branch of §4.1): each stage's 16-entry fp16 tables arrive by TMA and the codes are looked
+    up in them; the MMA runs in fp16 on activations converted from bf16."""
+    pw, packed, lut = _lut16(wq, n, k, m * 5 + n + k)
+    x_bits = workloads.activations(m, k, workloads.PREFILL, n + 2 * m)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul_rows(oracle.LUT16, packed, lut, 64, x_bits)
+    _check(y, y_ref, bound)
+    assert wq.device_error() == 0
+
+
+def test_gemm_lut16_one_hot_exact(wq):
+    """x = e_c gives bf16 of the fp16 centroid each row's code at column c selects."""
+    n, k = 256, 512
+    pw, packed, lut = _lut16(wq, n, k, 23)
+    wd = oracle.fp16_to_f64(oracle.dequant(oracle.LUT16, packed, lut, 64))
+    cols = np.arange(1, k, 3)
+    x = np.zeros((len(cols), k))
+    x[np.arange(len(cols)), cols] = 1.0
+    y = wq.gemm(pw, to_dev_bits(workloads.f64_to_bf16_bits(x)))
+    want = workloads.f64_to_bf16_bits(wd[:, cols].T)
+    assert np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+@pytest.mark.parametrize("m,n,k", [(48, 1024, 8192), (256, None, 4096)])
+def test_gemm_lut16_workspace_paths(wq, m, n, k):
+    """Split-K (small m) and the last-wave split (whole waves plus a short tail): the fp32
+    partial sums sit in the workspace after the fp16 activations; sampled rows against the
+    oracle."""
+    if n is None:
+        n = 128 * (torch.cuda.get_device_properties(0).multi_processor_count + 10)
+    pw, packed, lut = _lut16(wq, n, k, m + 41)
+    need = wq.gemm_workspace_bytes(pw, m)
+    assert need > 2 * m * k                                 # activations + partial sums
+    x_bits = workloads.activations(m, k, workloads.PREFILL, m + 41)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+    rows = np.concatenate([np.arange(0, n, 97), [n - 1]])
+    ms = np.arange(0, m, 5)
+    y_ref, bound = oracle.matmul_rows(oracle.LUT16, packed, lut, 64, x_bits[ms], rows=rows)
+    got = f32(y)[np.ix_(ms, rows)]
+    assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))

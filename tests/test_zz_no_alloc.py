@@ -15,12 +15,23 @@ from _util import f32, matmul_tolerance, to_dev, to_dev_bits
 pytestmark = pytest.mark.gpu
 
 
-def test_static_scratch_gemm_matches_workspace_gemm(wq):
+@pytest.mark.parametrize("fmt", ["dyadic", "lut16"])
+def test_static_scratch_gemm_matches_workspace_gemm(wq, fmt):
+    """LUT16 also keeps its fp16 copy of the activations in the scratch."""
     n, k, m = 1024, 8192, 48                  # small m: K is split, so the scratch is used
-    w_bits = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 21)
-    s, c = oracle.dyadic_quantize(w_bits, 64)
+    if fmt == "dyadic":
+        w_bits = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 21)
+        s, c = oracle.dyadic_quantize(w_bits, 64)
+        code, aux = oracle.DYADIC4, s
+    else:
+        g = np.random.default_rng(21)
+        c = g.integers(0, 16, (n, k), dtype=np.uint8)
+        code, aux = oracle.LUT16, oracle.f64_to_fp16(np.sort(g.standard_normal((n, k // 64, 16)), -1) * 0.01)
     packed = oracle.pack(c)
-    pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(packed), to_dev_bits(s))
+    if fmt == "dyadic":
+        pw = wq.PackedWeight(wq.FMT_DYADIC4, 64, n, k, to_dev(packed), to_dev_bits(aux))
+    else:
+        pw = wq.PackedWeight(wq.FMT_LUT16, 64, n, k, to_dev(packed), to_dev_bits(aux, torch.float16))
     d = pw.desc()
     need = wq.gemm_workspace_bytes(pw, m)
     assert 0 < need <= (16 << 20)
@@ -40,7 +51,7 @@ def test_static_scratch_gemm_matches_workspace_gemm(wq):
                                    need, stream)
         assert st == wq.WQ_OK, wq.last_error()
         torch.cuda.synchronize()
-        _, bound = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x_bits, rows=rows)
+        _, bound = oracle.matmul_rows(code, packed, aux, 64, x_bits, rows=rows)
         a, b = f32(y_static)[:, rows], f32(y_ws)[:, rows]
         assert np.all(np.abs(a - b) <= matmul_tolerance(b, bound))
         assert wq.device_error() == 0

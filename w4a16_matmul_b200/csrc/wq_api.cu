@@ -463,8 +463,6 @@ wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16
     g_last_error[0] = 0;
     wq_status st = check_weight(w);
     if (st) return st;
-    if (w->fmt != WQ_FMT_DYADIC4 && w->fmt != WQ_FMT_LLOYD8S)
-        return fail(WQ_EUNSUPPORTED, "GEMM supports DYADIC4 and LLOYD8S weights (got format %d)", w->fmt);
     if (w->k % 64 != 0) return fail(WQ_EINVAL, "GEMM needs k %% 64 == 0 (k=%lld)", (long long)w->k);
     if (m < 1 || m > (1LL << 31) - 1) return fail(WQ_EINVAL, "m=%lld outside 1..2^31-1", (long long)m);
     if ((st = check_ptr(x, "x", false))) return st;

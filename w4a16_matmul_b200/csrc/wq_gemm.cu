@@ -21,12 +21,18 @@
 // alone: no bf16 tile is written to and read back from shared memory, whose bandwidth the
 // MMA's activation reads and the TMA writes already share, and the freed space holds six
 // pipeline stages.
+// The LLOYD8S and LUT16 formats run in the same pipeline: their per-group tables (8 fp32
+// levels per 32 columns, 16 fp16 centroids per 64) arrive by TMA with each stage and the
+// reconstruction warps look the codes up in them. LUT16 runs an fp16 MMA, so that its
+// centroids enter the product unrounded: its activations are converted to fp16 once, into
+// the workspace, by a small kernel ahead of the GEMM.
 // Every wait on an mbarrier is bounded; a wait that expires records an error word on the
 // device (see wq_device_error) and the CTA skips the rest of its work, still releasing its
 // tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "wq_internal.cuh"
@@ -152,11 +158,17 @@ __device__ __forceinline__ uint4 dyadic_row8_f32(uint32_t w, float step) {
 // as 216 KB hold, up to 16. Tensor-memory slots (32 columns each, the reconstructed
 // weights of one stage) only need to cover reconstruction-to-MMA latency; for BN <= 64 the
 // allocation stays at 256 columns so that two CTAs can share an SM.
-template <int BN, bool LL = false, int KB = 64>
+// Weight formats of the kernel (template parameter F): the dyadic step, the LLOYD8S levels
+// or the LUT16 table.
+constexpr int kFDy = 0, kFLl = 1, kFLu = 2;
+
+template <int BN, int F = kFDy, int KB = 64>
 struct Smem {
     static constexpr int B_BYTES = BN * KB * 2;          // KB/64 activation tiles (128-byte swizzle)
     static constexpr int P_BYTES = BM * KB / 2;          // packed weight tile
-    static constexpr int L_BYTES = LL ? BM * KB : 0;     // LLOYD8S: the stage's groups' fp32 levels
+    // the stage's per-group tables: LLOYD8S 8 fp32 levels per 32 columns, LUT16 16 fp16
+    // centroids per 64 columns
+    static constexpr int L_BYTES = F == kFLl ? BM * KB : F == kFLu ? BM * KB / 2 : 0;
     static constexpr int STAGE = B_BYTES + P_BYTES + L_BYTES;   // a multiple of 1024
     static constexpr int STAGES = (216 * 1024 / STAGE) < 16 ? (216 * 1024 / STAGE) : 16;
     static constexpr int BARS = 2 * STAGES + 2 * 8 + 1;
@@ -235,14 +247,17 @@ __device__ __forceinline__ void tmem_st_part(uint32_t taddr, const uint32_t* v) 
     }
 }
 
-// LL: LLOYD8S weights (groups of 32, 8 fp32 levels each, loaded per stage by TMA through
-// tmap_l; `scale` unused); otherwise DYADIC4 with group G.
-template <int BN, int G, bool PARTIAL, bool LL, int KB>
+// F == kFLl: LLOYD8S weights (groups of 32, 8 fp32 levels each, loaded per stage by TMA
+// through tmap_l; `scale` unused). F == kFLu: LUT16 weights (groups of 64, 16 fp16 centroids
+// each, loaded the same way), with fp16 activations and an fp16 MMA. Otherwise DYADIC4 with
+// group G.
+template <int BN, int G, bool PARTIAL, int F, int KB>
 __global__ void __launch_bounds__(threads_for(BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
             const __grid_constant__ CUtensorMap tmap_l, const uint16_t* __restrict__ scale,
             void* __restrict__ out, int M, int N, int K, int kt_per_split, int grid_n, int tile0) {
-    using S = Smem<BN, LL, KB>;
+    using S = Smem<BN, F, KB>;
+    constexpr bool LL = F == kFLl, LU = F == kFLu;
     constexpr int STAGES = S::STAGES;
     constexpr int RW = rw_for(BN);
     extern __shared__ uint8_t smem_raw[];
@@ -311,14 +326,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 for (int j = 0; j < KB / 64; ++j)
                     tma_load_2d(stage_b(s) + j * BN * 128, &tmap_x, kt * KB + 64 * j, m0, &full_tma[s]);
                 tma_load_2d(stage_p(s), &tmap_p, kt * (KB / 2), n0, &full_tma[s]);
-                if (LL) tma_load_2d(stage_l(s), &tmap_l, kt * (KB / 4), n0, &full_tma[s]);
+                // both tables hold KB / 4 elements of a row per stage
+                if (F != kFDy) tma_load_2d(stage_l(s), &tmap_l, kt * (KB / 4), n0, &full_tma[s]);
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer: A (weights) from tensor memory, B from shared ------
         if (lane == 0) {
-            constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                                       ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+            // fp32 accumulator; A and B both bf16 (format 1), or both fp16 (format 0) for LUT16
+            constexpr uint32_t ab = LU ? 0u : (1u << 7) | (1u << 10);
+            constexpr uint32_t idesc = (1u << 4) | ab | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
             int s = 0, a = 0;
             uint32_t aph = 0;
             for (int i = 0; i < nk; ++i) {
@@ -348,8 +365,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         // colbase .. colbase + 8 WPT - 1 of the stage
         constexpr int WPT = (KB / 8) / RW;
         // a thread's columns span one group, or two g32 groups (then aligned to them)
-        constexpr bool SPAN2 = !LL && WPT * 8 > G;
-        static_assert(WPT * 8 <= 2 * G || LL, "at most two scale groups per thread and stage");
+        constexpr bool SPAN2 = F == kFDy && WPT * 8 > G;
+        static_assert(WPT * 8 <= 2 * G || F != kFDy, "at most two scale groups per thread and stage");
+        static_assert(!LU || WPT * 8 <= 64, "a thread's LUT16 columns lie in one group of 64");
         const int q = warp & 3, part = (warp - 2) >> 2;
         const int colbase = part * WPT * 8;
         const int i = 32 * q + lane;
@@ -363,7 +381,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 #pragma unroll
         for (int u = 0; u < kPre; ++u) {
             ring0[u] = ring1[u] = 0;
-            if (!LL && row_ok && u < nk) {
+            if (F == kFDy && row_ok && u < nk) {
                 ring0[u] = ldg_u16(srow + (kt0 + u) * (KB / G));
                 ring1[u] = SPAN2 ? ldg_u16(srow + (kt0 + u) * (KB / G) + 1) : ring0[u];
             }
@@ -377,7 +395,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 const int it = base + u;
                 if (it >= nk) break;
                 const uint32_t sc0 = ring0[u], sc1 = ring1[u];
-                if (!LL && row_ok && it + kPre < nk) {
+                if (F == kFDy && row_ok && it + kPre < nk) {
                     ring0[u] = ldg_u16(srow + (kt0 + it + kPre) * (KB / G));
                     ring1[u] = SPAN2 ? ldg_u16(srow + (kt0 + it + kPre) * (KB / G) + 1) : ring0[u];
                 }
@@ -426,6 +444,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                         const int gi = c >> 2;
                         lloyd8_lookup4(wv[c], plo[gi], phi[gi], v[4 * c], v[4 * c + 1]);
                         lloyd8_lookup4(wv[c] >> 16, plo[gi], phi[gi], v[4 * c + 2], v[4 * c + 3]);
+                    }
+                } else if constexpr (LU) {
+                    // the 16 fp16 centroids of the group this thread's words lie in, as byte
+                    // planes (lo / hi[q]: low / high bytes of entries 4q .. 4q + 3), then the
+                    // same lookup as the GEMV's: the centroids enter the product unrounded
+                    const uint4* tv = (const uint4*)(stage_l(s) + i * (KB / 2) + (colbase / 64) * 32);
+                    const uint4 t0 = tv[0], t1 = tv[1];
+                    const uint32_t lo[4] = {prmt(t0.x, t0.y, 0x6420u), prmt(t0.z, t0.w, 0x6420u),
+                                            prmt(t1.x, t1.y, 0x6420u), prmt(t1.z, t1.w, 0x6420u)};
+                    const uint32_t hi[4] = {prmt(t0.x, t0.y, 0x7531u), prmt(t0.z, t0.w, 0x7531u),
+                                            prmt(t1.x, t1.y, 0x7531u), prmt(t1.z, t1.w, 0x7531u)};
+#pragma unroll
+                    for (int c = 0; c < WPT; ++c) {
+                        lut16_lookup4(wv[c], lo, hi, v[4 * c], v[4 * c + 1]);
+                        lut16_lookup4(wv[c] >> 16, lo, hi, v[4 * c + 2], v[4 * c + 3]);
                     }
                 } else {
                     const bool huge = ((sc0 & 0x7FFFu) >= 0x7D80u) || ((sc1 & 0x7FFFu) >= 0x7D80u);
@@ -520,6 +553,17 @@ splitk_reduce_kernel(const float* __restrict__ part, int splits, int ntl, int ti
 #pragma unroll 4
     for (int sp = 0; sp < splits; ++sp) v += __ldg(src + sp * plane);
     y[(size_t)m * N + n] = (uint16_t)float_to_bf16_bits(v);
+}
+
+// Activations for the LUT16 product: bf16 -> fp16, 8 per thread and iteration (exact for |x|
+// in [2^-14, 65504], as the GEMV's staging of LUT16 activations). n8 = elements / 8.
+__global__ void __launch_bounds__(256)
+x_to_f16_kernel(const uint4* __restrict__ x, uint4* __restrict__ xh, int64_t n8) {
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (int64_t)gridDim.x * 256) {
+        const uint4 v = ldg_nc_v4(x + i);
+        xh[i] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                           bf16x2_to_f16x2(v.w));
+    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -629,22 +673,22 @@ Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt) {
 
 // One launch over tiles [tile0, tile0 + ntl) with K split `splits` ways (partial sums to
 // `out` in the [split][tile][BN][BM] layout when partial, bf16 y otherwise).
-template <int BN, int G, bool LL, int KB>
+template <int BN, int G, int F, int KB>
 wq_status launch_bn(const Plan& p, bool partial, int tile0, int ntl, int splits, int kt_per_split,
                     const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMap& tl,
                     const uint16_t* scale, void* out, int M, int N, int K, cudaStream_t s) {
-    const int smem = Smem<BN, LL, KB>::TOTAL;
+    const int smem = Smem<BN, F, KB>::TOTAL;
     const dim3 grid(ntl, splits, 1);
     // the shared-memory opt-in is set once per kernel variant (a function attribute holds
     // for the process; the flags are per variant and only ever go from false to true)
     static bool raised[2] = {false, false};
     if (partial) {
-        auto k = gemm_kernel<BN, G, true, LL, KB>;
+        auto k = gemm_kernel<BN, G, true, F, KB>;
         if (!raised[1] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[1] = true;
         k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, kt_per_split, p.grid_n, tile0);
     } else {
-        auto k = gemm_kernel<BN, G, false, LL, KB>;
+        auto k = gemm_kernel<BN, G, false, F, KB>;
         if (!raised[0] && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess)
             raised[0] = true;
         k<<<grid, threads_for(BN), smem, s>>>(tx, tp, tl, scale, out, M, N, K, kt_per_split, p.grid_n, tile0);
@@ -654,7 +698,7 @@ wq_status launch_bn(const Plan& p, bool partial, int tile0, int ntl, int splits,
 
 // The plan's launches: one (unsplit, or split everywhere) or two (whole waves unsplit, then
 // the split tail), each split launch followed by its reduction.
-template <int BN, int G, bool LL, int KB>
+template <int BN, int G, int F, int KB>
 wq_status launch_plan(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tp, const CUtensorMap& tl,
                       const uint16_t* scale, uint16_t* y, void* ws, int M, int N, int K, cudaStream_t s) {
     const int tiles = p.grid_n * p.grid_m;
@@ -664,14 +708,14 @@ wq_status launch_plan(const Plan& p, const CUtensorMap& tx, const CUtensorMap& t
     };
     wq_status st;
     if (p.splits > 1) {
-        if ((st = launch_bn<BN, G, LL, KB>(p, true, 0, tiles, p.splits, p.kt_per_split, tx, tp, tl, scale, ws, M, N,
+        if ((st = launch_bn<BN, G, F, KB>(p, true, 0, tiles, p.splits, p.kt_per_split, tx, tp, tl, scale, ws, M, N,
                                            K, s)))
             return st;
         return reduce(p.splits, 0, tiles);
     }
-    if ((st = launch_bn<BN, G, LL, KB>(p, false, 0, p.full, 1, K / KB, tx, tp, tl, scale, y, M, N, K, s))) return st;
+    if ((st = launch_bn<BN, G, F, KB>(p, false, 0, p.full, 1, K / KB, tx, tp, tl, scale, y, M, N, K, s))) return st;
     if (p.full == tiles) return WQ_OK;
-    if ((st = launch_bn<BN, G, LL, KB>(p, true, p.full, tiles - p.full, p.tail_splits, p.tail_kt_per_split, tx, tp,
+    if ((st = launch_bn<BN, G, F, KB>(p, true, p.full, tiles - p.full, p.tail_splits, p.tail_kt_per_split, tx, tp,
                                        tl, scale, ws, M, N, K, s)))
         return st;
     return reduce(p.tail_splits, p.full, tiles - p.full);
@@ -688,14 +732,22 @@ wq_status launch_plan(const Plan& p, const CUtensorMap& tx, const CUtensorMap& t
 // "K-Means量化技术…" §4.1.
 constexpr int64_t kGemvMaxRows = 12;
 
+// Workspace layout: for LUT16 the fp16 copy of the activations [m, k] first (rounded up to
+// 1 KB), then the fp32 partial sums of split launches.
+size_t lut16_x_bytes(const wq_weight& w, int64_t m) {
+    if (w.fmt != WQ_FMT_LUT16) return 0;
+    return ((size_t)m * (size_t)w.k * 2 + 1023) & ~(size_t)1023;
+}
+
 size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
     if (m <= kGemvMaxRows) return 0;
     const Plan p = plan_for(m, w.n, w.k, w.fmt);
     const size_t tile = (size_t)BM * (size_t)p.bn * sizeof(float);
     const size_t tiles = (size_t)p.grid_n * (size_t)p.grid_m;
-    if (p.splits > 1) return (size_t)p.splits * tiles * tile;
-    if (p.full < (int)tiles) return (size_t)p.tail_splits * (tiles - (size_t)p.full) * tile;
-    return 0;
+    size_t partial = 0;
+    if (p.splits > 1) partial = (size_t)p.splits * tiles * tile;
+    else if (p.full < (int)tiles) partial = (size_t)p.tail_splits * (tiles - (size_t)p.full) * tile;
+    return lut16_x_bytes(w, m) + partial;
 }
 
 wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
@@ -708,13 +760,27 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
     const Plan p = plan_for(M, N, K, w.fmt);
     auto enc = encode_fn();
     if (!enc) return fail(WQ_ECUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    const size_t need = gemm_workspace_bytes(w, m);
+    if (need > 0 && (ws == nullptr || ws_bytes < need)) return fail(WQ_EINVAL, "workspace too small");
+    const bool lut = w.fmt == WQ_FMT_LUT16;
+    const void* xa = x;                    // the activations the MMA reads
+    if (lut) {
+        const int64_t n8 = m * (int64_t)K / 8;
+        const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, 8 * (int64_t)sm_count());
+        x_to_f16_kernel<<<(unsigned)blocks, 256, 0, s>>>((const uint4*)x, (uint4*)ws, n8);
+        wq_status cs = check_launch("gemm activations to fp16");
+        if (cs) return cs;
+        xa = ws;
+        ws = (uint8_t*)ws + lut16_x_bytes(w, m);
+    }
     CUtensorMap tx, tp;
     {
         cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
         cuuint64_t strides[1] = {(cuuint64_t)K * 2};
         cuuint32_t box[2] = {64, (cuuint32_t)p.bn};        // one 128-byte swizzle row wide
         cuuint32_t es[2] = {1, 1};
-        CUresult r = enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)x, dims, strides, box, es,
+        CUresult r = enc(&tx, lut ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                         (void*)xa, dims, strides, box, es,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(WQ_ECUDA, "tensor map for x failed (%d)", (int)r);
@@ -730,7 +796,18 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
         if (r != CUDA_SUCCESS) return fail(WQ_ECUDA, "tensor map for packed weights failed (%d)", (int)r);
     }
     CUtensorMap tl = tp;                   // unused by DYADIC4 launches
-    if (w.fmt == WQ_FMT_LLOYD8S) {
+    if (lut) {
+        // centroids [N, K/64, 16] fp16 as a 2D [N, K/4] array; a stage's KB/64 groups are
+        // KB/4 entries
+        cuuint64_t dims[2] = {(cuuint64_t)K / 4, (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+        cuuint32_t box[2] = {(cuuint32_t)(p.kb / 4), (cuuint32_t)BM};
+        cuuint32_t es[2] = {1, 1};
+        CUresult r = enc(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)w.aux, dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(WQ_ECUDA, "tensor map for LUT16 centroids failed (%d)", (int)r);
+    } else if (w.fmt == WQ_FMT_LLOYD8S) {
         // levels [N, K/32, 8] fp32 as a 2D [N, K/4] array; a stage's 2 groups are 16 floats
         cuuint64_t dims[2] = {(cuuint64_t)K / 4, (cuuint64_t)N};
         cuuint64_t strides[1] = {(cuuint64_t)K};
@@ -741,14 +818,13 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(WQ_ECUDA, "tensor map for LLOYD8S levels failed (%d)", (int)r);
     }
-    const size_t need = gemm_workspace_bytes(w, m);
-    if (need > 0 && (ws == nullptr || ws_bytes < need)) return fail(WQ_EINVAL, "workspace too small");
     const uint16_t* sc = (const uint16_t*)w.aux;
     wq_status st;
-#define WQ_BN(BNV, KBV)                                                                                  \
-    st = (w.fmt == WQ_FMT_LLOYD8S) ? launch_plan<BNV, 32, true, 64>(p, tx, tp, tl, sc, y, ws, M, N, K, s) \
-       : (w.group == 64) ? launch_plan<BNV, 64, false, KBV>(p, tx, tp, tl, sc, y, ws, M, N, K, s)         \
-                         : launch_plan<BNV, 32, false, KBV>(p, tx, tp, tl, sc, y, ws, M, N, K, s)
+#define WQ_BN(BNV, KBV)                                                                                   \
+    st = (w.fmt == WQ_FMT_LLOYD8S) ? launch_plan<BNV, 32, kFLl, 64>(p, tx, tp, tl, sc, y, ws, M, N, K, s) \
+       : lut                     ? launch_plan<BNV, 64, kFLu, KBV>(p, tx, tp, tl, sc, y, ws, M, N, K, s)  \
+       : (w.group == 64)         ? launch_plan<BNV, 64, kFDy, KBV>(p, tx, tp, tl, sc, y, ws, M, N, K, s)  \
+                                 : launch_plan<BNV, 32, kFDy, KBV>(p, tx, tp, tl, sc, y, ws, M, N, K, s)
     switch (p.bn) {
         case 16: WQ_BN(16, 64); break;
         case 32: WQ_BN(32, 64); break;

@@ -110,29 +110,6 @@ __device__ __forceinline__ void dyadic_pairs_scaled(uint32_t w, uint32_t c1, uin
     p[3] = bf16x2_fma(t & 0x00F000F0u, c2, d);
 }
 
-// LUT16 lookup of 4 codes (nibbles of the low 16 bits of s) in a 16-entry fp16 table held
-// as byte planes: lo[q] / hi[q] hold the low / high bytes of entries 4q..4q+3. Returns the
-// fp16 pairs (code0, code1) and (code2, code3).
-// The byte mask (0xFF where code >= 8) comes from prmt's sign-replicate selector mode: the
-// codes' bit 3 is the top bit of a byte of s (codes 1, 3) or of s << 4 (codes 0, 2).
-__device__ __forceinline__ void lut16_lookup4(uint32_t s, const uint32_t* lo, const uint32_t* hi,
-                                              uint32_t& p01, uint32_t& p23) {
-    const uint32_t s7 = s & 0x7777u;                                  // index within 8 entries
-    const uint32_t m = prmt(s, s << 4, 0x9D8Cu);                      // byte mask: code >= 8
-    const uint32_t l = (prmt(lo[0], lo[1], s7) & ~m) | (prmt(lo[2], lo[3], s7) & m);
-    const uint32_t h = (prmt(hi[0], hi[1], s7) & ~m) | (prmt(hi[2], hi[3], s7) & m);
-    p01 = prmt(l, h, 0x5140u);
-    p23 = prmt(l, h, 0x7362u);
-}
-
-// bf16x2 -> fp16x2 (round to nearest even; exact for |x| in [2^-14, 65504]).
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
-    const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
 enum Kind { kDyadic64 = 0, kDyadic32 = 1, kLut16 = 2, kLloyd8 = 3 };
 
 // Per-lane state of one 256-column step for R 16-row blocks: the 32 bytes of rows g and

@@ -196,6 +196,29 @@ __device__ __forceinline__ void lloyd8_lookup4(uint32_t s, const uint32_t* lo, c
     p23 = prmt(l, h, 0x7362u);
 }
 
+// LUT16 lookup of 4 codes (nibbles of the low 16 bits of s) in a 16-entry fp16 table held
+// as byte planes: lo[q] / hi[q] hold the low / high bytes of entries 4q..4q+3. Returns the
+// fp16 pairs (code0, code1) and (code2, code3).
+// The byte mask (0xFF where code >= 8) comes from prmt's sign-replicate selector mode: the
+// codes' bit 3 is the top bit of a byte of s (codes 1, 3) or of s << 4 (codes 0, 2).
+__device__ __forceinline__ void lut16_lookup4(uint32_t s, const uint32_t* lo, const uint32_t* hi,
+                                              uint32_t& p01, uint32_t& p23) {
+    const uint32_t s7 = s & 0x7777u;                                  // index within 8 entries
+    const uint32_t m = prmt(s, s << 4, 0x9D8Cu);                      // byte mask: code >= 8
+    const uint32_t l = (prmt(lo[0], lo[1], s7) & ~m) | (prmt(lo[2], lo[3], s7) & m);
+    const uint32_t h = (prmt(hi[0], hi[1], s7) & ~m) | (prmt(hi[2], hi[3], s7) & m);
+    p01 = prmt(l, h, 0x5140u);
+    p23 = prmt(l, h, 0x7362u);
+}
+
+// bf16x2 -> fp16x2 (round to nearest even; exact for |x| in [2^-14, 65504]).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+    const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // D += A * B on the legacy warp-level tensor-core path, m16n8k16, bf16 in, fp32 accumulate.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
