@@ -739,7 +739,8 @@ def run_reference(args):
 
 def run_profile_target(args):
     """A few launches of one kernel on one shape and nothing else, for ncu captures:
-    --profile gemm --shape N,K,M (prefill GEMM), quantize --shape N,K, dequant --shape N,K,
+    --profile gemm --shape N,K,M (prefill GEMM; gemm_lut16: its LUT16 form, with the
+    activation conversion), quantize --shape N,K, dequant --shape N,K,
     lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd), gumbel --shape N,K
     (Gumbel-ST backward at tau = step^2; gumbel1: at tau = 1.0), ste --shape N,K (STE forward),
     bf16x --shape N,K (BF16X encode + decode), wf --shape N,K
@@ -762,6 +763,14 @@ def run_profile_target(args):
         y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
         ws = torch.empty(max(16, wq.gemm_workspace_bytes(pw, m)), dtype=torch.uint8, device=dev)
         fn = lambda: wq.gemm(pw, x, out=y, workspace=ws)
+    elif args.profile == "gemm_lut16":
+        m = dims[2]
+        lut = (torch.randn((n, k // 64, 16), device=dev, generator=gen) * 0.01).to(torch.float16)
+        pl = wq.PackedWeight(wq.FMT_LUT16, 64, n, k, packed, lut)
+        x = torch.randn((m, k), device=dev, generator=gen).to(torch.bfloat16)
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, wq.gemm_workspace_bytes(pl, m)), dtype=torch.uint8, device=dev)
+        fn = lambda: wq.gemm(pl, x, out=y, workspace=ws)
     elif args.profile == "quantize":
         w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
         fn = lambda: wq.quantize_dyadic(w, 64)
