@@ -509,7 +509,19 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
                                       "quantize_Gweights/s": round(nw / ms_q / 1e6, 2),
                                       "dequant_us": round(ms_dq * 1e3, 1), "dequant_GB/s": round(dq_b / ms_dq / 1e6, 1),
                                       "dequant_frac_hbm": round(dq_b / ms_dq / 1e6 / peaks["hbm_gbs"], 4)}
-        del gq_, gdw, sc, wd, off, pk, dwf, wb
+        # the format's GEMV (weights rebuilt as the dequant does, fp32 products), batch 1 / 16
+        qwf = wq.WfWeight(n_l, k_l, sc, wd, off, pk, total)
+        for b in (1, 16):
+            xw = torch.randn((b, k_l), device=dev).to(torch.bfloat16)
+            yw = torch.empty((b, n_l), dtype=torch.bfloat16, device=dev)
+            gg = graph_of(torch, lambda: wq.gemv_wf(qwf, xw, out=yw))
+            ms_g = max_over_ranks(time_region(torch, stream, gg.replay, steps, warm, barrier))
+            g_b = total + side + 2 * b * (k_l + n_l)
+            out["water_filling_large"][f"gemv_b{b}"] = {
+                "us": round(ms_g * 1e3, 1), "GB/s": round(g_b / ms_g / 1e6, 1),
+                "frac_hbm": round(g_b / ms_g / 1e6 / peaks["hbm_gbs"], 4)}
+            del gg
+        del gq_, gdw, sc, wd, off, pk, dwf, wb, qwf
     except Exception as e:
         out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
     if args.extras in ("gemm", "all"):
@@ -744,7 +756,7 @@ def run_profile_target(args):
     lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd), gumbel --shape N,K
     (Gumbel-ST backward at tau = step^2; gumbel1: at tau = 1.0), ste --shape N,K (STE forward),
     bf16x --shape N,K (BF16X encode + decode), wf --shape N,K
-    (water-filling analyze + dequant). Random packed codes and
+    (water-filling analyze + dequant), wf_gemv --shape N,K,B (its GEMV). Random packed codes and
     scales (timing does not depend on the values); inputs stay on the device."""
     import torch
     import __graft_entry__
@@ -809,6 +821,14 @@ def run_profile_target(args):
         q = wq.quantize_wf(w, 1e-6)
         out = torch.empty_like(w)
         fn = lambda: (wq.wf_analyze(w, 1e-6), wq.dequant_wf(q, out=out))
+    elif args.profile == "wf_gemv":
+        b = dims[2]
+        w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+        q = wq.quantize_wf(w, 1e-6)
+        del w
+        x = torch.randn((b, k), device=dev, generator=gen).to(torch.bfloat16)
+        y = torch.empty((b, n), dtype=torch.bfloat16, device=dev)
+        fn = lambda: wq.gemv_wf(q, x, out=y)
     elif args.profile == "lloyd":
         w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
         fn = lambda: wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)

@@ -361,6 +361,19 @@ wq_status wq_dequant_wf(const uint8_t* packed, int64_t packed_bytes, const uint1
                         const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                         uint16_t* out, wq_stream stream);
 
+/* y[i, r] = sum_c Wdeq[r, c] * x[i, c] for i < batch on water-filled weights, Wdeq the
+ * reconstruction of wq_dequant_wf (bf16, bit-exact), fp32 products and accumulation, bf16
+ * output: the decode-side consumer of the format. The pages give the format (one index
+ * space for the 3/4/5-bit codebooks, [DG] §2.1, §6) but no kernel that consumes it; this
+ * is the dyadic GEMV's contract on it.
+ *   x      bf16 [batch, k]; batch 1 .. 16.
+ *   y      out bf16 [batch, n].
+ * Same tolerance as wq_gemv_w4a16. A block outside packed_bytes, or a width outside 3..5,
+ * contributes nothing and is flagged for wq_device_error (WQ_EDATA). */
+wq_status wq_gemv_wf(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
+                     const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
+                     const uint16_t* x, int32_t batch, uint16_t* y, wq_stream stream);
+
 /* The GEMM above without a caller workspace, for callers that cannot allocate device
  * memory: e.g. an inference server whose caching allocator owns the whole device memory
  * budget and forbids any other cudaMalloc, a plugin that may only use the buffers its host

@@ -420,3 +420,16 @@ def wf_dequant(packed: np.ndarray, scale: np.ndarray, width: np.ndarray, blk_off
     _rows_parallel(n, lambda r0, r1: _L().orc_wf_dequant(_p(packed), _p(scale), _p(width), _p(blk_off),
                                                          n, k, r0, r1, _p(out)), threads)
     return out
+
+
+def wf_matmul_rows(packed: np.ndarray, scale: np.ndarray, width: np.ndarray, blk_off: np.ndarray,
+                   n: int, k: int, x_bits: np.ndarray, rows: np.ndarray | None = None):
+    """The product a consumer of the water-filled format computes, by its definition:
+    y[b, j] = sum_c Wdeq[rows[j], c] * x[b, c] in double with Wdeq = wf_dequant (the
+    reconstruction through the 5-bit index space, "MiniCPM5-1B 验证…" §2.1), and the error
+    scale bound[b, j] = sum_c |Wdeq[rows[j], c]| |x[b, c]|. x is bf16 bits [m, k]."""
+    wd = bf16_to_f64(wf_dequant(packed, scale, width, blk_off, n, k))
+    if rows is not None:
+        wd = wd[np.asarray(rows, np.int64)]
+    x = bf16_to_f64(np.atleast_2d(np.asarray(x_bits, np.uint16)))
+    return x @ wd.T, np.abs(x) @ np.abs(wd).T

@@ -77,6 +77,12 @@ def test_shape_and_group_checks_fail_before_any_cuda_call(wq):
     assert lib.wq_quantize_wf_pack(p, 4, 64, p, p, p, p, -1, None) == wq.WQ_EINVAL
     assert lib.wq_dequant_wf(p, -1, p, p, p, 4, 64, p, None) == wq.WQ_EINVAL
     assert lib.wq_dequant_wf(p, 16, p, p, p, 0, 64, p, None) == wq.WQ_EINVAL
+    # the water-filled GEMV: the same shape rules, batch 1..16
+    assert lib.wq_gemv_wf(p, 16, p, p, p, 4, 96, p, 1, p, None) == wq.WQ_EINVAL
+    assert lib.wq_gemv_wf(p, -1, p, p, p, 4, 64, p, 1, p, None) == wq.WQ_EINVAL
+    for batch in (0, 17):
+        assert lib.wq_gemv_wf(p, 16, p, p, p, 4, 64, p, batch, p, None) == wq.WQ_EINVAL
+        assert "batch" in wq.last_error()
 
 
 def test_gemv_plan_rejects_bad_arguments_and_keeps_nothing(wq):

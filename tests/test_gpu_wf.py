@@ -3,7 +3,8 @@ level index space; §6: water-filling) with the oracle, through the C ABI: scale
 the three fp64 distortions, block offsets, packed bit streams and the reconstruction are all
 bit-exact, over water levels from zero to infinity, ragged shapes, zero blocks, scales far
 outside the fast range, and sampled rows of a full-size launch; a too-small packed buffer is
-flagged without any access past it."""
+flagged without any access past it. The format's GEMV is checked against the oracle's
+product on the oracle's own encodings."""
 import ctypes
 
 import numpy as np
@@ -12,7 +13,7 @@ import torch
 
 import oracle
 import workloads
-from _util import bits, to_dev_bits
+from _util import bits, f32, matmul_tolerance, to_dev_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -118,3 +119,96 @@ def test_short_packed_buffer_is_flagged_not_overrun(wq):
     code = ctypes.c_int32(0)
     assert wq._lib.wq_device_error(ctypes.byref(code)) == wq.WQ_EDATA and code.value == 2001
     assert wq.device_error() == 0                            # the flag was cleared by the read
+
+
+def _oracle_encoding(wq, w_bits, lam):
+    """The oracle's water-filled encoding of w, and the same bytes on the device."""
+    n, k = w_bits.shape
+    s, wd, _ = oracle.wf_analyze(w_bits, lam)
+    off = oracle.wf_offsets(wd)
+    p = oracle.wf_pack(w_bits, s, wd, off)
+    dev = torch.device("cuda")
+    packed = torch.zeros(max(p.size, 16), dtype=torch.uint8, device=dev)
+    packed[:p.size] = torch.from_numpy(p).to(dev)
+    q = wq.WfWeight(n, k, to_dev_bits(s), torch.from_numpy(wd).to(dev),
+                    torch.from_numpy(off.view(np.int32)).to(dev), packed, int(p.size))
+    return q, (p, s, wd, off)
+
+
+def _gemv_check(wq, q, enc, x_bits, rows=None):
+    y = wq.gemv_wf(q, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.wf_matmul_rows(*enc, q.n, q.k, x_bits, rows=rows)
+    got = f32(y) if rows is None else f32(y)[:, rows]
+    assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound)), \
+        f"max err/bound {np.max(np.abs(got - y_ref) / np.maximum(bound, 1e-300)):.3g}"
+    assert wq.device_error() == 0
+
+
+@pytest.mark.parametrize("n,k", [(1, 64), (5, 2112), (33, 1024), (64, 4096), (19, 28672)])
+@pytest.mark.parametrize("batch", [1, 2, 3, 8, 9, 16])
+def test_gemv_matches_oracle(wq, n, k, batch):
+    """The format's GEMV ("MiniCPM5-1B 验证…" §2.1, §6 blocks; the dyadic GEMV's contract) on
+    mixed 3/4/5-bit rows: ragged row counts, a row tail of fewer than 32 blocks, batches
+    that are not a multiple of the kernel's 8 activation rows per launch."""
+    w = _weights(n * 3 + k, n, k)
+    _, _, d = oracle.wf_analyze(w, 0.0)
+    q, enc = _oracle_encoding(wq, w, float(np.median(d[..., 1]) / 64))
+    _gemv_check(wq, q, enc, workloads.activations(batch, k, workloads.LUT16, n + batch))
+
+
+def test_gemv_zero_blocks_subnormals_and_extreme_scales(wq):
+    w = _weights(11, 8, 512).astype(np.uint16)
+    w[0, :64] = 0
+    w[1, :] = np.arange(512) % 128                           # subnormal weights and scales
+    w[2:4] = workloads.f64_to_bf16_bits(oracle.bf16_to_f64(w[2:4]) * 2.0 ** 100)
+    w[4:6] = workloads.f64_to_bf16_bits(oracle.bf16_to_f64(w[4:6]) * 2.0 ** -110)
+    x = workloads.activations(4, 512, workloads.LUT16, 5)
+    for lam in (0.0, float("inf")):
+        q, enc = _oracle_encoding(wq, w, lam)
+        _gemv_check(wq, q, enc, x)
+
+
+def test_gemv_one_hot_exact(wq):
+    """x = e_c gives column c of the reconstruction, bit for bit."""
+    n, k = 40, 1024
+    w = _weights(17, n, k)
+    _, _, d = oracle.wf_analyze(w, 0.0)
+    q, enc = _oracle_encoding(wq, w, float(np.median(d[..., 1]) / 64))
+    wd = oracle.wf_dequant(*enc, n, k)
+    cols = np.array([0, 5, 63, 64, 500, 1023, 777, 128, 129, 300, 640, 1000, 2, 3, 4, 6])
+    x = np.zeros((16, k))
+    x[np.arange(16), cols] = 1.0
+    y = wq.gemv_wf(q, to_dev_bits(workloads.f64_to_bf16_bits(x)))
+    assert np.array_equal(bits(y), wd[:, cols].T)
+
+
+def test_gemv_full_size_sampled_rows(wq):
+    """The 8192 x 28672 launch bench.py times (batch 1 and 16), the encoding made by the
+    oracle, rows by sample."""
+    n, k = workloads.LUT16_SHAPE
+    g = np.random.default_rng(7)
+    w = workloads.f64_to_bf16_bits(g.standard_normal((n, k)) * 0.01)
+    q, enc = _oracle_encoding(wq, w, 8e-7)
+    rows = np.array([0, 1, 777, 4097, n - 2, n - 1])
+    for batch in (1, 16):
+        _gemv_check(wq, q, enc, workloads.activations(batch, k, workloads.LUT16, batch), rows=rows)
+
+
+def test_gemv_bad_block_is_flagged_not_read(wq):
+    """A width outside 3..5 or a block past packed_bytes contributes nothing and is flagged."""
+    n, k = 4, 256
+    w = _weights(19, n, k)
+    q, enc = _oracle_encoding(wq, w, 0.0)                     # every block 5 bits
+    x = to_dev_bits(workloads.activations(1, k, workloads.LUT16, 1))
+    q.width[1, 2] = 7
+    y = wq.gemv_wf(q, x)
+    torch.cuda.synchronize()
+    code = ctypes.c_int32(0)
+    assert wq._lib.wq_device_error(ctypes.byref(code)) == wq.WQ_EDATA and code.value == 2002
+    wd = oracle.bf16_to_f64(oracle.wf_dequant(*enc, n, k))
+    wd[1, 128:192] = 0.0                                      # the flagged block drops out
+    xd = oracle.bf16_to_f64(bits(x))
+    y_ref, bound = xd @ wd.T, np.abs(xd) @ np.abs(wd).T
+    assert np.all(np.abs(f32(y) - y_ref) <= matmul_tolerance(y_ref, bound))
+    assert wq.device_error() == 0

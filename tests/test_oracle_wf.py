@@ -152,3 +152,48 @@ def test_reconstruction_through_the_five_bit_index_space():
             assert np.array_equal(rec[r, 64 * g_:64 * g_ + 64], want)
     # and the storage: 8 * width bytes per block, plus a bf16 scale and a width byte
     assert off[-1] == 8 * int(wd.astype(np.int64).sum())
+
+
+def _bitstream(codes, b):
+    """Codes of b bits, code j in bits [b j, b j + b) from bit 0 of the first byte."""
+    acc = 0
+    for j, c in enumerate(codes):
+        acc |= int(c) << (b * j)
+    return acc.to_bytes(len(codes) * b // 8, "little")
+
+
+def test_product_hand_worked_blocks():
+    """One row of two blocks: a 3-bit block with every code 6 at scale 2 (value
+    (2 / 16)(6 * 4 - 16) = 1) and a 5-bit block with every code 3 at scale 1/2 (value
+    (1 / 32)(3 - 16) = -13/32). With x = 1 everywhere y = 64 - 26 = 38; with one-hot x the
+    product is the weight itself."""
+    packed = np.frombuffer(_bitstream([6] * 64, 3) + _bitstream([3] * 64, 5), np.uint8)
+    assert packed.size == 24 + 40
+    scale = workloads.f64_to_bf16_bits(np.array([[2.0, 0.5]]))
+    width = np.array([[3, 5]], np.uint8)
+    off = np.array([0, 24, 64], np.uint32)
+    ones = workloads.f64_to_bf16_bits(np.ones((1, 128)))
+    y, bound = oracle.wf_matmul_rows(packed, scale, width, off, 1, 128, ones)
+    assert y[0, 0] == 38.0 and bound[0, 0] == 64 + 26
+    eye = workloads.f64_to_bf16_bits(np.eye(128)[[0, 63, 64, 127]])
+    y, _ = oracle.wf_matmul_rows(packed, scale, width, off, 1, 128, eye)
+    assert list(y[:, 0]) == [1.0, 1.0, -13 / 32, -13 / 32]
+
+
+def test_product_at_four_bits_is_the_dyadic_product():
+    """With every block at 4 bits the format is the dyadic g64 format (same bytes, same
+    scales, same values), so the product must agree with the dyadic one."""
+    n, k = 24, 512
+    w = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 3)
+    s, c = oracle.dyadic_quantize(w, 64)
+    packed = oracle.pack(c)
+    width = np.full((n, k // 64), 4, np.uint8)
+    off = (32 * np.arange(n * k // 64 + 1)).astype(np.uint32)
+    x = workloads.activations(3, k, workloads.PREFILL, 3)
+    y, bound = oracle.wf_matmul_rows(packed.reshape(-1), s, width, off, n, k, x)
+    y4, bound4 = oracle.matmul_rows(oracle.DYADIC4, packed, s, 64, x)
+    assert np.allclose(y, y4, rtol=0, atol=1e-13 * bound4.max())
+    assert np.allclose(bound, bound4, rtol=1e-13)
+    rows = np.array([0, 7, 23])
+    yr, _ = oracle.wf_matmul_rows(packed.reshape(-1), s, width, off, n, k, x, rows=rows)
+    assert np.array_equal(yr, y[:, rows])

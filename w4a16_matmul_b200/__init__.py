@@ -70,6 +70,7 @@ _SIG = {
     "wq_quantize_wf_analyze": ([_vp, _i64, _i64, ctypes.c_double, _vp, _vp, _vp, _vp, _vp], _i32),
     "wq_quantize_wf_pack": ([_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp], _i32),
     "wq_dequant_wf": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp], _i32),
+    "wq_gemv_wf": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i32, _vp, _vp], _i32),
     "wq_bf16x_superblocks": ([_i64, _i64], _i64),
     "wq_bf16x_count": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "wq_bf16x_encode": ([_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp], _i32),
@@ -461,4 +462,15 @@ def dequant_wf(q: WfWeight, out: torch.Tensor | None = None) -> torch.Tensor:
         out = torch.empty((q.n, q.k), dtype=torch.bfloat16, device=q.packed.device)
     _check(_lib.wq_dequant_wf(_ptr(q.packed), q.packed.numel(), _ptr(q.scale), _ptr(q.width),
                               _ptr(q.blk_off), q.n, q.k, _ptr(out), _stream(out)))
+    return out
+
+
+def gemv_wf(q: WfWeight, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = x Wdeq^T for water-filled weights; x bf16 [batch, k] (batch 1..16) -> bf16 [batch, n]."""
+    _cuda(x, torch.bfloat16, "x")
+    batch = x.shape[0]
+    if out is None:
+        out = torch.empty((batch, q.n), dtype=torch.bfloat16, device=x.device)
+    _check(_lib.wq_gemv_wf(_ptr(q.packed), q.packed.numel(), _ptr(q.scale), _ptr(q.width), _ptr(q.blk_off),
+                           q.n, q.k, _ptr(x), batch, _ptr(out), _stream(x)))
     return out

@@ -228,6 +228,24 @@ wq_status wq_dequant_wf(const uint8_t* packed, int64_t packed_bytes, const uint1
     return launch_wf_dequant(packed, packed_bytes, scale, width, blk_off, n, k, out, (cudaStream_t)stream);
 }
 
+wq_status wq_gemv_wf(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
+                     const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
+                     const uint16_t* x, int32_t batch, uint16_t* y, wq_stream stream) {
+    g_last_error[0] = 0;
+    wq_status st = check_wf_shape(n, k);
+    if (st) return st;
+    if (packed_bytes < 0) return fail(WQ_EINVAL, "packed_bytes must be >= 0");
+    if (batch < 1 || batch > 16) return fail(WQ_EINVAL, "batch=%d outside 1..16", batch);
+    if ((st = check_ptr(packed, "packed", false))) return st;
+    if ((st = check_ptr(scale, "scale", false))) return st;
+    if ((st = check_ptr(width, "width", false))) return st;
+    if ((st = check_ptr(blk_off, "blk_off", false))) return st;
+    if ((st = check_ptr(x, "x", false))) return st;
+    if ((st = check_ptr(y, "y", false))) return st;
+    if ((st = check_injected())) return st;
+    return launch_wf_gemv(packed, packed_bytes, scale, width, blk_off, n, k, x, batch, y, (cudaStream_t)stream);
+}
+
 int64_t wq_bf16x_superblocks(int64_t n, int64_t k) {
     if (n < 1 || k < 1 || k % 16 != 0) return -1;
     return bf16x_superblocks(n, k);

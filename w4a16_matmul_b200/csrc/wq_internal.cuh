@@ -94,6 +94,9 @@ wq_status launch_wf_pack(const uint16_t* w, int64_t n, int64_t k, const uint16_t
 wq_status launch_wf_dequant(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
                             const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                             uint16_t* out, cudaStream_t s);
+wq_status launch_wf_gemv(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
+                         const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
+                         const uint16_t* x, int batch, uint16_t* y, cudaStream_t s);
 wq_status read_wf_error(int32_t* code);
 
 // Number of SMs of the current device (cached per device).

@@ -23,7 +23,8 @@
 // Kernels: analyze (scale, the three distortions, width, the scan's tile totals), the shared
 // in-place tile scan of the block sizes, pack (codes at the chosen width), dequant (eight
 // threads per block: each rebuilds 8 weights from b whole bytes and stores 16 bytes, so a
-// block's 128 output bytes leave in one coalesced run).
+// block's 128 output bytes leave in one coalesced run), and a GEMV that rebuilds the
+// weights the same way and multiplies them in fp32 (the format's decode-side consumer).
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -204,6 +205,53 @@ wf_pack_kernel(const uint4* __restrict__ w, int64_t nblk, const uint16_t* __rest
     }
 }
 
+// The b bytes at byte0 of the bit streams (8 codes of b bits), as the low bits of a 64-bit
+// word. Reads the 8-byte word holding byte0 and, when the bytes run past it, the next one:
+// both lie inside the block when byte0 = off + b t (t < 8) with off a multiple of 8 and the
+// block's 8 b bytes inside the buffer.
+__device__ __forceinline__ unsigned long long wf_bytes(const uint8_t* packed, int64_t byte0, int bw) {
+    const unsigned long long* src = reinterpret_cast<const unsigned long long*>(packed);
+    const int64_t q = byte0 >> 3;
+    const int sh = (int)(byte0 & 7) * 8;
+    unsigned long long v = __ldg(src + q) >> sh;
+    if (sh + 8 * bw > 64) v |= __ldg(src + q + 1) << (64 - sh);
+    return v;
+}
+
+// bf16((scale / 16) * (idx_5 - 16)) of the 8 codes of b bits in v (code j in bits b j ..),
+// as bf16 pairs in column order; sb = the block's bf16 scale bits.
+__device__ __forceinline__ void wf_decode8(unsigned long long v, int bw, uint32_t sb, uint32_t (&o)[4]) {
+    const uint32_t mask = (1u << bw) - 1u;
+    if ((sb & 0x7FFFu) >= 0x0400u) {
+        // scale >= 2^-119: every nonzero (scale / 16) (idx_5 - 16) is a normal bf16.
+        // Two codes at a time: idx_5 | 0x4300 is the bf16 number 128 + idx_5, minus 144
+        // is idx_5 - 16 exactly, and one bf16x2 multiply by scale / 16 (the exponent
+        // field minus 4) rounds the product once, as the definition reads.
+        const uint32_t s16x2 = prmt(sb - 0x0200u, 0u, 0x1010u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t c0 = (uint32_t)(v >> (bw * 2 * j)) & mask;
+            const uint32_t c1 = (uint32_t)(v >> (bw * (2 * j + 1))) & mask;
+            const uint32_t m = ((c0 | (c1 << 16)) << (5 - bw)) | 0x43004300u;
+            const uint32_t d = bf16x2_fma(m, 0x3F803F80u, 0xC310C310u);    // idx_5 - 16
+            o[j] = bf16x2_fma(d, s16x2, 0x80008000u);
+        }
+    } else {
+        const float s16 = bf16_bits_to_float(sb) * 0.0625f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i0 = (int)(((uint32_t)(v >> (bw * 2 * j)) & mask) << (5 - bw));
+            const int i1 = (int)(((uint32_t)(v >> (bw * (2 * j + 1))) & mask) << (5 - bw));
+            o[j] = pack_bf16x2(s16 * (float)(i0 - 16), s16 * (float)(i1 - 16));
+        }
+    }
+}
+
+// True when a block's width and offset are consistent with a buffer of packed_bytes.
+__device__ __forceinline__ bool wf_block_ok(int bw, int64_t off, int64_t packed_bytes) {
+    return bw >= 3 && bw <= 5 && (off & 7) == 0 && off + 8 * bw <= packed_bytes;
+}
+
 __global__ void __launch_bounds__(kThreads)
 wf_dequant_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const uint16_t* __restrict__ scale,
                   const uint8_t* __restrict__ width, const uint32_t* __restrict__ blk_off, int64_t nblk,
@@ -215,43 +263,99 @@ wf_dequant_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, cons
         const int bw = __ldg(width + i);
         const int64_t off = (int64_t)ldg_u32(blk_off + i);
         uint32_t o[4] = {0, 0, 0, 0};
-        if (bw < 3 || bw > 5 || (off & 7) != 0 || off + 8 * bw > packed_bytes) {
+        if (!wf_block_ok(bw, off, packed_bytes)) {
             report(2000);
         } else {
             // this thread's 8 codes are the b bytes at off + b t (8 codes of b bits)
-            const int64_t byte0 = off + (int64_t)bw * t;
-            const int64_t w0 = byte0 & ~7ll;
-            const int sh = (int)(byte0 & 7) * 8;
-            const unsigned long long* src = reinterpret_cast<const unsigned long long*>(packed);
-            unsigned long long v = __ldg(src + (w0 >> 3)) >> sh;
-            if (sh + 8 * bw > 64) v |= __ldg(src + (w0 >> 3) + 1) << (64 - sh);
-            const uint32_t sb = ldg_u16(scale + i);
-            const uint32_t mask = (1u << bw) - 1u;
-            if ((sb & 0x7FFFu) >= 0x0400u) {
-                // scale >= 2^-119: every nonzero (scale / 16) (idx_5 - 16) is a normal bf16.
-                // Two codes at a time: idx_5 | 0x4300 is the bf16 number 128 + idx_5, minus 144
-                // is idx_5 - 16 exactly, and one bf16x2 multiply by scale / 16 (the exponent
-                // field minus 4) rounds the product once, as the definition reads.
-                const uint32_t s16x2 = prmt(sb - 0x0200u, 0u, 0x1010u);
+            wf_decode8(wf_bytes(packed, off + (int64_t)bw * t, bw), bw, ldg_u16(scale + i), o);
+        }
+        stg_cs_v4(out + gid, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+}
+
+// GEMV on the water-filled weights: y[i, r] = sum_c Wdeq[r, c] x[i, c] for NB activation
+// rows, Wdeq rebuilt exactly as wf_dequant_kernel does (bf16), products and sums in fp32.
+// One warp per weight row; 8 lanes per 64-weight block (lane t: columns 8t .. 8t + 7, the b
+// bytes at the block's offset + b t), 4 blocks per step. The row's widths, offsets and
+// scales are read 32 blocks at a time, one block per lane, checked, and handed to the
+// decoding lanes by shuffles; the packed words of those 32 blocks (8 steps) are all loaded
+// before the first is decoded, to keep bytes in flight. A block whose width or offset is
+// inconsistent with the buffer is reported and contributes nothing.
+constexpr int kGemvWarps = 8;
+
+template <int NB>
+__global__ void __launch_bounds__(32 * kGemvWarps)
+wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const uint16_t* __restrict__ scale,
+               const uint8_t* __restrict__ width, const uint32_t* __restrict__ blk_off, int n, int k,
+               const uint16_t* __restrict__ x, uint16_t* __restrict__ y) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * kGemvWarps + (threadIdx.x >> 5);
+    if (row >= n) return;                        // the whole warp leaves; no CTA-wide barrier
+    const int kb = k >> 6;
+    const int64_t rb = (int64_t)row * kb;
+    const int t = lane & 7, sub = lane >> 3;
+    // two accumulators per activation row when there are one or two rows (shorter FMA
+    // chains), one otherwise (the rows are independent chains already)
+    constexpr int NA = NB <= 2 ? 2 : 1;
+    float acc[NB][NA];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t c0 = (uint32_t)(v >> (bw * 2 * j)) & mask;
-                    const uint32_t c1 = (uint32_t)(v >> (bw * (2 * j + 1))) & mask;
-                    const uint32_t m = ((c0 | (c1 << 16)) << (5 - bw)) | 0x43004300u;
-                    const uint32_t d = bf16x2_fma(m, 0x3F803F80u, 0xC310C310u);    // idx_5 - 16
-                    o[j] = bf16x2_fma(d, s16x2, 0x80008000u);
-                }
-            } else {
-                const float s16 = bf16_bits_to_float(sb) * 0.0625f;
+    for (int i = 0; i < NB; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int i0 = (int)(((uint32_t)(v >> (bw * 2 * j)) & mask) << (5 - bw));
-                    const int i1 = (int)(((uint32_t)(v >> (bw * (2 * j + 1))) & mask) << (5 - bw));
-                    o[j] = pack_bf16x2(s16 * (float)(i0 - 16), s16 * (float)(i1 - 16));
+        for (int a = 0; a < NA; ++a) acc[i][a] = 0.f;
+    for (int c0 = 0; c0 < kb; c0 += 32) {
+        const int nb = min(32, kb - c0);
+        int bw = 0;
+        uint32_t off = 0, sb = 0;
+        if (lane < nb) {
+            bw = __ldg(width + rb + c0 + lane);
+            off = ldg_u32(blk_off + rb + c0 + lane);
+            sb = ldg_u16(scale + rb + c0 + lane);
+            if (!wf_block_ok(bw, off, packed_bytes)) {
+                report(2002);
+                bw = 0;
+            }
+        }
+        unsigned long long v[8];
+        int w8[8];
+        uint32_t s8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int blk = 4 * j + sub;         // block of the chunk this lane decodes at step j
+            w8[j] = __shfl_sync(0xFFFFFFFFu, bw, blk);       // 0 past the row's end (lane >= nb)
+            const uint32_t o = __shfl_sync(0xFFFFFFFFu, off, blk);
+            s8[j] = __shfl_sync(0xFFFFFFFFu, sb, blk);
+            v[j] = w8[j] ? wf_bytes(packed, (int64_t)o + w8[j] * t, w8[j]) : 0ull;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (w8[j] == 0) continue;
+            uint32_t o[4];
+            wf_decode8(v[j], w8[j], s8[j], o);
+            float wv[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                wv[2 * q] = __uint_as_float(o[q] << 16);
+                wv[2 * q + 1] = __uint_as_float(o[q] & 0xFFFF0000u);
+            }
+            const int col = (c0 + 4 * j + sub) * 64 + 8 * t;
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                const uint4 xv = ldg_v4(x + (size_t)i * k + col);
+                const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[i][0] = fmaf(wv[2 * q], __uint_as_float(xs[q] << 16), acc[i][0]);
+                    acc[i][NA - 1] = fmaf(wv[2 * q + 1], __uint_as_float(xs[q] & 0xFFFF0000u), acc[i][NA - 1]);
                 }
             }
         }
-        stg_cs_v4(out + gid, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+        float r = NA == 2 ? acc[i][0] + acc[i][NA - 1] : acc[i][0];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+        if (lane == 0) y[(size_t)i * n + row] = (uint16_t)float_to_bf16_bits(r);
     }
 }
 
@@ -290,6 +394,35 @@ wq_status launch_wf_dequant(const uint8_t* packed, int64_t packed_bytes, const u
     wf_dequant_kernel<<<grid_cap((nblk * 8 + kThreads - 1) / kThreads), kThreads, 0, s>>>(
         packed, packed_bytes, scale, width, blk_off, nblk, (uint4*)out);
     return check_launch("wf dequant");
+}
+
+wq_status launch_wf_gemv(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
+                         const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
+                         const uint16_t* x, int batch, uint16_t* y, cudaStream_t s) {
+    const unsigned grid = (unsigned)((n + kGemvWarps - 1) / kGemvWarps);
+    // activation rows 8 at a time (x rows i .. i + 7 give y rows i .. i + 7)
+    for (int i0 = 0; i0 < batch; i0 += 8) {
+        const int nb = batch - i0 < 8 ? batch - i0 : 8;
+        const uint16_t* xi = x + (size_t)i0 * k;
+        uint16_t* yi = y + (size_t)i0 * n;
+#define WQ_WF_GEMV(NBV)                                                                              \
+    wf_gemv_kernel<NBV><<<grid, 32 * kGemvWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off, \
+                                                        (int)n, (int)k, xi, yi)
+        switch (nb) {
+            case 1: WQ_WF_GEMV(1); break;
+            case 2: WQ_WF_GEMV(2); break;
+            case 3: WQ_WF_GEMV(3); break;
+            case 4: WQ_WF_GEMV(4); break;
+            case 5: WQ_WF_GEMV(5); break;
+            case 6: WQ_WF_GEMV(6); break;
+            case 7: WQ_WF_GEMV(7); break;
+            default: WQ_WF_GEMV(8); break;
+        }
+#undef WQ_WF_GEMV
+        wq_status st = check_launch("wf gemv");
+        if (st) return st;
+    }
+    return WQ_OK;
 }
 
 wq_status read_wf_error(int32_t* code) {
