@@ -220,30 +220,38 @@ __device__ __forceinline__ unsigned long long wf_bytes(const uint8_t* packed, in
 
 // bf16((scale / 16) * (idx_5 - 16)) of the 8 codes of b bits in v (code j in bits b j ..),
 // as bf16 pairs in column order; sb = the block's bf16 scale bits.
+// Each code is brought to bits 5 - b .. 4, where its value is idx_5 = code << (5 - b), by one
+// 32-bit funnel shift of the 40 bits (the bits below it hold its neighbour and are masked
+// off); a pair of codes is joined into the two halves of one word by a byte permute.
 __device__ __forceinline__ void wf_decode8(unsigned long long v, int bw, uint32_t sb, uint32_t (&o)[4]) {
-    const uint32_t mask = (1u << bw) - 1u;
+    const uint32_t lo = (uint32_t)v, hi = (uint32_t)(v >> 32);
+    const int s5 = 5 - bw;
+    const uint32_t mp = (((1u << bw) - 1u) * 0x00010001u) << s5;      // idx_5 fields of a pair
+    uint32_t m[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // code 2j starts at bit 2 j b, code 2j + 1 at (2j + 1) b; shifted right by that minus
+        // s5 (>= 0 but for code 0, which is shifted left; < 32 but for code 7 at b = 5, bit 35)
+        const uint32_t c0 = j == 0 ? lo << s5 : __funnelshift_r(lo, hi, 2 * j * bw - s5);
+        const uint32_t c1 = (j == 3 && bw == 5) ? hi >> 3 : __funnelshift_r(lo, hi, (2 * j + 1) * bw - s5);
+        m[j] = prmt(c0, c1, 0x5410u) & mp;                               // (idx_5 of 2j, of 2j + 1)
+    }
     if ((sb & 0x7FFFu) >= 0x0400u) {
         // scale >= 2^-119: every nonzero (scale / 16) (idx_5 - 16) is a normal bf16.
-        // Two codes at a time: idx_5 | 0x4300 is the bf16 number 128 + idx_5, minus 144
-        // is idx_5 - 16 exactly, and one bf16x2 multiply by scale / 16 (the exponent
-        // field minus 4) rounds the product once, as the definition reads.
+        // idx_5 | 0x4300 is the bf16 number 128 + idx_5, minus 144 is idx_5 - 16 exactly, and
+        // one bf16x2 multiply by scale / 16 (the exponent field minus 4) rounds the product
+        // once, as the definition reads.
         const uint32_t s16x2 = prmt(sb - 0x0200u, 0u, 0x1010u);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint32_t c0 = (uint32_t)(v >> (bw * 2 * j)) & mask;
-            const uint32_t c1 = (uint32_t)(v >> (bw * (2 * j + 1))) & mask;
-            const uint32_t m = ((c0 | (c1 << 16)) << (5 - bw)) | 0x43004300u;
-            const uint32_t d = bf16x2_fma(m, 0x3F803F80u, 0xC310C310u);    // idx_5 - 16
+            const uint32_t d = bf16x2_fma(m[j] | 0x43004300u, 0x3F803F80u, 0xC310C310u);   // idx_5 - 16
             o[j] = bf16x2_fma(d, s16x2, 0x80008000u);
         }
     } else {
         const float s16 = bf16_bits_to_float(sb) * 0.0625f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i0 = (int)(((uint32_t)(v >> (bw * 2 * j)) & mask) << (5 - bw));
-            const int i1 = (int)(((uint32_t)(v >> (bw * (2 * j + 1))) & mask) << (5 - bw));
-            o[j] = pack_bf16x2(s16 * (float)(i0 - 16), s16 * (float)(i1 - 16));
-        }
+        for (int j = 0; j < 4; ++j)
+            o[j] = pack_bf16x2(s16 * (float)((int)(m[j] & 0xFFFFu) - 16), s16 * (float)((int)(m[j] >> 16) - 16));
     }
 }
 
@@ -276,12 +284,20 @@ wf_dequant_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, cons
 // GEMV on the water-filled weights: y[i, r] = sum_c Wdeq[r, c] x[i, c] for NB activation
 // rows, Wdeq rebuilt exactly as wf_dequant_kernel does (bf16), products and sums in fp32.
 // One warp per weight row; 8 lanes per 64-weight block (lane t: columns 8t .. 8t + 7, the b
-// bytes at the block's offset + b t), 4 blocks per step. The row's widths, offsets and
-// scales are read 32 blocks at a time, one block per lane, checked, and handed to the
-// decoding lanes by shuffles; the packed words of those 32 blocks (8 steps) are all loaded
-// before the first is decoded, to keep bytes in flight. A block whose width or offset is
-// inconsistent with the buffer is reported and contributes nothing.
+// bytes at the block's offset + b t), 4 blocks per step, 8 steps per chunk of 32 blocks.
+// A chunk's widths, offsets and scales are read one block per lane, checked, and handed to
+// the decoding lanes by shuffles. Software pipeline: the metadata is read two chunks
+// ahead and the packed words one chunk ahead, so that a chunk's loads are in flight while
+// the previous chunk is decoded. A block whose width or offset is inconsistent with the
+// buffer is reported and contributes nothing.
 constexpr int kGemvWarps = 8;
+
+// One chunk's packed words and, per step, the block width (0: nothing) and scale bits.
+struct WfChunk {
+    unsigned long long v[8];
+    uint32_t wpk;                    // width of step j in bits 4j .. 4j + 3
+    uint32_t spk[4];                 // scale bits of steps 2i (low half) and 2i + 1 (high half)
+};
 
 template <int NB>
 __global__ void __launch_bounds__(32 * kGemvWarps)
@@ -292,67 +308,80 @@ wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const u
     const int row = blockIdx.x * kGemvWarps + (threadIdx.x >> 5);
     if (row >= n) return;                        // the whole warp leaves; no CTA-wide barrier
     const int kb = k >> 6;
+    const int nch = (kb + 31) >> 5;
     const int64_t rb = (int64_t)row * kb;
     const int t = lane & 7, sub = lane >> 3;
-    // two accumulators per activation row when there are one or two rows (shorter FMA
-    // chains), one otherwise (the rows are independent chains already)
-    constexpr int NA = NB <= 2 ? 2 : 1;
-    float acc[NB][NA];
-#pragma unroll
-    for (int i = 0; i < NB; ++i)
-#pragma unroll
-        for (int a = 0; a < NA; ++a) acc[i][a] = 0.f;
-    for (int c0 = 0; c0 < kb; c0 += 32) {
-        const int nb = min(32, kb - c0);
-        int bw = 0;
-        uint32_t off = 0, sb = 0;
-        if (lane < nb) {
-            bw = __ldg(width + rb + c0 + lane);
-            off = ldg_u32(blk_off + rb + c0 + lane);
-            sb = ldg_u16(scale + rb + c0 + lane);
-            if (!wf_block_ok(bw, off, packed_bytes)) {
-                report(2002);
-                bw = 0;
-            }
+
+    // this lane's block of chunk c: width (0 past the row's end), offset, scale bits
+    auto meta = [&](int c, int& bw, uint32_t& off, uint32_t& sb) {
+        const int bi = 32 * c + lane;
+        bw = 0; off = 0; sb = 0;
+        if (bi < kb) {
+            bw = __ldg(width + rb + bi);
+            off = ldg_u32(blk_off + rb + bi);
+            sb = ldg_u16(scale + rb + bi);
         }
-        unsigned long long v[8];
-        int w8[8];
-        uint32_t s8[8];
+    };
+    // check the lane's block, then issue the chunk's packed loads (the whole warp takes part)
+    auto fetch = [&](int c, int bw, uint32_t off, uint32_t sb, WfChunk& ch) {
+        if (32 * c + lane < kb && !wf_block_ok(bw, off, packed_bytes)) {
+            report(2002);
+            bw = 0;
+        }
+        ch.wpk = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const int blk = 4 * j + sub;         // block of the chunk this lane decodes at step j
-            w8[j] = __shfl_sync(0xFFFFFFFFu, bw, blk);       // 0 past the row's end (lane >= nb)
+            const int blk = 4 * j + sub;
+            const int b = __shfl_sync(0xFFFFFFFFu, bw, blk);
             const uint32_t o = __shfl_sync(0xFFFFFFFFu, off, blk);
-            s8[j] = __shfl_sync(0xFFFFFFFFu, sb, blk);
-            v[j] = w8[j] ? wf_bytes(packed, (int64_t)o + w8[j] * t, w8[j]) : 0ull;
+            const uint32_t sj = __shfl_sync(0xFFFFFFFFu, sb, blk);
+            ch.wpk |= (uint32_t)b << (4 * j);
+            if (j & 1) ch.spk[j >> 1] |= sj << 16; else ch.spk[j >> 1] = sj;
+            ch.v[j] = b ? wf_bytes(packed, (int64_t)o + b * t, b) : 0ull;
+        }
+    };
+
+    float2 acc[NB];
+#pragma unroll
+    for (int i = 0; i < NB; ++i) acc[i] = make_float2(0.f, 0.f);
+
+    WfChunk cur;
+    int bw;
+    uint32_t off, sb;
+    meta(0, bw, off, sb);
+    fetch(0, bw, off, sb, cur);
+    if (nch > 1) meta(1, bw, off, sb);
+    for (int c = 0; c < nch; ++c) {
+        WfChunk nxt;
+        if (c + 1 < nch) {                       // uniform across the warp
+            fetch(c + 1, bw, off, sb, nxt);
+            if (c + 2 < nch) meta(c + 2, bw, off, sb);
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            if (w8[j] == 0) continue;
+            const int b = (int)(cur.wpk >> (4 * j)) & 15;
+            if (b == 0) continue;
+            const uint32_t sj = (j & 1) ? cur.spk[j >> 1] >> 16 : cur.spk[j >> 1] & 0xFFFFu;
             uint32_t o[4];
-            wf_decode8(v[j], w8[j], s8[j], o);
-            float wv[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                wv[2 * q] = __uint_as_float(o[q] << 16);
-                wv[2 * q + 1] = __uint_as_float(o[q] & 0xFFFF0000u);
-            }
-            const int col = (c0 + 4 * j + sub) * 64 + 8 * t;
+            wf_decode8(cur.v[j], b, sj, o);
+            const int col = (32 * c + 4 * j + sub) * 64 + 8 * t;
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
                 const uint4 xv = ldg_v4(x + (size_t)i * k + col);
                 const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    acc[i][0] = fmaf(wv[2 * q], __uint_as_float(xs[q] << 16), acc[i][0]);
-                    acc[i][NA - 1] = fmaf(wv[2 * q + 1], __uint_as_float(xs[q] & 0xFFFF0000u), acc[i][NA - 1]);
+                    const float2 w2 = make_float2(__uint_as_float(o[q] << 16), __uint_as_float(o[q] & 0xFFFF0000u));
+                    const float2 x2 = make_float2(__uint_as_float(xs[q] << 16), __uint_as_float(xs[q] & 0xFFFF0000u));
+                    acc[i] = __ffma2_rn(w2, x2, acc[i]);
                 }
             }
         }
+        if (c + 1 < nch) cur = nxt;
     }
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
-        float r = NA == 2 ? acc[i][0] + acc[i][NA - 1] : acc[i][0];
+        float r = acc[i].x + acc[i].y;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
         if (lane == 0) y[(size_t)i * n + row] = (uint16_t)float_to_bf16_bits(r);
