@@ -209,12 +209,20 @@ wf_pack_kernel(const uint4* __restrict__ w, int64_t nblk, const uint16_t* __rest
 // word. Reads the 8-byte word holding byte0 and, when the bytes run past it, the next one:
 // both lie inside the block when byte0 = off + b t (t < 8) with off a multiple of 8 and the
 // block's 8 b bytes inside the buffer.
+// The bytes are read once, so they bypass L1 (which then keeps what is reused, such as the
+// GEMV's activations).
+__device__ __forceinline__ unsigned long long ldg_na_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm("ld.global.nc.L1::no_allocate.u64 %0, [%1];" : "=l"(v) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ unsigned long long wf_bytes(const uint8_t* packed, int64_t byte0, int bw) {
     const unsigned long long* src = reinterpret_cast<const unsigned long long*>(packed);
     const int64_t q = byte0 >> 3;
     const int sh = (int)(byte0 & 7) * 8;
-    unsigned long long v = __ldg(src + q) >> sh;
-    if (sh + 8 * bw > 64) v |= __ldg(src + q + 1) << (64 - sh);
+    unsigned long long v = ldg_na_u64(src + q) >> sh;
+    if (sh + 8 * bw > 64) v |= ldg_na_u64(src + q + 1) << (64 - sh);
     return v;
 }
 
@@ -367,7 +375,8 @@ wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const u
             const int col = (32 * c + 4 * j + sub) * 64 + 8 * t;
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
-                const uint4 xv = ldg_v4(x + (size_t)i * k + col);
+                // cached in L1: every warp of the SM reads the same activations
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)i * k + col));
                 const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
