@@ -15,7 +15,8 @@ def test_library_exports_every_header_function(wq):
                 "wq_debug_fail_next_launches", "wq_device_error", "wq_gemm_w4a16_static",
                 "wq_gemv_plan_create", "wq_gemv_plan_launch", "wq_gemv_plan_destroy",
                 "wq_fake_quant_ste", "wq_bf16x_superblocks", "wq_bf16x_count", "wq_bf16x_encode",
-                "wq_bf16x_decode"}
+                "wq_bf16x_decode", "wq_gumbel_st_backward", "wq_quantize_wf_analyze",
+                "wq_quantize_wf_pack", "wq_dequant_wf", "wq_gemv_wf"}
     assert expected <= set(names), set(names) ^ expected
     for n in names:
         assert hasattr(wq._lib, n), n
@@ -122,3 +123,24 @@ def test_binding_refuses_cpu_tensors(wq):
         wq.quantize_dyadic(torch.zeros(4, 64, dtype=torch.bfloat16))
     with pytest.raises(ValueError):
         wq.pack(torch.zeros(4, 64, dtype=torch.uint8))
+
+
+def test_gemm_workspace_sizes(wq):
+    """Host-side GEMM planning (no GPU: the SM count falls back to the B200's 148). Up to 12
+    activation rows run on the GEMV and need nothing; on 4096 x 11008 the large m runs in
+    whole waves without scratch and m = 512 splits the tail. LUT16 plans the same launches
+    as DYADIC4 and adds its fp16 activations, 2 m k bytes rounded up to 1 KB, in front."""
+    def ws(fmt, group, n, k, m):
+        d = wq.WqWeight(fmt, group, n, k, None, None)
+        return int(wq._lib.wq_gemm_workspace_bytes(ctypes.byref(d), m))
+
+    n, k = 4096, 11008
+    for fmt, group in [(wq.FMT_DYADIC4, 64), (wq.FMT_LUT16, 64), (wq.FMT_LLOYD8S, 32)]:
+        assert ws(fmt, group, n, k, 12) == 0
+    assert ws(wq.FMT_DYADIC4, 64, n, k, 4096) == 0
+    assert ws(wq.FMT_DYADIC4, 64, n, k, 512) == 16 << 20
+    for m in (13, 16, 48, 100, 128, 200, 512, 4096):
+        for nn, kk in [(n, k), (11008, 4096), (200, 320)]:
+            x_bytes = -(-2 * m * kk // 1024) * 1024
+            assert ws(wq.FMT_LUT16, 64, nn, kk, m) == ws(wq.FMT_DYADIC4, 64, nn, kk, m) + x_bytes
+    assert ws(wq.FMT_LUT16, 64, n, k, 0) == 0
