@@ -230,3 +230,22 @@ def test_gemm_lut16_workspace_paths(wq, m, n, k):
     y_ref, bound = oracle.matmul_rows(oracle.LUT16, packed, lut, 64, x_bits[ms], rows=rows)
     got = f32(y)[np.ix_(ms, rows)]
     assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
+
+
+@pytest.mark.parametrize("m", [512, 4096])
+def test_gemm_lut16_bench_launch_sampled(wq, m):
+    """The LUT16 GEMM in the launches bench.py times (4096 x 11008; m = 512 splits K in two,
+    m = 4096 runs whole waves of 256-row activation tiles), random codes and sorted fp16
+    centroids; 64 sampled weight rows x 64 sampled activation rows against the oracle."""
+    n, k = workloads.PREFILL_SHAPES[0]
+    pw, packed, lut = _lut16(wq, n, k, 6)
+    x_bits = workloads.activations(m, k, workloads.PREFILL, m + 7)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+    rng = np.random.default_rng(m)
+    rows = np.sort(rng.choice(n, 64, replace=False))
+    ms = np.sort(rng.choice(m, 64, replace=False))
+    y_ref, bound = oracle.matmul_rows(oracle.LUT16, packed, lut, 64, x_bits[ms], rows=rows)
+    got = f32(y)[np.ix_(ms, rows)]
+    assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
