@@ -346,6 +346,22 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
     """Secondary rows of the hot path, each on its own workload, timed the same way."""
     out = {}
     steps, warm = max(args.steps, 5), max(args.warmup, 3)
+    # the headline's launch with 10 steps captured in one graph: its difference to the
+    # headline's per-step time (one graph replay per step) is the gap between graph launches
+    try:
+        run10 = wq.GroupedGemv(packed, xs, ys)
+        g10 = graph_of(torch, lambda: [run10() for _ in range(10)])
+        reps = max(steps // 10, 3)
+        ms10 = max_over_ranks(time_region(torch, stream, g10.replay, reps, 3, barrier)) / 10
+        pk, sc, xb, yb = sweep_bytes(mats, args.batch)
+        out["headline_10_steps_per_graph"] = {
+            "ms_per_step": round(ms10, 5), "GB/s": round((pk + sc) / ms10 / 1e6, 1),
+            "frac_hbm_algorithmic": round((pk + sc + xb + yb) / ms10 / 1e6 / peaks["hbm_gbs"], 4),
+            "replays": reps}
+        del g10
+        run10.close()
+    except Exception as e:  # report, never hide
+        out["headline_10_steps_per_graph"] = {"error": repr(e)[:200]}
     # decode sweep as 168 dependent-order launches captured in one CUDA graph
     try:
         g = torch.cuda.CUDAGraph()
