@@ -275,9 +275,11 @@ wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16
 /* Reads and clears the library's device-side error words. Kernels that wait on the GPU
  * (the GEMM pipeline's mbarrier waits) give up after a bounded time instead of hanging and
  * record a nonzero code; the BF16X kernels record one when an overflow-table index would
- * pass ovf_bytes (the access is skipped). *code receives the code (0 = none). Synchronous
- * (copies two ints from the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_EDATA
- * for inconsistent BF16X data, WQ_OK otherwise. */
+ * pass ovf_bytes, and the water-filling kernels one when a block's width is outside 3..5
+ * or its bytes do not fit packed_bytes (2000 dequant, 2001 pack, 2002 GEMV; the access is
+ * skipped in every case). *code receives the code (0 = none). Synchronous (copies three
+ * ints from the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_EDATA for
+ * inconsistent BF16X or water-filling data, WQ_OK otherwise. */
 wq_status wq_device_error(int32_t* code);
 
 /* ------------------------------------------------------------------------------------ */

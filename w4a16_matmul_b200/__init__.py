@@ -104,8 +104,9 @@ def last_error() -> str:
 
 
 def device_error() -> int:
-    """Reads and clears the device error words (nonzero: a bounded GPU wait expired, or a
-    BF16X kernel met an overflow index past its table)."""
+    """Reads and clears the device error words (nonzero: a bounded GPU wait expired, a BF16X
+    kernel met an overflow index past its table, or a water-filling kernel met a block whose
+    width or offset does not fit its buffer)."""
     code = _i32(0)
     st = _lib.wq_device_error(ctypes.byref(code))
     if st not in (WQ_OK, WQ_ETIMEOUT, WQ_EDATA):
