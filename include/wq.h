@@ -137,8 +137,12 @@ typedef struct wq_lloyd_params {
  *   codebook  out, see wq_lloyd_mode.
  *   params    out uint8 [n, k/32] (G32_WARM only), may be NULL.
  *   mse_trace out fp32, see wq_lloyd_mode, may be NULL.
- * Both modes take their decisions in double precision (G32_WARM screens the 112
- * candidates in fp32 first and re-ranks the near-best ones in double). */
+ * Both modes take their decisions in double precision. G32_WARM screens the 112
+ * candidates in fp32, bounding each candidate's exact MSE from both sides, and evaluates
+ * again in double, with the steps of [G32] §1.3 and the squared errors summed in index
+ * order, every candidate whose lower bound does not exceed the smallest upper bound; the
+ * lowest double MSE wins (lowest candidate on a tie). Lloyd and k-means member sums run in
+ * index order, so repeated calls give identical bits. */
 wq_status wq_quantize_lloyd(const uint16_t* w, int64_t n, int64_t k, const wq_lloyd_params* p,
                             uint8_t* codes, uint8_t* packed, void* codebook, uint8_t* params,
                             float* mse_trace, wq_stream stream);

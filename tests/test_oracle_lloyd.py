@@ -212,3 +212,87 @@ def test_kmeans_init_reading_and_properties():
     wd = oracle.fp16_to_f64(oracle.dequant(oracle.LUT16, oracle.pack(res["codes"]), res["lut"], 64))
     err = ((wd.reshape(16, 4, 64) - v) ** 2).mean(-1)
     assert np.allclose(err, tr[..., -1], rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
+# Brute force of the candidate search ([G32] §1.2 grid, §1.3 step 1), written apart from the
+# oracle: the grid from the page's printed lists, the transforms with Python's own pow and
+# tanh, every inverse level by scipy's Brent root finder on f(L) = q/7 * fmax (no closed
+# forms), round half to even, and all 112 MSEs compared one by one with the oracle forced to
+# each candidate.
+# ---------------------------------------------------------------------------------------
+
+def _page_grid():
+    gold = _golden()
+    lo, hi = (math.log10(v) for v in gold["rational_b_rel_endpoints"])
+    grid = []
+    for r in range(15):
+        for beta in gold["rational_beta"]:
+            grid.append((0, 10 ** (lo + (hi - lo) * r / 14), beta))
+    grid += [(1, br, 1.0) for br in gold["tanh_b_rel"]]
+    return grid
+
+
+def _brute_mses(a):
+    from scipy.optimize import brentq
+    gmax = max(a)
+    out = []
+    for fam, b_rel, beta in _page_grid():
+        b = b_rel * gmax
+        if fam == 0:
+            f = lambda v, b=b, beta=beta: v / (b + v ** beta)
+        else:
+            f = lambda v, b=b: math.tanh(v / b)
+        fmax = f(gmax)
+        levels = [0.0] + [brentq(lambda v, t=q / 7 * fmax: f(v) - t, 0.0, gmax, xtol=1e-300,
+                                 rtol=8.9e-16, maxiter=400) for q in range(1, 7)] + [gmax]
+        se = 0.0
+        for v in a:
+            q = min(max(int(np.rint(7 * f(v) / fmax)), 0), 7)      # rint: half to even
+            se += (v - levels[q]) ** 2
+        out.append(se / len(a))
+    return np.array(out)
+
+
+def _groups_for_brute_force():
+    rng = np.random.default_rng(11)
+    groups = [workloads.f64_to_bf16_bits(rng.laplace(0, 0.015, 32) * s) for s in (0.5, 1.0, 2.0)]
+    g = workloads.f64_to_bf16_bits(rng.normal(0, 0.02, 32))
+    g[rng.integers(32)] = workloads.f64_to_bf16_bits(np.array([0.4]))[0]      # one outlier x20
+    groups.append(g)
+    groups.append(workloads.f64_to_bf16_bits(rng.laplace(0, 1.0, 8)))          # a tiny group
+    return groups
+
+
+@pytest.mark.parametrize("gi", range(5))
+def test_candidate_search_matches_brute_force(gi):
+    g = _groups_for_brute_force()[gi]
+    a = [abs(float(v)) for v in oracle.bf16_to_f64(g)]
+    brute = _brute_mses(a)
+    size = len(a)
+    w = g.reshape(1, size)
+    ref = oracle.lloyd(w, size, 0)
+    # every candidate's MSE, the oracle forced to it
+    for c in range(112):
+        forced = oracle.lloyd(w, size, 0, force_cand=np.array([c], np.int32))
+        assert forced["trace"][0, 0, 0] == pytest.approx(brute[c], rel=1e-9, abs=1e-30), c
+    order = np.argsort(brute, kind="stable")
+    best, second = brute[order[0]], brute[order[1]]
+    assert second > best * (1 + 1e-6)          # a clear winner: no near-tie in these groups
+    assert ref["cand"][0, 0] == order[0]
+    assert ref["trace"][0, 0, 0] == pytest.approx(best, rel=1e-12)
+    assert ref["cand_gap"][0, 0] == pytest.approx(second - best, rel=1e-6)
+
+
+def test_candidate_search_exact_tie_takes_lowest_index():
+    """Magnitudes only 0 and gmax (and one just below gmax, which every candidate's concave
+    transform sends to the top level): every candidate reconstructs them with its exact end
+    levels, so all 112 MSEs are the same number and the lowest index, 0, must win."""
+    vals = np.array([0.0, 1.5, -1.5, 0.0, 1.5, -1.4921875] * 5 + [1.5, -0.0])
+    g = workloads.f64_to_bf16_bits(vals)
+    a = [abs(float(v)) for v in oracle.bf16_to_f64(g)]
+    brute = _brute_mses(a)
+    assert np.all(brute == brute[0]) and brute[0] > 0
+    ref = oracle.lloyd(g.reshape(1, 32), 32, 0)
+    assert ref["cand"][0, 0] == 0 and ref["params"][0, 0] == 0
+    assert ref["trace"][0, 0, 0] == brute[0]
