@@ -213,8 +213,12 @@ wq_status wq_gumbel_st_backward(const float* z, int64_t n, int64_t k, int32_t gr
 /* Decode-side W4A16 GEMV ([DG] §2.5/§3.2 fused unpack; [KM] §2.2, §4.1 small batch):
  * y[b, r] = sum_c Wdeq[r, c] * x[b, c], fp32 accumulation, bf16 output (rounded to
  * nearest even), for b < batch. Wdeq is the reconstruction wq_dequant gives (bf16 for
- * DYADIC4 / LLOYD8S; for LUT16 the fp16 centroid, with x converted to fp16, exact for
- * |x| in [2^-14, 65504]; |x| > 65504 is outside the contract).
+ * DYADIC4 / LLOYD8S; for LUT16 the fp16 centroid, multiplied by fp16 activations: each
+ * batch row's chunk of x that a thread block stages is converted as x * 2^e, with the
+ * power of two chosen from the chunk's largest |x| so that it lands in [2^15, 2^16), and
+ * the chunk's fp32 sums are multiplied by 2^-e. Every finite bf16 x is in range; an
+ * element more than 2^32 below its chunk's largest magnitude may lose low bits, by less
+ * than 2^-40 of that magnitude).
  *   w      packed weight (any format).
  *   x      bf16 [batch, k].
  *   batch  1..16.
@@ -256,6 +260,19 @@ wq_status wq_gemv_plan_create(const wq_weight* ws, const uint16_t* const* xs,
 wq_status wq_gemv_plan_launch(wq_gemv_plan plan, wq_stream stream);
 void wq_gemv_plan_destroy(wq_gemv_plan plan);
 
+/* Lets each later launch of the plan overlap the kernel before it in the stream
+ * (programmatic dependent launch), for decode loops where back-to-back launches would
+ * otherwise leave the GPU idle between kernels and during each kernel's last wave. With
+ * enable = 1, a launch's thread blocks may start, and load the plan's weights (packed codes
+ * and per-group scales, levels or centroids), while the previous kernel's last blocks are
+ * still running; they read the activations and write the outputs only after that kernel
+ * has completed and its writes are visible. Enable it only when the kernel launched just
+ * before the plan does not write the plan's weights (a previous launch of the plan, or any
+ * kernel that only produces its activations, is fine). enable = 0 (the default) restores
+ * plain stream order. Returns WQ_EINVAL for a NULL plan or another value. Host only; takes
+ * effect at the next wq_gemv_plan_launch. The pages describe no such mode. */
+wq_status wq_gemv_plan_set_overlap(wq_gemv_plan plan, int32_t enable);
+
 /* Bytes of device workspace wq_gemm_w4a16 needs for this weight and m (0 if none). */
 size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
 
@@ -264,14 +281,16 @@ size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
  * accumulation in tensor memory, bf16 output. Formats DYADIC4 (group 64 or 32), LLOYD8S
  * (the 8-level codebook plus sign of [G32] §5.2, rebuilt per stage from the group's levels)
  * and LUT16 (the per-block-64 centroid table of [KM] §2.2, looked up per stage; the product
- * runs in fp16 with the activations converted bf16 -> fp16 into the workspace, exact for
- * |x| in [2^-14, 65504] as in wq_gemv_w4a16). For m <= 12 the decode-shaped case runs on the
+ * runs in fp16 on the activations converted into the workspace as x * 2^e per activation
+ * row, the power of two chosen from the row's largest |x| as in wq_gemv_w4a16, and the
+ * epilogue multiplies the row's sums by 2^-e). For m <= 12 the decode-shaped case runs on the
  * GEMV kernel of wq_gemv_w4a16 (the kernel choice by batch size of [KM] §4.1), with the same
  * tolerance and no workspace.
  *   x      bf16 [m, k]; m >= 1; k % 64 == 0.
  *   y      out bf16 [m, n].
  *   ws     device workspace of at least wq_gemm_workspace_bytes(w, m) bytes (NULL if 0);
- *          for LUT16 it includes 2*m*k bytes for the fp16 activations.
+ *          for LUT16 it includes 2*m*k bytes for the scaled fp16 activations and 4*m for
+ *          the rows' factors 2^-e (each rounded up to 1 KB).
  * Same tolerance as wq_gemv_w4a16. */
 wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y,
                         void* ws, size_t ws_bytes, wq_stream stream);
@@ -398,7 +417,9 @@ wq_status wq_gemv_wf(const uint8_t* packed, int64_t packed_bytes, const uint16_t
  *     work overlaps (e.g. on two streams) race on it: serialise them.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) once and caches it; make that first call before any stream
- *     capture. */
+ *     capture. The cache remembers the context it was filled in: after cudaDeviceReset
+ *     the next call on that device looks the address up again (make it, too, outside a
+ *     capture). LUT16 also keeps its scaled fp16 activations in the array. */
 #define WQ_GEMM_STATIC_SCRATCH_BYTES (16u << 20)
 wq_status wq_gemm_w4a16_static(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y,
                                wq_stream stream);

@@ -13,7 +13,7 @@ def test_library_exports_every_header_function(wq):
                 "wq_quantize_lloyd", "wq_pack", "wq_unpack", "wq_dequant", "wq_gemv_w4a16",
                 "wq_gemv_w4a16_grouped", "wq_gemm_workspace_bytes", "wq_gemm_w4a16",
                 "wq_debug_fail_next_launches", "wq_device_error", "wq_gemm_w4a16_static",
-                "wq_gemv_plan_create", "wq_gemv_plan_launch", "wq_gemv_plan_destroy",
+                "wq_gemv_plan_create", "wq_gemv_plan_launch", "wq_gemv_plan_destroy", "wq_gemv_plan_set_overlap",
                 "wq_fake_quant_ste", "wq_bf16x_superblocks", "wq_bf16x_count", "wq_bf16x_encode",
                 "wq_bf16x_decode", "wq_gumbel_st_backward", "wq_quantize_wf_analyze",
                 "wq_quantize_wf_pack", "wq_dequant_wf", "wq_gemv_wf"}
@@ -101,6 +101,7 @@ def test_gemv_plan_rejects_bad_arguments_and_keeps_nothing(wq):
     assert lib.wq_gemv_plan_create(ctypes.byref(d), arr, arr, 1, 1, ctypes.byref(plan)) == wq.WQ_EINVAL
     assert plan.value is None
     assert lib.wq_gemv_plan_launch(None, None) == wq.WQ_EINVAL
+    assert lib.wq_gemv_plan_set_overlap(None, 1) == wq.WQ_EINVAL
     lib.wq_gemv_plan_destroy(None)                       # a no-op
 
 
@@ -129,7 +130,8 @@ def test_gemm_workspace_sizes(wq):
     """Host-side GEMM planning (no GPU: the SM count falls back to the B200's 148). Up to 12
     activation rows run on the GEMV and need nothing; on 4096 x 11008 the large m runs in
     whole waves without scratch and m = 512 splits the tail. LUT16 plans the same launches
-    as DYADIC4 and adds its fp16 activations, 2 m k bytes rounded up to 1 KB, in front."""
+    as DYADIC4 and adds, in front, its scaled fp16 activations (2 m k bytes) and the rows'
+    fp32 factors (4 m bytes), each rounded up to 1 KB."""
     def ws(fmt, group, n, k, m):
         d = wq.WqWeight(fmt, group, n, k, None, None)
         return int(wq._lib.wq_gemm_workspace_bytes(ctypes.byref(d), m))
@@ -141,6 +143,6 @@ def test_gemm_workspace_sizes(wq):
     assert ws(wq.FMT_DYADIC4, 64, n, k, 512) == 16 << 20
     for m in (13, 16, 48, 100, 128, 200, 512, 4096):
         for nn, kk in [(n, k), (11008, 4096), (200, 320)]:
-            x_bytes = -(-2 * m * kk // 1024) * 1024
+            x_bytes = -(-2 * m * kk // 1024) * 1024 + -(-4 * m // 1024) * 1024
             assert ws(wq.FMT_LUT16, 64, nn, kk, m) == ws(wq.FMT_DYADIC4, 64, nn, kk, m) + x_bytes
     assert ws(wq.FMT_LUT16, 64, n, k, 0) == 0

@@ -172,6 +172,11 @@ def test_gemm_last_wave_split(wq):
     assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
     # the same through the static-scratch entry point (the tail's scratch stays within it)
     assert wq.gemm_workspace_bytes(pw, m) <= (16 << 20)
+    ys = wq.gemm_static(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+    got = f32(ys)[np.ix_(ms, rows)]
+    assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
 
 
 def _lut16(wq, n, k, seed):

@@ -1,7 +1,8 @@
 """wq_gemm_w4a16_static: the GEMM for callers that cannot allocate device memory (its
-split-K scratch lives in a static device array of the library). Called through the C ABI
-and compared with wq_gemm_w4a16 given a caller workspace, within the tolerance of the other
-GEMM tests, on two calls in a row. This file is collected last on purpose."""
+split-K scratch lives in a static device array of the library). Called through the C ABI,
+on two calls in a row, and compared within the tolerance of the other GEMM tests both with
+the oracle's fp64 product and with wq_gemm_w4a16 given a caller workspace. This file is
+collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -15,9 +16,10 @@ from _util import f32, matmul_tolerance, to_dev, to_dev_bits
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("fmt", ["dyadic", "lut16"])
+@pytest.mark.parametrize("fmt", ["dyadic", "lut16", "lut16_small_x"])
 def test_static_scratch_gemm_matches_workspace_gemm(wq, fmt):
-    """LUT16 also keeps its fp16 copy of the activations in the scratch."""
+    """LUT16 also keeps its scaled fp16 copy of the activations and their row factors in the
+    scratch; lut16_small_x feeds it activations around 1e-8, mixed with 1e2 in odd rows."""
     n, k, m = 1024, 8192, 48                  # small m: K is split, so the scratch is used
     if fmt == "dyadic":
         w_bits = workloads.gaussian_outlier_weight(n, k, workloads.PREFILL, 21)
@@ -39,6 +41,10 @@ def test_static_scratch_gemm_matches_workspace_gemm(wq, fmt):
     rows = np.arange(0, n, 5)
     for call in range(2):
         x_bits = workloads.activations(m, k, workloads.PREFILL, 100 + call)
+        if fmt == "lut16_small_x":
+            xv = oracle.bf16_to_f64(x_bits) * 1e-8
+            xv[1::2, ::3] *= 1e10
+            x_bits = workloads.f64_to_bf16_bits(xv)
         x = to_dev_bits(x_bits)
         y_static = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
         st = wq._lib.wq_gemm_w4a16_static(ctypes.byref(d), ctypes.c_void_p(x.data_ptr()), m,
@@ -51,8 +57,10 @@ def test_static_scratch_gemm_matches_workspace_gemm(wq, fmt):
                                    need, stream)
         assert st == wq.WQ_OK, wq.last_error()
         torch.cuda.synchronize()
-        _, bound = oracle.matmul_rows(code, packed, aux, 64, x_bits, rows=rows)
+        y_ref, bound = oracle.matmul_rows(code, packed, aux, 64, x_bits, rows=rows)
         a, b = f32(y_static)[:, rows], f32(y_ws)[:, rows]
+        assert np.all(np.abs(a - y_ref) <= matmul_tolerance(y_ref, bound))
+        assert np.all(np.abs(b - y_ref) <= matmul_tolerance(y_ref, bound))
         assert np.all(np.abs(a - b) <= matmul_tolerance(b, bound))
         assert wq.device_error() == 0
 

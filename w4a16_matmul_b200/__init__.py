@@ -62,6 +62,7 @@ _SIG = {
                              ctypes.POINTER(_vp)], _i32),
     "wq_gemv_plan_launch": ([_vp, _vp], _i32),
     "wq_gemv_plan_destroy": ([_vp], None),
+    "wq_gemv_plan_set_overlap": ([_vp, _i32], _i32),
     "wq_gemm_workspace_bytes": ([_WP, _i64], _sz),
     "wq_gemm_w4a16": ([_WP, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
     "wq_gemm_w4a16_static": ([_WP, _vp, _i64, _vp, _vp], _i32),
@@ -302,9 +303,12 @@ class GroupedGemv:
     """A prepared grouped GEMV (wq_gemv_plan): the arguments are checked and the kernel is
     chosen once, at construction; each call only enqueues the kernel, on the current stream
     (or `stream`), reading whatever the bound x buffers hold by then. The tensors are kept
-    alive for the plan's lifetime."""
+    alive for the plan's lifetime. overlap=True lets each launch overlap the kernel before it
+    in the stream (wq_gemv_plan_set_overlap): only where that kernel does not write the
+    weights."""
 
-    def __init__(self, ws: list[PackedWeight], xs: list[torch.Tensor], ys: list[torch.Tensor]):
+    def __init__(self, ws: list[PackedWeight], xs: list[torch.Tensor], ys: list[torch.Tensor],
+                 overlap: bool = False):
         if not (len(ws) == len(xs) == len(ys)):
             raise ValueError("ws, xs and ys must have the same length")
         for x in xs:
@@ -319,6 +323,11 @@ class GroupedGemv:
         yp = (_vp * self.cnt)(*[y.data_ptr() for y in ys])
         self._plan = _vp(None)
         _check(_lib.wq_gemv_plan_create(arr, xp, yp, self.cnt, self.batch, ctypes.byref(self._plan)))
+        if overlap:
+            self.set_overlap(True)
+
+    def set_overlap(self, on: bool) -> None:
+        _check(_lib.wq_gemv_plan_set_overlap(self._plan, 1 if on else 0))
 
     def __call__(self, stream=None) -> None:
         s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
@@ -352,6 +361,17 @@ def gemm(w: PackedWeight, x: torch.Tensor, out: torch.Tensor | None = None,
     d = w.desc()
     _check(_lib.wq_gemm_w4a16(ctypes.byref(d), _ptr(x), m, _ptr(y), _ptr(workspace),
                               need, _stream(x)))
+    return y
+
+
+def gemm_static(w: PackedWeight, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """gemm() with its scratch in the library's static device array (wq_gemm_w4a16_static):
+    no workspace is allocated for the call."""
+    _cuda(x, torch.bfloat16, "x")
+    m = x.shape[0]
+    y = out if out is not None else torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device)
+    d = w.desc()
+    _check(_lib.wq_gemm_w4a16_static(ctypes.byref(d), _ptr(x), m, _ptr(y), _stream(x)))
     return y
 
 

@@ -450,6 +450,14 @@ wq_status wq_gemv_plan_launch(wq_gemv_plan plan, wq_stream stream) {
     return gemv_plan_launch(plan, (cudaStream_t)stream);
 }
 
+wq_status wq_gemv_plan_set_overlap(wq_gemv_plan plan, int32_t enable) {
+    g_last_error[0] = 0;
+    if (!plan) return fail(WQ_EINVAL, "plan is NULL");
+    if (enable != 0 && enable != 1) return fail(WQ_EINVAL, "enable must be 0 or 1, got %d", enable);
+    gemv_plan_set_overlap(plan, enable == 1);
+    return WQ_OK;
+}
+
 void wq_gemv_plan_destroy(wq_gemv_plan plan) {
     if (plan) gemv_plan_free(plan);
 }

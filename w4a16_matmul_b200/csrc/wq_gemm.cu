@@ -514,12 +514,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     for (int j = 0; j < 16; ++j) {
                         const int m = m0 + c0 + j;
                         if (m < M) {
+                            // LUT16: the activation row was scaled by 2^e; undo it (exact)
+                            const float val = LU ? __uint_as_float(v[j]) * reinterpret_cast<const float*>(scale)[m]
+                                                 : __uint_as_float(v[j]);
                             if (PARTIAL)                 // [split][tile of the launch][BN][BM]
                                 ((float*)out)[(((size_t)blockIdx.y * gridDim.x + blockIdx.x) * BN + c0 + j) * BM +
-                                              (n - n0)] = __uint_as_float(v[j]);
+                                              (n - n0)] = val;
                             else
-                                ((uint16_t*)out)[(size_t)m * N + n] =
-                                    (uint16_t)float_to_bf16_bits(__uint_as_float(v[j]));
+                                ((uint16_t*)out)[(size_t)m * N + n] = (uint16_t)float_to_bf16_bits(val);
                         }
                     }
                 }
@@ -555,14 +557,32 @@ splitk_reduce_kernel(const float* __restrict__ part, int splits, int ntl, int ti
     y[(size_t)m * N + n] = (uint16_t)float_to_bf16_bits(v);
 }
 
-// Activations for the LUT16 product: bf16 -> fp16, 8 per thread and iteration (exact for |x|
-// in [2^-14, 65504], as the GEMV's staging of LUT16 activations). n8 = elements / 8.
+// Activations for the LUT16 product, one CTA per activation row: the row's largest
+// magnitude picks the power of two 2^e that brings it into [2^15, 2^16) (lut_x_exponent),
+// the row is written as fp16(x * 2^e), and inv[row] = 2^-e for the epilogue. The row is
+// read twice (the second pass mostly from L1/L2). K % 8 == 0.
 __global__ void __launch_bounds__(256)
-x_to_f16_kernel(const uint4* __restrict__ x, uint4* __restrict__ xh, int64_t n8) {
-    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (int64_t)gridDim.x * 256) {
-        const uint4 v = ldg_nc_v4(x + i);
-        xh[i] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                           bf16x2_to_f16x2(v.w));
+x_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xh, float* __restrict__ inv, int K) {
+    __shared__ uint32_t red[8];
+    const int64_t row = blockIdx.x;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+    uint4* hr = reinterpret_cast<uint4*>(xh + row * K);
+    const int n8 = K / 8;
+    uint32_t mx = 0;
+    for (int i = threadIdx.x; i < n8; i += 256) mx = max(mx, bf16x8_max_mag(ldg_v4(xr + i)));
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) mx = max(mx, red[w]);
+    const int e = lut_x_exponent(mx);
+    if (threadIdx.x == 0) inv[row] = pow2_f32(-e);
+    const float s1 = pow2_f32(e >> 1), s2 = pow2_f32(e - (e >> 1));
+    for (int i = threadIdx.x; i < n8; i += 256) {
+        const uint4 v = ldg_v4(xr + i);
+        hr[i] = make_uint4(bf16x2_to_f16x2_scaled(v.x, s1, s2), bf16x2_to_f16x2_scaled(v.y, s1, s2),
+                           bf16x2_to_f16x2_scaled(v.z, s1, s2), bf16x2_to_f16x2_scaled(v.w, s1, s2));
     }
 }
 
@@ -732,11 +752,15 @@ wq_status launch_plan(const Plan& p, const CUtensorMap& tx, const CUtensorMap& t
 // "K-Means量化技术…" §4.1.
 constexpr int64_t kGemvMaxRows = 12;
 
-// Workspace layout: for LUT16 the fp16 copy of the activations [m, k] first (rounded up to
-// 1 KB), then the fp32 partial sums of split launches.
+// Workspace layout: for LUT16 the scaled fp16 copy of the activations [m, k] (rounded up to
+// 1 KB) and the per-row factors 2^-e (fp32 [m], rounded up to 1 KB) first, then the fp32
+// partial sums of split launches.
+size_t lut16_xh_bytes(const wq_weight& w, int64_t m) {
+    return ((size_t)m * (size_t)w.k * 2 + 1023) & ~(size_t)1023;
+}
 size_t lut16_x_bytes(const wq_weight& w, int64_t m) {
     if (w.fmt != WQ_FMT_LUT16) return 0;
-    return ((size_t)m * (size_t)w.k * 2 + 1023) & ~(size_t)1023;
+    return lut16_xh_bytes(w, m) + (((size_t)m * 4 + 1023) & ~(size_t)1023);
 }
 
 size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
@@ -764,13 +788,15 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
     if (need > 0 && (ws == nullptr || ws_bytes < need)) return fail(WQ_EINVAL, "workspace too small");
     const bool lut = w.fmt == WQ_FMT_LUT16;
     const void* xa = x;                    // the activations the MMA reads
+    const float* xinv = nullptr;           // LUT16: per activation row, 2^-e
     if (lut) {
-        const int64_t n8 = m * (int64_t)K / 8;
-        const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, 8 * (int64_t)sm_count());
-        x_to_f16_kernel<<<(unsigned)blocks, 256, 0, s>>>((const uint4*)x, (uint4*)ws, n8);
+        uint16_t* xh = (uint16_t*)ws;
+        float* inv = (float*)((uint8_t*)ws + lut16_xh_bytes(w, m));
+        x_to_f16_kernel<<<(unsigned)m, 256, 0, s>>>(x, xh, inv, K);
         wq_status cs = check_launch("gemm activations to fp16");
         if (cs) return cs;
-        xa = ws;
+        xa = xh;
+        xinv = inv;
         ws = (uint8_t*)ws + lut16_x_bytes(w, m);
     }
     CUtensorMap tx, tp;
@@ -818,7 +844,9 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(WQ_ECUDA, "tensor map for LLOYD8S levels failed (%d)", (int)r);
     }
-    const uint16_t* sc = (const uint16_t*)w.aux;
+    // the kernel's `scale`: DYADIC4 the bf16 scales; LUT16 the activation rows' factors
+    // (the centroids travel through tmap_l); LLOYD8S unused
+    const uint16_t* sc = lut ? (const uint16_t*)xinv : (const uint16_t*)w.aux;
     wq_status st;
 #define WQ_BN(BNV, KBV)                                                                                   \
     st = (w.fmt == WQ_FMT_LLOYD8S) ? launch_plan<BNV, 32, kFLl, 64>(p, tx, tp, tl, sc, y, ws, M, N, K, s) \

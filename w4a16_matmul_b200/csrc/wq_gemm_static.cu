@@ -4,7 +4,12 @@
 // The scratch is a file-scope __device__ array of kStaticScratchBytes, present on every
 // GPU that loads this library until the process exits. Host code cannot use the array's
 // name as a device address (it names a host-side shadow), so the device address is looked
-// up once per device with cudaGetSymbolAddress and cached.
+// up with cudaGetSymbolAddress, with the device current, on the first call on a device, and
+// cached. The cache entry remembers the CUDA context it was resolved in: after
+// cudaDeviceReset the device's next context loads the module again, possibly elsewhere,
+// and the next call resolves the address anew.
+#include <cuda.h>
+
 #include <mutex>
 #include <vector>
 
@@ -17,23 +22,56 @@ constexpr size_t kStaticScratchBytes = WQ_GEMM_STATIC_SCRATCH_BYTES;
 
 static __device__ __align__(256) unsigned char g_gemm_scratch[kStaticScratchBytes];
 
-// Device address of g_gemm_scratch on the current device, resolved on first use.
+// The unique ID of the calling thread's current context (0 if the driver cannot tell).
+unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = (GetCurrent)p;
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = (GetId)p;
+        cudaGetLastError();
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS)
+        return id;
+    return 0;
+}
+
+// Device address of g_gemm_scratch on the current device, resolved on the first use in
+// each context of the device.
 wq_status scratch_address(void** out) {
+    struct Entry {
+        void* addr;
+        unsigned long long ctx;
+    };
     static std::mutex mu;
-    static std::vector<void*> cache;
+    static std::vector<Entry> cache;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(WQ_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    // (0 when no context is current yet: then the lookup, which creates it, runs again)
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lock(mu);
-    if ((int)cache.size() <= dev) cache.resize(dev + 1, nullptr);
-    if (cache[dev] == nullptr) {
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, Entry{nullptr, 0});
+    if (cache[dev].addr == nullptr || cache[dev].ctx != ctx || ctx == 0) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_gemm_scratch);
         if (e != cudaSuccess || p == nullptr)
             return fail(WQ_ECUDA, "cudaGetSymbolAddress(static GEMM scratch): %s", cudaGetErrorString(e));
-        cache[dev] = p;
+        cache[dev] = Entry{p, ctx};
     }
-    *out = cache[dev];
+    *out = cache[dev].addr;
     return WQ_OK;
 }
 

@@ -401,12 +401,15 @@ __device__ __forceinline__ bool step_scales_in_range(const Step<KIND, R>& st) {
 // eight rows one 128-bit shared load phase touches start on distinct banks); inside a row,
 // step s of the chunk at 512 * s, sub-step u at 64 * u, quad position t at 16 * t: the
 // 8 columns 256 * s + 64 * t + 8 * u .. +7 in B-fragment order. Dyadic: bf16 times 2^64,
-// columns paired (0,4), (1,5), (2,6), (3,7); LUT16: fp16 in natural order. Columns at or
-// beyond K are zero. Stages steps [c0, c0 + ns) of all B rows with the whole CTA; returns
-// (dyadic) whether some staged |x| reaches 2^64 or is not finite.
+// columns paired (0,4), (1,5), (2,6), (3,7); LUT16: fp16 in natural order, each batch row's
+// 256 columns of a step times the power of two 2^e that puts their largest magnitude in
+// [2^15, 2^16) (lut_x_exponent), with 2^-e in xf[b * ns + step] for the step's sums (a warp
+// stages exactly one row's step: its 32 consecutive 8-column blocks); LLOYD8S: bf16 in
+// natural order. Columns at or beyond K are zero. Stages steps [c0, c0 + ns) of all B rows
+// with the whole CTA; returns (dyadic) whether some staged |x| reaches 2^64 or is not finite.
 template <int KIND, int THREADS>
 __device__ __forceinline__ bool stage_x(uint8_t* xs, const uint16_t* x, int B, int K, int c0,
-                                        int ns, int rs) {
+                                        int ns, int rs, float* xf) {
     const int per_row = ns * 32;                 // 16-byte blocks of 8 columns
     const int total = B * per_row;
     uint32_t bad = 0;
@@ -430,8 +433,18 @@ __device__ __forceinline__ bool stage_x(uint8_t* xs, const uint16_t* x, int B, i
             const int b = i / per_row, j = i - b * per_row;
             uint4 f;
             if (KIND == kLut16) {
-                f.x = bf16x2_to_f16x2(v[u].x); f.y = bf16x2_to_f16x2(v[u].y);
-                f.z = bf16x2_to_f16x2(v[u].z); f.w = bf16x2_to_f16x2(v[u].w);
+                // the warp's 32 blocks are row b's step j >> 5 (a row is ns * 32 blocks)
+                const int e = lut_x_exponent(__reduce_max_sync(0xFFFFFFFFu, bf16x8_max_mag(v[u])));
+                if ((threadIdx.x & 31) == 0) xf[b * ns + (j >> 5)] = pow2_f32(-e);
+                if (e <= 127) {                         // (warp-uniform) 2^e is a bf16 number
+                    const uint32_t p2 = bf16_pow2_bits(e) * 0x10001u;
+                    f.x = bf16x2_to_f16x2_pow2(v[u].x, p2); f.y = bf16x2_to_f16x2_pow2(v[u].y, p2);
+                    f.z = bf16x2_to_f16x2_pow2(v[u].z, p2); f.w = bf16x2_to_f16x2_pow2(v[u].w, p2);
+                } else {                                // a step whose largest |x| is below 2^-112
+                    const float s1 = pow2_f32(e >> 1), s2 = pow2_f32(e - (e >> 1));
+                    f.x = bf16x2_to_f16x2_scaled(v[u].x, s1, s2); f.y = bf16x2_to_f16x2_scaled(v[u].y, s1, s2);
+                    f.z = bf16x2_to_f16x2_scaled(v[u].z, s1, s2); f.w = bf16x2_to_f16x2_scaled(v[u].w, s1, s2);
+                }
             } else if (KIND == kLloyd8) {
                 f = v[u];                               // bf16 in natural order
             } else {
@@ -487,6 +500,9 @@ constexpr int cta_warps(int wk, int fw) { return wk == 1 ? fw : 4; }
 #ifndef WQ_GEMV_LUT_CAP
 #define WQ_GEMV_LUT_CAP 4
 #endif
+#ifndef WQ_GEMV_LUT_FW
+#define WQ_GEMV_LUT_FW 8
+#endif
 #ifndef WQ_GEMV_LLOYD_CAP
 #define WQ_GEMV_LLOYD_CAP 1
 #endif
@@ -515,6 +531,10 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     const int wr = warp % WR, wk = warp / WR;
     const int tb = (int)blockIdx.x / CL;             // row tile (clusters are CL consecutive CTAs)
     const int crank = (int)blockIdx.x % CL;
+    // A launch made with programmatic stream serialization (a plan with overlap enabled) may
+    // start while the kernel before it finishes: let the next launch do the same with this
+    // one as soon as all of this grid's CTAs are running. (No effect on other launches.)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // ---- which problem / row tile (a tile = the 16*R*WR rows of one CTA) -----------------
     int p = 0;
     if (MAXP > 1) {
@@ -557,11 +577,34 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
         else if (s < full_steps) load_step<KIND, R, true>(st, pb, row0, g, s * 256 + t * 64, N, K);
         else load_step<KIND, R, false>(st, pb, row0, g, s * 256 + t * 64, N, K);
     };
+    // LUT16: each step's staged activations carry their own power of two (stage_x), so a
+    // step's products are summed apart and added to acc times the step's 2^-e per batch row
+    // (exact); the sums below then hold plain values
+    float* xf = reinterpret_cast<float*>(xs + (size_t)B * rs);
     auto run_step = [&](const Step<KIND, R>& st, int s, int c0, bool xbad) {
-        if (KIND >= kLut16 || (!xbad && __all_sync(0xFFFFFFFFu, step_scales_in_range<KIND, R>(st))))
+        if constexpr (KIND == kLut16) {
+            float sacc[R][NB][4];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) sacc[r][nb][0] = sacc[r][nb][1] = sacc[r][nb][2] = sacc[r][nb][3] = 0.f;
+            compute_step_staged<KIND, NB, R>(st, sacc, xs0 + 512 * (s - c0), xs1 + 512 * (s - c0));
+            const int ns = min(cs, steps - c0);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float f = xf[min(8 * nb + 2 * t + h, B - 1) * ns + (s - c0)];
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+#pragma unroll
+                        for (int j = h; j < 4; j += 2) acc[r][nb][j] = fmaf(sacc[r][nb][j], f, acc[r][nb][j]);
+                }
+        } else if (KIND == kLloyd8 || (!xbad && __all_sync(0xFFFFFFFFu, step_scales_in_range<KIND, R>(st)))) {
             compute_step_staged<KIND, NB, R>(st, acc, xs0 + 512 * (s - c0), xs1 + 512 * (s - c0));
-        else
+        } else {
             compute_step_exact<KIND, NB, R>(pb, row0, g, s * 256 + t * 64, N, K, B, acc);
+        }
     };
     // D register buffers in rotation: the bytes of D - 1 steps are in flight while one step
     // computes, and the first D - 1 steps' loads are issued before the activations are
@@ -574,10 +617,14 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
         for (int i = 0; i < D - 1; ++i)
             if (s_lo + wk + i * WK < steps) load(buf[i], s_lo + wk + i * WK);
     }
+    // Activations are read, and outputs written, only once the kernel before this launch has
+    // completed and its writes are visible (immediate without programmatic serialization);
+    // the weight loads above may run beside that kernel's tail.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int c0 = s_lo; c0 < steps; c0 += cs) {
         if (c0 > s_lo) __syncthreads();            // every warp is done with the last chunk
         const int ns = min(cs, steps - c0);
-        const bool xbad = __syncthreads_or(stage_x<KIND, THREADS>(xs, pb.x, B, K, c0, ns, rs)) != 0;
+        const bool xbad = __syncthreads_or(stage_x<KIND, THREADS>(xs, pb.x, B, K, c0, ns, rs, xf)) != 0;
         if (!live) continue;
         const int cend = c0 + ns;
         for (int s0 = c0 + wk; s0 < cend; s0 += D * WK) {
@@ -666,6 +713,7 @@ struct Prepared {
     int cl;                      // cluster size (CTAs splitting one tile's K)
     int threads;
     size_t smem;
+    bool overlap = false;        // launch with programmatic stream serialization
 };
 
 template <int KIND, int NB, int R, int WK, int FW, int MAXP, int CL = 1>
@@ -678,6 +726,7 @@ wq_status prepare_variant(Prepared<MAXP>& pr, const GemvProblem* probs, int tile
     cs = max(unit, cs - cs % unit);
     prm.chunk_steps = min(cs, max_steps);
     pr.smem = (size_t)prm.batch * (512 * prm.chunk_steps + 64);
+    if (KIND == kLut16) pr.smem += (size_t)prm.batch * prm.chunk_steps * sizeof(float);   // step factors
     pr.kern = gemv_kernel<KIND, NB, R, WK, FW, MAXP, CL>;
     pr.tiles = tiles;
     pr.cl = CL;
@@ -710,6 +759,10 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
     // 32-row warps pay off once the activation fragment is shared by more batch rows
     // (measured on the decode sweep: 16-row warps win up to batch 8, 32-row warps at 9..16)
     constexpr int BIGR = (KIND >= kLut16) ? 1 : 2;
+    // warps (of 16 rows) per CTA where a CTA stages its whole K range at batch 1 and in the
+    // cluster split: LUT16 takes 8 (each staged activation chunk, converted to fp16 with its
+    // scale, then serves 128 weight rows; the CTAs per SM halve at the same 128 registers)
+    constexpr int FWL = (KIND == kLut16) ? WQ_GEMV_LUT_FW : 4;
     // full-K CTAs: 4 row warps at batch 1, WQ_GEMV_WARPS_BATCHED above (measured on the
     // decode sweep: 8 warps +9 / +13 / +14 % at batch 4 / 8 / 16, neutral at batch 1)
     if (BIGR == 2 && batch > WQ_GEMV_R2_MIN_BATCH && rows16 >= 12 * sms * 2) {
@@ -717,7 +770,7 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
         return prepare_variant<KIND, NB, BIGR, 1, FWB, MAXP>(pr, probs, tiles_for(16 * FWB * BIGR));
     }
     if (rows16 >= 8 * sms) {
-        if (batch == 1) return prepare_variant<KIND, NB, 1, 1, 4, MAXP>(pr, probs, tiles_for(64));
+        if (batch == 1) return prepare_variant<KIND, NB, 1, 1, FWL, MAXP>(pr, probs, tiles_for(16 * FWL));
         constexpr int FWB = WQ_GEMV_WARPS_BATCHED;
         return prepare_variant<KIND, NB, 1, 1, FWB, MAXP>(pr, probs, tiles_for(16 * FWB));
     }
@@ -737,9 +790,9 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
         int64_t want = (WQ_GEMV_CL_WARPS * sms + 4 * tiles64 - 1) / (4 * tiles64);
         int cl = weights < ((int64_t)1 << 24) ? 1 : want >= 8 ? 8 : want >= 4 ? 4 : want >= 2 ? 2 : 1;
         while (cl > 1 && max_steps / cl < 2) cl >>= 1;
-        if (cl == 8) return prepare_variant<KIND, NB, 1, 1, 4, MAXP, 8>(pr, probs, tiles_for(64));
-        if (cl == 4) return prepare_variant<KIND, NB, 1, 1, 4, MAXP, 4>(pr, probs, tiles_for(64));
-        if (cl == 2) return prepare_variant<KIND, NB, 1, 1, 4, MAXP, 2>(pr, probs, tiles_for(64));
+        if (cl == 8) return prepare_variant<KIND, NB, 1, 1, FWL, MAXP, 8>(pr, probs, tiles_for(16 * FWL));
+        if (cl == 4) return prepare_variant<KIND, NB, 1, 1, FWL, MAXP, 4>(pr, probs, tiles_for(16 * FWL));
+        if (cl == 2) return prepare_variant<KIND, NB, 1, 1, FWL, MAXP, 2>(pr, probs, tiles_for(16 * FWL));
     }
 #endif
     if (rows16 >= 2 * sms) return prepare_variant<KIND, NB, 1, 2, 4, MAXP>(pr, probs, tiles_for(32));
@@ -782,7 +835,7 @@ wq_status prepare(int fmt, int group, const GemvProblem* probs, int count, int b
 
 template <int MAXP>
 wq_status launch_prepared(const Prepared<MAXP>& pr, cudaStream_t s) {
-    if (pr.cl == 1) {
+    if (pr.cl == 1 && !pr.overlap) {
         pr.kern<<<pr.tiles, pr.threads, pr.smem, s>>>(pr.prm);
         return check_launch("gemv");
     }
@@ -791,15 +844,24 @@ wq_status launch_prepared(const Prepared<MAXP>& pr, cudaStream_t s) {
     cfg.blockDim = dim3(pr.threads);
     cfg.dynamicSmemBytes = pr.smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = pr.cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pr.cl > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = pr.cl;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pr.overlap) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, pr.kern, pr.prm) != cudaSuccess) return check_launch("gemv (cluster)");
-    return check_launch("gemv (cluster)");
+    cfg.numAttrs = na;
+    cudaLaunchKernelEx(&cfg, pr.kern, pr.prm);
+    return check_launch(pr.cl > 1 ? "gemv (cluster)" : "gemv");
 }
 
 template <int MAXP>
@@ -827,6 +889,10 @@ wq_status gemv_plan_build(int fmt, int group, const GemvProblem* probs, int coun
     if (st != WQ_OK) { delete pr; return st; }
     *plan = pr;
     return WQ_OK;
+}
+
+void gemv_plan_set_overlap(void* plan, bool on) {
+    static_cast<Prepared<kMaxProblems>*>(plan)->overlap = on;
 }
 
 wq_status gemv_plan_launch(const void* plan, cudaStream_t s) {

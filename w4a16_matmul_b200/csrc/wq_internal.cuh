@@ -54,6 +54,7 @@ wq_status launch_gemv(int fmt, int group, const GemvProblem* probs, int count, i
 wq_status gemv_plan_build(int fmt, int group, const GemvProblem* probs, int count, int batch,
                           void** plan);
 wq_status gemv_plan_launch(const void* plan, cudaStream_t s);
+void gemv_plan_set_overlap(void* plan, bool on);
 void gemv_plan_free(void* plan);
 
 wq_status launch_lloyd_g32(const uint16_t* w, int64_t n, int64_t k, int rounds, uint8_t* codes,
@@ -217,6 +218,56 @@ __device__ __forceinline__ void lut16_lookup4(uint32_t s, const uint32_t* lo, co
 // bf16x2 -> fp16x2 (round to nearest even; exact for |x| in [2^-14, 65504]).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// fp16 activations for the LUT16 products. A bf16 row (or chunk) is converted as x * 2^e,
+// with e chosen from its largest magnitude so that this maximum lands in [2^15, 2^16) (all
+// of bf16's binades map into fp16 that way, and every magnitude of the row down to 2^-17 *
+// 2^-e converts exactly); the fp32 sums are multiplied back by 2^-e. `mag` is the largest
+// bf16 magnitude (bits & 0x7FFF); 0 or a non-finite maximum gives e = 0. e lies in
+// [-113, 148].
+__device__ __forceinline__ int lut_x_exponent(uint32_t mag) {
+    if (mag == 0 || mag >= 0x7F80u) return 0;
+    const int E = (int)(mag >> 7);                 // biased exponent; 0 for subnormals
+    return E ? 142 - E : 117 + __clz(mag & 0x7Fu);
+}
+// 2^e as an fp32 for e in [-149, 127] (subnormal below -126), exact.
+__device__ __forceinline__ float pow2_f32(int e) {
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
+}
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+// The largest magnitude among the eight (finite) bf16 values of v, as bits.
+__device__ __forceinline__ uint32_t bf16x8_max_mag(uint4 v) {
+    const uint32_t m = bf16x2_max(bf16x2_max(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                  bf16x2_max(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16);
+}
+// bf16 pair -> fp16 pair of the values times 2^e for e in [-133, 127] (2^e a bf16 number,
+// given as the pair p2 = (2^e, 2^e)): one exact bf16 product (wherever fp16 can hold the
+// result), then one rounding to fp16.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_pow2(uint32_t v, uint32_t p2) {
+    const uint32_t m = bf16x2_fma(v, p2, 0x80008000u);
+    const float lo = __uint_as_float(m << 16), hi = __uint_as_float(m & 0xFFFF0000u);
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// The bf16 bits of 2^e, e in [-133, 127].
+__device__ __forceinline__ uint32_t bf16_pow2_bits(int e) {
+    return e >= -126 ? (uint32_t)(e + 127) << 7 : 1u << (e + 133);
+}
+// bf16 pair -> fp16 pair of the values times 2^e, one rounding to nearest even (the fp32
+// products by s1 = 2^(e>>1) and s2 = 2^(e - (e>>1)) are exact wherever fp16 can hold the
+// result).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t v, float s1, float s2) {
+    const float lo = __uint_as_float(v << 16) * s1 * s2, hi = __uint_as_float(v & 0xFFFF0000u) * s1 * s2;
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
