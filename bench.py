@@ -156,6 +156,20 @@ def sweep_bytes(mats, batch):
 # our arm
 # ---------------------------------------------------------------------------------------
 
+class nvtx_range:
+    """An NVTX range around one bench phase (visible in nsys/ncu timelines)."""
+
+    def __init__(self, torch, name: str):
+        self.torch, self.name = torch, name
+
+    def __enter__(self):
+        self.torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        self.torch.cuda.nvtx.range_pop()
+        return False
+
+
 def graph_of(torch, fn):
     """fn's launches captured once in a CUDA graph (after one eager call for any one-time
     setup); replaying it keeps per-call host work (argument checks, allocation) out of a
@@ -254,8 +268,9 @@ def run_ours(args):
     regions = REGIONS
     g_warm.replay()
     clocks.start()
-    region_ms = [time_region(torch, stream, g_steps.replay, 1, 0, barrier) / args.steps
-                 for _ in range(regions)]
+    with nvtx_range(torch, "headline: decode sweep GEMV"):
+        region_ms = [time_region(torch, stream, g_steps.replay, 1, 0, barrier) / args.steps
+                     for _ in range(regions)]
     clk = clocks.stop()
     ms = max_over_ranks(float(np.median(region_ms)))
     value = replica_value(world, weight_bytes, ms)
@@ -312,8 +327,9 @@ def run_ours(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     s_in.wait_stream(stream)
-    for e in e2e_steps(args.steps):
-        stream.wait_event(e)
+    with nvtx_range(torch, "e2e: host copies + decode sweep GEMV"):
+        for e in e2e_steps(args.steps):
+            stream.wait_event(e)
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -324,8 +340,9 @@ def run_ours(args):
 
     extras = {}
     if not args.no_extras:
-        extras = run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrier,
-                            max_over_ranks)
+        with nvtx_range(torch, "extras"):
+            extras = run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrier,
+                                max_over_ranks)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -627,9 +644,11 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
     except Exception as e:
         out["quantize_dyadic_layer"] = {"error": repr(e)[:200]}
     if args.extras in ("gemm", "all"):
-        out["prefill_gemm"] = bench_gemm(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks)
+        with nvtx_range(torch, "extras: prefill GEMM"):
+            out["prefill_gemm"] = bench_gemm(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks)
     if args.extras in ("producers", "all"):
-        out.update(bench_producers(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks))
+        with nvtx_range(torch, "extras: producers and codebook GEMVs"):
+            out.update(bench_producers(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks))
     return out
 
 

@@ -302,7 +302,20 @@ wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16
  * or its bytes do not fit packed_bytes (2000 dequant, 2001 pack, 2002 GEMV; the access is
  * skipped in every case). *code receives the code (0 = none). Synchronous (copies three
  * ints from the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_EDATA for
- * inconsistent BF16X or water-filling data, WQ_OK otherwise. */
+ * inconsistent BF16X or water-filling data, WQ_OK otherwise.
+ * The debug build of the library (libwq_debug.so, compiled with -DWQ_DEBUG=1) also checks
+ * on the device what the normal build takes as preconditions, records the first failed
+ * check of each kernel family and reports it here with WQ_EDATA (the kernels never trap):
+ *   3001 / 3010 / 3011 / 3020 / 3030 / 3031  a derived index out of range (dequant scale
+ *        index; GEMV problem and tile, staged chunk; GEMM tile and K range; Lloyd candidate;
+ *        k-means rank);
+ *   3101 / 3102 / 3103  a NaN or Inf weight given to wq_quantize_dyadic / the G32_WARM /
+ *        the KMEANS16 producer;
+ *   3201 / 3202 / 3203  a NaN or Inf activation given to the GEMV / the LUT16 GEMM / the
+ *        other GEMMs;
+ *   3301 / 3302 / 3303  a NaN or Inf latent (wq_fake_quant_ste / wq_gumbel_st_backward) or
+ *        upstream gradient (wq_gumbel_st_backward).
+ * The normal build skips these checks and never reports these codes. */
 wq_status wq_device_error(int32_t* code);
 
 /* ------------------------------------------------------------------------------------ */

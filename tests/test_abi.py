@@ -146,3 +146,19 @@ def test_gemm_workspace_sizes(wq):
             x_bytes = -(-2 * m * kk // 1024) * 1024 + -(-4 * m // 1024) * 1024
             assert ws(wq.FMT_LUT16, 64, nn, kk, m) == ws(wq.FMT_DYADIC4, 64, nn, kk, m) + x_bytes
     assert ws(wq.FMT_LUT16, 64, n, k, 0) == 0
+
+
+def test_debug_library_builds_and_exports_every_header_function(wq):
+    """The WQ_DEBUG build (device-side index and finite-input checks) is the same ABI."""
+    import importlib.util
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("_wq_build", os.path.join(root, "w4a16_matmul_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    path = b.build(debug=True)
+    lib = ctypes.CDLL(path)
+    for n in wq.header_functions():
+        assert hasattr(lib, n), n
+    lib.wq_status_string.restype = ctypes.c_char_p
+    assert lib.wq_status_string(0).decode() == "WQ_OK"

@@ -17,12 +17,15 @@ from dataclasses import dataclass
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libwq.so")
+# WQ_DEBUG=1 selects the debug build of the same library (device-side index and finite-input
+# checks, reported through device_error()); it is built with `build.py --debug`
+DEBUG = os.environ.get("WQ_DEBUG", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libwq_debug.so" if DEBUG else "libwq.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "wq.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python w4a16_matmul_b200/build.py` "
-                      "(nvcc, sm_100a). There is no fallback implementation.")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python w4a16_matmul_b200/build.py"
+                      f"{' --debug' if DEBUG else ''}` (nvcc, sm_100a). There is no fallback implementation.")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

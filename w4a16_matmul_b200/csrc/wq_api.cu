@@ -166,6 +166,19 @@ wq_status wq_device_error(int32_t* code) {
         *code = wf;
         return fail(WQ_EDATA, "water-filling block outside packed_bytes or bad width (code %d)", wf);
     }
+    // debug build: the first failed device-side check of each kernel family
+    wq_status (*readers[])(int32_t*) = {read_debug_dyadic, read_debug_gemv, read_debug_gemm,
+                                        read_debug_lloyd, read_debug_ste};
+    int32_t first = 0;
+    for (auto rd : readers) {
+        int32_t v = 0;
+        if ((st = rd(&v))) return st;
+        if (first == 0) first = v;
+    }
+    if (first != 0) {
+        *code = first;
+        return fail(WQ_EDATA, "a device-side debug check failed (code %d)", first);
+    }
     return WQ_OK;
 }
 

@@ -7,6 +7,8 @@
 #include "wq_internal.cuh"
 
 namespace wq {
+
+WQ_DEBUG_WORD(dyadic)
 namespace {
 
 constexpr int kThreads = 256;
@@ -148,6 +150,7 @@ quantize_dyadic_kernel(const uint4* __restrict__ w, I n_chunks, uint16_t* __rest
         for (int u = 0; u < U; ++u) {
             const I c = c0 + 32 * u + lane;
             v[u] = c < n_chunks ? ldg_nc_v4(w + c) : make_uint4(0, 0, 0, 0);
+            WQ_DCHECK(bf16x8_finite(v[u]), kDbgNonFiniteWeight + 1);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -221,6 +224,7 @@ dequant_dyadic_kernel(const uint32_t* __restrict__ packed, const uint16_t* __res
             p[u] = 0x88888888u;
             sc[u] = 0;
             if (i < n_words) {
+                WQ_DCHECK((i >> gshift) <= ((n_words - 1) >> gshift), kDbgIndex + 1);
                 p[u] = __ldg(packed + i);
                 sc[u] = ldg_u16(scale + (i >> gshift));
             }

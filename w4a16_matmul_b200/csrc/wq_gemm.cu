@@ -39,6 +39,8 @@
 
 namespace wq {
 
+WQ_DEBUG_WORD(gemm)
+
 __device__ int g_device_error;     // 0, or the code of the first expired device wait
 
 namespace {
@@ -280,6 +282,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     const int kt0 = blockIdx.y * kt_per_split;
     const int kt1 = min(KT, kt0 + kt_per_split);
     const int nk = kt1 - kt0;
+    WQ_DCHECK(n0 < N && m0 < M && kt0 < KT && kt1 <= KT, kDbgIndex + 20);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -569,7 +572,11 @@ x_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xh, float
     uint4* hr = reinterpret_cast<uint4*>(xh + row * K);
     const int n8 = K / 8;
     uint32_t mx = 0;
-    for (int i = threadIdx.x; i < n8; i += 256) mx = max(mx, bf16x8_max_mag(ldg_v4(xr + i)));
+    for (int i = threadIdx.x; i < n8; i += 256) {
+        const uint4 v = ldg_v4(xr + i);
+        WQ_DCHECK(bf16x8_finite(v), kDbgNonFiniteActivation + 2);
+        mx = max(mx, bf16x8_max_mag(v));
+    }
     mx = __reduce_max_sync(0xFFFFFFFFu, mx);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
     __syncthreads();
@@ -585,6 +592,15 @@ x_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xh, float
                            bf16x2_to_f16x2_scaled(v.z, s1, s2), bf16x2_to_f16x2_scaled(v.w, s1, s2));
     }
 }
+
+#if WQ_DEBUG
+// Debug build only: the finite-activation check for the formats whose activations reach the
+// MMA by TMA without passing through a kernel of this library first.
+__global__ void __launch_bounds__(256) debug_scan_x_kernel(const uint4* __restrict__ x, int64_t n8) {
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (int64_t)gridDim.x * 256)
+        WQ_DCHECK(bf16x8_finite(ldg_v4(x + i)), kDbgNonFiniteActivation + 3);
+}
+#endif
 
 // ---------------------------------------------------------------------------------------
 // host side
@@ -799,6 +815,15 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
         xinv = inv;
         ws = (uint8_t*)ws + lut16_x_bytes(w, m);
     }
+#if WQ_DEBUG
+    if (!lut) {
+        const int64_t n8 = m * (int64_t)K / 8;
+        debug_scan_x_kernel<<<(unsigned)std::min<int64_t>((n8 + 255) / 256, 4 * (int64_t)sm_count()), 256, 0, s>>>(
+            (const uint4*)x, n8);
+        wq_status cs = check_launch("gemm debug activation scan");
+        if (cs) return cs;
+    }
+#endif
     CUtensorMap tx, tp;
     {
         cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};

@@ -41,6 +41,8 @@
 #include "wq_internal.cuh"
 
 namespace wq {
+
+WQ_DEBUG_WORD(gemv)
 namespace {
 
 constexpr int kMaxProblems = WQ_GEMV_MAX_GROUPED;
@@ -424,6 +426,7 @@ __device__ __forceinline__ bool stage_x(uint8_t* xs, const uint16_t* x, int B, i
                 const int b = i / per_row, j = i - b * per_row;
                 const int col = c0 * 256 + 8 * j;
                 if (col < K) v[u] = ldg_v4(x + (size_t)b * K + col);
+                WQ_DCHECK(b < B && bf16x8_finite(v[u]), kDbgNonFiniteActivation + 1);
             }
         }
 #pragma unroll
@@ -545,6 +548,7 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
         }
         p = lo;
     }
+    WQ_DCHECK(p >= 0 && p < prm.count && tb >= prm.tile_start[p] && tb < prm.tile_start[p + 1], kDbgIndex + 10);
     const GemvProblem& pb = prm.prob[p];
     const int N = pb.n, K = pb.k, B = prm.batch;
     const int row0 = (tb - prm.tile_start[p]) * (16 * R * WR) + wr * 16 * R;
@@ -624,6 +628,7 @@ gemv_kernel(const __grid_constant__ GemvParams<MAXP> prm) {
     for (int c0 = s_lo; c0 < steps; c0 += cs) {
         if (c0 > s_lo) __syncthreads();            // every warp is done with the last chunk
         const int ns = min(cs, steps - c0);
+        WQ_DCHECK(ns >= 1 && ns <= cs && c0 + ns <= all_steps, kDbgIndex + 11);
         const bool xbad = __syncthreads_or(stage_x<KIND, THREADS>(xs, pb.x, B, K, c0, ns, rs, xf)) != 0;
         if (!live) continue;
         const int cend = c0 + ns;

@@ -13,6 +13,73 @@
 namespace wq {
 
 // ---------------------------------------------------------------------------------------
+// Debug build (-DWQ_DEBUG=1, libwq_debug.so): device-side checks of derived indices and of
+// the finite-input precondition. A failed check records its code in the translation
+// unit's debug word (the first code wins), skips nothing else and never traps; the host
+// reads and clears the words through wq_device_error (WQ_EDATA). In the normal build the
+// checks compile to nothing and the readers report 0.
+// ---------------------------------------------------------------------------------------
+#ifndef WQ_DEBUG
+#define WQ_DEBUG 0
+#endif
+enum : int {
+    kDbgIndex = 3000,              // + site: a derived index outside its range
+    kDbgNonFiniteWeight = 3100,    // + site: a NaN / Inf weight reached a producer
+    kDbgNonFiniteActivation = 3200,  // + site: a NaN / Inf activation reached a consumer
+    kDbgNonFiniteLatent = 3300,    // + site: a NaN / Inf latent or gradient reached the STE kernels
+};
+#if WQ_DEBUG
+// Defines this translation unit's debug word, debug_fail() and the reader read_debug_<name>.
+#define WQ_DEBUG_WORD(name)                                                                   \
+    static __device__ int g_debug_word;                                                       \
+    __device__ __forceinline__ void debug_fail(int code) { atomicCAS(&g_debug_word, 0, code); } \
+    wq_status read_debug_##name(int32_t* code) {                                              \
+        int v = 0;                                                                            \
+        if (cudaMemcpyFromSymbol(&v, g_debug_word, sizeof v) != cudaSuccess)                  \
+            return fail(WQ_ECUDA, "reading the debug word of " #name);                         \
+        if (v != 0) {                                                                         \
+            const int zero = 0;                                                               \
+            cudaMemcpyToSymbol(g_debug_word, &zero, sizeof zero);                             \
+        }                                                                                     \
+        *code = v;                                                                            \
+        return WQ_OK;                                                                         \
+    }
+#define WQ_DCHECK(cond, code)                 \
+    do {                                      \
+        if (!(cond)) debug_fail(code);        \
+    } while (0)
+#else
+#define WQ_DEBUG_WORD(name)                          \
+    wq_status read_debug_##name(int32_t* code) {     \
+        *code = 0;                                   \
+        return WQ_OK;                                \
+    }
+#define WQ_DCHECK(cond, code) \
+    do {                      \
+    } while (0)
+#endif
+wq_status read_debug_dyadic(int32_t* code);
+wq_status read_debug_gemv(int32_t* code);
+wq_status read_debug_gemm(int32_t* code);
+wq_status read_debug_lloyd(int32_t* code);
+wq_status read_debug_ste(int32_t* code);
+
+// True when none of the eight bf16 values of v is a NaN or an infinity.
+__host__ __device__ __forceinline__ bool bf16x8_finite(uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ok = ok && (w[i] & 0x7F80u) != 0x7F80u && (w[i] & 0x7F800000u) != 0x7F800000u;
+    return ok;
+}
+
+// True when none of the four fp32 values (bits) of v is a NaN or an infinity.
+__host__ __device__ __forceinline__ bool f32x4_finite(uint4 v) {
+    return (v.x & 0x7F800000u) != 0x7F800000u && (v.y & 0x7F800000u) != 0x7F800000u &&
+           (v.z & 0x7F800000u) != 0x7F800000u && (v.w & 0x7F800000u) != 0x7F800000u;
+}
+
+// ---------------------------------------------------------------------------------------
 // Host-side status plumbing (wq_api.cu)
 // ---------------------------------------------------------------------------------------
 

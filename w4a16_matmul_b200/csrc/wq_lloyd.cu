@@ -28,6 +28,8 @@
 #include "wq_internal.cuh"
 
 namespace wq {
+
+WQ_DEBUG_WORD(lloyd)
 namespace {
 
 constexpr int kCand = 112;
@@ -206,6 +208,7 @@ lloyd_g32_kernel(const uint16_t* __restrict__ w, int64_t n_groups, int rounds,
 
     for (int64_t g = (int64_t)blockIdx.x * kWarps + wi; g < n_groups; g += warps_total) {
         const uint32_t hb = w[g * 32 + lane];
+        WQ_DCHECK((hb & 0x7F80u) != 0x7F80u, kDbgNonFiniteWeight + 2);
         const float wf = bf16_bits_to_float(hb);
         const float af = fabsf(wf);
         const int sgn = wf < 0.f ? 1 : 0;                 // -0.0 counts as positive
@@ -297,6 +300,7 @@ lloyd_g32_kernel(const uint16_t* __restrict__ w, int64_t n_groups, int rounds,
             unsigned m = __ballot_sync(0xFFFFFFFFu, cl < kCand && !(s_lo[wi][cl] > thr));
             while (m) {
                 const int cc = base + __ffs(m) - 1;
+                WQ_DCHECK(cc < kCand, kDbgIndex + 30);
                 m &= m - 1;
                 double Lc[8];
                 const double mse = candidate_mse64(cc, a, gmax, lane, ct, Lc);
@@ -386,6 +390,8 @@ kmeans16_kernel(const uint16_t* __restrict__ w, int64_t n_blocks, int rounds,
     const int64_t warps_total = (int64_t)gridDim.x * kWarps;
     const int T = rounds + 1;
     for (int64_t g = (int64_t)blockIdx.x * kWarps + wi; g < n_blocks; g += warps_total) {
+        WQ_DCHECK((w[g * 64 + lane] & 0x7F80u) != 0x7F80u && (w[g * 64 + 32 + lane] & 0x7F80u) != 0x7F80u,
+                  kDbgNonFiniteWeight + 3);
         const double v0 = (double)bf16_bits_to_float(w[g * 64 + lane]);
         const double v1 = (double)bf16_bits_to_float(w[g * 64 + 32 + lane]);
         s_v[wi][lane] = v0;
@@ -399,6 +405,7 @@ kmeans16_kernel(const uint16_t* __restrict__ w, int64_t n_blocks, int rounds,
             r0 += (vm < v0) || (vm == v0 && m < i0);
             r1 += (vm < v1) || (vm == v1 && m < i1);
         }
+        WQ_DCHECK(r0 < 64 && r1 < 64 && r0 != r1, kDbgIndex + 31);
         if ((r0 & 3) == 2) s_c[wi][r0 >> 2] = v0;
         if ((r1 & 3) == 2) s_c[wi][r1 >> 2] = v1;
         __syncwarp();

@@ -29,6 +29,8 @@
 #include "wq_internal.cuh"
 
 namespace wq {
+
+WQ_DEBUG_WORD(ste)
 namespace {
 
 constexpr int kThreads = 256;
@@ -85,6 +87,7 @@ fake_quant_ste_kernel(const float4* __restrict__ z, const uint16_t* __restrict__
             sc[u] = 0;
             if (i < n8) {
                 const uint4 va = ldg_nc_v4(z + 2 * i), vb = ldg_nc_v4(z + 2 * i + 1);
+                WQ_DCHECK(f32x4_finite(va) && f32x4_finite(vb), kDbgNonFiniteLatent + 1);
                 a[u] = make_float4(__uint_as_float(va.x), __uint_as_float(va.y), __uint_as_float(va.z), __uint_as_float(va.w));
                 b[u] = make_float4(__uint_as_float(vb.x), __uint_as_float(vb.y), __uint_as_float(vb.z), __uint_as_float(vb.w));
                 sc[u] = ldg_u16(scale + i / per_group);
@@ -250,6 +253,8 @@ gumbel_st_backward_kernel(const float4* __restrict__ z, const uint16_t* __restri
         if (i < n8) {
             const uint4 za = ldg_nc_v4(z + 2 * i), zb = ldg_nc_v4(z + 2 * i + 1);
             const uint4 ga = ldg_nc_v4(gq + 2 * i), gb = ldg_nc_v4(gq + 2 * i + 1);
+            WQ_DCHECK(f32x4_finite(za) && f32x4_finite(zb), kDbgNonFiniteLatent + 2);
+            WQ_DCHECK(f32x4_finite(ga) && f32x4_finite(gb), kDbgNonFiniteLatent + 3);
             const float s = bf16_bits_to_float(ldg_u16(scale + i / per_group));
             const bool fast = s >= 0x1p-96f && s <= 0x1p96f;
             const float c8 = fast ? 8.0f * rcp_fast(s) : 0.0f;
