@@ -179,6 +179,46 @@ def test_gemm_last_wave_split(wq):
     assert np.all(np.abs(got - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
 
 
+@pytest.mark.parametrize("fmt", ["dyadic", "lloyd8s", "lut16"])
+@pytest.mark.parametrize("m", [48, 128, 300])
+def test_gemm_split_k_across_many_ctas(wq, fmt, m):
+    """8 weight-row tiles and K = 8192: the plans split K across many CTAs (narrow 128 x 64
+    tiles at m = 48, 128 x 128 tiles with 128-column stages at m = 128, 128 x 256 at
+    m = 300), so each tile's sum is assembled from many fp32 partials in the workspace.
+    Every weight row of sampled activation rows against the oracle, for each weight format,
+    and the static-scratch entry point the same where its scratch holds the partials."""
+    n, k = 1024, 8192
+    if fmt == "dyadic":
+        pw, packed, aux = _weight(wq, n, k, 64, 50 + m)
+        code, group = oracle.DYADIC4, 64
+    elif fmt == "lloyd8s":
+        g = np.random.default_rng(m)
+        codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+        aux = np.sort(np.abs(g.standard_normal((n, k // 32, 8))) * 0.02, -1).astype(np.float32)
+        packed = oracle.pack(codes)
+        pw = wq.PackedWeight(wq.FMT_LLOYD8S, 32, n, k, to_dev(packed), torch.from_numpy(aux).cuda())
+        code, group = oracle.LLOYD8S, 32
+    else:
+        pw, packed, aux = _lut16(wq, n, k, m)
+        code, group = oracle.LUT16, 64
+    assert wq.gemm_workspace_bytes(pw, m) > 0
+    x_bits = workloads.activations(m, k, workloads.PREFILL, 70 + m)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    try:
+        ys = wq.gemm_static(pw, to_dev_bits(x_bits))
+    except wq.WqError as e:          # LUT16 at m = 300: activations + partials pass 16 MiB
+        assert e.status == wq.WQ_EINVAL and "static scratch" in str(e)
+        ys = None
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+    ms = np.arange(0, m, 7)
+    y_ref, bound = oracle.matmul_rows(code, packed, aux, group, x_bits[ms])
+    tol = matmul_tolerance(y_ref, bound, TOL)
+    assert np.all(np.abs(f32(y)[ms] - y_ref) <= tol)
+    if ys is not None:
+        assert np.all(np.abs(f32(ys)[ms] - y_ref) <= tol)
+
+
 def _lut16(wq, n, k, seed):
     g = np.random.default_rng(seed)
     codes = g.integers(0, 16, (n, k), dtype=np.uint8)
