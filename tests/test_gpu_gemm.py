@@ -219,6 +219,37 @@ def test_gemm_split_k_across_many_ctas(wq, fmt, m):
         assert np.all(np.abs(f32(ys)[ms] - y_ref) <= tol)
 
 
+@pytest.mark.parametrize("fmt", ["dyadic", "lloyd8s", "lut16"])
+@pytest.mark.parametrize("m", [768, 700])
+def test_gemm_384_row_activation_tiles(wq, fmt, m):
+    """74 weight-row tiles: 384-row activation tiles need one wave where 256-row ones need
+    two (at most 0.7 times the waves), so the plan takes them (two N = 192 MMAs per reconstructed weight slot, the
+    activation tile loaded as two 192-row boxes; at m = 700 the second box of the last tile
+    runs past the last row). Sampled activation rows, every weight row, against the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n, k = 128 * (sms // 2), 1024
+    if fmt == "dyadic":
+        pw, packed, aux = _weight(wq, n, k, 64, 90 + m)
+        code, group = oracle.DYADIC4, 64
+    elif fmt == "lloyd8s":
+        g = np.random.default_rng(m + 1)
+        codes = g.integers(0, 16, (n, k), dtype=np.uint8)
+        aux = np.sort(np.abs(g.standard_normal((n, k // 32, 8))) * 0.02, -1).astype(np.float32)
+        packed = oracle.pack(codes)
+        pw = wq.PackedWeight(wq.FMT_LLOYD8S, 32, n, k, to_dev(packed), torch.from_numpy(aux).cuda())
+        code, group = oracle.LLOYD8S, 32
+    else:
+        pw, packed, aux = _lut16(wq, n, k, m + 2)
+        code, group = oracle.LUT16, 64
+    x_bits = workloads.activations(m, k, workloads.PREFILL, 95 + m)
+    y = wq.gemm(pw, to_dev_bits(x_bits))
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+    ms = np.concatenate([np.arange(0, m, 37), [191, 192, 383, 384, 575, 576, m - 1]])
+    y_ref, bound = oracle.matmul_rows(code, packed, aux, group, x_bits[ms])
+    assert np.all(np.abs(f32(y)[ms] - y_ref) <= matmul_tolerance(y_ref, bound, TOL))
+
+
 def _lut16(wq, n, k, seed):
     g = np.random.default_rng(seed)
     codes = g.integers(0, 16, (n, k), dtype=np.uint8)

@@ -260,6 +260,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             void* __restrict__ out, int M, int N, int K, int kt_per_split, int grid_n, int tile0) {
     using S = Smem<BN, F, KB>;
     constexpr bool LL = F == kFLl, LU = F == kFLu;
+    constexpr int XBOXES = BN > 256 ? 2 : 1;        // TMA boxes span at most 256 rows
     constexpr int STAGES = S::STAGES;
     constexpr int RW = rw_for(BN);
     extern __shared__ uint8_t smem_raw[];
@@ -327,7 +328,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 const int kt = kt0 + i;
 #pragma unroll
                 for (int j = 0; j < KB / 64; ++j)
-                    tma_load_2d(stage_b(s) + j * BN * 128, &tmap_x, kt * KB + 64 * j, m0, &full_tma[s]);
+#pragma unroll
+                    for (int h = 0; h < XBOXES; ++h)   // activation boxes of BN / XBOXES rows
+                        tma_load_2d(stage_b(s) + j * BN * 128 + h * (BN / XBOXES) * 128, &tmap_x,
+                                    kt * KB + 64 * j, m0 + h * (BN / XBOXES), &full_tma[s]);
                 tma_load_2d(stage_p(s), &tmap_p, kt * (KB / 2), n0, &full_tma[s]);
                 // both tables hold KB / 4 elements of a row per stage
                 if (F != kFDy) tma_load_2d(stage_l(s), &tmap_l, kt * (KB / 4), n0, &full_tma[s]);
@@ -338,7 +342,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         if (lane == 0) {
             // fp32 accumulator; A and B both bf16 (format 1), or both fp16 (format 0) for LUT16
             constexpr uint32_t ab = LU ? 0u : (1u << 7) | (1u << 10);
-            constexpr uint32_t idesc = (1u << 4) | ab | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+            // BN = 384: two MMAs of N = 192 per K step read the same weight slot, into the two
+            // halves of the accumulator, from the two halves of the activation tile
+            constexpr int NH = BN > 256 ? 2 : 1, NM = BN / NH;
+            constexpr uint32_t idesc = (1u << 4) | ab | ((uint32_t)(NM >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
             int s = 0, a = 0;
             uint32_t aph = 0;
             for (int i = 0; i < nk; ++i) {
@@ -349,7 +356,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 #pragma unroll
                 for (int k = 0; k < KB / 16; ++k) {  // 16 values of K: 8 A columns, +2 in B descriptor units
                     const uint64_t db = sw128_desc(smem_u32(stage_b(s) + (k / 4) * BN * 128));
-                    umma_f16_ts(tmem, ta + 8u * (uint32_t)k, db + 2 * (k % 4), idesc, (i > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        // descriptor address units are 16 bytes: + NM rows of 128 bytes
+                        const uint64_t dbh = db + (uint64_t)(h * NM * 128 / 16);
+                        umma_f16_ts(tmem + (uint32_t)(h * NM), ta + 8u * (uint32_t)k, dbh + 2 * (k % 4), idesc,
+                                    (i > 0 || k > 0) ? 1u : 0u);
+                    }
                 }
                 umma_commit(&empty[s]);           // fire once these MMAs have read the stage ...
                 if constexpr (!S::COUPLED) umma_commit(&slot_free[a]);   // ... and the slot
@@ -639,6 +652,9 @@ constexpr size_t kTailScratchBytes = (size_t)16 << 20;
 #ifndef WQ_GEMM_KB128
 #define WQ_GEMM_KB128 1
 #endif
+#ifndef WQ_GEMM_BN384
+#define WQ_GEMM_BN384 1
+#endif
 
 Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt) {
     Plan p;
@@ -650,6 +666,20 @@ Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt) {
     // narrower tiles run out of (measured: BN 128 / 192 at 0.5-0.9x of BN 256 throughput even
     // where they leave fewer SMs idle in the last wave).
     p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= WQ_GEMM_BN128_MAX ? 128 : 256;
+    // 384-row activation tiles (two N = 192 MMAs from each reconstructed weight slot) where
+    // they need at most 0.7 times the waves of 256-row ones. Each weight is rebuilt once per
+    // tile either way, but a 384-row tile takes about 1.35 times as long (4 pipeline stages
+    // instead of 6, and shared memory near its bandwidth: the TMA writes plus the MMA's reads
+    // of the activation tile), so fewer waves pay only where they are much fewer. Measured:
+    // 11008 x 4096 at m = 4096 (7 waves instead of 10) 353 -> 337 us; 4096 x 11008 at
+    // m = 4096 (3 instead of 4) 339 -> 344 us and 11008 x 4096 at m = 2048 (4 instead of 5)
+    // 179 -> 194 us, which keep 256 rows.
+    if (WQ_GEMM_BN384 && p.bn == 256) {
+        const int64_t gn = (N + BM - 1) / BM;
+        const int64_t w256 = (gn * ((M + 255) / 256) + sms - 1) / sms;
+        const int64_t w384 = (gn * ((M + 383) / 384) + sms - 1) / sms;
+        if (gn * ((M + 383) / 384) >= sms && 10 * w384 <= 7 * w256) p.bn = 384;
+    }
     // 128-column stages for 128-wide activation tiles where K allows: there they halve the
     // per-stage bookkeeping of the reconstruction, which this m is bound by (measured 1.4x at
     // m = 128); the 256-wide tiles keep 64-column stages, whose finer ring overlaps better
@@ -828,7 +858,8 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
     {
         cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
         cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        cuuint32_t box[2] = {64, (cuuint32_t)p.bn};        // one 128-byte swizzle row wide
+        // one 128-byte swizzle row wide, at most 256 rows (a 384-row tile loads two boxes)
+        cuuint32_t box[2] = {64, (cuuint32_t)(p.bn > 256 ? p.bn / 2 : p.bn)};
         cuuint32_t es[2] = {1, 1};
         CUresult r = enc(&tx, lut ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                          (void*)xa, dims, strides, box, es,
@@ -885,6 +916,7 @@ wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t
         case 128:
             if (p.kb == 128) { WQ_BN(128, 128); } else { WQ_BN(128, 64); }
             break;
+        case 384: WQ_BN(384, 64); break;
         default: WQ_BN(256, 64); break;
     }
 #undef WQ_BN
