@@ -289,8 +289,25 @@ wf_dequant_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, cons
     }
 }
 
-// GEMV on the water-filled weights: y[i, r] = sum_c Wdeq[r, c] x[i, c] for NB activation
-// rows, Wdeq rebuilt exactly as wf_dequant_kernel does (bf16), products and sums in fp32.
+// Larger batches: y[i, r] = sum_c Wdeq[r, c] x[i, c] for up to 16 activation rows in one
+// pass over the weights, Wdeq rebuilt exactly as wf_dequant_kernel does (bf16), products on
+// the tensor cores (mma.sync m16n8k16, fp32 accumulation).
+//   * A warp owns 16 weight rows; step = one 64-weight block column. Lane (g, t) decodes
+//     words t and t + 4 (codes 8t .. 8t + 7 and 32 + 8t .. 32 + 8t + 7) of the blocks of rows
+//     g and g + 8. Pair u of word t (codes 8t + 2u, + 1) is its A operand at k-slots 2t, 2t + 1
+//     of the step's MMA u, pair u of word t + 4 at k-slots 2t + 8, 2t + 9: every lane's A
+//     comes from its own words, and the 4 MMAs of a step cover the block's 64 columns.
+//   * The B operand is then x[g][block + 8t .. + 7] and x[g][block + 32 + 8t .. + 7] in
+//     natural order (word u of each 16-byte load for MMA u), read through L1 (every warp
+//     of the SM reads the same activations).
+//   * The 8 warps of a CTA take every 8th block of the same 16 rows and add up their sums
+//     in shared memory at the end.
+//   * Software pipeline: a block's metadata is read two steps ahead, its packed words and
+//     activations one step ahead.
+// A block whose width or offset is inconsistent with the buffer is reported (2002) and
+// contributes nothing.
+// Small batches: y[i, r] = sum_c Wdeq[r, c] x[i, c] for NB <= 8 activation
+// rows on the CUDA cores, Wdeq rebuilt exactly as wf_dequant_kernel does (bf16), products and sums in fp32.
 // One warp per weight row; 8 lanes per 64-weight block (lane t: columns 8t .. 8t + 7, the b
 // bytes at the block's offset + b t), 4 blocks per step, 8 steps per chunk of 32 blocks.
 // A chunk's widths, offsets and scales are read one block per lane, checked, and handed to
@@ -298,7 +315,7 @@ wf_dequant_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, cons
 // ahead and the packed words one chunk ahead, so that a chunk's loads are in flight while
 // the previous chunk is decoded. A block whose width or offset is inconsistent with the
 // buffer is reported and contributes nothing.
-constexpr int kGemvWarps = 8;
+constexpr int kFmaWarps = 8;
 
 // One chunk's packed words and, per step, the block width (0: nothing) and scale bits.
 struct WfChunk {
@@ -308,12 +325,12 @@ struct WfChunk {
 };
 
 template <int NB>
-__global__ void __launch_bounds__(32 * kGemvWarps)
-wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const uint16_t* __restrict__ scale,
+__global__ void __launch_bounds__(32 * kFmaWarps)
+wf_gemv_fma_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const uint16_t* __restrict__ scale,
                const uint8_t* __restrict__ width, const uint32_t* __restrict__ blk_off, int n, int k,
                const uint16_t* __restrict__ x, uint16_t* __restrict__ y) {
     const int lane = threadIdx.x & 31;
-    const int row = blockIdx.x * kGemvWarps + (threadIdx.x >> 5);
+    const int row = blockIdx.x * kFmaWarps + (threadIdx.x >> 5);
     if (row >= n) return;                        // the whole warp leaves; no CTA-wide barrier
     const int kb = k >> 6;
     const int nch = (kb + 31) >> 5;
@@ -397,6 +414,147 @@ wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const u
     }
 }
 
+#ifndef WQ_WF_WARPS
+#define WQ_WF_WARPS 4                  // warps per CTA (splitting the row group's blocks)
+#endif
+#ifndef WQ_WF_BPS
+#define WQ_WF_BPS 1                    // blocks per warp step (loads issued together)
+#endif
+constexpr int kWfWarps = WQ_WF_WARPS;
+constexpr int kWfBps = WQ_WF_BPS;
+
+struct WfMeta {
+    int b[2];            // widths of rows g, g + 8 (0: none)
+    uint32_t off[2];
+    uint32_t sb[2];
+};
+
+template <int NB>
+__global__ void __launch_bounds__(32 * kWfWarps)
+wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const uint16_t* __restrict__ scale,
+               const uint8_t* __restrict__ width, const uint32_t* __restrict__ blk_off, int n, int k,
+               const uint16_t* __restrict__ x, int batch, uint16_t* __restrict__ y) {
+    __shared__ float red[kWfWarps][NB][4][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int kb = k >> 6;
+    const int row[2] = {(int)blockIdx.x * 16 + g, (int)blockIdx.x * 16 + g + 8};
+    const uint16_t* xr[2] = {x + (size_t)min(g, batch - 1) * k, x + (size_t)min(g + 8, batch - 1) * k};
+    constexpr int STRIDE = kWfWarps * kWfBps;     // blocks between a warp's steps
+
+    auto meta = [&](int blk, WfMeta& m) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            m.b[h] = 0; m.off[h] = 0; m.sb[h] = 0;
+            if (blk < kb && row[h] < n) {
+                const int64_t i = (int64_t)row[h] * kb + blk;
+                m.b[h] = __ldg(width + i);
+                m.off[h] = ldg_u32(blk_off + i);
+                m.sb[h] = ldg_u16(scale + i);
+                if (!wf_block_ok(m.b[h], m.off[h], packed_bytes)) {
+                    report(2002);
+                    m.b[h] = 0;
+                }
+            }
+        }
+    };
+    auto words = [&](const WfMeta& m, unsigned long long (&v)[2][2]) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int b = m.b[h];
+            v[h][0] = b ? wf_bytes(packed, (int64_t)m.off[h] + b * t, b) : 0ull;
+            v[h][1] = b ? wf_bytes(packed, (int64_t)m.off[h] + b * (t + 4), b) : 0ull;
+        }
+    };
+    auto acts = [&](int blk, uint4 (&xa)[NB][2]) {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            xa[nb][0] = xa[nb][1] = make_uint4(0, 0, 0, 0);
+            if (blk < kb) {
+                xa[nb][0] = __ldg(reinterpret_cast<const uint4*>(xr[nb] + blk * 64 + 8 * t));
+                xa[nb][1] = __ldg(reinterpret_cast<const uint4*>(xr[nb] + blk * 64 + 32 + 8 * t));
+            }
+        }
+    };
+
+    float acc[NB][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+
+    // step = kWfBps blocks kWfWarps apart, starting at block warp; pipeline: a step's
+    // metadata two steps ahead, its words and activations one step ahead
+    WfMeta m0[kWfBps], m1[kWfBps];
+    unsigned long long v0[kWfBps][2][2];
+    uint4 x0[kWfBps][NB][2];
+#pragma unroll
+    for (int q = 0; q < kWfBps; ++q) {
+        meta(warp + q * kWfWarps, m0[q]);
+        words(m0[q], v0[q]);
+        acts(warp + q * kWfWarps, x0[q]);
+        meta(warp + q * kWfWarps + STRIDE, m1[q]);
+    }
+    for (int blk = warp; blk < kb; blk += STRIDE) {
+        unsigned long long v1[kWfBps][2][2];
+        uint4 x1[kWfBps][NB][2];
+        WfMeta m2[kWfBps];
+#pragma unroll
+        for (int q = 0; q < kWfBps; ++q) {
+            words(m1[q], v1[q]);
+            acts(blk + q * kWfWarps + STRIDE, x1[q]);
+            meta(blk + q * kWfWarps + 2 * STRIDE, m2[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < kWfBps; ++q) {
+            // decode rows g, g + 8 (4 bf16 pairs per word), 4 MMAs per 8 batch rows
+            uint32_t a[2][2][4];                 // [row][word][pair]
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    if (m0[q].b[h]) {
+                        wf_decode8(v0[q][h][w], m0[q].b[h], m0[q].sb[h], a[h][w]);
+                    } else {
+                        a[h][w][0] = a[h][w][1] = a[h][w][2] = a[h][w][3] = 0u;
+                    }
+                }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const uint32_t xb0[4] = {x0[q][nb][0].x, x0[q][nb][0].y, x0[q][nb][0].z, x0[q][nb][0].w};
+                const uint32_t xb1[4] = {x0[q][nb][1].x, x0[q][nb][1].y, x0[q][nb][1].z, x0[q][nb][1].w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    mma_bf16_16816(acc[nb], a[0][0][u], a[1][0][u], a[0][1][u], a[1][1][u], xb0[u], xb1[u]);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kWfBps; ++q) {
+            m0[q] = m1[q]; m1[q] = m2[q];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) { v0[q][h][0] = v1[q][h][0]; v0[q][h][1] = v1[q][h][1]; }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) { x0[q][nb][0] = x1[q][nb][0]; x0[q][nb][1] = x1[q][nb][1]; }
+        }
+    }
+    // the CTA's warps add up their K slices; lane (g, t) holds rows g, g + 8 and batch
+    // columns 8 nb + 2t, + 1
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[warp][nb][j][lane] = acc[nb][j];
+    __syncthreads();
+    if (warp != 0) return;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWfWarps; ++w) v += red[w][nb][j][lane];
+            const int r = row[j >> 1], bcol = 8 * nb + 2 * t + (j & 1);
+            if (r < n && bcol < batch) y[(size_t)bcol * n + r] = (uint16_t)float_to_bf16_bits(v);
+        }
+}
+
 int grid_cap(int64_t want) {
     const int64_t cap = (int64_t)sm_count() * 8;
     if (want > cap) want = cap;
@@ -434,33 +592,46 @@ wq_status launch_wf_dequant(const uint8_t* packed, int64_t packed_bytes, const u
     return check_launch("wf dequant");
 }
 
+// Batch 1 takes the CUDA-core kernel, larger batches the tensor-core one (measured on
+// 8192 x 28672 at 4.5 bits per weight: 189 us against 245 us at batch 1; from batch 2 the
+// tensor-core kernel runs one pass in 245-256 us where the CUDA-core one takes 262 us at
+// batch 2, 435 us at 8 and two passes, 896 us, at 16). The tensor-core kernel reads each
+// block's width, offset and scale at 16 different rows per warp step, scattered over many
+// cache lines, which is what holds it at about 0.65 TB/s.
+#ifndef WQ_WF_FMA_MAX
+#define WQ_WF_FMA_MAX 1                // largest batch the CUDA-core kernel takes
+#endif
+
 wq_status launch_wf_gemv(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
                          const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                          const uint16_t* x, int batch, uint16_t* y, cudaStream_t s) {
-    const unsigned grid = (unsigned)((n + kGemvWarps - 1) / kGemvWarps);
-    // activation rows 8 at a time (x rows i .. i + 7 give y rows i .. i + 7)
-    for (int i0 = 0; i0 < batch; i0 += 8) {
-        const int nb = batch - i0 < 8 ? batch - i0 : 8;
-        const uint16_t* xi = x + (size_t)i0 * k;
-        uint16_t* yi = y + (size_t)i0 * n;
-#define WQ_WF_GEMV(NBV)                                                                              \
-    wf_gemv_kernel<NBV><<<grid, 32 * kGemvWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off, \
-                                                        (int)n, (int)k, xi, yi)
-        switch (nb) {
-            case 1: WQ_WF_GEMV(1); break;
-            case 2: WQ_WF_GEMV(2); break;
-            case 3: WQ_WF_GEMV(3); break;
-            case 4: WQ_WF_GEMV(4); break;
-            case 5: WQ_WF_GEMV(5); break;
-            case 6: WQ_WF_GEMV(6); break;
-            case 7: WQ_WF_GEMV(7); break;
-            default: WQ_WF_GEMV(8); break;
+    if (batch <= WQ_WF_FMA_MAX) {
+        const unsigned grid = (unsigned)((n + kFmaWarps - 1) / kFmaWarps);
+#define WQ_WF_FMA(NBV)                                                                                    \
+    wf_gemv_fma_kernel<NBV><<<grid, 32 * kFmaWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off, \
+                                                            (int)n, (int)k, x, y)
+        switch (batch) {
+            case 1: WQ_WF_FMA(1); break;
+            case 2: WQ_WF_FMA(2); break;
+            case 3: WQ_WF_FMA(3); break;
+            case 4: WQ_WF_FMA(4); break;
+            case 5: WQ_WF_FMA(5); break;
+            case 6: WQ_WF_FMA(6); break;
+            case 7: WQ_WF_FMA(7); break;
+            default: WQ_WF_FMA(8); break;
         }
-#undef WQ_WF_GEMV
-        wq_status st = check_launch("wf gemv");
-        if (st) return st;
+#undef WQ_WF_FMA
+        return check_launch("wf gemv");
     }
-    return WQ_OK;
+    static_assert(WQ_WF_FMA_MAX <= 8, "the CUDA-core kernel takes at most 8 activation rows");
+    const unsigned grid = (unsigned)((n + 15) / 16);
+    if (batch <= 8)
+        wf_gemv_kernel<1><<<grid, 32 * kWfWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off, (int)n,
+                                                         (int)k, x, batch, y);
+    else
+        wf_gemv_kernel<2><<<grid, 32 * kWfWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off, (int)n,
+                                                         (int)k, x, batch, y);
+    return check_launch("wf gemv");
 }
 
 wq_status read_wf_error(int32_t* code) {
