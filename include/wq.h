@@ -283,7 +283,7 @@ size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
  * and LUT16 (the per-block-64 centroid table of [KM] §2.2, looked up per stage; the product
  * runs in fp16 on the activations converted into the workspace as x * 2^e per activation
  * row, the power of two chosen from the row's largest |x| as in wq_gemv_w4a16, and the
- * epilogue multiplies the row's sums by 2^-e). For m <= 12 the decode-shaped case runs on the
+ * epilogue multiplies the row's sums by 2^-e). For m <= 16 the decode-shaped case runs on the
  * GEMV kernel of wq_gemv_w4a16 (the kernel choice by batch size of [KM] §4.1), with the same
  * tolerance and no workspace.
  *   x      bf16 [m, k]; m >= 1; k % 64 == 0.

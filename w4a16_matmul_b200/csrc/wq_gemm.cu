@@ -792,11 +792,14 @@ wq_status launch_plan(const Plan& p, const CUtensorMap& tx, const CUtensorMap& t
 // Up to this many activation rows the product is decode-shaped: the GEMV kernel (weights
 // rebuilt in registers, mma.sync, no TMA/TMEM pipeline) runs it faster than the
 // tensor-memory pipeline, whose per-stage bookkeeping dominates when BN is this small.
-// Measured on 4096x11008 and 11008x4096: at m = 8, 14.9 / 12.2 us against about 23 us; at
-// m = 12, 18.4 / 19.3 us against 20.9 / 22.5 us; at m = 16 the two are even, so the GEMV's
-// second batch fragment stops at 12 rows. This is the kernel choice by batch size of
-// "K-Means量化技术…" §4.1.
-constexpr int64_t kGemvMaxRows = 12;
+// Measured on 4096x11008 and 11008x4096: at m = 8, 13.3 / 12.0 us against about 23 us; at
+// m = 12, 16.6 / 17.9 us against 20.9 / 22.5 us; at m = 16, 17.9 / 19.9 us against 20.8 /
+// 23.4 us (with the GEMV's 128-row CTAs in its cluster split). This is the kernel choice by
+// batch size of "K-Means量化技术…" §4.1.
+#ifndef WQ_GEMM_GEMV_MAX_ROWS
+#define WQ_GEMM_GEMV_MAX_ROWS 16
+#endif
+constexpr int64_t kGemvMaxRows = WQ_GEMM_GEMV_MAX_ROWS;
 
 // Workspace layout: for LUT16 the scaled fp16 copy of the activations [m, k] (rounded up to
 // 1 KB) and the per-row factors 2^-e (fp32 [m], rounded up to 1 KB) first, then the fp32

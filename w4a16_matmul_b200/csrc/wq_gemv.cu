@@ -506,6 +506,9 @@ constexpr int cta_warps(int wk, int fw) { return wk == 1 ? fw : 4; }
 #ifndef WQ_GEMV_LUT_FW
 #define WQ_GEMV_LUT_FW 8
 #endif
+#ifndef WQ_GEMV_CL_FW
+#define WQ_GEMV_CL_FW 8               // warps per CTA in the cluster split, other formats, batch >= 4
+#endif
 #ifndef WQ_GEMV_LLOYD_CAP
 #define WQ_GEMV_LLOYD_CAP 1
 #endif
@@ -768,6 +771,12 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
     // cluster split: LUT16 takes 8 (each staged activation chunk, converted to fp16 with its
     // scale, then serves 128 weight rows; the CTAs per SM halve at the same 128 registers)
     constexpr int FWL = (KIND == kLut16) ? WQ_GEMV_LUT_FW : 4;
+    // the cluster split: 8 warps (128 rows) per CTA for LUT16, and for the other formats
+    // from batch 4 on, where staging the activations is a large share of a CTA's work
+    // (measured on 4096 x 11008 and 11008 x 4096 at m = 8 / 12 / 16: 12.5 -> 12.0 / 19.7 ->
+    // 17.9 / 22.9 -> 19.9 us and 14.5 -> 13.3 / 18.7 -> 16.6 / 21.4 -> 17.9 us; at batch 1
+    // it was up to 0.9 us slower)
+    constexpr int FWC = (KIND == kLut16) ? WQ_GEMV_LUT_FW : WQ_GEMV_CL_FW;
     // full-K CTAs: 4 row warps at batch 1, WQ_GEMV_WARPS_BATCHED above (measured on the
     // decode sweep: 8 warps +9 / +13 / +14 % at batch 4 / 8 / 16, neutral at batch 1)
     if (BIGR == 2 && batch > WQ_GEMV_R2_MIN_BATCH && rows16 >= 12 * sms * 2) {
@@ -795,9 +804,15 @@ wq_status pick_split(Prepared<MAXP>& pr, const GemvProblem* probs, int count, in
         int64_t want = (WQ_GEMV_CL_WARPS * sms + 4 * tiles64 - 1) / (4 * tiles64);
         int cl = weights < ((int64_t)1 << 24) ? 1 : want >= 8 ? 8 : want >= 4 ? 4 : want >= 2 ? 2 : 1;
         while (cl > 1 && max_steps / cl < 2) cl >>= 1;
-        if (cl == 8) return prepare_variant<KIND, NB, 1, 1, FWL, MAXP, 8>(pr, probs, tiles_for(16 * FWL));
-        if (cl == 4) return prepare_variant<KIND, NB, 1, 1, FWL, MAXP, 4>(pr, probs, tiles_for(16 * FWL));
-        if (cl == 2) return prepare_variant<KIND, NB, 1, 1, FWL, MAXP, 2>(pr, probs, tiles_for(16 * FWL));
+        if (cl == 8) return batch >= 4 || KIND == kLut16
+                                  ? prepare_variant<KIND, NB, 1, 1, FWC, MAXP, 8>(pr, probs, tiles_for(16 * FWC))
+                                  : prepare_variant<KIND, NB, 1, 1, 4, MAXP, 8>(pr, probs, tiles_for(64));
+        if (cl == 4) return batch >= 4 || KIND == kLut16
+                                  ? prepare_variant<KIND, NB, 1, 1, FWC, MAXP, 4>(pr, probs, tiles_for(16 * FWC))
+                                  : prepare_variant<KIND, NB, 1, 1, 4, MAXP, 4>(pr, probs, tiles_for(64));
+        if (cl == 2) return batch >= 4 || KIND == kLut16
+                                  ? prepare_variant<KIND, NB, 1, 1, FWC, MAXP, 2>(pr, probs, tiles_for(16 * FWC))
+                                  : prepare_variant<KIND, NB, 1, 1, 4, MAXP, 2>(pr, probs, tiles_for(64));
     }
 #endif
     if (rows16 >= 2 * sms) return prepare_variant<KIND, NB, 1, 2, 4, MAXP>(pr, probs, tiles_for(32));
