@@ -379,10 +379,44 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args, mats, seconds=args.cpu_seconds)
+    # last on the line, so that a reader of only its tail still sees every row's headline
+    line["rows"] = summarize(extras, line)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def summarize(extras: dict, line: dict) -> dict:
+    """One short entry per row of the hot path (fractions of the measured peaks; GEMM in
+    TFLOP/s with the dequantise + cuBLAS bf16 line beside it), from the full results."""
+    def get(d, *path):
+        for p in path:
+            if not isinstance(d, dict) or p not in d:
+                return None
+            d = d[p]
+        return d
+    r = {"headline_frac": line["roofline"]["frac"], "headline_frac_packed_only": line["roofline"]["frac_packed_only"],
+         "sweep_b4_frac": get(extras, "sweep_batch4", "frac_hbm"),
+         "sweep_b16_frac": get(extras, "sweep_batch16", "frac_hbm"),
+         "single_2048_us": [get(extras, "single_matrix_2048", k, "us") for k in ("quantize_pack", "dequant", "gemv_b1")],
+         "quantize_8192x28672_frac": get(extras, "quantize_dyadic_large", "frac_hbm"),
+         "dequant_8192x28672_frac": get(extras, "dequant_large", "frac_hbm")}
+    g = extras.get("prefill_gemm", {})
+    for shape in ("4096x11008", "11008x4096"):
+        r[f"gemm_{shape}_TFLOPs_m16_128_512_2048_4096"] = [get(g, f"{shape}_m{m}", "TFLOP/s") for m in (16, 128, 512, 2048, 4096)]
+        r[f"cublas_{shape}_TFLOPs"] = [get(g, f"{shape}_m{m}", "cublas_bf16_materialized_TFLOP/s")
+                                       for m in (16, 128, 512, 2048, 4096)]
+    r["gemm_lloyd8s_lut16_TFLOPs_m512_4096"] = [get(g, f"{f}_4096x11008_m{m}", "TFLOP/s")
+                                                for f in ("lloyd8s", "lut16") for m in (512, 4096)]
+    r["lut16_gemv_frac_b1_8_16"] = [get(extras, f"lut16_gemv_b{b}", "frac_hbm") for b in (1, 8, 16)]
+    r["lloyd8s_gemv_frac_b1"] = get(extras, "lloyd8s_gemv_b1", "frac_hbm")
+    r["wf_gemv_frac_b1_16"] = [get(extras, "water_filling_large", f"gemv_b{b}", "frac_hbm") for b in (1, 16)]
+    r["lloyd_g32_ms_per_matrix"] = get(extras, "lloyd_g32", "ms_per_matrix")
+    r["kmeans16_ms"] = get(extras, "kmeans16", "ms")
+    r["ste_frac"] = get(extras, "fake_quant_ste_large", "frac_hbm")
+    r["bf16x_frac_enc_dec"] = [get(extras, "bf16x_large", "encode_frac_hbm"), get(extras, "bf16x_large", "decode_frac_hbm")]
+    return r
 
 
 def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrier, max_over_ranks):
@@ -876,6 +910,7 @@ def run_profile_target(args):
     activation conversion), quantize --shape N,K, dequant --shape N,K,
     lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd), gumbel --shape N,K
     (Gumbel-ST backward at tau = step^2; gumbel1: at tau = 1.0), ste --shape N,K (STE forward),
+    kmeans --shape N,K (16-centroid k-means),
     bf16x --shape N,K (BF16X encode + decode), wf --shape N,K
     (water-filling analyze + dequant), wf_gemv --shape N,K,B (its GEMV). Random packed codes and
     scales (timing does not depend on the values); inputs stay on the device."""
@@ -953,6 +988,9 @@ def run_profile_target(args):
     elif args.profile == "lloyd":
         w = (torch.randn((n, k), device=dev, generator=gen) * 0.02).to(torch.bfloat16)
         fn = lambda: wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)
+    elif args.profile == "kmeans":
+        w = (torch.randn((n, k), device=dev, generator=gen) * 0.01).to(torch.bfloat16)
+        fn = lambda: wq.quantize_lloyd(w, wq.LLOYD_KMEANS16, 25)
     else:
         raise SystemExit(f"unknown --profile {args.profile}")
     for _ in range(3):
