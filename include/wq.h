@@ -296,13 +296,14 @@ wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16
                         void* ws, size_t ws_bytes, wq_stream stream);
 
 /* Reads and clears the library's device-side error words. Kernels that wait on the GPU
- * (the GEMM pipeline's mbarrier waits) give up after a bounded time instead of hanging and
- * record a nonzero code; the BF16X kernels record one when an overflow-table index would
- * pass ovf_bytes, and the water-filling kernels one when a block's width is outside 3..5
- * or its bytes do not fit packed_bytes (2000 dequant, 2001 pack, 2002 GEMV; the access is
- * skipped in every case). *code receives the code (0 = none). Synchronous (copies three
- * ints from the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_EDATA for
- * inconsistent BF16X or water-filling data, WQ_OK otherwise.
+ * (the GEMM pipeline's mbarrier waits, the water-filled GEMV's waits for its staged bytes)
+ * give up after a bounded time instead of hanging and record a nonzero code (the GEMV's
+ * is 2100); the BF16X kernels record one when an overflow-table index would pass
+ * ovf_bytes, and the water-filling kernels one when a block's width is outside 3..5 or its
+ * bytes do not fit packed_bytes (2000 dequant, 2001 pack, 2002 GEMV; the access is skipped
+ * in every case). *code receives the code (0 = none). Synchronous (copies three ints from
+ * the device). Returns WQ_ETIMEOUT if a wait had expired, WQ_EDATA for inconsistent BF16X
+ * or water-filling data, WQ_OK otherwise.
  * The debug build of the library (libwq_debug.so, compiled with -DWQ_DEBUG=1) also checks
  * on the device what the normal build takes as preconditions, records the first failed
  * check of each kernel family and reports it here with WQ_EDATA (the kernels never trap):
@@ -407,7 +408,10 @@ wq_status wq_dequant_wf(const uint8_t* packed, int64_t packed_bytes, const uint1
  *   x      bf16 [batch, k]; batch 1 .. 16.
  *   y      out bf16 [batch, n].
  * Same tolerance as wq_gemv_w4a16. A block outside packed_bytes, or a width outside 3..5,
- * contributes nothing and is flagged for wq_device_error (WQ_EDATA). */
+ * contributes nothing and is flagged for wq_device_error (WQ_EDATA). For batches 1 and 2
+ * each row's blocks are read in runs of 32: a run whose offsets do not describe whole
+ * blocks back to back inside packed_bytes is not read at all (all of its blocks count as
+ * flagged), and a block whose width disagrees with the offsets is flagged. */
 wq_status wq_gemv_wf(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
                      const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                      const uint16_t* x, int32_t batch, uint16_t* y, wq_stream stream);

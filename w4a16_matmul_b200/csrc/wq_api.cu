@@ -162,6 +162,10 @@ wq_status wq_device_error(int32_t* code) {
         *code = data;
         return fail(WQ_EDATA, "BF16X overflow index past ovf_bytes (code %d)", data);
     }
+    if (wf >= 2100) {
+        *code = wf;
+        return fail(WQ_ETIMEOUT, "a water-filled GEMV's wait for its staged bytes expired (code %d)", wf);
+    }
     if (wf != 0) {
         *code = wf;
         return fail(WQ_EDATA, "water-filling block outside packed_bytes or bad width (code %d)", wf);

@@ -48,57 +48,10 @@ namespace {
 constexpr int BM = 128;            // weight rows per CTA (MMA M)
 // Columns per stage, KB: 64 (one 128-byte swizzle row of bf16) or 128 (two such tiles, used
 // when K % 128 == 0: twice the reconstruction work per stage for the same bookkeeping).
-constexpr uint64_t kWaitNs = 2000000000ull;   // a wait longer than 2 s is declared dead
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-#ifndef WQ_GEMM_SUSPEND_NS
-#define WQ_GEMM_SUSPEND_NS 20000
-#endif
 #ifndef WQ_GEMM_BIG_SLOTS
 #define WQ_GEMM_BIG_SLOTS 0
 #endif
-// Bounded wait for the completion of phase `parity`: gives up after about two seconds of
-// wall time and returns false. Each try_wait may suspend the thread for up to
-// WQ_GEMM_SUSPEND_NS nanoseconds (it wakes as soon as the phase completes), so a waiting
-// warp does not spin on the issue slots the reconstruction warps need.
-// `abort` (shared memory) is polled only while the wait spins, so that a CTA whose other
-// role gave up stops waiting at once instead of timing out wait by wait.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, const int* abort = nullptr) {
-    const uint32_t a = smem_u32(b);
-    uint64_t deadline = 0;
-    for (uint32_t i = 0;; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
-            : "=r"(done) : "r"(a), "r"(parity), "r"((uint32_t)WQ_GEMM_SUSPEND_NS) : "memory");
-        if (done) return true;
-        if ((i & 7) == 0) {
-            if (abort && *(volatile const int*)abort) return false;
-            const uint64_t now = global_ns();
-            if (deadline == 0) deadline = now + kWaitNs;
-            else if (now > deadline) return false;
-        }
-    }
-}
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
     asm volatile(

@@ -216,6 +216,63 @@ __device__ __forceinline__ uint4 ldg_v4(const void* p) {
     return v;
 }
 
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// mbarrier helpers (shared::cta): init, plain arrive, arrive that also announces the bytes
+// the asynchronous copies of the phase will deliver, and a bounded wait.
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+constexpr uint64_t kWaitNs = 2000000000ull;   // a device wait longer than 2 s is declared dead
+#ifndef WQ_MBAR_SUSPEND_NS
+#define WQ_MBAR_SUSPEND_NS 20000
+#endif
+// Bounded wait for the completion of phase `parity`: gives up after about two seconds of
+// wall time and returns false. Each try_wait may suspend the thread for up to
+// WQ_MBAR_SUSPEND_NS nanoseconds (it wakes as soon as the phase completes), so a waiting
+// warp does not spin on issue slots other warps need.
+// `abort` (shared memory) is polled only while the wait spins, so that a CTA whose other
+// role gave up stops waiting at once instead of timing out wait by wait.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, const int* abort = nullptr) {
+    const uint32_t a = smem_u32(b);
+    uint64_t deadline = 0;
+    for (uint32_t i = 0;; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+            : "=r"(done) : "r"(a), "r"(parity), "r"((uint32_t)WQ_MBAR_SUSPEND_NS) : "memory");
+        if (done) return true;
+        if ((i & 7) == 0) {
+            if (abort && *(volatile const int*)abort) return false;
+            const uint64_t now = global_ns();
+            if (deadline == 0) deadline = now + kWaitNs;
+            else if (now > deadline) return false;
+        }
+    }
+}
+
+// Asynchronous bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from
+// global to this CTA's shared memory, completing on `bar` (complete_tx). No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
 // Asks the L2 to fetch [p, p + bytes) from memory ahead of use (a hint; p and bytes must be
 // multiples of 16 and the range must lie inside one allocation).
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {

@@ -23,8 +23,10 @@
 // Kernels: analyze (scale, the three distortions, width, the scan's tile totals), the shared
 // in-place tile scan of the block sizes, pack (codes at the chosen width), dequant (eight
 // threads per block: each rebuilds 8 weights from b whole bytes and stores 16 bytes, so a
-// block's 128 output bytes leave in one coalesced run), and a GEMV that rebuilds the
-// weights the same way and multiplies them in fp32 (the format's decode-side consumer).
+// block's 128 output bytes leave in one coalesced run), and two GEMVs (the format's
+// decode-side consumers) that rebuild the weights as the dequant does and multiply them on
+// the tensor cores with fp32 accumulation: batches of 1 and 2 with the packed bytes staged
+// in shared memory by bulk copies, larger batches 16 rows per warp.
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -226,16 +228,16 @@ __device__ __forceinline__ unsigned long long wf_bytes(const uint8_t* packed, in
     return v;
 }
 
-// bf16((scale / 16) * (idx_5 - 16)) of the 8 codes of b bits in v (code j in bits b j ..),
-// as bf16 pairs in column order; sb = the block's bf16 scale bits.
-// Each code is brought to bits 5 - b .. 4, where its value is idx_5 = code << (5 - b), by one
-// 32-bit funnel shift of the 40 bits (the bits below it hold its neighbour and are masked
-// off); a pair of codes is joined into the two halves of one word by a byte permute.
-__device__ __forceinline__ void wf_decode8(unsigned long long v, int bw, uint32_t sb, uint32_t (&o)[4]) {
+// idx_5 of the 8 codes of b bits in v (code j in bits b j ..), as pairs in column order (the
+// two halves of each word). Each code is brought to bits 5 - b .. 4, where its value is
+// idx_5 = code << (5 - b), by one 32-bit funnel shift of the 40 bits (the bits below it hold
+// its neighbour and are masked off); a pair of codes is joined into one word by a byte
+// permute. wf_decode8 then gives bf16((scale / 16) * (idx_5 - 16)) of each, as bf16 pairs;
+// sb = the block's bf16 scale bits.
+__device__ __forceinline__ void wf_fields8(unsigned long long v, int bw, uint32_t (&m)[4]) {
     const uint32_t lo = (uint32_t)v, hi = (uint32_t)(v >> 32);
     const int s5 = 5 - bw;
     const uint32_t mp = (((1u << bw) - 1u) * 0x00010001u) << s5;      // idx_5 fields of a pair
-    uint32_t m[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         // code 2j starts at bit 2 j b, code 2j + 1 at (2j + 1) b; shifted right by that minus
@@ -244,17 +246,28 @@ __device__ __forceinline__ void wf_decode8(unsigned long long v, int bw, uint32_
         const uint32_t c1 = (j == 3 && bw == 5) ? hi >> 3 : __funnelshift_r(lo, hi, (2 * j + 1) * bw - s5);
         m[j] = prmt(c0, c1, 0x5410u) & mp;                               // (idx_5 of 2j, of 2j + 1)
     }
-    if ((sb & 0x7FFFu) >= 0x0400u) {
-        // scale >= 2^-119: every nonzero (scale / 16) (idx_5 - 16) is a normal bf16.
-        // idx_5 | 0x4300 is the bf16 number 128 + idx_5, minus 144 is idx_5 - 16 exactly, and
-        // one bf16x2 multiply by scale / 16 (the exponent field minus 4) rounds the product
-        // once, as the definition reads.
-        const uint32_t s16x2 = prmt(sb - 0x0200u, 0u, 0x1010u);
+}
+
+// The reconstruction for a scale >= 2^-119, where every nonzero (scale / 16) (idx_5 - 16) is
+// a normal bf16: idx_5 | 0x4300 is the bf16 number 128 + idx_5, minus 144 is idx_5 - 16
+// exactly, and one bf16x2 multiply by scale / 16 (the exponent field minus 4) rounds the
+// product once, as the definition reads.
+__device__ __forceinline__ void wf_finish_normal(const uint32_t (&m)[4], uint32_t sb, uint32_t (&o)[4]) {
+    const uint32_t s16x2 = prmt(sb - 0x0200u, 0u, 0x1010u);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t d = bf16x2_fma(m[j] | 0x43004300u, 0x3F803F80u, 0xC310C310u);   // idx_5 - 16
-            o[j] = bf16x2_fma(d, s16x2, 0x80008000u);
-        }
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t d = bf16x2_fma(m[j] | 0x43004300u, 0x3F803F80u, 0xC310C310u);   // idx_5 - 16
+        o[j] = bf16x2_fma(d, s16x2, 0x80008000u);
+    }
+}
+
+__device__ __forceinline__ bool wf_scale_normal(uint32_t sb) { return (sb & 0x7FFFu) >= 0x0400u; }
+
+__device__ __forceinline__ void wf_decode8(unsigned long long v, int bw, uint32_t sb, uint32_t (&o)[4]) {
+    uint32_t m[4];
+    wf_fields8(v, bw, m);
+    if (wf_scale_normal(sb)) {
+        wf_finish_normal(m, sb, o);
     } else {
         const float s16 = bf16_bits_to_float(sb) * 0.0625f;
 #pragma unroll
@@ -306,114 +319,6 @@ wf_dequant_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, cons
 //     activations one step ahead.
 // A block whose width or offset is inconsistent with the buffer is reported (2002) and
 // contributes nothing.
-// Small batches: y[i, r] = sum_c Wdeq[r, c] x[i, c] for NB <= 8 activation
-// rows on the CUDA cores, Wdeq rebuilt exactly as wf_dequant_kernel does (bf16), products and sums in fp32.
-// One warp per weight row; 8 lanes per 64-weight block (lane t: columns 8t .. 8t + 7, the b
-// bytes at the block's offset + b t), 4 blocks per step, 8 steps per chunk of 32 blocks.
-// A chunk's widths, offsets and scales are read one block per lane, checked, and handed to
-// the decoding lanes by shuffles. Software pipeline: the metadata is read two chunks
-// ahead and the packed words one chunk ahead, so that a chunk's loads are in flight while
-// the previous chunk is decoded. A block whose width or offset is inconsistent with the
-// buffer is reported and contributes nothing.
-constexpr int kFmaWarps = 8;
-
-// One chunk's packed words and, per step, the block width (0: nothing) and scale bits.
-struct WfChunk {
-    unsigned long long v[8];
-    uint32_t wpk;                    // width of step j in bits 4j .. 4j + 3
-    uint32_t spk[4];                 // scale bits of steps 2i (low half) and 2i + 1 (high half)
-};
-
-template <int NB>
-__global__ void __launch_bounds__(32 * kFmaWarps)
-wf_gemv_fma_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const uint16_t* __restrict__ scale,
-               const uint8_t* __restrict__ width, const uint32_t* __restrict__ blk_off, int n, int k,
-               const uint16_t* __restrict__ x, uint16_t* __restrict__ y) {
-    const int lane = threadIdx.x & 31;
-    const int row = blockIdx.x * kFmaWarps + (threadIdx.x >> 5);
-    if (row >= n) return;                        // the whole warp leaves; no CTA-wide barrier
-    const int kb = k >> 6;
-    const int nch = (kb + 31) >> 5;
-    const int64_t rb = (int64_t)row * kb;
-    const int t = lane & 7, sub = lane >> 3;
-
-    // this lane's block of chunk c: width (0 past the row's end), offset, scale bits
-    auto meta = [&](int c, int& bw, uint32_t& off, uint32_t& sb) {
-        const int bi = 32 * c + lane;
-        bw = 0; off = 0; sb = 0;
-        if (bi < kb) {
-            bw = __ldg(width + rb + bi);
-            off = ldg_u32(blk_off + rb + bi);
-            sb = ldg_u16(scale + rb + bi);
-        }
-    };
-    // check the lane's block, then issue the chunk's packed loads (the whole warp takes part)
-    auto fetch = [&](int c, int bw, uint32_t off, uint32_t sb, WfChunk& ch) {
-        if (32 * c + lane < kb && !wf_block_ok(bw, off, packed_bytes)) {
-            report(2002);
-            bw = 0;
-        }
-        ch.wpk = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int blk = 4 * j + sub;
-            const int b = __shfl_sync(0xFFFFFFFFu, bw, blk);
-            const uint32_t o = __shfl_sync(0xFFFFFFFFu, off, blk);
-            const uint32_t sj = __shfl_sync(0xFFFFFFFFu, sb, blk);
-            ch.wpk |= (uint32_t)b << (4 * j);
-            if (j & 1) ch.spk[j >> 1] |= sj << 16; else ch.spk[j >> 1] = sj;
-            ch.v[j] = b ? wf_bytes(packed, (int64_t)o + b * t, b) : 0ull;
-        }
-    };
-
-    float2 acc[NB];
-#pragma unroll
-    for (int i = 0; i < NB; ++i) acc[i] = make_float2(0.f, 0.f);
-
-    WfChunk cur;
-    int bw;
-    uint32_t off, sb;
-    meta(0, bw, off, sb);
-    fetch(0, bw, off, sb, cur);
-    if (nch > 1) meta(1, bw, off, sb);
-    for (int c = 0; c < nch; ++c) {
-        WfChunk nxt;
-        if (c + 1 < nch) {                       // uniform across the warp
-            fetch(c + 1, bw, off, sb, nxt);
-            if (c + 2 < nch) meta(c + 2, bw, off, sb);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int b = (int)(cur.wpk >> (4 * j)) & 15;
-            if (b == 0) continue;
-            const uint32_t sj = (j & 1) ? cur.spk[j >> 1] >> 16 : cur.spk[j >> 1] & 0xFFFFu;
-            uint32_t o[4];
-            wf_decode8(cur.v[j], b, sj, o);
-            const int col = (32 * c + 4 * j + sub) * 64 + 8 * t;
-#pragma unroll
-            for (int i = 0; i < NB; ++i) {
-                // cached in L1: every warp of the SM reads the same activations
-                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)i * k + col));
-                const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 w2 = make_float2(__uint_as_float(o[q] << 16), __uint_as_float(o[q] & 0xFFFF0000u));
-                    const float2 x2 = make_float2(__uint_as_float(xs[q] << 16), __uint_as_float(xs[q] & 0xFFFF0000u));
-                    acc[i] = __ffma2_rn(w2, x2, acc[i]);
-                }
-            }
-        }
-        if (c + 1 < nch) cur = nxt;
-    }
-#pragma unroll
-    for (int i = 0; i < NB; ++i) {
-        float r = acc[i].x + acc[i].y;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
-        if (lane == 0) y[(size_t)i * n + row] = (uint16_t)float_to_bf16_bits(r);
-    }
-}
-
 #ifndef WQ_WF_WARPS
 #define WQ_WF_WARPS 4                  // warps per CTA (splitting the row group's blocks)
 #endif
@@ -555,6 +460,290 @@ wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const u
         }
 }
 
+// Batches of 1 and 2: y[i, r] = sum_c Wdeq[r, c] x[i, c] with the packed bytes staged in
+// shared memory by bulk asynchronous copies, products on the tensor cores.
+//   * A warp owns 4 weight rows. Its blocks come in chunks of 32 block columns: one lane
+//     reads each block's offset, width and scale (coalesced), checks them, and writes a
+//     packed descriptor to shared memory; one lane then copies each row's bytes of the chunk,
+//     a contiguous run of the bit streams, into shared memory with one cp.async.bulk (from
+//     the 16-byte boundary at or below the run's start; the run's last 8 bytes by a plain
+//     load when its end is not on a 16-byte boundary), completing on the stage's mbarrier.
+//     WQ_WF_ST_STAGES stages per warp: while one chunk is decoded the next ones are in
+//     flight, with no registers held for them.
+//   * One mma.sync m16n8k16 per block column covers the 4 rows x 64 columns: lane (g, t)
+//     decodes word t + 4 (g >> 2) (codes 8w .. 8w + 7) of row g & 3's block, its pairs
+//     0 and 1 as A row g (quarter g >> 2 of the columns), pairs 2 and 3 as A row g + 8
+//     (quarter 2 + (g >> 2)). B column 4 i + q holds activation row i at the columns of
+//     quarter q (4 consecutive values per lane: one 8-byte load), so D[rho][4 i + q(rho)]
+//     are the useful sums (16 of the 128 outputs) and y[i][row] adds four of them.
+// A chunk whose offsets do not describe a contiguous run inside packed_bytes is not read;
+// a block whose width or offset is inconsistent is not decoded; both are reported (2002)
+// and contribute nothing. An expired wait for a copy is reported as 2100.
+#ifndef WQ_WF_ST_WARPS
+#define WQ_WF_ST_WARPS 1               // warps per CTA (each independent)
+#endif
+#ifndef WQ_WF_ST_STAGES
+#define WQ_WF_ST_STAGES 2              // chunks staged per warp
+#endif
+constexpr int kStWarps = WQ_WF_ST_WARPS;
+constexpr int kStStages = WQ_WF_ST_STAGES;
+constexpr int kStRowBytes = 32 * 40 + 32;      // a chunk of 5-bit blocks, the alignment and read slack
+
+struct WfStage {
+    alignas(16) uint8_t data[4][kStRowBytes];  // row i's run, from its 16-byte boundary
+    uint4 meta[4][32];                         // per block: its descriptor (wf_st_desc)
+};
+struct WfWarpSmem {
+    WfStage st[kStStages];
+    uint4 tbl[3];                              // descriptor words .y (the mask), .z, .w for b = 3, 4, 5
+    uint64_t bar[kStStages];
+};
+
+// Block descriptor of the staged GEMV (zero for a block that is not decoded):
+//   .x  the bf16x2 pair (scale * 4, scale * 4), or, where that pair would not give the exact
+//       reconstruction (a scale below 2^-119, from 2^126 on, negative or not finite), the
+//       scale's bf16 bits with bit 31 set;
+//   .y  the block's byte offset in its row's staged run << 21 | width b << 8 | the mask of
+//       the idx_5 fields of a code pair (bits 5 - b .. 4 and 21 - b .. 20);
+//   .z  2^(32 - 2b);  .w  2^21 + 2^(5 + b).
+__device__ __forceinline__ bool wf_st_pair_scale(uint32_t sb) { return sb >= 0x0400u && sb < 0x7E80u; }
+
+__device__ __forceinline__ uint4 wf_st_desc(uint32_t sb, uint32_t b, uint32_t off) {
+    const uint32_t sx = wf_st_pair_scale(sb) ? prmt(sb + 0x0100u, 0u, 0x1010u) : (sb | 0x80000000u);
+    const uint32_t mp = (((1u << b) - 1u) << (5 - b)) * 0x00010001u;
+    return make_uint4(sx, (off << 21) | (b << 8) | mp, 1u << (32 - 2 * b), (1u << 21) + (1u << (5 + b)));
+}
+
+// One block column of the staged GEMV: the lane decodes word wd (codes 8 wd .. 8 wd + 7) of
+// its row's block and issues the column's MMA. The word's b bytes start at byte b wd of the
+// block. Pair j (codes 2j, 2j + 1) is the window shifted right by 2jb (a funnel shift, h);
+// h * 2^(32 - 2b) keeps just the pair, at the top of the word, and the high half of its
+// product with 2^21 + 2^(5 + b) is the pair shifted right by 11 (code 2j + 1 at bits
+// 21 - b .. 20) plus the pair shifted right by 27 - b (code 2j at bits 5 - b .. 4): both
+// shifts are exact and the two ranges do not overlap, so no carry disturbs the idx_5
+// fields, which the mask then isolates. As bf16 numbers the fields are idx_5 * 2^-133;
+// times 2^127 minus 1/4 that is (idx_5 - 16) * 2^-6 exactly, and times (scale * 4) it is
+// (scale / 16) (idx_5 - 16) rounded once, the reconstruction. FAST: every block of the
+// chunk is valid with a pair-form scale, so nothing branches.
+template <bool FAST>
+__device__ __forceinline__ void wf_st_step(const uint8_t* rowdata, uint4 d, uint32_t wd, uint2 xv, float (&acc)[4]) {
+    const uint32_t b = FAST ? (d.y >> 8) & 7u : max((d.y >> 8) & 7u, 3u);     // 0: not decoded
+    const uint32_t bw = b * wd;
+    const uint32_t* wp = reinterpret_cast<const uint32_t*>(rowdata + (d.y >> 21) + (bw & ~3u));
+    const uint32_t sh = (bw & 3u) * 8;
+    const uint32_t lo = __funnelshift_r(wp[0], wp[1], sh), hi = wp[1] >> sh;
+    const uint32_t h[4] = {lo, __funnelshift_r(lo, hi, 2 * b), __funnelshift_r(lo, hi, 4 * b),
+                           __funnelshift_r(lo, hi, 6 * b)};
+    uint32_t m[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m[j] = __umulhi(h[j] * d.z, d.w) & d.y & 0x001F001Fu;
+    uint32_t o[4];
+    if (FAST || (d.x >> 31) == 0u) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            o[j] = bf16x2_fma(bf16x2_fma(m[j], 0x7F007F00u, 0xBE80BE80u), d.x, 0x80008000u);
+    } else {
+        const float s16 = bf16_bits_to_float(d.x & 0xFFFFu) * 0.0625f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            o[j] = pack_bf16x2(s16 * (float)((int)(m[j] & 0xFFFFu) - 16), s16 * (float)((int)(m[j] >> 16) - 16));
+    }
+    if (!FAST && d.y == 0u) o[0] = o[1] = o[2] = o[3] = 0u;
+    mma_bf16_16816(acc, o[0], o[2], o[1], o[3], xv.x, xv.y);
+}
+
+// The block columns J0 .. J0 + nb - 1 of one staged chunk, in groups of 4 whose activation
+// pieces were loaded 8 columns ahead (xa: the group at hand, xb: the next); after a group
+// is used its registers take the pieces 8 columns further on. FULL: nb == 32.
+template <bool FAST, bool FULL, typename XLoad>
+__device__ __forceinline__ void wf_st_chunk(const WfStage& st, int ri, uint32_t wd, int J0, int nb, XLoad& xload4,
+                                            uint2 (&xa)[4], uint2 (&xb)[4], float (&acc)[2][4]) {
+    const uint8_t* rowdata = st.data[ri];
+    const uint4* meta = st.meta[ri];
+#pragma unroll 1
+    for (int jg = 0; jg < 32; jg += 8) {
+        if (!FULL && jg >= nb) break;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (FULL || jg + u < nb) wf_st_step<FAST>(rowdata, meta[jg + u], wd, xa[u], acc[u & 1]);
+        xload4(J0 + jg + 8, xa);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (FULL || jg + 4 + u < nb) wf_st_step<FAST>(rowdata, meta[jg + 4 + u], wd, xb[u], acc[u & 1]);
+        xload4(J0 + jg + 12, xb);
+    }
+}
+
+template <int NB>
+__global__ void __launch_bounds__(32 * kStWarps)
+wf_gemv_staged_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const uint16_t* __restrict__ scale,
+                      const uint8_t* __restrict__ width, const uint32_t* __restrict__ blk_off, int n, int k,
+                      const uint16_t* __restrict__ x, int batch, uint16_t* __restrict__ y) {
+    __shared__ WfWarpSmem smem[kStWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    WfWarpSmem& S = smem[warp];
+    const int g = lane >> 2, t = lane & 3;
+    const int row0 = ((int)blockIdx.x * kStWarps + warp) * 4;
+    if (row0 >= n) return;                       // the whole warp leaves; warps share nothing
+    const int kb = k >> 6, nch = (kb + 31) >> 5;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < kStStages; ++s) mbar_init(&S.bar[s], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (lane < 3) {
+        const uint4 d = wf_st_desc(0x3F80u, (uint32_t)lane + 3, 0);
+        S.tbl[lane] = make_uint4(0u, d.y & 0x001F001Fu, d.z, d.w);
+    }
+    __syncwarp();
+
+    // lane l's block of chunk c in each row (offset; scale << 16 | width); lanes 0-3: the
+    // offsets of the first block of row `lane`'s chunk and just past its last block
+    const uint32_t rb0 = (uint32_t)row0 * (uint32_t)kb;          // n * kb < 2^27
+    uint32_t m_off[4], m_wsb[4], m_lo, m_end;
+    auto load_meta = [&](int c) {
+        const int j = 32 * c + lane;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            m_off[i] = 0; m_wsb[i] = 0;
+            if (row0 + i < n && j < kb) {
+                const uint32_t bi = rb0 + (uint32_t)(i * kb + j);
+                m_off[i] = ldg_u32(blk_off + bi);
+                m_wsb[i] = (uint32_t)__ldg(width + bi) | (ldg_u16(scale + bi) << 16);
+            }
+        }
+        m_lo = 0; m_end = 0;
+        if (lane < 4 && row0 + lane < n) {
+            const uint32_t bi = rb0 + (uint32_t)(lane * kb + 32 * c);
+            m_lo = ldg_u32(blk_off + bi);
+            m_end = ldg_u32(blk_off + bi + min(32, kb - 32 * c));
+        }
+    };
+    // start the copies of chunk c into stage s, check its blocks and write their
+    // descriptors; true when some block of the chunk is missing, inconsistent or has a
+    // scale without the pair form, so that the chunk takes the general decode
+    auto publish = [&](int c, int s) -> bool {
+        WfStage& st = S.st[s];
+        const int nb = min(32, kb - 32 * c);
+        // lanes 0-3: row `lane`'s run [lo, hi) must be whole 8-byte blocks, at least one and
+        // at most 32 of them at 5 bits, inside the buffer
+        const bool rok = lane < 4 && row0 + lane < n && ((m_lo | m_end) & 7u) == 0 && m_end >= m_lo + 24 &&
+                         m_end - m_lo <= 32 * 40 && (int64_t)m_end <= packed_bytes;
+        const uint32_t base = m_lo & ~15u;
+        const uint32_t bytes = rok ? (m_end & ~15u) - base : 0u;  // >= 16 when the run is sound
+        uint32_t tot = bytes;
+        tot += __shfl_xor_sync(0xFFFFFFFFu, tot, 1);
+        tot += __shfl_xor_sync(0xFFFFFFFFu, tot, 2);
+        if (lane == 0) mbar_expect_tx(&S.bar[s], tot);
+        if (rok) {
+            bulk_load(st.data[lane], packed + base, bytes, &S.bar[s]);
+            if ((m_end & 15u) == 8u)        // the run's last 8 bytes end off a 16-byte boundary
+                *reinterpret_cast<unsigned long long*>(st.data[lane] + (m_end - 8 - base)) =
+                    ldg_na_u64(reinterpret_cast<const unsigned long long*>(packed + m_end - 8));
+        }
+        const uint32_t lr = m_lo | (rok ? 1u : 0u);
+        bool special = false;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lri = __shfl_sync(0xFFFFFFFFu, lr, i), hi = __shfl_sync(0xFFFFFFFFu, m_end, i);
+            const uint32_t lo = lri & ~1u, off = m_off[i], b = m_wsb[i] & 0xFFu, sb = m_wsb[i] >> 16;
+            uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, off, 1);
+            if (lane == nb - 1) nxt = hi;
+            // a decodable block: inside the run, 8-byte aligned, b in 3..5, and followed by
+            // the next block (or the run's end) exactly 8 b bytes later
+            const bool ok = (lri & 1u) && lane < nb && b - 3u <= 2u && (off & 7u) == 0 && off >= lo &&
+                            nxt <= hi && nxt - off == 8 * b;
+            const bool rv = row0 + i < n;
+            if (rv && lane < nb && !ok) report(2002);
+            const uint4 tb = S.tbl[ok ? b - 3 : 0];
+            uint4 d = make_uint4(0u, 0u, 0u, 0u);
+            if (ok) {
+                d.x = wf_st_pair_scale(sb) ? prmt(sb + 0x0100u, 0u, 0x1010u) : (sb | 0x80000000u);
+                d.y = ((off - (lo & ~15u)) << 21) | (b << 8) | tb.y;
+                d.z = tb.z;
+                d.w = tb.w;
+            }
+            st.meta[i][lane] = d;
+            special |= !rv || (lane < nb && !(ok && wf_st_pair_scale(sb)));
+        }
+        return __any_sync(0xFFFFFFFFu, special);
+    };
+
+    // this lane's activation columns: row bi, quarter q = g & 3 of each block column
+    const int bi = min(NB == 1 ? 0 : g >> 2, batch - 1);
+    const int q = g & 3;
+    const uint16_t* xl = x + (size_t)bi * k + 32 * (q & 1) + 8 * t + 4 * (q >> 1);
+    const int ri = g & 3;
+    const uint32_t wd = (uint32_t)(t + 4 * (g >> 2));   // decoded row and word
+    // the activation pieces of steps J .. J + 3 (J: block column; past the row's end a
+    // repeated in-bounds load whose value is not used)
+    auto xload4 = [&](int J, uint2 (&xr)[4]) {
+        if (J + 3 < kb) {
+            const uint2* p = reinterpret_cast<const uint2*>(xl + (size_t)J * 64);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) xr[u] = __ldg(p + 16 * u);
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                xr[u] = __ldg(reinterpret_cast<const uint2*>(xl + (size_t)min(J + u, kb - 1) * 64));
+        }
+    };
+
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    uint2 xa[4], xb[4];                          // steps 8 apart: the next two groups of 4
+    xload4(0, xa);
+    xload4(4, xb);
+    uint32_t slow = 0;                           // bit s: stage s holds a chunk for the general loop
+    bool dead = false;
+    load_meta(0);
+    for (int p = 0; p < kStStages - 1 && p < nch; ++p) {
+        slow |= (uint32_t)publish(p, p) << p;
+        if (p + 1 < nch) load_meta(p + 1);
+    }
+    int c = 0;
+    for (; c < nch; ++c) {
+        const int pc = c + kStStages - 1;
+        if (pc < nch) {
+            const int ps = pc % kStStages;
+            slow = (slow & ~(1u << ps)) | ((uint32_t)publish(pc, ps) << ps);
+            if (pc + 1 < nch) load_meta(pc + 1);
+        }
+        const int s = c % kStStages;
+        if (!mbar_wait(&S.bar[s], (uint32_t)(c / kStStages) & 1u)) {
+            report(2100);
+            dead = true;
+            break;
+        }
+        __syncwarp();                            // the descriptors and tail bytes other lanes wrote
+        const WfStage& st = S.st[s];
+        const int nb = min(32, kb - 32 * c);
+        if (nb == 32 && !((slow >> s) & 1u))
+            wf_st_chunk<true, true>(st, ri, wd, 32 * c, 32, xload4, xa, xb, acc);
+        else if (nb == 32)
+            wf_st_chunk<false, true>(st, ri, wd, 32 * c, 32, xload4, xa, xb, acc);
+        else
+            wf_st_chunk<false, false>(st, ri, wd, 32 * c, nb, xload4, xa, xb, acc);
+        __syncwarp();                            // stage s is refilled next
+    }
+    if (dead) {
+        // chunks c .. c + stages - 1 were started: give their copies (again a bounded wait)
+        // the chance to land before the warp's shared memory goes away
+        for (int d = c; d < nch && d < c + kStStages; ++d)
+            mbar_wait(&S.bar[d % kStStages], (uint32_t)(d / kStStages) & 1u);
+        return;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[0][e] += acc[1][e];
+    // lane (g, t): t even holds the quarter-0/1 sums, t odd the quarter-2/3 sums of batch row t >> 1
+    float v = (t & 1) ? (g < 4 ? acc[0][2] : acc[0][3]) : (g < 4 ? acc[0][0] : acc[0][1]);
+    v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+    v += __shfl_xor_sync(0xFFFFFFFFu, v, 16);
+    const int ob = t >> 1;
+    if (g < 4 && !(t & 1) && ob < NB && ob < batch && row0 + g < n)
+        y[(size_t)ob * n + row0 + g] = (uint16_t)float_to_bf16_bits(v);
+}
+
 int grid_cap(int64_t want) {
     const int64_t cap = (int64_t)sm_count() * 8;
     if (want > cap) want = cap;
@@ -592,38 +781,23 @@ wq_status launch_wf_dequant(const uint8_t* packed, int64_t packed_bytes, const u
     return check_launch("wf dequant");
 }
 
-// Batch 1 takes the CUDA-core kernel, larger batches the tensor-core one (measured on
-// 8192 x 28672 at 4.5 bits per weight: 189 us against 245 us at batch 1; from batch 2 the
-// tensor-core kernel runs one pass in 245-256 us where the CUDA-core one takes 262 us at
-// batch 2, 435 us at 8 and two passes, 896 us, at 16). The tensor-core kernel reads each
-// block's width, offset and scale at 16 different rows per warp step, scattered over many
-// cache lines, which is what holds it at about 0.65 TB/s.
-#ifndef WQ_WF_FMA_MAX
-#define WQ_WF_FMA_MAX 1                // largest batch the CUDA-core kernel takes
-#endif
-
+// Batches of 1 and 2 take the staged kernel, larger ones the 16-row one (8192 x 28672 at
+// 4.5 bits per weight: the staged kernel runs batch 1 and 2 in about 100 us, the 16-row
+// one batches 3 to 16 in 245-256 us: it reads each block's width, offset and scale at 16
+// different rows per warp step, scattered over many cache lines, with no staging).
 wq_status launch_wf_gemv(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
                          const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                          const uint16_t* x, int batch, uint16_t* y, cudaStream_t s) {
-    if (batch <= WQ_WF_FMA_MAX) {
-        const unsigned grid = (unsigned)((n + kFmaWarps - 1) / kFmaWarps);
-#define WQ_WF_FMA(NBV)                                                                                    \
-    wf_gemv_fma_kernel<NBV><<<grid, 32 * kFmaWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off, \
-                                                            (int)n, (int)k, x, y)
-        switch (batch) {
-            case 1: WQ_WF_FMA(1); break;
-            case 2: WQ_WF_FMA(2); break;
-            case 3: WQ_WF_FMA(3); break;
-            case 4: WQ_WF_FMA(4); break;
-            case 5: WQ_WF_FMA(5); break;
-            case 6: WQ_WF_FMA(6); break;
-            case 7: WQ_WF_FMA(7); break;
-            default: WQ_WF_FMA(8); break;
-        }
-#undef WQ_WF_FMA
+    if (batch <= 2) {
+        const unsigned sgrid = (unsigned)((n + 4 * kStWarps - 1) / (4 * kStWarps));
+        if (batch == 1)
+            wf_gemv_staged_kernel<1><<<sgrid, 32 * kStWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off,
+                                                                    (int)n, (int)k, x, batch, y);
+        else
+            wf_gemv_staged_kernel<2><<<sgrid, 32 * kStWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off,
+                                                                    (int)n, (int)k, x, batch, y);
         return check_launch("wf gemv");
     }
-    static_assert(WQ_WF_FMA_MAX <= 8, "the CUDA-core kernel takes at most 8 activation rows");
     const unsigned grid = (unsigned)((n + 15) / 16);
     if (batch <= 8)
         wf_gemv_kernel<1><<<grid, 32 * kWfWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off, (int)n,
