@@ -47,8 +47,9 @@ def load_peaks():
         d = json.load(open(p))
         return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
                     bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
-                    source="measured")
-    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+                    sm_max_mhz=float(d.get("sm_max_mhz", 1965.0)), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, sm_max_mhz=1965.0,
+                source="fallback")
 
 
 # ---------------------------------------------------------------------------------------
@@ -411,8 +412,9 @@ def summarize(extras: dict, line: dict) -> dict:
                                                 for f in ("lloyd8s", "lut16") for m in (512, 4096)]
     r["lut16_gemv_frac_b1_8_16"] = [get(extras, f"lut16_gemv_b{b}", "frac_hbm") for b in (1, 8, 16)]
     r["lloyd8s_gemv_frac_b1"] = get(extras, "lloyd8s_gemv_b1", "frac_hbm")
-    r["wf_gemv_frac_b1_16"] = [get(extras, "water_filling_large", f"gemv_b{b}", "frac_hbm") for b in (1, 16)]
+    r["wf_gemv_frac_b1_2_16"] = [get(extras, "water_filling_large", f"gemv_b{b}", "frac_hbm") for b in (1, 2, 16)]
     r["lloyd_g32_ms_per_matrix"] = get(extras, "lloyd_g32", "ms_per_matrix")
+    r["lloyd_g32_xu_frac"] = get(extras, "lloyd_g32", "roofline", "frac")
     r["kmeans16_ms"] = get(extras, "kmeans16", "ms")
     r["ste_frac"] = get(extras, "fake_quant_ste_large", "frac_hbm")
     r["bf16x_frac_enc_dec"] = [get(extras, "bf16x_large", "encode_frac_hbm"), get(extras, "bf16x_large", "decode_frac_hbm")]
@@ -662,9 +664,9 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
                                       "quantize_Gweights/s": round(nw / ms_q / 1e6, 2),
                                       "dequant_us": round(ms_dq * 1e3, 1), "dequant_GB/s": round(dq_b / ms_dq / 1e6, 1),
                                       "dequant_frac_hbm": round(dq_b / ms_dq / 1e6 / peaks["hbm_gbs"], 4)}
-        # the format's GEMV (weights rebuilt as the dequant does, fp32 products), batch 1 / 16
+        # the format's GEMV (weights rebuilt as the dequant does, fp32 products), batch 1 / 2 / 16
         qwf = wq.WfWeight(n_l, k_l, sc, wd, off, pk, total)
-        for b in (1, 16):
+        for b in (1, 2, 16):
             xw = torch.randn((b, k_l), device=dev).to(torch.bfloat16)
             yw = torch.empty((b, n_l), dtype=torch.bfloat16, device=dev)
             gg = graph_of(torch, lambda: wq.gemv_wf(qwf, xw, out=yw))
@@ -780,9 +782,20 @@ def bench_producers(args, wq, torch, dev, stream, peaks, barrier, max_over_ranks
                 made.append(wq.quantize_lloyd(w, wq.LLOYD_G32_WARM, 25)[0])
         ms = max_over_ranks(time_region(torch, stream, lloyd, 2, 1, barrier))
         n_w = nm * 2048 * 2048
+        # special-function roofline: the screen evaluates every (weight, candidate) pair, and
+        # each evaluation needs at least one special-function result (the reciprocal of the
+        # rational transform's denominator, or tanh); the unit gives 16 per clock per SM
+        evals = n_w * 112
+        xu_peak = 16 * torch.cuda.get_device_properties(dev).multi_processor_count * peaks["sm_max_mhz"] * 1e6
         out["lloyd_g32"] = {"Gweights/s": round(n_w / ms / 1e6, 3), "ms_per_matrix": round(ms / nm, 3),
                             "sample": f"{nm} of the 224 matrices 2048x2048",
-                            "extrapolated_224_s": round(ms / nm * 224 / 1e3, 3)}
+                            "extrapolated_224_s": round(ms / nm * 224 / 1e3, 3),
+                            "roofline": {"bound": "xu", "unit": "G candidate evaluations/s",
+                                         "achieved": round(evals / ms / 1e6, 1),
+                                         "peak": round(xu_peak / 1e9, 1),
+                                         "frac": round(evals / ms * 1e3 / xu_peak, 4),
+                                         "peak_basis": "one special-function result per evaluation, "
+                                                       "16 per clock per SM"}}
         del ws
         # the fused LLOYD8S consumer: one grouped GEMV over those matrices, batch 1 (codes
         # 0.5 B + fp32 levels 1 B per weight)
