@@ -525,13 +525,21 @@ __device__ __forceinline__ uint4 wf_st_desc(uint32_t sb, uint32_t b, uint32_t of
 // times 2^127 minus 1/4 that is (idx_5 - 16) * 2^-6 exactly, and times (scale * 4) it is
 // (scale / 16) (idx_5 - 16) rounded once, the reconstruction. FAST: every block of the
 // chunk is valid with a pair-form scale, so nothing branches.
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
 template <bool FAST>
-__device__ __forceinline__ void wf_st_step(const uint8_t* rowdata, uint4 d, uint32_t wd, uint2 xv, float (&acc)[4]) {
-    const uint32_t b = FAST ? (d.y >> 8) & 7u : max((d.y >> 8) & 7u, 3u);     // 0: not decoded
-    const uint32_t bw = b * wd;
-    const uint32_t* wp = reinterpret_cast<const uint32_t*>(rowdata + (d.y >> 21) + (bw & ~3u));
-    const uint32_t sh = (bw & 3u) * 8;
-    const uint32_t lo = __funnelshift_r(wp[0], wp[1], sh), hi = wp[1] >> sh;
+__device__ __forceinline__ void wf_st_step(uint4 d, uint32_t b, uint32_t w0, uint32_t w1, uint32_t sh, uint2 xv,
+                                           float (&acc)[4]) {
+    const uint32_t lo = __funnelshift_r(w0, w1, sh), hi = w1 >> sh;
     const uint32_t h[4] = {lo, __funnelshift_r(lo, hi, 2 * b), __funnelshift_r(lo, hi, 4 * b),
                            __funnelshift_r(lo, hi, 6 * b)};
     uint32_t m[4];
@@ -552,24 +560,43 @@ __device__ __forceinline__ void wf_st_step(const uint8_t* rowdata, uint4 d, uint
     mma_bf16_16816(acc, o[0], o[2], o[1], o[3], xv.x, xv.y);
 }
 
+// Four block columns: the shared-memory loads of all four (descriptors, then the words) are
+// issued before any is decoded, so that their latencies overlap.
+template <bool FAST>
+__device__ __forceinline__ void wf_st_group(uint32_t rowdata, uint32_t meta, uint32_t wd, int nvalid,
+                                            const uint2 (&xv)[4], float (&acc)[2][4]) {
+    uint4 d[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) d[u] = lds_v4(meta + 16 * u);
+    uint32_t b[4], w0[4], w1[4], sh[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        b[u] = FAST ? (d[u].y >> 8) & 7u : max((d[u].y >> 8) & 7u, 3u);     // 0: not decoded
+        const uint32_t bw = b[u] * wd;
+        const uint32_t wa = rowdata + (d[u].y >> 21) + (bw & ~3u);
+        w0[u] = lds_u32(wa);
+        w1[u] = lds_u32(wa + 4);
+        sh[u] = (bw & 3u) * 8;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        if (u < nvalid) wf_st_step<FAST>(d[u], b[u], w0[u], w1[u], sh[u], xv[u], acc[u & 1]);
+}
+
 // The block columns J0 .. J0 + nb - 1 of one staged chunk, in groups of 4 whose activation
 // pieces were loaded 8 columns ahead (xa: the group at hand, xb: the next); after a group
 // is used its registers take the pieces 8 columns further on. FULL: nb == 32.
 template <bool FAST, bool FULL, typename XLoad>
 __device__ __forceinline__ void wf_st_chunk(const WfStage& st, int ri, uint32_t wd, int J0, int nb, XLoad& xload4,
                                             uint2 (&xa)[4], uint2 (&xb)[4], float (&acc)[2][4]) {
-    const uint8_t* rowdata = st.data[ri];
-    const uint4* meta = st.meta[ri];
+    const uint32_t rowdata = smem_u32(st.data[ri]);
+    const uint32_t meta = smem_u32(st.meta[ri]);
 #pragma unroll 1
     for (int jg = 0; jg < 32; jg += 8) {
         if (!FULL && jg >= nb) break;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (FULL || jg + u < nb) wf_st_step<FAST>(rowdata, meta[jg + u], wd, xa[u], acc[u & 1]);
+        wf_st_group<FAST>(rowdata, meta + 16 * jg, wd, FULL ? 4 : nb - jg, xa, acc);
         xload4(J0 + jg + 8, xa);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (FULL || jg + 4 + u < nb) wf_st_step<FAST>(rowdata, meta[jg + 4 + u], wd, xb[u], acc[u & 1]);
+        wf_st_group<FAST>(rowdata, meta + 16 * (jg + 4), wd, FULL ? 4 : nb - jg - 4, xb, acc);
         xload4(J0 + jg + 12, xb);
     }
 }
@@ -789,6 +816,17 @@ wq_status launch_wf_gemv(const uint8_t* packed, int64_t packed_bytes, const uint
                          const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                          const uint16_t* x, int batch, uint16_t* y, cudaStream_t s) {
     if (batch <= 2) {
+        // one warp of 14.6 KB of static shared memory per CTA: ask for the largest shared
+        // memory carve-out, or the driver may leave room for only about 4 CTAs per SM
+        static const bool carve = [] {
+            cudaFuncSetAttribute(wf_gemv_staged_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+            cudaFuncSetAttribute(wf_gemv_staged_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+            cudaGetLastError();
+            return true;
+        }();
+        (void)carve;
         const unsigned sgrid = (unsigned)((n + 4 * kStWarps - 1) / (4 * kStWarps));
         if (batch == 1)
             wf_gemv_staged_kernel<1><<<sgrid, 32 * kStWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off,
