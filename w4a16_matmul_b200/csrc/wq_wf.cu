@@ -491,7 +491,9 @@ constexpr int kStRowBytes = 32 * 40 + 32;      // a chunk of 5-bit blocks, the a
 
 struct WfStage {
     alignas(16) uint8_t data[4][kStRowBytes];  // row i's run, from its 16-byte boundary
-    uint4 meta[4][32];                         // per block: its descriptor (wf_st_desc)
+    uint4 meta[4][33];                         // per block: its descriptor (wf_st_desc); rows one
+                                               // entry apart in the banks, so that a column's four
+                                               // descriptors load without a bank conflict
 };
 struct WfWarpSmem {
     WfStage st[kStStages];
@@ -658,14 +660,18 @@ wf_gemv_staged_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, 
         const bool rok = lane < 4 && row0 + lane < n && ((m_lo | m_end) & 7u) == 0 && m_end >= m_lo + 24 &&
                          m_end - m_lo <= 32 * 40 && (int64_t)m_end <= packed_bytes;
         const uint32_t base = m_lo & ~15u;
-        const uint32_t bytes = rok ? (m_end & ~15u) - base : 0u;  // >= 16 when the run is sound
+        // the copy runs to the 16-byte boundary at or past the run's end when that stays
+        // inside the buffer (a few bytes of the next run come along), else to the one below
+        const uint32_t up = (m_end + 15u) & ~15u;
+        const bool whole = (int64_t)up <= packed_bytes;
+        const uint32_t bytes = rok ? (whole ? up : m_end & ~15u) - base : 0u;   // >= 16 when sound
         uint32_t tot = bytes;
         tot += __shfl_xor_sync(0xFFFFFFFFu, tot, 1);
         tot += __shfl_xor_sync(0xFFFFFFFFu, tot, 2);
         if (lane == 0) mbar_expect_tx(&S.bar[s], tot);
         if (rok) {
             bulk_load(st.data[lane], packed + base, bytes, &S.bar[s]);
-            if ((m_end & 15u) == 8u)        // the run's last 8 bytes end off a 16-byte boundary
+            if (!whole && (m_end & 15u) == 8u)   // the run's last 8 bytes, at the buffer's end
                 *reinterpret_cast<unsigned long long*>(st.data[lane] + (m_end - 8 - base)) =
                     ldg_na_u64(reinterpret_cast<const unsigned long long*>(packed + m_end - 8));
         }
