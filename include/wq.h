@@ -409,9 +409,10 @@ wq_status wq_dequant_wf(const uint8_t* packed, int64_t packed_bytes, const uint1
  *   y      out bf16 [batch, n].
  * Same tolerance as wq_gemv_w4a16. A block outside packed_bytes, or a width outside 3..5,
  * contributes nothing and is flagged for wq_device_error (WQ_EDATA). For batches 1 and 2
- * each row's blocks are read in runs of 32: a run whose offsets do not describe whole
- * blocks back to back inside packed_bytes is not read at all (all of its blocks count as
- * flagged), and a block whose width disagrees with the offsets is flagged. */
+ * each row's blocks are read in runs of 32: a run whose first or end offset is not a
+ * multiple of 8, or that does not lie inside packed_bytes, is not read at all (all of its
+ * blocks count as flagged); inside a run, a block is decoded only when the next block's
+ * offset (or the run's end) lies exactly 8 * width bytes past its own. */
 wq_status wq_gemv_wf(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
                      const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                      const uint16_t* x, int32_t batch, uint16_t* y, wq_stream stream);

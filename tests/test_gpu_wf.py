@@ -212,3 +212,37 @@ def test_gemv_bad_block_is_flagged_not_read(wq):
     y_ref, bound = xd @ wd.T, np.abs(xd) @ np.abs(wd).T
     assert np.all(np.abs(f32(y) - y_ref) <= matmul_tolerance(y_ref, bound))
     assert wq.device_error() == 0
+
+
+@pytest.mark.parametrize("batch", [1, 2])
+def test_gemv_shifted_offset_drops_both_neighbours(wq, batch):
+    """Batches 1-2 check each block against the next block's offset: shifting block 5's
+    offset by 8 bytes breaks blocks 4 and 5 of that row (both flagged, both left out)."""
+    n, k = 4, 1024
+    w = _weights(23, n, k)
+    q, enc = _oracle_encoding(wq, w, 0.0)                     # every block 5 bits
+    x = to_dev_bits(workloads.activations(batch, k, workloads.LUT16, 2))
+    kb = k // 64
+    q.blk_off[2 * kb + 5] += 8
+    y = wq.gemv_wf(q, x)
+    torch.cuda.synchronize()
+    code = ctypes.c_int32(0)
+    assert wq._lib.wq_device_error(ctypes.byref(code)) == wq.WQ_EDATA and code.value == 2002
+    wd = oracle.bf16_to_f64(oracle.wf_dequant(*enc, n, k))
+    wd[2, 4 * 64:6 * 64] = 0.0
+    xd = oracle.bf16_to_f64(bits(x))
+    y_ref, bound = xd @ wd.T, np.abs(xd) @ np.abs(wd).T
+    assert np.all(np.abs(f32(y) - y_ref) <= matmul_tolerance(y_ref, bound))
+    assert wq.device_error() == 0
+
+
+@pytest.mark.parametrize("batch", [1, 2])
+def test_gemv_run_ending_at_the_buffer_end(wq, batch):
+    """All blocks at 3 bits (24 bytes): 9 blocks end 8 bytes short of a 16-byte boundary,
+    exactly at the end of the buffer, so the last run's tail is read apart from its bulk
+    copy; 3 rows leave a row of the warp empty."""
+    n, k = 3, 192
+    w = _weights(29, n, k)
+    q, enc = _oracle_encoding(wq, w, float("inf"))
+    assert q.total == 216 and q.packed.numel() == 216
+    _gemv_check(wq, q, enc, workloads.activations(batch, k, workloads.LUT16, 4))
