@@ -516,17 +516,8 @@ __device__ __forceinline__ uint4 wf_st_desc(uint32_t sb, uint32_t b, uint32_t of
     return make_uint4(sx, (off << 21) | (b << 8) | mp, 1u << (32 - 2 * b), (1u << 21) + (1u << (5 + b)));
 }
 
-// One block column of the staged GEMV: the lane decodes word wd (codes 8 wd .. 8 wd + 7) of
-// its row's block and issues the column's MMA. The word's b bytes start at byte b wd of the
-// block. Pair j (codes 2j, 2j + 1) is the window shifted right by 2jb (a funnel shift, h);
-// h * 2^(32 - 2b) keeps just the pair, at the top of the word, and the high half of its
-// product with 2^21 + 2^(5 + b) is the pair shifted right by 11 (code 2j + 1 at bits
-// 21 - b .. 20) plus the pair shifted right by 27 - b (code 2j at bits 5 - b .. 4): both
-// shifts are exact and the two ranges do not overlap, so no carry disturbs the idx_5
-// fields, which the mask then isolates. As bf16 numbers the fields are idx_5 * 2^-133;
-// times 2^127 minus 1/4 that is (idx_5 - 16) * 2^-6 exactly, and times (scale * 4) it is
-// (scale / 16) (idx_5 - 16) rounded once, the reconstruction. FAST: every block of the
-// chunk is valid with a pair-form scale, so nothing branches.
+// Shared-memory loads by 32-bit shared address (volatile: they stay after the stage's
+// mbarrier wait, which the compiler sees only as an asm with a memory clobber).
 __device__ __forceinline__ uint4 lds_v4(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
@@ -538,6 +529,17 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
     return v;
 }
 
+// One block column of the staged GEMV: the lane decodes word wd (codes 8 wd .. 8 wd + 7) of
+// its row's block and issues the column's MMA. The word's b bytes start at byte b wd of the
+// block. Pair j (codes 2j, 2j + 1) is the window shifted right by 2jb (a funnel shift, h);
+// h * 2^(32 - 2b) keeps just the pair, at the top of the word, and the high half of its
+// product with 2^21 + 2^(5 + b) is the pair shifted right by 11 (code 2j + 1 at bits
+// 21 - b .. 20) plus the pair shifted right by 27 - b (code 2j at bits 5 - b .. 4): both
+// shifts are exact and the two ranges do not overlap, so no carry disturbs the idx_5
+// fields, which the mask then isolates. As bf16 numbers the fields are idx_5 * 2^-133;
+// times 2^127 minus 1/4 that is (idx_5 - 16) * 2^-6 exactly, and times (scale * 4) it is
+// (scale / 16) (idx_5 - 16) rounded once, the reconstruction. FAST: every block of the
+// chunk is valid with a pair-form scale, so nothing branches.
 template <bool FAST>
 __device__ __forceinline__ void wf_st_step(uint4 d, uint32_t b, uint32_t w0, uint32_t w1, uint32_t sh, uint2 xv,
                                            float (&acc)[4]) {
