@@ -49,10 +49,6 @@ constexpr int BM = 128;            // weight rows per CTA (MMA M)
 // Columns per stage, KB: 64 (one 128-byte swizzle row of bf16) or 128 (two such tiles, used
 // when K % 128 == 0: twice the reconstruction work per stage for the same bookkeeping).
 
-#ifndef WQ_GEMM_BIG_SLOTS
-#define WQ_GEMM_BIG_SLOTS 0
-#endif
-
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
