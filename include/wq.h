@@ -273,7 +273,10 @@ void wq_gemv_plan_destroy(wq_gemv_plan plan);
  * effect at the next wq_gemv_plan_launch. The pages describe no such mode. */
 wq_status wq_gemv_plan_set_overlap(wq_gemv_plan plan, int32_t enable);
 
-/* Bytes of device workspace wq_gemm_w4a16 needs for this weight and m (0 if none). */
+/* Bytes of device workspace wq_gemm_w4a16 needs for this weight and m (0 if none): fp32
+ * partial sums where K is split across CTAs (small m, or a last wave of at most half the
+ * SMs after up to three whole waves, its partial sums up to 64 MiB), plus LUT16's converted
+ * activations. */
 size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m);
 
 /* Prefill-side W4A16 GEMM on the tcgen05 tensor cores ([KM] §4.1 large batch; [DG] §3.2
@@ -426,10 +429,12 @@ wq_status wq_gemv_wf(const uint8_t* packed, int64_t packed_bytes, const uint16_t
  * that the library allocates statically (a file-scope device array of
  * WQ_GEMM_STATIC_SCRATCH_BYTES); every GPU that loads libwq holds that array until the
  * process exits. This entry point itself allocates and frees nothing.
- *   - Same arguments, layout, tolerance and results as wq_gemm_w4a16.
- *   - A problem whose scratch need (wq_gemm_workspace_bytes) exceeds
- *     WQ_GEMM_STATIC_SCRATCH_BYTES is rejected with WQ_EINVAL; use wq_gemm_w4a16 with a
- *     workspace for it.
+ *   - Same arguments, layout, tolerance and results as wq_gemm_w4a16. A last wave is split
+ *     only as far as its partial sums fit the array, so the launches may differ from
+ *     wq_gemm_w4a16's where that one would use more.
+ *   - A problem whose scratch need still exceeds WQ_GEMM_STATIC_SCRATCH_BYTES (e.g. the
+ *     split-K partial sums of a small m) is rejected with WQ_EINVAL; use wq_gemm_w4a16 with
+ *     a workspace for it.
  *   - All calls share the one array, which keeps the last call's contents (every call
  *     writes all the scratch it reads, so nothing has to start at zero). Calls whose GPU
  *     work overlaps (e.g. on two streams) race on it: serialise them.

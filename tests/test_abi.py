@@ -128,10 +128,11 @@ def test_binding_refuses_cpu_tensors(wq):
 
 def test_gemm_workspace_sizes(wq):
     """Host-side GEMM planning (no GPU: the SM count falls back to the B200's 148). Up to 16
-    activation rows run on the GEMV and need nothing; on 4096 x 11008 the large m runs in
-    whole waves without scratch and m = 512 splits the tail. LUT16 plans the same launches
-    as DYADIC4 and adds, in front, its scaled fp16 activations (2 m k bytes) and the rows'
-    fp32 factors (4 m bytes), each rounded up to 1 KB."""
+    activation rows run on the GEMV and need nothing; on 4096 x 11008, m = 512 splits K two
+    ways (64 tiles of 128 x 256) and m = 4096 runs 3 whole waves and splits its last 68
+    tiles two ways. LUT16 plans the same launches as DYADIC4 and adds, in front, its scaled
+    fp16 activations (2 m k bytes) and the rows' fp32 factors (4 m bytes), each rounded up
+    to 1 KB."""
     def ws(fmt, group, n, k, m):
         d = wq.WqWeight(fmt, group, n, k, None, None)
         return int(wq._lib.wq_gemm_workspace_bytes(ctypes.byref(d), m))
@@ -139,7 +140,7 @@ def test_gemm_workspace_sizes(wq):
     n, k = 4096, 11008
     for fmt, group in [(wq.FMT_DYADIC4, 64), (wq.FMT_LUT16, 64), (wq.FMT_LLOYD8S, 32)]:
         assert ws(fmt, group, n, k, 12) == 0 and ws(fmt, group, n, k, 16) == 0
-    assert ws(wq.FMT_DYADIC4, 64, n, k, 4096) == 0
+    assert ws(wq.FMT_DYADIC4, 64, n, k, 4096) == 2 * 68 * 128 * 256 * 4
     assert ws(wq.FMT_DYADIC4, 64, n, k, 512) == 16 << 20
     for m in (17, 48, 100, 128, 200, 512, 4096):
         for nn, kk in [(n, k), (11008, 4096), (200, 320)]:

@@ -124,6 +124,25 @@ wq_status check_bf16x_shape(int64_t n, int64_t k) {
 }
 
 }  // namespace
+wq_status gemm_checked(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
+                       size_t ws_bytes, cudaStream_t stream, size_t tail_cap) {
+    g_last_error[0] = 0;
+    wq_status st = check_weight(w);
+    if (st) return st;
+    if (w->k % 64 != 0) return fail(WQ_EINVAL, "GEMM needs k %% 64 == 0 (k=%lld)", (long long)w->k);
+    if (m < 1 || m > (1LL << 31) - 1) return fail(WQ_EINVAL, "m=%lld outside 1..2^31-1", (long long)m);
+    if ((st = check_ptr(x, "x", false))) return st;
+    if ((st = check_ptr(y, "y", false))) return st;
+    size_t need = gemm_workspace_bytes(*w, m, tail_cap);
+    if (need > 0) {
+        if ((st = check_ptr(ws, "ws", false))) return st;
+        if (ws_bytes < need)
+            return fail(WQ_EINVAL, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
+    }
+    if ((st = check_injected())) return st;
+    return launch_gemm(*w, x, m, y, ws, ws_bytes, stream, tail_cap);
+}
+
 }  // namespace wq
 
 using namespace wq;
@@ -501,23 +520,10 @@ size_t wq_gemm_workspace_bytes(const wq_weight* w, int64_t m) {
     return gemm_workspace_bytes(*w, m);
 }
 
+
 wq_status wq_gemm_w4a16(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
                         size_t ws_bytes, wq_stream stream) {
-    g_last_error[0] = 0;
-    wq_status st = check_weight(w);
-    if (st) return st;
-    if (w->k % 64 != 0) return fail(WQ_EINVAL, "GEMM needs k %% 64 == 0 (k=%lld)", (long long)w->k);
-    if (m < 1 || m > (1LL << 31) - 1) return fail(WQ_EINVAL, "m=%lld outside 1..2^31-1", (long long)m);
-    if ((st = check_ptr(x, "x", false))) return st;
-    if ((st = check_ptr(y, "y", false))) return st;
-    size_t need = gemm_workspace_bytes(*w, m);
-    if (need > 0) {
-        if ((st = check_ptr(ws, "ws", false))) return st;
-        if (ws_bytes < need)
-            return fail(WQ_EINVAL, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
-    }
-    if ((st = check_injected())) return st;
-    return launch_gemm(*w, x, m, y, ws, ws_bytes, (cudaStream_t)stream);
+    return gemm_checked(w, x, m, y, ws, ws_bytes, (cudaStream_t)stream, kGemmTailScratch);
 }
 
 }  // extern "C"

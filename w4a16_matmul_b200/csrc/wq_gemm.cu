@@ -591,9 +591,9 @@ struct Plan {
     int full, tail_splits, tail_kt_per_split;
 };
 
-// Scratch the last-wave split may use (it then stays within the static scratch of
-// wq_gemm_w4a16_static).
-constexpr size_t kTailScratchBytes = (size_t)16 << 20;
+#ifndef WQ_GEMM_TAIL_WAVES
+#define WQ_GEMM_TAIL_WAVES 3           // the last-wave split runs after at most this many whole waves
+#endif
 
 #ifndef WQ_GEMM_BN128_MAX
 #define WQ_GEMM_BN128_MAX 128
@@ -605,7 +605,7 @@ constexpr size_t kTailScratchBytes = (size_t)16 << 20;
 #define WQ_GEMM_BN384 1
 #endif
 
-Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt) {
+Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt, size_t tail_cap) {
     Plan p;
     const int sms = sm_count();
     p.kb = 64;
@@ -660,22 +660,22 @@ Plan plan_for(int64_t M, int64_t N, int64_t K, int fmt) {
     }
     p.kt_per_split = (KT + splits - 1) / splits;
     p.splits = (KT + p.kt_per_split - 1) / p.kt_per_split;
-    // One or two whole waves of wide tiles plus a tail of at most half a wave: a single pass
+    // One to three whole waves of wide tiles plus a tail of at most half a wave: a single pass
     // spends a full wave's time on the tail. Run the whole waves as they are, then the tail
     // tiles with K split s ways (s tail CTAs per tile fit one wave: the tail then takes about
-    // 1/s of a wave), each split keeping >= 512 columns, the partial sums within
-    // kTailScratchBytes. (Measured on 11008 x 4096: m = 512, 1 wave + 24 tiles, 1.25x; with
-    // 9 waves + 44 tiles at m = 4096 the second launch and its reduction cost what the tail
-    // saves, hence the two-wave limit.)
+    // 1/s of a wave), each split keeping >= 512 columns, the partial sums within tail_cap.
+    // (Measured on 11008 x 4096: m = 512, 1 wave + 24 tiles, 1.25x; with 9 waves + 44 tiles
+    // at m = 4096 the second launch and its reduction cost what the tail saves, hence the
+    // limit on whole waves.)
     p.full = (int)tiles;
     p.tail_splits = 1;
     p.tail_kt_per_split = KT;
     if (p.bn >= 128 && p.splits == 1) {
         const int64_t full = tiles / sms * sms, tail = tiles - full;
-        if (full > 0 && full <= 2 * sms && tail > 0 && 2 * tail <= sms) {
+        if (full > 0 && full <= WQ_GEMM_TAIL_WAVES * sms && tail > 0 && 2 * tail <= sms) {
             int64_t sp = sms / tail;
             while (sp > 1 && KT / sp < min_narrow) --sp;
-            while (sp > 1 && (size_t)sp * tail * BM * p.bn * sizeof(float) > kTailScratchBytes) --sp;
+            while (sp > 1 && (size_t)sp * tail * BM * p.bn * sizeof(float) > tail_cap) --sp;
             if (sp > 1) {
                 p.tail_kt_per_split = (KT + (int)sp - 1) / (int)sp;
                 p.tail_splits = (KT + p.tail_kt_per_split - 1) / p.tail_kt_per_split;
@@ -761,9 +761,9 @@ size_t lut16_x_bytes(const wq_weight& w, int64_t m) {
     return lut16_xh_bytes(w, m) + (((size_t)m * 4 + 1023) & ~(size_t)1023);
 }
 
-size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
+size_t gemm_workspace_bytes(const wq_weight& w, int64_t m, size_t tail_cap) {
     if (m <= kGemvMaxRows) return 0;
-    const Plan p = plan_for(m, w.n, w.k, w.fmt);
+    const Plan p = plan_for(m, w.n, w.k, w.fmt, tail_cap);
     const size_t tile = (size_t)BM * (size_t)p.bn * sizeof(float);
     const size_t tiles = (size_t)p.grid_n * (size_t)p.grid_m;
     size_t partial = 0;
@@ -773,16 +773,16 @@ size_t gemm_workspace_bytes(const wq_weight& w, int64_t m) {
 }
 
 wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
-                      size_t ws_bytes, cudaStream_t s) {
+                      size_t ws_bytes, cudaStream_t s, size_t tail_cap) {
     const int M = (int)m, N = (int)w.n, K = (int)w.k;
     if (m <= kGemvMaxRows) {
         const GemvProblem prob{w.packed, w.aux, x, y, N, K};
         return launch_gemv(w.fmt, w.group, &prob, 1, M, s);
     }
-    const Plan p = plan_for(M, N, K, w.fmt);
+    const Plan p = plan_for(M, N, K, w.fmt, tail_cap);
     auto enc = encode_fn();
     if (!enc) return fail(WQ_ECUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
-    const size_t need = gemm_workspace_bytes(w, m);
+    const size_t need = gemm_workspace_bytes(w, m, tail_cap);
     if (need > 0 && (ws == nullptr || ws_bytes < need)) return fail(WQ_EINVAL, "workspace too small");
     const bool lut = w.fmt == WQ_FMT_LUT16;
     const void* xa = x;                    // the activations the MMA reads

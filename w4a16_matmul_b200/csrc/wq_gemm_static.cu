@@ -82,7 +82,8 @@ extern "C" wq_status wq_gemm_w4a16_static(const wq_weight* w, const uint16_t* x,
                                           uint16_t* y, wq_stream stream) {
     using namespace wq;
     if (!w) return fail(WQ_EINVAL, "weight descriptor is NULL");
-    const size_t need = wq_gemm_workspace_bytes(w, m);
+    // planned so that a last-wave split stays within the static scratch
+    const size_t need = m < 1 ? 0 : gemm_workspace_bytes(*w, m, kStaticScratchBytes);
     if (need > kStaticScratchBytes)
         return fail(WQ_EINVAL,
                     "this GEMM (n=%lld, k=%lld, m=%lld) needs %zu bytes of scratch; the static scratch "
@@ -93,5 +94,6 @@ extern "C" wq_status wq_gemm_w4a16_static(const wq_weight* w, const uint16_t* x,
         wq_status st = scratch_address(&scratch);
         if (st) return st;
     }
-    return wq_gemm_w4a16(w, x, m, y, scratch, need > 0 ? kStaticScratchBytes : 0, stream);
+    return gemm_checked(w, x, m, y, scratch, need > 0 ? kStaticScratchBytes : 0, (cudaStream_t)stream,
+                        kStaticScratchBytes);
 }

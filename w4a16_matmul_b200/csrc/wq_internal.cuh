@@ -130,9 +130,15 @@ wq_status launch_lloyd_g32(const uint16_t* w, int64_t n, int64_t k, int rounds, 
 wq_status launch_kmeans16(const uint16_t* w, int64_t n, int64_t k, int rounds, uint8_t* codes,
                           uint8_t* packed, uint16_t* lut, float* trace, cudaStream_t s);
 
-size_t gemm_workspace_bytes(const wq_weight& w, int64_t m);
+// The GEMM's last-wave split may use up to tail_cap bytes of fp32 partial sums (the static
+// scratch entry plans with its own, smaller cap).
+constexpr size_t kGemmTailScratch = (size_t)64 << 20;
+size_t gemm_workspace_bytes(const wq_weight& w, int64_t m, size_t tail_cap = kGemmTailScratch);
 wq_status launch_gemm(const wq_weight& w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
-                      size_t ws_bytes, cudaStream_t s);
+                      size_t ws_bytes, cudaStream_t s, size_t tail_cap = kGemmTailScratch);
+// wq_gemm_w4a16's argument checks and launch, planned with the given tail cap.
+wq_status gemm_checked(const wq_weight* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
+                       size_t ws_bytes, cudaStream_t s, size_t tail_cap);
 
 // Reads and clears the device error word written by expired bounded waits.
 wq_status read_device_error(int32_t* code);
