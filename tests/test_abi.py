@@ -141,6 +141,11 @@ def test_gemm_workspace_sizes(wq):
     for fmt, group in [(wq.FMT_DYADIC4, 64), (wq.FMT_LUT16, 64), (wq.FMT_LLOYD8S, 32)]:
         assert ws(fmt, group, n, k, 12) == 0 and ws(fmt, group, n, k, 16) == 0
     assert ws(wq.FMT_DYADIC4, 64, n, k, 4096) == 2 * 68 * 128 * 256 * 4
+    # 11008 x 4096 at m = 4096 takes 384-row tiles (6 whole waves + 58 tiles: more than
+    # three whole waves) and at m = 2048 has 4 waves + 96 tiles (more than half a wave
+    # left): neither splits its last wave
+    assert ws(wq.FMT_DYADIC4, 64, 11008, 4096, 4096) == 0
+    assert ws(wq.FMT_DYADIC4, 64, 11008, 4096, 2048) == 0
     assert ws(wq.FMT_DYADIC4, 64, n, k, 512) == 16 << 20
     for m in (17, 48, 100, 128, 200, 512, 4096):
         for nn, kk in [(n, k), (11008, 4096), (200, 320)]:
