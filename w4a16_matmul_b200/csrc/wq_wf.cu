@@ -464,21 +464,23 @@ wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const u
 // shared memory by bulk asynchronous copies, products on the tensor cores.
 //   * A warp owns 4 weight rows. Its blocks come in chunks of 32 block columns: one lane
 //     reads each block's offset, width and scale (coalesced), checks them, and writes a
-//     packed descriptor to shared memory; one lane then copies each row's bytes of the chunk,
+//     16-byte descriptor to shared memory; lanes 0-3 each copy one row's bytes of the chunk,
 //     a contiguous run of the bit streams, into shared memory with one cp.async.bulk (from
-//     the 16-byte boundary at or below the run's start; the run's last 8 bytes by a plain
-//     load when its end is not on a 16-byte boundary), completing on the stage's mbarrier.
-//     WQ_WF_ST_STAGES stages per warp: while one chunk is decoded the next ones are in
-//     flight, with no registers held for them.
+//     the 16-byte boundary at or below the run's start to the one at or past its end; at
+//     the end of the buffer, to the one below, and the run's last 8 bytes by a plain load),
+//     completing on the stage's mbarrier. WQ_WF_ST_STAGES stages per warp: while one chunk
+//     is decoded the next ones are in flight, with no registers held for them.
 //   * One mma.sync m16n8k16 per block column covers the 4 rows x 64 columns: lane (g, t)
 //     decodes word t + 4 (g >> 2) (codes 8w .. 8w + 7) of row g & 3's block, its pairs
 //     0 and 1 as A row g (quarter g >> 2 of the columns), pairs 2 and 3 as A row g + 8
 //     (quarter 2 + (g >> 2)). B column 4 i + q holds activation row i at the columns of
 //     quarter q (4 consecutive values per lane: one 8-byte load), so D[rho][4 i + q(rho)]
 //     are the useful sums (16 of the 128 outputs) and y[i][row] adds four of them.
-// A chunk whose offsets do not describe a contiguous run inside packed_bytes is not read;
-// a block whose width or offset is inconsistent is not decoded; both are reported (2002)
-// and contribute nothing. An expired wait for a copy is reported as 2100.
+// A chunk whose first or end offset is not a multiple of 8, or whose run does not lie inside
+// packed_bytes, is not read; inside a run, a block is decoded only when its width is 3..5
+// and the next block's offset (or the run's end) lies 8 * width bytes past its own. Both
+// are reported (2002) and contribute nothing. An expired wait for a copy is reported as
+// 2100.
 #ifndef WQ_WF_ST_WARPS
 #define WQ_WF_ST_WARPS 1               // warps per CTA (each independent)
 #endif
