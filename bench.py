@@ -412,7 +412,7 @@ def summarize(extras: dict, line: dict) -> dict:
                                                 for f in ("lloyd8s", "lut16") for m in (512, 4096)]
     r["lut16_gemv_frac_b1_8_16"] = [get(extras, f"lut16_gemv_b{b}", "frac_hbm") for b in (1, 8, 16)]
     r["lloyd8s_gemv_frac_b1"] = get(extras, "lloyd8s_gemv_b1", "frac_hbm")
-    r["wf_gemv_frac_b1_2_16"] = [get(extras, "water_filling_large", f"gemv_b{b}", "frac_hbm") for b in (1, 2, 16)]
+    r["wf_gemv_frac_b1_2_4_16"] = [get(extras, "water_filling_large", f"gemv_b{b}", "frac_hbm") for b in (1, 2, 4, 16)]
     r["lloyd_g32_ms_per_matrix"] = get(extras, "lloyd_g32", "ms_per_matrix")
     r["lloyd_g32_xu_frac"] = get(extras, "lloyd_g32", "roofline", "frac")
     r["kmeans16_ms"] = get(extras, "kmeans16", "ms")
@@ -664,9 +664,9 @@ def run_extras(args, wq, torch, dev, stream, packed, mats, xs, ys, peaks, barrie
                                       "quantize_Gweights/s": round(nw / ms_q / 1e6, 2),
                                       "dequant_us": round(ms_dq * 1e3, 1), "dequant_GB/s": round(dq_b / ms_dq / 1e6, 1),
                                       "dequant_frac_hbm": round(dq_b / ms_dq / 1e6 / peaks["hbm_gbs"], 4)}
-        # the format's GEMV (weights rebuilt as the dequant does, fp32 products), batch 1 / 2 / 16
+        # the format's GEMV (weights rebuilt as the dequant does, fp32 products), batch 1 / 2 / 4 / 16
         qwf = wq.WfWeight(n_l, k_l, sc, wd, off, pk, total)
-        for b in (1, 2, 16):
+        for b in (1, 2, 4, 16):
             xw = torch.randn((b, k_l), device=dev).to(torch.bfloat16)
             yw = torch.empty((b, n_l), dtype=torch.bfloat16, device=dev)
             gg = graph_of(torch, lambda: wq.gemv_wf(qwf, xw, out=yw))

@@ -411,7 +411,7 @@ wq_status wq_dequant_wf(const uint8_t* packed, int64_t packed_bytes, const uint1
  *   x      bf16 [batch, k]; batch 1 .. 16.
  *   y      out bf16 [batch, n].
  * Same tolerance as wq_gemv_w4a16. A block outside packed_bytes, or a width outside 3..5,
- * contributes nothing and is flagged for wq_device_error (WQ_EDATA). For batches 1 and 2
+ * contributes nothing and is flagged for wq_device_error (WQ_EDATA). For batches 1 to 4
  * each row's blocks are read in runs of 32: a run whose first or end offset is not a
  * multiple of 8, or that does not lie inside packed_bytes, is not read at all (all of its
  * blocks count as flagged); inside a run, a block is decoded only when the next block's

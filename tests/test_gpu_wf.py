@@ -146,7 +146,7 @@ def _gemv_check(wq, q, enc, x_bits, rows=None):
 
 
 @pytest.mark.parametrize("n,k", [(1, 64), (5, 2112), (33, 1024), (64, 4096), (19, 28672)])
-@pytest.mark.parametrize("batch", [1, 2, 3, 8, 9, 16])
+@pytest.mark.parametrize("batch", [1, 2, 3, 4, 8, 9, 16])
 def test_gemv_matches_oracle(wq, n, k, batch):
     """The format's GEMV ("MiniCPM5-1B 验证…" §2.1, §6 blocks; the dyadic GEMV's contract) on
     mixed 3/4/5-bit rows: ragged row counts, a row tail of fewer than 32 blocks, batches
@@ -191,7 +191,7 @@ def test_gemv_full_size_sampled_rows(wq):
     w = workloads.f64_to_bf16_bits(g.standard_normal((n, k)) * 0.01)
     q, enc = _oracle_encoding(wq, w, 8e-7)
     rows = np.array([0, 1, 777, 4097, n - 2, n - 1])
-    for batch in (1, 16):
+    for batch in (1, 4, 16):
         _gemv_check(wq, q, enc, workloads.activations(batch, k, workloads.LUT16, batch), rows=rows)
 
 
@@ -214,9 +214,9 @@ def test_gemv_bad_block_is_flagged_not_read(wq):
     assert wq.device_error() == 0
 
 
-@pytest.mark.parametrize("batch", [1, 2])
+@pytest.mark.parametrize("batch", [1, 2, 4])
 def test_gemv_shifted_offset_drops_both_neighbours(wq, batch):
-    """Batches 1-2 check each block against the next block's offset: shifting block 5's
+    """Batches 1-4 check each block against the next block's offset: shifting block 5's
     offset by 8 bytes breaks blocks 4 and 5 of that row (both flagged, both left out)."""
     n, k = 4, 1024
     w = _weights(23, n, k)
@@ -236,7 +236,7 @@ def test_gemv_shifted_offset_drops_both_neighbours(wq, batch):
     assert wq.device_error() == 0
 
 
-@pytest.mark.parametrize("batch", [1, 2])
+@pytest.mark.parametrize("batch", [1, 2, 3])
 def test_gemv_run_ending_at_the_buffer_end(wq, batch):
     """All blocks at 3 bits (24 bytes): 9 blocks end 8 bytes short of a 16-byte boundary,
     exactly at the end of the buffer, so the last run's tail is read apart from its bulk

@@ -460,8 +460,9 @@ wf_gemv_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, const u
         }
 }
 
-// Batches of 1 and 2: y[i, r] = sum_c Wdeq[r, c] x[i, c] with the packed bytes staged in
-// shared memory by bulk asynchronous copies, products on the tensor cores.
+// Batches of 1 to 4: y[i, r] = sum_c Wdeq[r, c] x[i, c] with the packed bytes staged in
+// shared memory by bulk asynchronous copies, products on the tensor cores (one MMA per
+// block column and pair of batch rows, all from the same decoded weights).
 //   * A warp owns 4 weight rows. Its blocks come in chunks of 32 block columns: one lane
 //     reads each block's offset, width and scale (coalesced), checks them, and writes a
 //     16-byte descriptor to shared memory; lanes 0-3 each copy one row's bytes of the chunk,
@@ -542,9 +543,9 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
 // times 2^127 minus 1/4 that is (idx_5 - 16) * 2^-6 exactly, and times (scale * 4) it is
 // (scale / 16) (idx_5 - 16) rounded once, the reconstruction. FAST: every block of the
 // chunk is valid with a pair-form scale, so nothing branches.
-template <bool FAST>
-__device__ __forceinline__ void wf_st_step(uint4 d, uint32_t b, uint32_t w0, uint32_t w1, uint32_t sh, uint2 xv,
-                                           float (&acc)[4]) {
+template <bool FAST, int NM>
+__device__ __forceinline__ void wf_st_step(uint4 d, uint32_t b, uint32_t w0, uint32_t w1, uint32_t sh,
+                                           const uint2 (&xv)[NM], float (&acc)[NM][4]) {
     const uint32_t lo = __funnelshift_r(w0, w1, sh), hi = w1 >> sh;
     const uint32_t h[4] = {lo, __funnelshift_r(lo, hi, 2 * b), __funnelshift_r(lo, hi, 4 * b),
                            __funnelshift_r(lo, hi, 6 * b)};
@@ -563,14 +564,15 @@ __device__ __forceinline__ void wf_st_step(uint4 d, uint32_t b, uint32_t w0, uin
             o[j] = pack_bf16x2(s16 * (float)((int)(m[j] & 0xFFFFu) - 16), s16 * (float)((int)(m[j] >> 16) - 16));
     }
     if (!FAST && d.y == 0u) o[0] = o[1] = o[2] = o[3] = 0u;
-    mma_bf16_16816(acc, o[0], o[2], o[1], o[3], xv.x, xv.y);
+#pragma unroll
+    for (int mi = 0; mi < NM; ++mi) mma_bf16_16816(acc[mi], o[0], o[2], o[1], o[3], xv[mi].x, xv[mi].y);
 }
 
 // Four block columns: the shared-memory loads of all four (descriptors, then the words) are
 // issued before any is decoded, so that their latencies overlap.
-template <bool FAST>
+template <bool FAST, int NM>
 __device__ __forceinline__ void wf_st_group(uint32_t rowdata, uint32_t meta, uint32_t wd, int nvalid,
-                                            const uint2 (&xv)[4], float (&acc)[2][4]) {
+                                            const uint2 (&xv)[NM][4], float (&acc)[2][NM][4]) {
     uint4 d[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) d[u] = lds_v4(meta + 16 * u);
@@ -586,23 +588,28 @@ __device__ __forceinline__ void wf_st_group(uint32_t rowdata, uint32_t meta, uin
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-        if (u < nvalid) wf_st_step<FAST>(d[u], b[u], w0[u], w1[u], sh[u], xv[u], acc[u & 1]);
+        if (u < nvalid) {
+            uint2 xs[NM];
+#pragma unroll
+            for (int mi = 0; mi < NM; ++mi) xs[mi] = xv[mi][u];
+            wf_st_step<FAST, NM>(d[u], b[u], w0[u], w1[u], sh[u], xs, acc[u & 1]);
+        }
 }
 
 // The block columns J0 .. J0 + nb - 1 of one staged chunk, in groups of 4 whose activation
 // pieces were loaded 8 columns ahead (xa: the group at hand, xb: the next); after a group
 // is used its registers take the pieces 8 columns further on. FULL: nb == 32.
-template <bool FAST, bool FULL, typename XLoad>
+template <bool FAST, bool FULL, int NM, typename XLoad>
 __device__ __forceinline__ void wf_st_chunk(const WfStage& st, int ri, uint32_t wd, int J0, int nb, XLoad& xload4,
-                                            uint2 (&xa)[4], uint2 (&xb)[4], float (&acc)[2][4]) {
+                                            uint2 (&xa)[NM][4], uint2 (&xb)[NM][4], float (&acc)[2][NM][4]) {
     const uint32_t rowdata = smem_u32(st.data[ri]);
     const uint32_t meta = smem_u32(st.meta[ri]);
 #pragma unroll 1
     for (int jg = 0; jg < 32; jg += 8) {
         if (!FULL && jg >= nb) break;
-        wf_st_group<FAST>(rowdata, meta + 16 * jg, wd, FULL ? 4 : nb - jg, xa, acc);
+        wf_st_group<FAST, NM>(rowdata, meta + 16 * jg, wd, FULL ? 4 : nb - jg, xa, acc);
         xload4(J0 + jg + 8, xa);
-        wf_st_group<FAST>(rowdata, meta + 16 * (jg + 4), wd, FULL ? 4 : nb - jg - 4, xb, acc);
+        wf_st_group<FAST, NM>(rowdata, meta + 16 * (jg + 4), wd, FULL ? 4 : nb - jg - 4, xb, acc);
         xload4(J0 + jg + 12, xb);
     }
 }
@@ -707,28 +714,41 @@ wf_gemv_staged_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, 
         return __any_sync(0xFFFFFFFFu, special);
     };
 
-    // this lane's activation columns: row bi, quarter q = g & 3 of each block column
-    const int bi = min(NB == 1 ? 0 : g >> 2, batch - 1);
+    // this lane's activation columns: in MMA mi, row 2 mi + (g >> 2) (row 0 at batch 1),
+    // quarter q = g & 3 of each block column
+    constexpr int NM = (NB + 1) / 2;             // MMAs per block column (2 batch rows each)
     const int q = g & 3;
-    const uint16_t* xl = x + (size_t)bi * k + 32 * (q & 1) + 8 * t + 4 * (q >> 1);
+    const uint16_t* xl[NM];
+#pragma unroll
+    for (int mi = 0; mi < NM; ++mi) {
+        const int bi = min(NB == 1 ? 0 : 2 * mi + (g >> 2), batch - 1);
+        xl[mi] = x + (size_t)bi * k + 32 * (q & 1) + 8 * t + 4 * (q >> 1);
+    }
     const int ri = g & 3;
     const uint32_t wd = (uint32_t)(t + 4 * (g >> 2));   // decoded row and word
     // the activation pieces of steps J .. J + 3 (J: block column; past the row's end a
     // repeated in-bounds load whose value is not used)
-    auto xload4 = [&](int J, uint2 (&xr)[4]) {
-        if (J + 3 < kb) {
-            const uint2* p = reinterpret_cast<const uint2*>(xl + (size_t)J * 64);
+    auto xload4 = [&](int J, uint2 (&xr)[NM][4]) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) xr[u] = __ldg(p + 16 * u);
-        } else {
+        for (int mi = 0; mi < NM; ++mi) {
+            if (J + 3 < kb) {
+                const uint2* p = reinterpret_cast<const uint2*>(xl[mi] + (size_t)J * 64);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                xr[u] = __ldg(reinterpret_cast<const uint2*>(xl + (size_t)min(J + u, kb - 1) * 64));
+                for (int u = 0; u < 4; ++u) xr[mi][u] = __ldg(p + 16 * u);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    xr[mi][u] = __ldg(reinterpret_cast<const uint2*>(xl[mi] + (size_t)min(J + u, kb - 1) * 64));
+            }
         }
     };
 
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    uint2 xa[4], xb[4];                          // steps 8 apart: the next two groups of 4
+    float acc[2][NM][4];
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int mi = 0; mi < NM; ++mi) acc[e][mi][0] = acc[e][mi][1] = acc[e][mi][2] = acc[e][mi][3] = 0.f;
+    uint2 xa[NM][4], xb[NM][4];                  // steps 8 apart: the next two groups of 4
     xload4(0, xa);
     xload4(4, xb);
     uint32_t slow = 0;                           // bit s: stage s holds a chunk for the general loop
@@ -756,11 +776,11 @@ wf_gemv_staged_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, 
         const WfStage& st = S.st[s];
         const int nb = min(32, kb - 32 * c);
         if (nb == 32 && !((slow >> s) & 1u))
-            wf_st_chunk<true, true>(st, ri, wd, 32 * c, 32, xload4, xa, xb, acc);
+            wf_st_chunk<true, true, NM>(st, ri, wd, 32 * c, 32, xload4, xa, xb, acc);
         else if (nb == 32)
-            wf_st_chunk<false, true>(st, ri, wd, 32 * c, 32, xload4, xa, xb, acc);
+            wf_st_chunk<false, true, NM>(st, ri, wd, 32 * c, 32, xload4, xa, xb, acc);
         else
-            wf_st_chunk<false, false>(st, ri, wd, 32 * c, nb, xload4, xa, xb, acc);
+            wf_st_chunk<false, false, NM>(st, ri, wd, 32 * c, nb, xload4, xa, xb, acc);
         __syncwarp();                            // stage s is refilled next
     }
     if (dead) {
@@ -771,14 +791,19 @@ wf_gemv_staged_kernel(const uint8_t* __restrict__ packed, int64_t packed_bytes, 
         return;
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[0][e] += acc[1][e];
-    // lane (g, t): t even holds the quarter-0/1 sums, t odd the quarter-2/3 sums of batch row t >> 1
-    float v = (t & 1) ? (g < 4 ? acc[0][2] : acc[0][3]) : (g < 4 ? acc[0][0] : acc[0][1]);
-    v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-    v += __shfl_xor_sync(0xFFFFFFFFu, v, 16);
-    const int ob = t >> 1;
-    if (g < 4 && !(t & 1) && ob < NB && ob < batch && row0 + g < n)
-        y[(size_t)ob * n + row0 + g] = (uint16_t)float_to_bf16_bits(v);
+    for (int mi = 0; mi < NM; ++mi) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[0][mi][e] += acc[1][mi][e];
+        // lane (g, t): t even holds the quarter-0/1 sums, t odd the quarter-2/3 sums of the
+        // MMA's batch row t >> 1
+        const float* a = acc[0][mi];
+        float v = (t & 1) ? (g < 4 ? a[2] : a[3]) : (g < 4 ? a[0] : a[1]);
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, 16);
+        const int ob = 2 * mi + (t >> 1);
+        if (g < 4 && !(t & 1) && ob < NB && ob < batch && row0 + g < n)
+            y[(size_t)ob * n + row0 + g] = (uint16_t)float_to_bf16_bits(v);
+    }
 }
 
 int grid_cap(int64_t want) {
@@ -818,20 +843,22 @@ wq_status launch_wf_dequant(const uint8_t* packed, int64_t packed_bytes, const u
     return check_launch("wf dequant");
 }
 
-// Batches of 1 and 2 take the staged kernel, larger ones the 16-row one (8192 x 28672 at
-// 4.5 bits per weight: the staged kernel runs batch 1 and 2 in about 100 us, the 16-row
-// one batches 3 to 16 in 245-256 us: it reads each block's width, offset and scale at 16
+// Batches of 1 to 4 take the staged kernel, larger ones the 16-row one (8192 x 28672 at
+// 4.5 bits per weight: the staged kernel runs batch 1 and 2 in about 97 us, the 16-row one
+// batches 3 to 16 in 245-256 us: it reads each block's width, offset and scale at 16
 // different rows per warp step, scattered over many cache lines, with no staging).
 wq_status launch_wf_gemv(const uint8_t* packed, int64_t packed_bytes, const uint16_t* scale,
                          const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                          const uint16_t* x, int batch, uint16_t* y, cudaStream_t s) {
-    if (batch <= 2) {
+    if (batch <= 4) {
         // one warp of 14.6 KB of static shared memory per CTA: ask for the largest shared
         // memory carve-out, or the driver may leave room for only about 4 CTAs per SM
         static const bool carve = [] {
             cudaFuncSetAttribute(wf_gemv_staged_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
             cudaFuncSetAttribute(wf_gemv_staged_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+            cudaFuncSetAttribute(wf_gemv_staged_kernel<4>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
             cudaGetLastError();
             return true;
@@ -841,8 +868,11 @@ wq_status launch_wf_gemv(const uint8_t* packed, int64_t packed_bytes, const uint
         if (batch == 1)
             wf_gemv_staged_kernel<1><<<sgrid, 32 * kStWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off,
                                                                     (int)n, (int)k, x, batch, y);
-        else
+        else if (batch == 2)
             wf_gemv_staged_kernel<2><<<sgrid, 32 * kStWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off,
+                                                                    (int)n, (int)k, x, batch, y);
+        else
+            wf_gemv_staged_kernel<4><<<sgrid, 32 * kStWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off,
                                                                     (int)n, (int)k, x, batch, y);
         return check_launch("wf gemv");
     }
