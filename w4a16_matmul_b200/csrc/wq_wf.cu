@@ -851,19 +851,6 @@ wq_status launch_wf_gemv(const uint8_t* packed, int64_t packed_bytes, const uint
                          const uint8_t* width, const uint32_t* blk_off, int64_t n, int64_t k,
                          const uint16_t* x, int batch, uint16_t* y, cudaStream_t s) {
     if (batch <= 4) {
-        // one warp of 14.6 KB of static shared memory per CTA: ask for the largest shared
-        // memory carve-out, or the driver may leave room for only about 4 CTAs per SM
-        static const bool carve = [] {
-            cudaFuncSetAttribute(wf_gemv_staged_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-            cudaFuncSetAttribute(wf_gemv_staged_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-            cudaFuncSetAttribute(wf_gemv_staged_kernel<4>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-            cudaGetLastError();
-            return true;
-        }();
-        (void)carve;
         const unsigned sgrid = (unsigned)((n + 4 * kStWarps - 1) / (4 * kStWarps));
         if (batch == 1)
             wf_gemv_staged_kernel<1><<<sgrid, 32 * kStWarps, 0, s>>>(packed, packed_bytes, scale, width, blk_off,
