@@ -921,7 +921,8 @@ def run_profile_target(args):
     """A few launches of one kernel on one shape and nothing else, for ncu captures:
     --profile gemm --shape N,K,M (prefill GEMM; gemm_lut16: its LUT16 form, with the
     activation conversion), quantize --shape N,K, dequant --shape N,K,
-    lut16 --shape N,K,B (LUT16 GEMV), lloyd --shape N,K (g32 Lloyd), gumbel --shape N,K
+    lut16 --shape N,K,B (LUT16 GEMV), lloyd8s --shape N,K,B (the fused LLOYD8S GEMV),
+    lloyd --shape N,K (g32 Lloyd), gumbel --shape N,K
     (Gumbel-ST backward at tau = step^2; gumbel1: at tau = 1.0), ste --shape N,K (STE forward),
     kmeans --shape N,K (16-centroid k-means),
     bf16x --shape N,K (BF16X encode + decode), wf --shape N,K
@@ -962,6 +963,13 @@ def run_profile_target(args):
         b = dims[2]
         lut = (torch.randn((n, k // 64, 16), device=dev, generator=gen) * 0.01).to(torch.float16)
         pl = wq.PackedWeight(wq.FMT_LUT16, 64, n, k, packed, lut)
+        x = torch.randn((b, k), device=dev, generator=gen).to(torch.bfloat16)
+        y = torch.empty((b, n), dtype=torch.bfloat16, device=dev)
+        fn = lambda: wq.gemv(pl, x, out=y)
+    elif args.profile == "lloyd8s":
+        b = dims[2]
+        levels = torch.sort(torch.rand((n, k // 32, 8), device=dev, generator=gen) * 0.05, dim=-1).values
+        pl = wq.PackedWeight(wq.FMT_LLOYD8S, 32, n, k, packed, levels.contiguous())
         x = torch.randn((b, k), device=dev, generator=gen).to(torch.bfloat16)
         y = torch.empty((b, n), dtype=torch.bfloat16, device=dev)
         fn = lambda: wq.gemv(pl, x, out=y)
